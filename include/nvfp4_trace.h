@@ -1,0 +1,231 @@
+/*
+ * nvfp4_trace.h -- C ABI of libnvfp4trace.so: NVFP4 block quantization with
+ * train/rollout rounding alignment (TRACE-style guidance), for sm_100a.
+ *
+ * Sources cited below (pages are named by title; none has numbered sections):
+ *   [TRACE]  "TRACE explainer" -- blog.ontle.kr/blog/286
+ *   [RLQ]    "Quantization in RL training" -- ai-systems-engineering.com/posts/rl-quantized-training
+ *   [TML4]   "Thinking Machines Lab releases 4-bit training" -- metallab.ai/2026/11/thinking-machines-4bit-training
+ *
+ * ---------------------------------------------------------------------------
+ * Number format (one definition for both the rollout and the train side, the
+ * "same quantization convention on both engines" of [RLQ], shared-convention
+ * paragraph):
+ *
+ *   * 16 consecutive values of a row share one scale ([TML4], paragraph on the
+ *     forward/backward mismatch); 4 bits per code + 8 bits per 16 values =
+ *     4.5 bits per value ([TRACE], guidance-volume paragraph; [TML4], format
+ *     comparison table).
+ *   * Code: E2M1, 4 bits = sign<<3 | m, magnitude index m in 0..7 selects
+ *     G = {0, 0.5, 1, 1.5, 2, 3, 4, 6} (16 representable values, [TML4]).
+ *   * Block scale: one E4M3 byte (OCP "fn": bias 7, max 448, no inf,
+ *     min subnormal 2^-9).  Tensor scale: one FP32 decode multiplier s_t.
+ *   * Decoded value = (G[m] * sb) * s_t with the sign applied: code times scale
+ *     ([RLQ], "code 3 with scale 0.1 is 0.3, with scale 0.2 it is 0.6").
+ *
+ * Scale recipe (all FP32 ops IEEE round-to-nearest-even, no FMA, no FTZ):
+ *   A    = max |x| over the tensor
+ *   s_t  = A / 2688            (2688 = 6 * 448);  A == 0  ->  s_t = 1
+ *   sb   = E4M3_RNE_satfinite((amax_block / 6) / s_t)
+ *   inv  = 1 / (sb * s_t)      sb == 0  ->  every code of the block is sign<<3
+ *   v    = x * inv;  m = RNE onto G of |v| (ties to even m; |v| > 6 -> 6);
+ *   sign = sign bit of x.
+ *
+ * Storage layouts (row-major, caller-owned device buffers):
+ *   x       [rows, cols]        BF16 bit patterns (uint16), cols % 16 == 0
+ *   codes   [rows, cols/2]      bytes; element 2j in the low nibble of byte j
+ *   scales  [rows, cols/16]     E4M3 bytes, block b covers elements 16b..16b+15
+ *   hints   ceil(n*bits/8)      element i at byte (i*bits)>>3, bit (i*bits)&7
+ *   ws      NVFP4_WS_WORDS uint32 words of device scratch (see below)
+ *
+ * Conventions for every call:
+ *   * Pointers are DEVICE pointers unless stated; the library never allocates,
+ *     frees or keeps them.  Every pointer must be 16-byte aligned
+ *     (NVFP4_ERR_MISALIGNED otherwise).
+ *   * `stream` is a cudaStream_t (NULL = legacy default stream).  Calls are
+ *     asynchronous on it; they return once the kernels are enqueued.
+ *   * Arguments are validated before anything is enqueued: a call that returns
+ *     an error has written nothing.  Inputs are never modified.
+ *   * n = rows * cols must be below 2^40 (NVFP4_ERR_SHAPE otherwise).
+ *   * NVFP4_ERR_CUDA means a launch failed; cudaGetLastError() has been
+ *     consumed, the stream's earlier work is unaffected.
+ *   * Non-finite inputs are outside the contract: they never fault, the
+ *     outputs are unspecified and bit NVFP4_WARN_NONFINITE is set in ws[1].
+ */
+#ifndef NVFP4_TRACE_H_
+#define NVFP4_TRACE_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef int nvfp4_status;
+
+#define NVFP4_OK                0
+#define NVFP4_ERR_INVALID_ARG   1   /* null pointer, negative size, bad flag */
+#define NVFP4_ERR_MISALIGNED    2   /* a pointer is not 16-byte aligned */
+#define NVFP4_ERR_SHAPE         3   /* cols % 16 (RHT: % 32), rows % 16 (SR), size >= 2^40 */
+#define NVFP4_ERR_CUDA          4   /* a kernel launch failed */
+#define NVFP4_ERR_UNSUPPORTED   5   /* hint_bits not in {1, 2, 4} */
+
+/* Scratch words written by the amax pass and read by the quantize pass. */
+#define NVFP4_WS_WORDS          4   /* ws[0] = bits of A (FP32), ws[1] = warning bits */
+#define NVFP4_WARN_NONFINITE    1u  /* ws[1]: an input was Inf or NaN */
+
+/* flags */
+#define NVFP4_AMAX_PRECOMPUTED  1   /* ws[0] already holds A (e.g. from nvfp4_tensor_amax) */
+
+/* stats8 indices (nvfp4_mismatch_stats). "pos" is the signed grid position
+ * (s ? -m : m), so +0 and -0 are the same position. */
+#define NVFP4_STAT_ELEMENTS      0  /* elements compared */
+#define NVFP4_STAT_CODE_MISMATCH 1  /* pos_a != pos_b */
+#define NVFP4_STAT_ADJACENT      2  /* |pos_a - pos_b| == 1 */
+#define NVFP4_STAT_FAR           3  /* |pos_a - pos_b| >= 2 */
+#define NVFP4_STAT_SUM_ABS_DELTA 4  /* sum of |pos_a - pos_b| */
+#define NVFP4_STAT_SCALE_MISMATCH 5 /* 16-blocks whose E4M3 scale bytes differ */
+#define NVFP4_STAT_VALUE_MISMATCH 6 /* decoded FP32 values differ (-0 == +0) */
+#define NVFP4_STATS8_WORDS       8  /* word 7 is reserved (written 0) */
+
+/* stats4 indices (nvfp4_guided_requant) */
+#define NVFP4_GSTAT_CONSULTED    0  /* off-grid and |v| < 6: the hint decided */
+#define NVFP4_GSTAT_CHANGED      1  /* guided code != round-to-nearest code */
+#define NVFP4_GSTAT_OUTSIDE      2  /* hint matched neither bracket end: RTN kept */
+#define NVFP4_STATS4_WORDS       4  /* word 3 is reserved (written 0) */
+
+/*
+ * nvfp4_tensor_amax -- A = max |x| over n BF16 values.
+ *   Defines the per-tensor scale's input ([TML4]: a shared scale needs the
+ *   group maximum).  ws[0] receives the FP32 bit pattern of A (exact: the
+ *   maximum of BF16 magnitudes is a BF16 value), ws[1] the warning bits.
+ *   ws is cleared by this call.  n == 0 gives A = 0.
+ */
+nvfp4_status nvfp4_tensor_amax(const uint16_t* x_bf16, int64_t n, uint32_t* ws,
+                               void* stream);
+
+/*
+ * nvfp4_quantize_rtn -- rollout-side round-to-nearest NVFP4 quantization, with
+ * an optional fused hint emit.
+ *   [TRACE], rounding-analogy paragraph: each engine rounds to the nearest
+ *   cell; the compaction paragraph: the rollout ships only the low bits that
+ *   tell adjacent cells apart.
+ *   x [rows, cols] BF16 -> codes, scales, *tensor_scale = s_t.
+ *   ws: scratch; unless flags has NVFP4_AMAX_PRECOMPUTED the call first runs
+ *   the amax pass into it.
+ *   hints: NULL for none (hint_bits ignored), else hint_bits in {1, 2, 4}:
+ *   1 -> m & 1, 2 -> m & 3 (magnitude bits, no sign), 4 -> the full code.
+ *   rows == 0 or cols == 0: writes *tensor_scale = 1 and nothing else.
+ */
+nvfp4_status nvfp4_quantize_rtn(const uint16_t* x_bf16, int64_t rows, int64_t cols,
+                                uint32_t* ws, int flags,
+                                uint8_t* codes, uint8_t* scales, float* tensor_scale,
+                                uint8_t* hints, int hint_bits, void* stream);
+
+/*
+ * nvfp4_emit_hint -- standalone compact hint from already-quantized codes.
+ *   [TRACE], compaction paragraph (>99% of mismatches are one cell apart, so a
+ *   few low bits of the code pick the rollout's cell).
+ *   codes: n/2 bytes (n % 16 == 0) -> hints: ceil(n*hint_bits/8) bytes.
+ */
+nvfp4_status nvfp4_emit_hint(const uint8_t* codes, int64_t n, int hint_bits,
+                             uint8_t* hints, void* stream);
+
+/*
+ * nvfp4_guided_requant -- train-side re-quantization that follows the
+ * rollout's cell.
+ *   [TRACE], prescription paragraph: near a boundary the train side takes the
+ *   cell the rollout chose instead of the nearest one.
+ *   The train tensor gets its own A, s_t, sb, inv and v exactly as in
+ *   nvfp4_quantize_rtn.  With a = |v| and lo = #{g in G, g > 0, g <= a}:
+ *     a >= 6            -> m = 7
+ *     a == G[lo]        -> m = lo (no rounding decision, hint ignored)
+ *     otherwise         -> hi = lo + 1;  m = lo if h == lo (mod 2^bits),
+ *                          hi if h == hi (mod 2^bits), else round-to-nearest.
+ *   hint_bits 1 or 2 compare magnitudes; the sign comes from x.  hint_bits 4
+ *   compares signed grid positions (the bracket is the pair of signed grid
+ *   points around v).  hints == NULL gives plain round-to-nearest.
+ *   stats4: NULL, or NVFP4_STATS4_WORDS uint64 counters that are ADDED to
+ *   (the caller zeroes them).
+ */
+nvfp4_status nvfp4_guided_requant(const uint16_t* x_train_bf16, int64_t rows, int64_t cols,
+                                  const uint8_t* hints, int hint_bits,
+                                  uint32_t* ws, int flags,
+                                  uint8_t* codes, uint8_t* scales, float* tensor_scale,
+                                  uint64_t* stats4, void* stream);
+
+/*
+ * nvfp4_mismatch_stats -- train/rollout discrepancy counters between two NVFP4
+ * tensors of the same shape.
+ *   [TRACE]: the distance between the two paths is the quantity to shrink
+ *   (opening and prescription paragraphs); most mismatches are one cell apart
+ *   (compaction paragraph).
+ *   ts_a, ts_b: device pointers to the two FP32 tensor scales.
+ *   stats8: NVFP4_STATS8_WORDS uint64 counters that are ADDED to (the caller
+ *   zeroes them); indices NVFP4_STAT_*.  Decoded values use
+ *   (G[m] * sb) * s_t in FP32 (the first product is exact).
+ */
+nvfp4_status nvfp4_mismatch_stats(const uint8_t* codes_a, const uint8_t* scales_a,
+                                  const float* ts_a,
+                                  const uint8_t* codes_b, const uint8_t* scales_b,
+                                  const float* ts_b,
+                                  int64_t rows, int64_t cols, uint64_t* stats8,
+                                  void* stream);
+
+/*
+ * nvfp4_sr_transpose_requant -- dequantize, transpose, stochastic-rounding
+ * re-quantize, for a stack of `batch` independent [rows, cols] matrices.
+ *   [TML4], forward/backward mismatch paragraph: transposing changes which 16
+ *   values share a scale, so return to high precision, transpose, and
+ *   re-quantize with stochastic rounding (2.25 -> 2 three times in four, 3
+ *   once; the mean is kept).
+ *   Per matrix e: y = (G[m] * sb) * s_t[e];  y^T is [cols, rows]; it gets its
+ *   own A', s_t', sb', inv' by the recipe above; v = y * inv'; with a = |v|,
+ *   a >= 6 -> 6; on-grid values stay; otherwise lo/hi bracket a and
+ *     p = (a - G[lo]) / (G[hi] - G[lo]),
+ *     r = Philox4x32-10(key = (seed lo32, seed hi32),
+ *                       counter = (i lo32, i hi32, draw, 0)).x0,
+ *     round up iff (r >> 8) < p * 2^24,
+ *   i = row-major index of the element in the OUTPUT stack [batch, cols, rows].
+ *   Philox4x32-10: Salmon, Moraes, Dror, Shaw, "Parallel random numbers: as
+ *   easy as 1, 2, 3", SC'11.
+ *   codes [batch, rows, cols/2], scales [batch, rows, cols/16],
+ *   tensor_scale [batch] -> codes_t [batch, cols, rows/2],
+ *   scales_t [batch, cols, rows/16], tensor_scale_t [batch].
+ *   ws: batch uint32 words of scratch (per-matrix amax of y), cleared here.
+ *   rows % 16 == 0 and cols % 16 == 0 (NVFP4_ERR_SHAPE).
+ */
+nvfp4_status nvfp4_sr_transpose_requant(const uint8_t* codes, const uint8_t* scales,
+                                        const float* tensor_scale,
+                                        int64_t batch, int64_t rows, int64_t cols,
+                                        uint64_t seed, uint32_t draw, uint32_t* ws,
+                                        uint8_t* codes_t, uint8_t* scales_t,
+                                        float* tensor_scale_t, void* stream);
+
+/*
+ * nvfp4_rht_quantize -- 32-point random Hadamard transform, then NVFP4
+ * round-to-nearest quantization.
+ *   [TML4], communication paragraph: a 32-dimensional random Hadamard
+ *   transform precedes the low-bit combine payload.
+ *   For each contiguous group of 32 values of a row:
+ *     y = (H32 * (sigma (.) x)) * fl32(1/sqrt(32)),
+ *   H32 the Sylvester Hadamard matrix H[i][j] = (-1)^popcount(i & j),
+ *   sigma_j = (Philox4x32-10(key = (seed lo32, seed hi32),
+ *                            counter = (j, 0, 0, 0)).x0 & 1) ? -1 : +1,
+ *   one sign vector for the whole tensor.  Then A, s_t, sb, codes as in
+ *   nvfp4_quantize_rtn on the FP32 y.  cols % 32 == 0 (NVFP4_ERR_SHAPE).
+ *   y_out: NULL, or [rows, cols] FP32 receiving y (for verification).
+ */
+nvfp4_status nvfp4_rht_quantize(const uint16_t* x_bf16, int64_t rows, int64_t cols,
+                                uint64_t sign_seed, uint32_t* ws,
+                                uint8_t* codes, uint8_t* scales, float* tensor_scale,
+                                float* y_out, void* stream);
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* nvfp4_status_string(nvfp4_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NVFP4_TRACE_H_ */

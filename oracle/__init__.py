@@ -1,0 +1,275 @@
+"""CPU oracle for NVFP4 quantization with train/rollout rounding alignment.
+
+TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
+CPU-baseline / reference legs of ``bench.py`` may import this package.  The
+product path (``train_rollout_alignment_b200``) never imports it and has no CPU
+fallback.
+
+The arithmetic lives in ``nvfp4_oracle.c`` (plain scalar C, every FP32 step one
+IEEE round-to-nearest operation).  This module only compiles it with gcc and
+marshals numpy arrays.  ctypes releases the GIL during each call, so callers
+may run independent tensors on a thread pool.
+
+Pages followed: "TRACE explainer" (blog.ontle.kr/blog/286), "Quantization in RL
+training" (ai-systems-engineering.com) and "Thinking Machines Lab releases 4-bit
+training" (metallab.ai); the C file cites the paragraph behind each step.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "nvfp4_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle_nvfp4.so")
+_lock = threading.Lock()
+_lib = None
+
+CFLAGS = ["-O2", "-ffp-contract=off", "-fno-fast-math", "-fPIC", "-shared", "-std=c11"]
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle shared library (gcc) if missing or stale."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + ".tmp.%d" % os.getpid()
+        subprocess.check_call(["gcc", *CFLAGS, _SRC, "-o", tmp, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            build()
+            lib = ctypes.CDLL(_LIB)
+            P = ctypes.c_void_p
+            I64 = ctypes.c_int64
+            F = ctypes.c_float
+            sig = {
+                "oracle_e2m1_value": (ctypes.c_double, [ctypes.c_int]),
+                "oracle_e2m1_rne": (ctypes.c_int, [F]),
+                "oracle_e4m3_value": (ctypes.c_double, [ctypes.c_int]),
+                "oracle_e4m3_rne_satfinite": (ctypes.c_int, [F]),
+                "oracle_bf16_to_f32": (F, [ctypes.c_uint16]),
+                "oracle_amax_f32": (F, [P, I64]),
+                "oracle_amax_bf16": (F, [P, I64]),
+                "oracle_tensor_scale": (F, [F]),
+                "oracle_block_scale": (ctypes.c_int, [F, F]),
+                "oracle_quantize_f32": (None, [P, I64, I64, F, P, P, P]),
+                "oracle_emit_hint": (None, [P, I64, ctypes.c_int, P]),
+                "oracle_quantize_rtn_bf16": (None, [P, I64, I64, F, P, P, P, P, ctypes.c_int]),
+                "oracle_guided_bf16": (None, [P, I64, I64, F, P, ctypes.c_int, P, P, P, P]),
+                "oracle_dequant_one": (F, [ctypes.c_int, ctypes.c_int, F]),
+                "oracle_dequant": (None, [P, P, F, I64, P]),
+                "oracle_mismatch_stats": (None, [P, P, F, P, P, F, I64, I64, P]),
+                "oracle_philox4x32_10": (None, [P, P, P]),
+                "oracle_sr_magnitude": (ctypes.c_int, [F, ctypes.c_uint32]),
+                "oracle_sr_transpose_requant": (
+                    None, [P, P, P, I64, I64, I64, ctypes.c_uint64, ctypes.c_uint32, P, P, P]),
+                "oracle_rht_signs": (None, [ctypes.c_uint64, P]),
+                "oracle_rht32_f64": (None, [P, I64, I64, ctypes.c_uint64, P]),
+                "oracle_rht_quantize": (None, [P, I64, I64, ctypes.c_uint64, P, P, P, P]),
+            }
+            for name, (res, args) in sig.items():
+                fn = getattr(lib, name)
+                fn.restype = res
+                fn.argtypes = args
+            _lib = lib
+    return _lib
+
+
+def _ptr(a: np.ndarray):
+    assert a.flags["C_CONTIGUOUS"], "oracle arrays must be C-contiguous"
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _u16(x) -> np.ndarray:
+    x = np.ascontiguousarray(x)
+    assert x.dtype == np.uint16, "BF16 inputs are passed as uint16 bit patterns"
+    return x
+
+
+# --------------------------------------------------------------------------- scalars
+def e2m1_value(m: int) -> float:
+    return _load().oracle_e2m1_value(int(m))
+
+
+def e2m1_rne(a: float) -> int:
+    return _load().oracle_e2m1_rne(float(a))
+
+
+def e4m3_value(b: int) -> float:
+    return _load().oracle_e4m3_value(int(b))
+
+
+def e4m3_rne_satfinite(f: float) -> int:
+    return _load().oracle_e4m3_rne_satfinite(float(f))
+
+
+def tensor_scale(A: float) -> float:
+    return _load().oracle_tensor_scale(float(A))
+
+
+def block_scale(amax_block: float, s_t: float) -> int:
+    return _load().oracle_block_scale(float(amax_block), float(s_t))
+
+
+def sr_magnitude(a: float, r: int) -> int:
+    return _load().oracle_sr_magnitude(float(a), int(r) & 0xFFFFFFFF)
+
+
+def philox4x32_10(ctr, key) -> tuple:
+    c = np.asarray(ctr, dtype=np.uint32).copy()
+    k = np.asarray(key, dtype=np.uint32).copy()
+    out = np.zeros(4, dtype=np.uint32)
+    _load().oracle_philox4x32_10(_ptr(c), _ptr(k), _ptr(out))
+    return tuple(int(v) for v in out)
+
+
+def rht_signs(seed: int) -> np.ndarray:
+    s = np.zeros(32, dtype=np.int32)
+    _load().oracle_rht_signs(int(seed), _ptr(s))
+    return s
+
+
+# --------------------------------------------------------------------------- tensors
+def amax_bf16(x) -> float:
+    x = _u16(x)
+    return float(_load().oracle_amax_bf16(_ptr(x), x.size))
+
+
+def amax_f32(y) -> float:
+    y = np.ascontiguousarray(y, dtype=np.float32)
+    return float(_load().oracle_amax_f32(_ptr(y), y.size))
+
+
+def _alloc_q(rows, cols):
+    return (np.zeros((rows, cols // 2), np.uint8), np.zeros((rows, cols // 16), np.uint8),
+            np.zeros(1, np.float32))
+
+
+def quantize_f32(y, A: float | None = None):
+    """Round-to-nearest NVFP4 of an FP32 [rows, cols] array -> (codes, scales, s_t)."""
+    y = np.ascontiguousarray(y, dtype=np.float32)
+    rows, cols = y.shape
+    if A is None:
+        A = amax_f32(y)
+    codes, scales, ts = _alloc_q(rows, cols)
+    _load().oracle_quantize_f32(_ptr(y), rows, cols, float(A), _ptr(codes), _ptr(scales), _ptr(ts))
+    return codes, scales, float(ts[0])
+
+
+def quantize_rtn(x, A: float | None = None, hint_bits: int = 0):
+    """Rollout side: BF16 [rows, cols] -> (codes, scales, s_t, hints or None).
+
+    ``A`` is the tensor amax; pass the full tensor's amax when ``x`` holds only
+    some rows of it (sampled checking)."""
+    x = _u16(x)
+    rows, cols = x.shape
+    if A is None:
+        A = amax_bf16(x)
+    codes, scales, ts = _alloc_q(rows, cols)
+    hints = None
+    hp = None
+    if hint_bits:
+        hints = np.zeros((rows * cols * hint_bits + 7) // 8, np.uint8)
+        hp = _ptr(hints)
+    _load().oracle_quantize_rtn_bf16(_ptr(x), rows, cols, float(A), _ptr(codes), _ptr(scales),
+                                     _ptr(ts), hp, int(hint_bits))
+    return codes, scales, float(ts[0]), hints
+
+
+def emit_hint(codes, n: int, hint_bits: int) -> np.ndarray:
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    hints = np.zeros((n * hint_bits + 7) // 8, np.uint8)
+    _load().oracle_emit_hint(_ptr(codes), int(n), int(hint_bits), _ptr(hints))
+    return hints
+
+
+def guided_requant(x, hints, hint_bits: int, A: float | None = None):
+    """Train side: BF16 [rows, cols] + rollout hints -> (codes, scales, s_t, stats4)."""
+    x = _u16(x)
+    rows, cols = x.shape
+    if A is None:
+        A = amax_bf16(x)
+    codes, scales, ts = _alloc_q(rows, cols)
+    stats = np.zeros(4, np.uint64)
+    hp = None
+    if hints is not None:
+        hints = np.ascontiguousarray(hints, dtype=np.uint8)
+        hp = _ptr(hints)
+    _load().oracle_guided_bf16(_ptr(x), rows, cols, float(A), hp, int(hint_bits), _ptr(codes),
+                               _ptr(scales), _ptr(ts), _ptr(stats))
+    return codes, scales, float(ts[0]), stats
+
+
+def dequant_one(code: int, scale_byte: int, s_t: float) -> float:
+    return float(_load().oracle_dequant_one(int(code), int(scale_byte), float(s_t)))
+
+
+def dequant(codes, scales, s_t: float, n: int) -> np.ndarray:
+    """NVFP4 -> FP32 values, flat, n elements."""
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    scales = np.ascontiguousarray(scales, dtype=np.uint8)
+    out = np.zeros(n, np.float32)
+    _load().oracle_dequant(_ptr(codes), _ptr(scales), float(s_t), int(n), _ptr(out))
+    return out
+
+
+def mismatch_stats(codes_a, scales_a, ts_a, codes_b, scales_b, ts_b, rows, cols) -> np.ndarray:
+    ca = np.ascontiguousarray(codes_a, dtype=np.uint8)
+    sa = np.ascontiguousarray(scales_a, dtype=np.uint8)
+    cb = np.ascontiguousarray(codes_b, dtype=np.uint8)
+    sb = np.ascontiguousarray(scales_b, dtype=np.uint8)
+    stats = np.zeros(8, np.uint64)
+    _load().oracle_mismatch_stats(_ptr(ca), _ptr(sa), float(ts_a), _ptr(cb), _ptr(sb), float(ts_b),
+                                  int(rows), int(cols), _ptr(stats))
+    return stats
+
+
+def sr_transpose_requant(codes, scales, ts, batch, rows, cols, seed, draw):
+    """[batch, rows, cols] NVFP4 -> transposed [batch, cols, rows] NVFP4 by SR."""
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    scales = np.ascontiguousarray(scales, dtype=np.uint8)
+    ts = np.ascontiguousarray(ts, dtype=np.float32)
+    ct = np.zeros((batch, cols, rows // 2), np.uint8)
+    st = np.zeros((batch, cols, rows // 16), np.uint8)
+    tst = np.zeros(batch, np.float32)
+    _load().oracle_sr_transpose_requant(_ptr(codes), _ptr(scales), _ptr(ts), int(batch), int(rows),
+                                        int(cols), int(seed), int(draw) & 0xFFFFFFFF, _ptr(ct),
+                                        _ptr(st), _ptr(tst))
+    return ct, st, tst
+
+
+def rht32_f64(x, seed: int) -> np.ndarray:
+    x = _u16(x)
+    rows, cols = x.shape
+    y = np.zeros((rows, cols), np.float64)
+    _load().oracle_rht32_f64(_ptr(x), rows, cols, int(seed), _ptr(y))
+    return y
+
+
+def rht_quantize(x, seed: int):
+    """-> (codes, scales, s_t, y_f32) with y the FP32-rounded double transform."""
+    x = _u16(x)
+    rows, cols = x.shape
+    codes, scales, ts = _alloc_q(rows, cols)
+    y = np.zeros((rows, cols), np.float32)
+    _load().oracle_rht_quantize(_ptr(x), rows, cols, int(seed), _ptr(codes), _ptr(scales), _ptr(ts),
+                                _ptr(y))
+    return codes, scales, float(ts[0]), y
+
+
+# --------------------------------------------------------------------------- helpers
+def unpack_codes(codes, n: int | None = None) -> np.ndarray:
+    """Packed nibbles -> one uint8 code per element (element 2j = low nibble)."""
+    c = np.asarray(codes, dtype=np.uint8).reshape(-1)
+    out = np.empty(c.size * 2, np.uint8)
+    out[0::2] = c & 15
+    out[1::2] = c >> 4
+    return out if n is None else out[:n]

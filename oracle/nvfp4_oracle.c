@@ -1,0 +1,489 @@
+/*
+ * nvfp4_oracle.c -- plain, slow, scalar CPU oracle for NVFP4 quantization with
+ * train/rollout rounding alignment.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the test suite, the smoke check of the
+ * package entry module and the CPU-baseline leg of bench.py may load this.
+ * It shares no code, header, table or constant generator with the CUDA path.
+ *
+ * Compile with  gcc -O2 -ffp-contract=off -fno-fast-math  so that every float
+ * operation below is one IEEE binary32 operation rounded to nearest-even (no
+ * fused multiply-add, no flush-to-zero).  Rounding decisions onto the E2M1
+ * grid and the E4M3 scale set are taken by exhaustive search over all
+ * candidates, in double precision where every distance that can tie is exact.
+ *
+ * Pages followed (named by title):
+ *   [TRACE] "TRACE explainer" (blog.ontle.kr/blog/286)
+ *   [RLQ]   "Quantization in RL training" (ai-systems-engineering.com)
+ *   [TML4]  "Thinking Machines Lab releases 4-bit training" (metallab.ai)
+ * Numeric format: E2M1 codes, 16-value blocks with an E4M3 block scale and an
+ * FP32 tensor scale; the scale recipe and every reading the pages leave open
+ * are listed with the function that applies them.
+ *
+ * Parity pins: every function here is pinned by the tests under tests/
+ * (test_oracle_*.py) against library casts, brute force, closed forms and the
+ * pages' worked examples.  The per-tensor scale constants (2688 = 6 * 448) and
+ * the order of the two block-scale divisions are readings, not pinned values.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+/* ------------------------------------------------------------------------ */
+/* Element format: E2M1 magnitudes.  [TML4] format comparison: 4 bits give 16
+ * representable values (8 magnitudes x sign). */
+static const double GRID[8] = {0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0};
+
+double oracle_e2m1_value(int m) { return GRID[m & 7]; }
+
+/* Round a >= 0 to the nearest grid magnitude, ties to the even index (the
+ * IEEE rule: even index = zero mantissa bit), values above 6 saturate to 6.
+ * Exhaustive search over the eight candidates. */
+int oracle_e2m1_rne(float a)
+{
+    if (a != a) return 0;          /* NaN: outside the contract */
+    if (a >= 6.0f) return 7;       /* saturation (includes +inf) */
+    int best = 0;
+    double bestd = fabs((double)a - GRID[0]);
+    for (int m = 1; m < 8; ++m) {
+        double d = fabs((double)a - GRID[m]);
+        if (d < bestd || (d == bestd && (m % 2) == 0)) {
+            best = m;
+            bestd = d;
+        }
+    }
+    return best;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Block-scale format: E4M3 "fn" (bias 7, no infinities, 0x7F = NaN). */
+double oracle_e4m3_value(int byte)
+{
+    int e = (byte >> 3) & 15, mant = byte & 7;
+    double mag = (e == 0) ? ldexp((double)mant, -9) : ldexp((double)(8 + mant), e - 10);
+    return (byte & 0x80) ? -mag : mag;
+}
+
+/* Round f >= 0 to the nearest finite non-negative E4M3 value, ties to the
+ * even byte (even mantissa), saturating at 448.  Exhaustive search over the
+ * 127 finite non-negative encodings 0x00..0x7E. */
+int oracle_e4m3_rne_satfinite(float f)
+{
+    if (f != f) return 0x7F;       /* NaN: outside the contract */
+    if (f >= 448.0f) return 0x7E;  /* satfinite (includes +inf) */
+    int best = 0;
+    double bestd = fabs((double)f - oracle_e4m3_value(0));
+    for (int b = 1; b <= 0x7E; ++b) {
+        double d = fabs((double)f - oracle_e4m3_value(b));
+        if (d < bestd || (d == bestd && (b % 2) == 0)) {
+            best = b;
+            bestd = d;
+        }
+    }
+    return best;
+}
+
+/* ------------------------------------------------------------------------ */
+float oracle_bf16_to_f32(uint16_t b)
+{
+    uint32_t u = (uint32_t)b << 16;
+    float f;
+    memcpy(&f, &u, 4);
+    return f;
+}
+
+static int sign_of(float f) { return signbit(f) ? 1 : 0; }
+
+static int nibble_get(const uint8_t* p, int64_t i) { return (p[i >> 1] >> ((i & 1) * 4)) & 15; }
+
+static void nibble_put(uint8_t* p, int64_t i, int v)
+{
+    int sh = (int)(i & 1) * 4;
+    p[i >> 1] = (uint8_t)((p[i >> 1] & ~(15 << sh)) | ((v & 15) << sh));
+}
+
+/* ------------------------------------------------------------------------ */
+/* Step 1: tensor amax.  A shared scale is fitted to the largest magnitude of
+ * what it covers ([TML4], forward/backward mismatch paragraph: one large value
+ * sets the scale for the rest).  Exact: the result is one of the inputs. */
+float oracle_amax_f32(const float* y, int64_t n)
+{
+    float A = 0.0f;
+    for (int64_t i = 0; i < n; ++i) {
+        float a = fabsf(y[i]);
+        if (a > A) A = a;
+    }
+    return A;
+}
+
+float oracle_amax_bf16(const uint16_t* x, int64_t n)
+{
+    float A = 0.0f;
+    for (int64_t i = 0; i < n; ++i) {
+        float a = fabsf(oracle_bf16_to_f32(x[i]));
+        if (a > A) A = a;
+    }
+    return A;
+}
+
+/* Step 2: scales.  Tensor decode multiplier s_t = A / (6 * 448) so that the
+ * largest magnitude lands on the top of both formats; A == 0 -> 1.
+ * Block scale sb = E4M3((amax_block / 6) / s_t): two rounded divisions in that
+ * order.  Decoded value = code value * scale ([RLQ], code 3 x scale 0.1). */
+float oracle_tensor_scale(float A) { return (A == 0.0f) ? 1.0f : A / 2688.0f; }
+
+int oracle_block_scale(float amax_block, float s_t)
+{
+    float q = amax_block / 6.0f;
+    float sbf = q / s_t;
+    return oracle_e4m3_rne_satfinite(sbf);
+}
+
+/* Step 3: the per-element scaled value v = x * (1 / (sb * s_t)), three
+ * rounded FP32 operations in that order. */
+static float scaled_value(float x, float sbv, float s_t)
+{
+    float denom = sbv * s_t;
+    float inv = 1.0f / denom;
+    return x * inv;
+}
+
+/* Round-to-nearest NVFP4 quantization of an FP32 tensor whose amax A is given
+ * ([TRACE], rounding-analogy paragraph: each engine rounds to the nearest
+ * cell).  codes: rows*cols/2 bytes, scales: rows*cols/16 bytes. */
+void oracle_quantize_f32(const float* y, int64_t rows, int64_t cols, float A,
+                         uint8_t* codes, uint8_t* scales, float* tensor_scale)
+{
+    float s_t = oracle_tensor_scale(A);
+    *tensor_scale = s_t;
+    int64_t nblk = cols / 16;
+    for (int64_t r = 0; r < rows; ++r) {
+        for (int64_t b = 0; b < nblk; ++b) {
+            const float* blk = y + r * cols + b * 16;
+            float amax_b = 0.0f;
+            for (int k = 0; k < 16; ++k)
+                if (fabsf(blk[k]) > amax_b) amax_b = fabsf(blk[k]);
+            int sb = oracle_block_scale(amax_b, s_t);
+            scales[r * nblk + b] = (uint8_t)sb;
+            float sbv = (float)oracle_e4m3_value(sb);
+            for (int k = 0; k < 16; ++k) {
+                int m = 0;
+                if (sbv != 0.0f) m = oracle_e2m1_rne(fabsf(scaled_value(blk[k], sbv, s_t)));
+                nibble_put(codes, r * cols + b * 16 + k, (sign_of(blk[k]) << 3) | m);
+            }
+        }
+    }
+}
+
+static float* bf16_rows_to_f32(const uint16_t* x, int64_t n)
+{
+    float* y = (float*)malloc((size_t)(n > 0 ? n : 1) * sizeof(float));
+    for (int64_t i = 0; i < n; ++i) y[i] = oracle_bf16_to_f32(x[i]);
+    return y;
+}
+
+/* Step 4: compact hint ([TRACE], compaction paragraph).  bits 1 -> m & 1
+ * (the E2M1 mantissa bit, enough to tell two adjacent cells apart), 2 ->
+ * m & 3, 4 -> the whole code (the uncompacted guidance).  Element i occupies
+ * bits (i*bits) .. (i*bits + bits - 1) of the byte stream, LSB first. */
+void oracle_emit_hint(const uint8_t* codes, int64_t n, int bits, uint8_t* hints)
+{
+    int64_t nbytes = (n * bits + 7) / 8;
+    memset(hints, 0, (size_t)nbytes);
+    for (int64_t i = 0; i < n; ++i) {
+        int code = nibble_get(codes, i);
+        int h = (bits == 4) ? code : ((code & 7) & ((1 << bits) - 1));
+        int64_t pos = i * bits;
+        hints[pos >> 3] |= (uint8_t)(h << (pos & 7));
+    }
+}
+
+static int hint_get(const uint8_t* hints, int64_t i, int bits)
+{
+    int64_t pos = i * bits;
+    return (hints[pos >> 3] >> (pos & 7)) & ((1 << bits) - 1);
+}
+
+/* Rollout side: round-to-nearest codes of a BF16 tensor, plus its hints. */
+void oracle_quantize_rtn_bf16(const uint16_t* x, int64_t rows, int64_t cols, float A,
+                              uint8_t* codes, uint8_t* scales, float* tensor_scale,
+                              uint8_t* hints, int hint_bits)
+{
+    float* y = bf16_rows_to_f32(x, rows * cols);
+    oracle_quantize_f32(y, rows, cols, A, codes, scales, tensor_scale);
+    free(y);
+    if (hints) oracle_emit_hint(codes, rows * cols, hint_bits, hints);
+}
+
+/* Step 5: guided re-quantization on the train side ([TRACE], prescription
+ * paragraph: near a boundary take the cell the rollout chose, not the nearest
+ * one).  The train tensor derives its own scales (only cells are aligned).
+ * For off-grid |v| < 6 the two candidate cells are the grid points that
+ * bracket |v|: lo = the largest grid index with G[lo] <= |v|, hi = lo + 1.
+ * hint_bits 1/2 compare magnitude indices modulo 2^bits; hint_bits 4 compares
+ * signed grid positions.  No match -> round-to-nearest.  stats4 (may be NULL)
+ * is added to: [consulted, changed, outside-bracket, reserved]. */
+void oracle_guided_bf16(const uint16_t* x, int64_t rows, int64_t cols, float A,
+                        const uint8_t* hints, int hint_bits,
+                        uint8_t* codes, uint8_t* scales, float* tensor_scale,
+                        uint64_t* stats4)
+{
+    float s_t = oracle_tensor_scale(A);
+    *tensor_scale = s_t;
+    int64_t nblk = cols / 16;
+    uint64_t consulted = 0, changed = 0, outside = 0;
+    for (int64_t r = 0; r < rows; ++r) {
+        for (int64_t b = 0; b < nblk; ++b) {
+            float blk[16];
+            for (int k = 0; k < 16; ++k) blk[k] = oracle_bf16_to_f32(x[r * cols + b * 16 + k]);
+            float amax_b = 0.0f;
+            for (int k = 0; k < 16; ++k)
+                if (fabsf(blk[k]) > amax_b) amax_b = fabsf(blk[k]);
+            int sb = oracle_block_scale(amax_b, s_t);
+            scales[r * nblk + b] = (uint8_t)sb;
+            float sbv = (float)oracle_e4m3_value(sb);
+            for (int k = 0; k < 16; ++k) {
+                int64_t i = r * cols + b * 16 + k;
+                int sgn = sign_of(blk[k]);
+                int m = 0;
+                if (sbv != 0.0f) {
+                    float a = fabsf(scaled_value(blk[k], sbv, s_t));
+                    int m_rtn = oracle_e2m1_rne(a);
+                    m = m_rtn;
+                    if (hints != NULL && a < 6.0f) {
+                        int lo = 0;
+                        for (int g = 1; g < 8; ++g)
+                            if (GRID[g] <= (double)a) lo = g;
+                        if ((double)a != GRID[lo]) {
+                            int hi = lo + 1;
+                            int h = hint_get(hints, i, hint_bits);
+                            int take_lo, take_hi;
+                            consulted++;
+                            if (hint_bits == 4) {
+                                int pos_h = (h & 8) ? -(h & 7) : (h & 7);
+                                int pos_lo = sgn ? -lo : lo;
+                                int pos_hi = sgn ? -hi : hi;
+                                take_lo = (pos_h == pos_lo);
+                                take_hi = (pos_h == pos_hi);
+                            } else {
+                                int mask = (1 << hint_bits) - 1;
+                                take_lo = ((h & mask) == (lo & mask));
+                                take_hi = ((h & mask) == (hi & mask));
+                            }
+                            if (take_lo) m = lo;
+                            else if (take_hi) m = hi;
+                            else outside++;
+                            if (m != m_rtn) changed++;
+                        }
+                    }
+                }
+                nibble_put(codes, i, (sgn << 3) | m);
+            }
+        }
+    }
+    if (stats4) {
+        stats4[0] += consulted;
+        stats4[1] += changed;
+        stats4[2] += outside;
+    }
+}
+
+/* Decoded value of element i: sign * ((G[m] * sb) * s_t) in FP32; the first
+ * product is exact (2 x 4 significant bits).  [RLQ], shared-convention
+ * paragraph: a code means code value times scale (code 3 with scale 0.1 is
+ * 0.3, with scale 0.2 it is 0.6). */
+float oracle_dequant_one(int code, int scale_byte, float s_t)
+{
+    float sbv = (float)oracle_e4m3_value(scale_byte);
+    float val = ((float)GRID[code & 7] * sbv) * s_t;
+    return (code & 8) ? -val : val;
+}
+
+void oracle_dequant(const uint8_t* codes, const uint8_t* scales, float s_t, int64_t n, float* out)
+{
+    for (int64_t i = 0; i < n; ++i) out[i] = oracle_dequant_one(nibble_get(codes, i), scales[i / 16], s_t);
+}
+
+/* Step 6: mismatch counters between two NVFP4 tensors ([TRACE]: the
+ * train/rollout distance is the quantity to shrink; most mismatches are one
+ * cell apart).  Positions are signed grid indices (s ? -m : m); decoded values
+ * are compared in FP32 (-0 equals +0).  stats8 is added to. */
+void oracle_mismatch_stats(const uint8_t* codes_a, const uint8_t* scales_a, float ts_a,
+                           const uint8_t* codes_b, const uint8_t* scales_b, float ts_b,
+                           int64_t rows, int64_t cols, uint64_t* stats8)
+{
+    int64_t n = rows * cols;
+    for (int64_t i = 0; i < n; ++i) {
+        int ca = nibble_get(codes_a, i), cb = nibble_get(codes_b, i);
+        int pa = (ca & 8) ? -(ca & 7) : (ca & 7);
+        int pb = (cb & 8) ? -(cb & 7) : (cb & 7);
+        int d = abs(pa - pb);
+        stats8[0] += 1;
+        if (d != 0) stats8[1] += 1;
+        if (d == 1) stats8[2] += 1;
+        if (d >= 2) stats8[3] += 1;
+        stats8[4] += (uint64_t)d;
+        float ya = oracle_dequant_one(ca, scales_a[i / 16], ts_a);
+        float yb = oracle_dequant_one(cb, scales_b[i / 16], ts_b);
+        if (ya != yb) stats8[6] += 1;
+    }
+    for (int64_t b = 0; b < n / 16; ++b)
+        if (scales_a[b] != scales_b[b]) stats8[5] += 1;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Philox4x32-10, from its published definition (Salmon, Moraes, Dror, Shaw,
+ * "Parallel random numbers: as easy as 1, 2, 3", SC'11): ten rounds of two
+ * 32x32->64 multiplications with multipliers 0xD2511F53 and 0xCD9E8D57, the
+ * key bumped by the Weyl constants 0x9E3779B9 / 0xBB67AE85 between rounds. */
+void oracle_philox4x32_10(const uint32_t ctr[4], const uint32_t key[2], uint32_t out[4])
+{
+    uint32_t c0 = ctr[0], c1 = ctr[1], c2 = ctr[2], c3 = ctr[3];
+    uint32_t k0 = key[0], k1 = key[1];
+    for (int round = 0; round < 10; ++round) {
+        if (round > 0) {
+            k0 += 0x9E3779B9u;
+            k1 += 0xBB67AE85u;
+        }
+        uint64_t p0 = (uint64_t)0xD2511F53u * (uint64_t)c0;
+        uint64_t p1 = (uint64_t)0xCD9E8D57u * (uint64_t)c2;
+        uint32_t hi0 = (uint32_t)(p0 >> 32), lo0 = (uint32_t)p0;
+        uint32_t hi1 = (uint32_t)(p1 >> 32), lo1 = (uint32_t)p1;
+        uint32_t n0 = hi1 ^ c1 ^ k0;
+        uint32_t n1 = lo1;
+        uint32_t n2 = hi0 ^ c3 ^ k1;
+        uint32_t n3 = lo0;
+        c0 = n0; c1 = n1; c2 = n2; c3 = n3;
+    }
+    out[0] = c0; out[1] = c1; out[2] = c2; out[3] = c3;
+}
+
+/* Stochastic rounding of a magnitude a = |v| onto the grid with the random
+ * word r ([TML4]: 2.25 becomes 2 three times in four and 3 once, so the mean
+ * is kept).  p = (a - G[lo]) / (G[hi] - G[lo]); round up iff
+ * (r >> 8) < p * 2^24.  On-grid values stay, a >= 6 gives 6. */
+int oracle_sr_magnitude(float a, uint32_t r)
+{
+    if (a != a) return 0;
+    if (a >= 6.0f) return 7;
+    int lo = 0;
+    for (int g = 1; g < 8; ++g)
+        if (GRID[g] <= (double)a) lo = g;
+    if ((double)a == GRID[lo]) return lo;
+    int hi = lo + 1;
+    double p = ((double)a - GRID[lo]) / (GRID[hi] - GRID[lo]);
+    return ((double)(r >> 8) < p * 16777216.0) ? hi : lo;
+}
+
+/* Step 7: dequantize -> transpose -> stochastic re-quantize, per matrix of a
+ * stack ([TML4], forward/backward mismatch paragraph).  Each matrix e is its
+ * own tensor (own A', s_t').  The random word of output element i (row-major
+ * in the [batch, cols, rows] output stack) is Philox4x32-10 with key
+ * (seed lo32, seed hi32) and counter (i lo32, i hi32, draw, 0), word x0. */
+void oracle_sr_transpose_requant(const uint8_t* codes, const uint8_t* scales,
+                                 const float* tensor_scale, int64_t batch, int64_t rows,
+                                 int64_t cols, uint64_t seed, uint32_t draw,
+                                 uint8_t* codes_t, uint8_t* scales_t, float* tensor_scale_t)
+{
+    int64_t n = rows * cols;
+    float* y = (float*)malloc((size_t)(n > 0 ? n : 1) * sizeof(float));
+    float* yt = (float*)malloc((size_t)(n > 0 ? n : 1) * sizeof(float));
+    uint32_t key[2] = {(uint32_t)seed, (uint32_t)(seed >> 32)};
+    for (int64_t e = 0; e < batch; ++e) {
+        const uint8_t* ce = codes + e * n / 2;
+        const uint8_t* se = scales + e * n / 16;
+        oracle_dequant(ce, se, tensor_scale[e], n, y);
+        /* transpose [rows, cols] -> [cols, rows] */
+        for (int64_t r = 0; r < rows; ++r)
+            for (int64_t c = 0; c < cols; ++c) yt[c * rows + r] = y[r * cols + c];
+        float A = oracle_amax_f32(yt, n);
+        float s_t = oracle_tensor_scale(A);
+        tensor_scale_t[e] = s_t;
+        uint8_t* cte = codes_t + e * n / 2;
+        uint8_t* ste = scales_t + e * n / 16;
+        int64_t nblk = rows / 16;
+        for (int64_t c = 0; c < cols; ++c) {
+            for (int64_t b = 0; b < nblk; ++b) {
+                const float* blk = yt + c * rows + b * 16;
+                float amax_b = 0.0f;
+                for (int k = 0; k < 16; ++k)
+                    if (fabsf(blk[k]) > amax_b) amax_b = fabsf(blk[k]);
+                int sb = oracle_block_scale(amax_b, s_t);
+                ste[c * nblk + b] = (uint8_t)sb;
+                float sbv = (float)oracle_e4m3_value(sb);
+                for (int k = 0; k < 16; ++k) {
+                    int64_t local = c * rows + b * 16 + k;
+                    int64_t gi = e * n + local;
+                    int m = 0;
+                    if (sbv != 0.0f) {
+                        uint32_t ctr[4] = {(uint32_t)gi, (uint32_t)((uint64_t)gi >> 32), draw, 0u};
+                        uint32_t out[4];
+                        oracle_philox4x32_10(ctr, key, out);
+                        m = oracle_sr_magnitude(fabsf(scaled_value(blk[k], sbv, s_t)), out[0]);
+                    }
+                    nibble_put(cte, local, (sign_of(blk[k]) << 3) | m);
+                }
+            }
+        }
+    }
+    free(y);
+    free(yt);
+}
+
+/* ------------------------------------------------------------------------ */
+/* Step 8: 32-point random Hadamard transform ([TML4], communication
+ * paragraph).  Signs: sigma_j = -1 iff bit 0 of Philox4x32-10(key = (seed lo32,
+ * seed hi32), counter = (j, 0, 0, 0)).x0 is set.  The transform is the plain
+ * matrix product with the Sylvester matrix H[j][k] = (-1)^popcount(j & k),
+ * in double precision, scaled by 1/sqrt(32). */
+void oracle_rht_signs(uint64_t seed, int* sigma32)
+{
+    uint32_t key[2] = {(uint32_t)seed, (uint32_t)(seed >> 32)};
+    for (uint32_t j = 0; j < 32; ++j) {
+        uint32_t ctr[4] = {j, 0u, 0u, 0u}, out[4];
+        oracle_philox4x32_10(ctr, key, out);
+        sigma32[j] = (out[0] & 1u) ? -1 : 1;
+    }
+}
+
+static int popcount_u32(uint32_t v)
+{
+    int c = 0;
+    while (v) {
+        c += (int)(v & 1u);
+        v >>= 1;
+    }
+    return c;
+}
+
+void oracle_rht32_f64(const uint16_t* x, int64_t rows, int64_t cols, uint64_t seed, double* y)
+{
+    int sigma[32];
+    oracle_rht_signs(seed, sigma);
+    double norm = 1.0 / sqrt(32.0);
+    int64_t n = rows * cols;
+    for (int64_t g = 0; g < n; g += 32) {
+        for (int j = 0; j < 32; ++j) {
+            double s = 0.0;
+            for (int k = 0; k < 32; ++k) {
+                double h = (popcount_u32((uint32_t)(j & k)) % 2) ? -1.0 : 1.0;
+                s += h * (double)sigma[k] * (double)oracle_bf16_to_f32(x[g + k]);
+            }
+            y[g + j] = s * norm;
+        }
+    }
+}
+
+/* RHT then round-to-nearest quantization of the FP32-rounded transform. */
+void oracle_rht_quantize(const uint16_t* x, int64_t rows, int64_t cols, uint64_t seed,
+                         uint8_t* codes, uint8_t* scales, float* tensor_scale, float* y_f32)
+{
+    int64_t n = rows * cols;
+    double* yd = (double*)malloc((size_t)(n > 0 ? n : 1) * sizeof(double));
+    oracle_rht32_f64(x, rows, cols, seed, yd);
+    for (int64_t i = 0; i < n; ++i) y_f32[i] = (float)yd[i];
+    free(yd);
+    float A = oracle_amax_f32(y_f32, n);
+    oracle_quantize_f32(y_f32, rows, cols, A, codes, scales, tensor_scale);
+}
