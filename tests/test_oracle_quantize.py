@@ -198,6 +198,51 @@ def test_guided_distance_guarantee(noise):
             assert np.sum(p_g != p_ro) < np.sum(p_rtn != p_ro)
 
 
+def _exact_grid_tensor(seed):
+    """A tensor whose scaled values are exact: A = 2688 gives s_t = 1, a block
+    with max 6 * 2^j gets sb = 2^j and inv = 2^-j, so grid values times 2^j sit
+    exactly on the grid.  Returns (bf16 bits, on-grid mask)."""
+    rng = np.random.default_rng(seed)
+    rows, cols = 8, 64
+    x = np.zeros((rows, cols), np.float32)
+    grid = np.array(GRID, np.float32)
+    on = np.zeros((rows, cols), bool)
+    for r in range(rows):
+        for b in range(cols // 16):
+            j = int(rng.integers(-3, 4))
+            blk = rng.choice(grid, 16) * np.float32(2.0 ** j)
+            blk[0] = 6.0 * 2.0 ** j
+            off = rng.random(16) < 0.4
+            off[0] = False
+            blk[off] = (rng.uniform(0, 6, off.sum()) * 2.0 ** j).astype(np.float32)
+            blk *= rng.choice(np.array([-1, 1], np.float32), 16)
+            x[r, 16 * b:16 * b + 16] = blk
+            on[r, 16 * b:16 * b + 16] = ~off
+    x[0, 0] = 2688.0
+    on[0, :16] = False  # that block's scale is 448: not exact
+    xb = syn.bf16_bits(x)
+    on &= syn.bf16_to_f32(xb) == x  # off-grid draws that BF16 rounding put on-grid
+    return xb, on
+
+
+@pytest.mark.parametrize("bits", [1, 2, 4])
+def test_guided_ignores_hints_on_grid(bits):
+    xb, on = _exact_grid_tensor(5)
+    rows, cols = xb.shape
+    n = xb.size
+    rc, rs, rt, _ = oracle.quantize_rtn(xb)
+    assert rt == 1.0
+    rng = np.random.default_rng(bits)
+    hints = rng.integers(0, 256, (n * bits + 7) // 8).astype(np.uint8)  # adversarial
+    gc, gs, gt, st = oracle.guided_requant(xb, hints, bits)
+    c_rtn, c_g = _codes(rc, n).reshape(rows, cols), _codes(gc, n).reshape(rows, cols)
+    assert np.array_equal(c_g[on], c_rtn[on])
+    a, _ = _scaled_abs(xb, rs, rt)
+    exact_on = np.isin(a.reshape(rows, cols), np.array(GRID)) | (a.reshape(rows, cols) >= 6)
+    assert np.all(exact_on[on])
+    assert st[0] == np.sum(~exact_on)
+
+
 def test_guided_outside_bracket_count_two_bit():
     xt = syn.random_case((8, 128), 21, "normal")
     xr = syn.random_case((8, 128), 22, "normal")
