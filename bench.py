@@ -1,0 +1,476 @@
+"""Throughput of the NVFP4 train/rollout alignment path on B200.
+
+One step = the whole path over the 48-layer stack of 65536x4096 BF16
+activations (per-column scales log-uniform in [0.1, 10]), for every layer:
+  rollout: tensor amax -> round-to-nearest quantize (+ fused 2-bit hints on
+           layers 24..47)
+  train:   tensor amax -> guided re-quantize (hints on layers 24..47, plain
+           round-to-nearest before) with its counters
+  both:    mismatch counters between the rollout and the train codes.
+Inputs (48 GiB per GPU) are resident in HBM and larger than L2, so no L2 flush
+is needed between steps.  `value` is algorithmic GB/s (bytes each kernel must
+move, summed over the step, divided by the step time), `elements_per_s` the
+train + rollout elements processed per second.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--layers L] [--impl reference]
+
+With N > 1 (torchrun, one rank per GPU) every rank runs its own 48-layer stack
+(weak scaling, no collective on the data path); the time is the max over
+ranks.  `--impl reference` times the CPU oracle on a bounded sample of the
+same workload instead.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+METRIC = "NVFP4 quantize+guided-requant GB/s and elements/s; fraction of B200 HBM roofline"
+ROWS, COLS = 65536, 4096
+HINT_BITS = 2
+
+# Algorithmic bytes per element of each kernel (what it must read + write).
+BYTES = {
+    "amax": 2.0,                                   # BF16 in
+    "quantize_rtn": 2.0 + 0.5 + 1 / 16,            # BF16 in, codes + scales out
+    "quantize_rtn+hint": 2.0 + 0.5 + 1 / 16 + HINT_BITS / 8,
+    "guided_requant": 2.0 + 0.5 + 1 / 16,          # no hints: plain RTN
+    "guided_requant+hint": 2.0 + HINT_BITS / 8 + 0.5 + 1 / 16,
+    "mismatch_stats": 2 * (0.5 + 1 / 16),
+    "emit_hint": 0.5 + HINT_BITS / 8,
+}
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        p = json.load(open(path))
+        return float(p["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def _dist():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+# --------------------------------------------------------------------------- clocks
+CLOCK_QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+
+    def __init__(self, device_index: int):
+        self.proc = None
+        self.lines = []
+        try:
+            uuid = "GPU-" + str(torch.cuda.get_device_properties(device_index).uuid)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", uuid, "--query-gpu=" + CLOCK_QUERY, "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, smax, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            f = [t.strip() for t in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax = max(smax, float(f[2]))
+            except ValueError:
+                continue
+            for name, val in zip(names, f[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": smax, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# --------------------------------------------------------------------------- workload
+class Stack:
+    """Device-resident 48-layer workload and its output buffers."""
+
+    def __init__(self, layers: int, hint_from: int, device, rank: int):
+        from train_rollout_alignment_b200 import synthetic as syn
+        self.layers, self.hint_from, self.device = layers, hint_from, device
+        self.n = ROWS * COLS
+        self.xt, self.xr = [], []
+        for l in range(layers):
+            t, r = syn.cfg4_layer_device(l, device, rank)
+            self.xt.append(t)
+            self.xr.append(r)
+        u8 = dict(dtype=torch.uint8, device=device)
+        self.cr = [torch.empty((ROWS, COLS // 2), **u8) for _ in range(layers)]
+        self.sr = [torch.empty((ROWS, COLS // 16), **u8) for _ in range(layers)]
+        self.ct = [torch.empty((ROWS, COLS // 2), **u8) for _ in range(layers)]
+        self.st = [torch.empty((ROWS, COLS // 16), **u8) for _ in range(layers)]
+        self.hints = [torch.empty(self.n * HINT_BITS // 8, **u8) if l >= hint_from else None
+                      for l in range(layers)]
+        self.ts = torch.empty((layers, 2), dtype=torch.float32, device=device)
+        self.ws = torch.zeros((layers, 2, 4), dtype=torch.int32, device=device)
+        self.stats = torch.zeros((layers, 12), dtype=torch.int64, device=device)
+
+    def kernels_of_layer(self, l):
+        """(kernel label, algorithmic bytes) in launch order for layer l."""
+        hinted = l >= self.hint_from
+        return [("amax", BYTES["amax"] * self.n),
+                ("quantize_rtn", BYTES["quantize_rtn+hint" if hinted else "quantize_rtn"] * self.n),
+                ("amax", BYTES["amax"] * self.n),
+                ("guided_requant", BYTES["guided_requant+hint" if hinted else "guided_requant"] * self.n),
+                ("mismatch_stats", BYTES["mismatch_stats"] * self.n)]
+
+    def step_bytes(self):
+        return sum(b for l in range(self.layers) for _, b in self.kernels_of_layer(l))
+
+    def run_layer(self, b, l, xr, xt, events=None):
+        """The five kernels of layer l; events: list to append (start, end) pairs to."""
+        ws_r, ws_t = self.ws[l, 0], self.ws[l, 1]
+        ts_r, ts_t = self.ts[l, 0:1], self.ts[l, 1:2]
+        h = self.hints[l]
+        bits = HINT_BITS if h is not None else 0
+        st = self.stats[l]
+        calls = [
+            lambda: b.nvfp4_tensor_amax(xr, ws_r),
+            lambda: b.nvfp4_quantize_rtn(xr, ws_r, self.cr[l], self.sr[l], ts_r, h, bits,
+                                         flags=b.NVFP4_AMAX_PRECOMPUTED),
+            lambda: b.nvfp4_tensor_amax(xt, ws_t),
+            lambda: b.nvfp4_guided_requant(xt, h, HINT_BITS, ws_t, self.ct[l], self.st[l], ts_t, st[8:12],
+                                           flags=b.NVFP4_AMAX_PRECOMPUTED),
+            lambda: b.nvfp4_mismatch_stats(self.cr[l], self.sr[l], ts_r, self.ct[l], self.st[l], ts_t,
+                                           ROWS, COLS, st[0:8]),
+        ]
+        for fn in calls:
+            if events is not None:
+                e0 = torch.cuda.Event(enable_timing=True)
+                e1 = torch.cuda.Event(enable_timing=True)
+                e0.record()
+                fn()
+                e1.record()
+                events.append((e0, e1))
+            else:
+                fn()
+
+    def step(self, b, events=None):
+        self.stats.zero_()
+        for l in range(self.layers):
+            self.run_layer(b, l, self.xr[l], self.xt[l], events)
+
+
+# --------------------------------------------------------------------------- CPU oracle
+def _oracle_pipeline(xt, xr, hint_bits):
+    import oracle
+    A_r, A_t = oracle.amax_bf16(xr), oracle.amax_bf16(xt)
+    rc, rs, rt, h = oracle.quantize_rtn(xr, A_r, hint_bits)
+    gc, gs, gt, _ = oracle.guided_requant(xt, h, HINT_BITS, A_t)
+    oracle.mismatch_stats(rc, rs, rt, gc, gs, gt, xt.shape[0], xt.shape[1])
+
+
+def oracle_sample(device, rank, rows_per_core: int, cores: int):
+    """Host arrays for the CPU oracle: `cores` chunks of `rows_per_core` rows of
+    layer 24 (a hinted layer), each chunk quantized as a tensor of its own."""
+    from train_rollout_alignment_b200 import synthetic as syn
+    xt, xr = syn.cfg4_layer_device(24, device, rank)
+    rows = min(ROWS, rows_per_core * cores)
+    to_np = lambda t: t[:rows].contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+    xt_h, xr_h = to_np(xt), to_np(xr)
+    del xt, xr
+    return [(xt_h[i:i + rows_per_core], xr_h[i:i + rows_per_core]) for i in range(0, rows, rows_per_core)]
+
+
+def time_oracle(chunks):
+    """Wall time of the oracle pipeline over all chunks, one thread per chunk
+    (the C oracle releases the GIL)."""
+    from concurrent.futures import ThreadPoolExecutor
+    t0 = time.perf_counter()
+    with ThreadPoolExecutor(max_workers=len(chunks)) as ex:
+        list(ex.map(lambda c: _oracle_pipeline(c[0], c[1], HINT_BITS), chunks))
+    return time.perf_counter() - t0
+
+
+def oracle_bytes(chunks):
+    per_elem = (BYTES["amax"] * 2 + BYTES["quantize_rtn+hint"] + BYTES["guided_requant+hint"]
+                + BYTES["mismatch_stats"])
+    return sum(c[0].size for c in chunks) * per_elem, sum(c[0].size for c in chunks)
+
+
+def _cores():
+    return len(os.sched_getaffinity(0))
+
+
+# --------------------------------------------------------------------------- main
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--layers", type=int, default=48)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    args = ap.parse_args()
+    world, rank, local = _dist()
+    if args.impl == "reference":
+        return run_reference(args, world, rank, local)
+    return run_ours(args, world, rank, local)
+
+
+def _config(layers):
+    return {"workload": "%d-layer stack of %dx%d BF16 activations, N(0,1) x per-column log-uniform "
+                        "[0.1, 10] scales, seed 4: rollout RTN + 2-bit hints on layers %d-%d, train "
+                        "guided requant, mismatch stats" % (layers, ROWS, COLS, layers // 2, layers - 1),
+            "layers": layers, "rows": ROWS, "cols": COLS, "hint_bits": HINT_BITS,
+            "inputs_bf16_gib_per_gpu": round(layers * 2 * ROWS * COLS * 2 / 2 ** 30, 1),
+            "l2": "no flush: every input tensor (512 MiB) is larger than L2 (126 MB)"}
+
+
+def run_ours(args, world, rank, local):
+    from train_rollout_alignment_b200 import _binding as b
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    peak, peak_kind = _peaks()
+
+    stack = Stack(args.layers, args.layers // 2, device, rank)
+    torch.cuda.synchronize()
+    step_bytes = stack.step_bytes()
+    step_elems = 2 * stack.n * args.layers
+
+    for _ in range(args.warmup):
+        stack.step(b)
+    torch.cuda.synchronize()
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+
+    # ---- device-timed region: K steps, per-kernel events on the launching stream
+    sampler = ClockSampler(local)
+    time.sleep(0.3)
+    barrier()
+    torch.cuda.synchronize()
+    events = []
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record()
+    for _ in range(args.steps):
+        stack.step(b, events)
+    t_end.record()
+    torch.cuda.synchronize()
+    barrier()
+    clocks = sampler.stop()
+    elapsed = t_start.elapsed_time(t_end) / 1e3
+    t_max = torch.tensor([elapsed], dtype=torch.float64, device=device)
+    if world > 1:
+        torch.distributed.all_reduce(t_max, op=torch.distributed.ReduceOp.MAX)
+    t_max = float(t_max.item())
+
+    # per-kernel durations (average over launches in the timed region)
+    labels = [lab for l in range(args.layers) for lab, _ in stack.kernels_of_layer(l)] * args.steps
+    nbytes = [nb for l in range(args.layers) for _, nb in stack.kernels_of_layer(l)] * args.steps
+    per = {}
+    for lab, nb, (e0, e1) in zip(labels, nbytes, events):
+        d = per.setdefault(lab, {"launches": 0, "ms": 0.0, "bytes": 0.0})
+        d["launches"] += 1
+        d["ms"] += e0.elapsed_time(e1)
+        d["bytes"] += nb
+    total_ms = sum(d["ms"] for d in per.values())
+    kernels = {}
+    for lab, d in per.items():
+        gbs = d["bytes"] / (d["ms"] / 1e3) / 1e9
+        kernels[lab] = {"launches": d["launches"], "avg_us": round(1e3 * d["ms"] / d["launches"], 2),
+                        "share": round(d["ms"] / total_ms, 4), "GB/s": round(gbs, 1),
+                        "frac": round(gbs / peak, 4)}
+    dom = max(kernels, key=lambda k: kernels[k]["share"])
+    dom_bytes_per_launch = per[dom]["bytes"] / per[dom]["launches"]
+    dom_gbs = per[dom]["bytes"] / (per[dom]["ms"] / 1e3) / 1e9
+    traffic = _ncu_traffic(dom)
+
+    value = world * args.steps * step_bytes / t_max / 1e9
+    elems = world * args.steps * step_elems / t_max
+
+    # ---- end to end through the C ABI with host buffers (rank-local)
+    e2e = run_e2e(b, stack, device, steps=min(args.steps, 2))
+
+    # ---- CPU oracle baseline (rank 0, N = 1 only)
+    cpu = None
+    if world == 1:
+        cores = _cores()
+        chunks = oracle_sample(device, rank, rows_per_core=1024, cores=cores)
+        nbytes_cpu, nel = oracle_bytes(chunks)
+        dt = time_oracle(chunks)
+        cpu = {"value": round(nbytes_cpu / dt / 1e9, 3), "unit": "GB/s", "cores": len(chunks),
+               "kind": "oracle",
+               "sample": "%d rows x %d cols of layer 24 (train + rollout), split in %d chunks of 1024 "
+                         "rows each quantized as its own tensor, one thread per chunk; %.1f s wall"
+                         % (len(chunks) * 1024, COLS, len(chunks), dt),
+               "elements_per_s": round(2 * nel / dt, 1)}
+
+    launches = 5 * args.layers * args.steps
+    out = {
+        "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * t_max / args.steps, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic (seeded, generated on the GPU; BF16 inputs, FP32 arithmetic)",
+        "config": _config(args.layers),
+        "elements_per_s": round(elems, 1),
+        "roofline": {"bound": "hbm", "kernel": dom, "achieved": round(dom_gbs, 1), "peak": peak,
+                     "peak_kind": peak_kind, "unit": "GB/s", "frac": round(dom_gbs / peak, 4),
+                     "bytes_per_launch": dom_bytes_per_launch, "traffic": traffic},
+        "kernels": kernels,
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": launches,
+        "clocks": clocks,
+    }
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(out))
+
+
+def _ncu_traffic(kernel_label):
+    """DRAM bytes per launch of the dominant kernel from the committed ncu
+    summary, if it was taken on the current kernel sources (else None)."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "ncu_dram_traffic.txt")
+    if not os.path.exists(path):
+        return None
+    from train_rollout_alignment_b200 import build as bld
+    h = hashlib.sha256()
+    for f in bld.SOURCES + bld.HEADERS:
+        h.update(open(os.path.join(bld.CSRC, f), "rb").read())
+    src = h.hexdigest()[:16]
+    for line in open(path):
+        if line.startswith("#") or "=" not in line:
+            continue
+        kv = dict(tok.split("=", 1) for tok in line.split())
+        if kv.get("label") == kernel_label and kv.get("src_sha") == src:
+            return float(kv["dram_bytes_per_launch"])
+    return None
+
+
+def run_e2e(b, stack, device, steps):
+    """The same step with inputs copied from pinned host memory every step and
+    the hints + counters read back, timed on the host around the device work.
+    Host copies of 4 distinct layers are reused cyclically (host memory bound);
+    copies run on a second stream, double-buffered against the kernels."""
+    P = min(4, stack.layers)
+    pin = lambda t: t.cpu().pin_memory()
+    h_xr = [pin(stack.xr[l]) for l in range(P)]
+    h_xt = [pin(stack.xt[l]) for l in range(P)]
+    h_hints = [torch.empty(stack.n * HINT_BITS // 8, dtype=torch.uint8).pin_memory()
+               for l in range(stack.layers) if stack.hints[l] is not None]
+    h_stats = torch.empty_like(stack.stats, device="cpu").pin_memory()
+    slots_r = [torch.empty_like(stack.xr[0]) for _ in range(2)]
+    slots_t = [torch.empty_like(stack.xt[0]) for _ in range(2)]
+    copy = torch.cuda.Stream(device)
+    comp = torch.cuda.current_stream(device)
+    h2d = d2h = 0
+
+    def one_step():
+        nonlocal h2d, d2h
+        free = [torch.cuda.Event(), torch.cuda.Event()]
+        for e in free:
+            e.record(comp)
+        stack.stats.zero_()
+        hi = 0
+        for l in range(stack.layers):
+            s = l % 2
+            ready = torch.cuda.Event()
+            with torch.cuda.stream(copy):
+                copy.wait_event(free[s])
+                slots_r[s].copy_(h_xr[l % P], non_blocking=True)
+                slots_t[s].copy_(h_xt[l % P], non_blocking=True)
+                ready.record(copy)
+            h2d += 2 * slots_r[s].numel() * 2
+            comp.wait_event(ready)
+            stack.run_layer(b, l, slots_r[s], slots_t[s])
+            free[s].record(comp)
+            if stack.hints[l] is not None:
+                h_hints[hi].copy_(stack.hints[l], non_blocking=True)
+                d2h += stack.hints[l].numel()
+                hi += 1
+        h_stats.copy_(stack.stats, non_blocking=True)
+        d2h += stack.stats.numel() * 8
+
+    one_step()  # warm-up (pins, first copies)
+    torch.cuda.synchronize()
+    h2d = d2h = 0
+    t0 = time.perf_counter()
+    for _ in range(steps):
+        one_step()
+    torch.cuda.synchronize()
+    dt = time.perf_counter() - t0
+    return {"value": round(steps * stack.step_bytes() / dt / 1e9, 2), "unit": "GB/s",
+            "h2d_bytes_per_step": h2d // steps, "d2h_bytes_per_step": d2h // steps, "steps": steps,
+            "host_layers": "%d distinct layers in pinned host memory, used cyclically" % P}
+
+
+def run_reference(args, world, rank, local):
+    """The CPU oracle as the reference arm, on a bounded sample of the same
+    workload per step (rank 0 only; other ranks exit)."""
+    if rank != 0:
+        return
+    device = torch.device("cuda", local) if torch.cuda.is_available() else torch.device("cpu")
+    cores = _cores()
+    rows_per_core = 256
+    if device.type == "cuda":
+        chunks = oracle_sample(device, 0, rows_per_core=rows_per_core, cores=cores)
+    else:
+        from train_rollout_alignment_b200 import synthetic as syn
+        chunks = [syn.normal_pair((rows_per_core, COLS), 4 + i) for i in range(cores)]
+        chunks = [(t, r) for t, r in chunks]
+    nbytes, nel = oracle_bytes(chunks)
+    for _ in range(args.warmup):
+        time_oracle(chunks)
+    dts = [time_oracle(chunks) for _ in range(args.steps)]
+    dt = sum(dts)
+    value = args.steps * nbytes / dt / 1e9
+    sample = ("%d rows x %d cols of layer 24 (train + rollout) per step, %d chunks of %d rows, one "
+              "thread per chunk" % (len(chunks) * rows_per_core, COLS, len(chunks), rows_per_core))
+    out = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": "GB/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(1e3 * dt / args.steps, 3), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic (seeded)", "config": _config(args.layers),
+        "elements_per_s": round(args.steps * 2 * nel / dt, 1),
+        "cpu_baseline": {"value": round(value, 3), "unit": "GB/s", "cores": len(chunks), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(value, 3), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(out))
+
+
+if __name__ == "__main__":
+    main()

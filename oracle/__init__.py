@@ -71,6 +71,8 @@ def _load():
                 "oracle_sr_magnitude": (ctypes.c_int, [F, ctypes.c_uint32]),
                 "oracle_sr_transpose_requant": (
                     None, [P, P, P, I64, I64, I64, ctypes.c_uint64, ctypes.c_uint32, P, P, P]),
+                "oracle_sr_transpose_requant_from": (
+                    None, [P, P, P, I64, I64, I64, I64, ctypes.c_uint64, ctypes.c_uint32, P, P, P]),
                 "oracle_rht_signs": (None, [ctypes.c_uint64, P]),
                 "oracle_rht32_f64": (None, [P, I64, I64, ctypes.c_uint64, P]),
                 "oracle_rht_quantize": (None, [P, I64, I64, ctypes.c_uint64, P, P, P, P]),
@@ -232,17 +234,20 @@ def mismatch_stats(codes_a, scales_a, ts_a, codes_b, scales_b, ts_b, rows, cols)
     return stats
 
 
-def sr_transpose_requant(codes, scales, ts, batch, rows, cols, seed, draw):
-    """[batch, rows, cols] NVFP4 -> transposed [batch, cols, rows] NVFP4 by SR."""
+def sr_transpose_requant(codes, scales, ts, batch, rows, cols, seed, draw, first: int = 0):
+    """[batch, rows, cols] NVFP4 -> transposed [batch, cols, rows] NVFP4 by SR.
+
+    ``first``: index of the first given matrix within the whole stack (the
+    random counter is the element's index in the whole output stack)."""
     codes = np.ascontiguousarray(codes, dtype=np.uint8)
     scales = np.ascontiguousarray(scales, dtype=np.uint8)
     ts = np.ascontiguousarray(ts, dtype=np.float32)
     ct = np.zeros((batch, cols, rows // 2), np.uint8)
     st = np.zeros((batch, cols, rows // 16), np.uint8)
     tst = np.zeros(batch, np.float32)
-    _load().oracle_sr_transpose_requant(_ptr(codes), _ptr(scales), _ptr(ts), int(batch), int(rows),
-                                        int(cols), int(seed), int(draw) & 0xFFFFFFFF, _ptr(ct),
-                                        _ptr(st), _ptr(tst))
+    _load().oracle_sr_transpose_requant_from(_ptr(codes), _ptr(scales), _ptr(ts), int(first),
+                                             int(batch), int(rows), int(cols), int(seed),
+                                             int(draw) & 0xFFFFFFFF, _ptr(ct), _ptr(st), _ptr(tst))
     return ct, st, tst
 
 

@@ -376,6 +376,11 @@ int oracle_sr_magnitude(float a, uint32_t r)
     return ((double)(r >> 8) < p * 16777216.0) ? hi : lo;
 }
 
+void oracle_sr_transpose_requant_from(const uint8_t* codes, const uint8_t* scales,
+                                      const float* tensor_scale, int64_t first, int64_t batch,
+                                      int64_t rows, int64_t cols, uint64_t seed, uint32_t draw,
+                                      uint8_t* codes_t, uint8_t* scales_t, float* tensor_scale_t);
+
 /* Step 7: dequantize -> transpose -> stochastic re-quantize, per matrix of a
  * stack ([TML4], forward/backward mismatch paragraph).  Each matrix e is its
  * own tensor (own A', s_t').  The random word of output element i (row-major
@@ -385,6 +390,17 @@ void oracle_sr_transpose_requant(const uint8_t* codes, const uint8_t* scales,
                                  const float* tensor_scale, int64_t batch, int64_t rows,
                                  int64_t cols, uint64_t seed, uint32_t draw,
                                  uint8_t* codes_t, uint8_t* scales_t, float* tensor_scale_t)
+{
+    oracle_sr_transpose_requant_from(codes, scales, tensor_scale, 0, batch, rows, cols, seed, draw,
+                                     codes_t, scales_t, tensor_scale_t);
+}
+
+/* The same for matrices first .. first+batch-1 of a larger stack whose data
+ * starts at the given pointers (the counter keeps the whole stack's index). */
+void oracle_sr_transpose_requant_from(const uint8_t* codes, const uint8_t* scales,
+                                      const float* tensor_scale, int64_t first, int64_t batch,
+                                      int64_t rows, int64_t cols, uint64_t seed, uint32_t draw,
+                                      uint8_t* codes_t, uint8_t* scales_t, float* tensor_scale_t)
 {
     int64_t n = rows * cols;
     float* y = (float*)malloc((size_t)(n > 0 ? n : 1) * sizeof(float));
@@ -414,7 +430,7 @@ void oracle_sr_transpose_requant(const uint8_t* codes, const uint8_t* scales,
                 float sbv = (float)oracle_e4m3_value(sb);
                 for (int k = 0; k < 16; ++k) {
                     int64_t local = c * rows + b * 16 + k;
-                    int64_t gi = e * n + local;
+                    int64_t gi = (first + e) * n + local;
                     int m = 0;
                     if (sbv != 0.0f) {
                         uint32_t ctr[4] = {(uint32_t)gi, (uint32_t)((uint64_t)gi >> 32), draw, 0u};

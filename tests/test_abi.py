@@ -1,0 +1,78 @@
+"""The C-ABI library builds for sm_100a, loads without a GPU, exports every
+entry point that include/nvfp4_trace.h declares, and rejects bad arguments
+before touching the device (CPU only: validation never reaches CUDA)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _lib_path():
+    from train_rollout_alignment_b200 import build
+    return build.build()
+
+
+def _declared():
+    names = []
+    for fname in os.listdir(os.path.join(ROOT, "include")):
+        if fname.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", fname)).read()
+            names += re.findall(r"^\s*(?:nvfp4_status|const char\*)\s+(nvfp4_\w+)\s*\(", text, re.M)
+    return sorted(set(names))
+
+
+def test_header_declares_the_boundary():
+    want = {"nvfp4_quantize_rtn", "nvfp4_emit_hint", "nvfp4_guided_requant",
+            "nvfp4_sr_transpose_requant", "nvfp4_rht_quantize", "nvfp4_mismatch_stats",
+            "nvfp4_tensor_amax", "nvfp4_status_string"}
+    assert want <= set(_declared())
+
+
+def test_library_exports_every_declared_symbol():
+    lib = ctypes.CDLL(_lib_path())
+    missing = [n for n in _declared() if not hasattr(lib, n)]
+    assert not missing, missing
+
+
+def test_status_strings():
+    lib = ctypes.CDLL(_lib_path())
+    lib.nvfp4_status_string.restype = ctypes.c_char_p
+    for s in range(6):
+        assert lib.nvfp4_status_string(s)
+    assert b"unknown" in lib.nvfp4_status_string(99)
+
+
+def test_validation_rejects_bad_arguments_without_a_gpu():
+    lib = ctypes.CDLL(_lib_path())
+    P, I64, I = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
+    q = lib.nvfp4_quantize_rtn
+    q.restype = I
+    q.argtypes = [P, I64, I64, P, I, P, P, P, P, I, P]
+    fake = 1 << 20  # never dereferenced: every call below fails validation first
+    assert q(fake, 4, 40, fake, 0, fake, fake, fake, None, 0, None) == 3          # cols % 16
+    assert q(fake, -1, 64, fake, 0, fake, fake, fake, None, 0, None) == 1         # negative rows
+    assert q(None, 4, 64, fake, 0, fake, fake, fake, None, 0, None) == 1          # null input
+    assert q(fake + 16, 4, 64, fake, 0, fake, fake, fake, None, 0, None) == 2     # x not 32-B aligned
+    assert q(fake, 4, 64, fake, 0, fake + 8, fake, fake, None, 0, None) == 2      # codes misaligned
+    assert q(fake, 4, 64, fake, 0, fake, fake, fake, fake, 3, None) == 5          # hint bits
+    assert q(fake, 4, 64, fake, 2, fake, fake, fake, None, 0, None) == 1          # unknown flag
+    assert q(fake, 1 << 21, 1 << 20, fake, 0, fake, fake, fake, None, 0, None) == 3  # >= 2^40
+    r = lib.nvfp4_rht_quantize
+    r.restype = I
+    r.argtypes = [P, I64, I64, ctypes.c_uint64, P, P, P, P, P, P]
+    assert r(fake, 4, 48, 3, fake, fake, fake, fake, None, None) == 3              # cols % 32
+    s = lib.nvfp4_sr_transpose_requant
+    s.restype = I
+    s.argtypes = [P, P, P, I64, I64, I64, ctypes.c_uint64, ctypes.c_uint32, P, P, P, P, P]
+    assert s(fake, fake, fake, 2, 24, 32, 2, 0, fake, fake, fake, fake, None) == 3  # rows % 16
+    assert s(fake, fake, fake, 70000, 16, 16, 2, 0, fake, fake, fake, fake, None) == 3
+    assert s(fake, fake, fake, 0, 16, 16, 2, 0, None, None, None, None, None) == 0  # empty stack
+    e = lib.nvfp4_emit_hint
+    e.restype = I
+    e.argtypes = [P, I64, I, P, P]
+    assert e(fake, 32, 3, fake, None) == 5
+    assert e(fake, 24, 2, fake, None) == 3
+    assert e(fake, 32, 2, fake + 4, None) == 2

@@ -1,0 +1,241 @@
+"""GPU parity on small and adversarial inputs: every CUDA kernel, through the C
+ABI, against the CPU oracle, element by element.  Codes, scales, tensor scales,
+hints and counters must match bit for bit; RHT outputs follow the tolerance
+rule of the RHT tests below.  Sizes span several CTAs, ragged tails and the
+degenerate cases (one block, all zeros, subnormal block scales, exact ties)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from train_rollout_alignment_b200 import synthetic as syn
+
+from _gpu_util import (Buf, assert_codes_equal, dev_bf16, f32_bits, gpu_emit_hint, gpu_guided,
+                       gpu_rht, gpu_rtn, gpu_sr, gpu_stats, lib)
+
+pytestmark = pytest.mark.gpu
+
+SHAPES = [(1, 16), (3, 48), (37, 528), (64, 1024), (257, 2080)]
+KINDS = ["normal", "heavy", "tiny", "outlier", "zeros", "ties"]
+
+
+@pytest.mark.parametrize("shape", SHAPES)
+@pytest.mark.parametrize("kind", KINDS)
+def test_rtn_matches_oracle(shape, kind):
+    x = syn.random_case(shape, 1000 + shape[0], kind)
+    for bits in (0, 1, 2, 4):
+        g = gpu_rtn(x, bits)
+        c, s, t, h = oracle.quantize_rtn(x, hint_bits=bits)
+        assert f32_bits(g["ts"]) == f32_bits(t)
+        assert_codes_equal(g["scales"], s, "scales")
+        assert_codes_equal(g["codes"], c, "codes")
+        if bits:
+            assert_codes_equal(g["hints"], h, "hints")
+        assert f32_bits(np.uint32(g["ws"][0]).view(np.float32)) == f32_bits(oracle.amax_bf16(x))
+
+
+def test_amax_precomputed_flag_and_standalone_amax():
+    b = lib()
+    x = syn.random_case((128, 256), 5, "heavy")
+    xt = dev_bf16(x)
+    ws = torch.zeros(4, dtype=torch.int32, device="cuda")
+    b.nvfp4_tensor_amax(xt, ws)
+    torch.cuda.synchronize()
+    assert f32_bits(np.uint32(ws.cpu().numpy()[0]).view(np.float32)) == f32_bits(oracle.amax_bf16(x))
+    g = gpu_rtn(x, 0, ws=ws, flags=b.NVFP4_AMAX_PRECOMPUTED)
+    c, s, t, _ = oracle.quantize_rtn(x)
+    assert_codes_equal(g["codes"], c)
+    # a planted amax is used as given: scales follow A = 2 * true amax
+    ws2 = torch.tensor([f32_bits(2 * oracle.amax_bf16(x)), 0, 0, 0], dtype=torch.int64).to(torch.int32).cuda()
+    g2 = gpu_rtn(x, 0, ws=ws2, flags=b.NVFP4_AMAX_PRECOMPUTED)
+    c2, s2, t2, _ = oracle.quantize_rtn(x, A=2 * oracle.amax_bf16(x))
+    assert f32_bits(g2["ts"]) == f32_bits(t2)
+    assert_codes_equal(g2["codes"], c2)
+
+
+@pytest.mark.parametrize("shape", [(1, 16), (37, 528), (129, 2048)])
+@pytest.mark.parametrize("noise", [2.0 ** -8, 2.0 ** -3, None])
+def test_guided_matches_oracle(shape, noise):
+    rng = np.random.default_rng(shape[0])
+    xt = syn.random_case(shape, 2000 + shape[0], "heavy")
+    xr = syn.rollout_copy(xt, rng, noise) if noise else syn.random_case(shape, 77, "heavy")
+    for bits in (1, 2, 4):
+        _, _, _, hints = oracle.quantize_rtn(xr, hint_bits=bits)
+        g = gpu_guided(xt, hints, bits)
+        c, s, t, st = oracle.guided_requant(xt, hints, bits)
+        assert f32_bits(g["ts"]) == f32_bits(t)
+        assert_codes_equal(g["scales"], s, "scales")
+        assert_codes_equal(g["codes"], c, "guided codes")
+        assert list(g["stats"][:3]) == list(st[:3])
+    g = gpu_guided(xt, None, 2)
+    c, s, t, _ = oracle.quantize_rtn(xt)
+    assert_codes_equal(g["codes"], c)
+    assert not g["stats"].any()
+
+
+def test_guided_on_grid_values_ignore_hints():
+    x = syn.random_case((32, 256), 3, "ties")
+    rng = np.random.default_rng(1)
+    for bits in (1, 2, 4):
+        hints = rng.integers(0, 256, 32 * 256 * bits // 8).astype(np.uint8)
+        g = gpu_guided(x, hints, bits)
+        c, s, t, st = oracle.guided_requant(x, hints, bits)
+        assert_codes_equal(g["codes"], c)
+        assert list(g["stats"][:3]) == list(st[:3])
+
+
+@pytest.mark.parametrize("n", [16, 48, 16 * 1001, 1 << 20])
+def test_emit_hint_matches_oracle(n):
+    rng = np.random.default_rng(n)
+    codes = rng.integers(0, 256, n // 2).astype(np.uint8)
+    for bits in (1, 2, 4):
+        assert_codes_equal(gpu_emit_hint(codes, n, bits), oracle.emit_hint(codes, n, bits), "hints")
+
+
+@pytest.mark.parametrize("shape", [(1, 16), (37, 528), (200, 1024)])
+def test_mismatch_stats_matches_oracle(shape):
+    rng = np.random.default_rng(7)
+    rows, cols = shape
+    xt = syn.random_case(shape, 3000 + rows, "normal")
+    xr = syn.rollout_copy(xt, rng, 2.0 ** -6)
+    a = oracle.quantize_rtn(xr, hint_bits=2)
+    b = oracle.guided_requant(xt, a[3], 2)
+    r = oracle.quantize_rtn(xt)
+    for (ca, sa, ta), (cb, sb, tb) in [((a[0], a[1], a[2]), (b[0], b[1], b[2])),
+                                       ((a[0], a[1], a[2]), (r[0], r[1], r[2])),
+                                       ((r[0], r[1], r[2]), (r[0], r[1], r[2])),
+                                       ((a[0], a[1], a[2]), (a[0], a[1], np.float32(a[2]) * 3))]:
+        g = gpu_stats(ca, sa, ta, cb, sb, tb, rows, cols)
+        o = oracle.mismatch_stats(ca, sa, ta, cb, sb, tb, rows, cols)
+        assert list(g[:7]) == list(o[:7])
+        assert g[7] == 0
+
+
+def _rtn_stack(w):
+    batch = w.shape[0]
+    outs = [oracle.quantize_rtn(w[e]) for e in range(batch)]
+    return (np.stack([o[0] for o in outs]), np.stack([o[1] for o in outs]),
+            np.array([o[2] for o in outs], np.float32))
+
+
+@pytest.mark.parametrize("shape", [(1, 16, 16), (3, 32, 48), (2, 80, 208), (2, 128, 64)])
+@pytest.mark.parametrize("kind", ["normal", "heavy", "tiny", "zeros"])
+def test_sr_transpose_matches_oracle(shape, kind):
+    w = syn.random_case(shape, 4000 + shape[1], kind)
+    batch, rows, cols = shape
+    codes, scales, ts = _rtn_stack(w)
+    for seed, draw in ((2, 0), (2, 1), ((5 << 32) | 17, 123456)):
+        ct, st, tst = gpu_sr(codes, scales, ts, batch, rows, cols, seed, draw)
+        oc, osc, ots = oracle.sr_transpose_requant(codes, scales, ts, batch, rows, cols, seed, draw)
+        assert [f32_bits(v) for v in tst] == [f32_bits(v) for v in ots]
+        assert_codes_equal(st, osc, "transposed scales")
+        assert_codes_equal(ct, oc, "transposed SR codes")
+
+
+def _rht_check(x, seed):
+    g = gpu_rht(x, seed)
+    rows, cols = x.shape
+    # 1) the GPU transform is within 1e-6 * ||x_group||_2 of the double-precision one
+    yd = oracle.rht32_f64(x, seed)
+    xg = syn.bf16_to_f32(x).astype(np.float64).reshape(-1, 32)
+    norm = np.linalg.norm(xg, axis=1)
+    err = np.abs(g["y"].astype(np.float64).reshape(-1, 32) - yd.reshape(-1, 32))
+    assert np.all(err <= 1e-6 * norm[:, None] + 1e-45)
+    # 2) quantization of the GPU's own y is bit-exact
+    c, s, t = oracle.quantize_f32(g["y"])
+    assert f32_bits(g["ts"]) == f32_bits(t)
+    assert_codes_equal(g["scales"], s, "rht scales")
+    assert_codes_equal(g["codes"], c, "rht codes")
+    # 3) against the full oracle, codes may differ only where the oracle's value
+    #    is within the transform tolerance (propagated to the scaled domain) of
+    #    a rounding boundary: an E4M3 midpoint for the block scale, an E2M1
+    #    midpoint for the code.
+    oc, osc, ot, oy = oracle.rht_quantize(x, seed)
+    tol_y = 1e-6 * np.repeat(norm, 2)  # per 16-block: the bound of its 32-group
+    amax_b = np.abs(oy.reshape(-1, 16)).max(axis=1).astype(np.float64)
+    e4 = np.array([oracle.e4m3_value(k) for k in range(127)])
+    e4_mid = (e4[:-1] + e4[1:]) / 2
+    sbf = amax_b / 6.0 / ot
+    near_sb = np.min(np.abs(sbf[:, None] - e4_mid[None, :]), axis=1) <= (tol_y / 6.0 / ot) * 1.01 + 1e-6 * sbf
+    blk_diff = osc.reshape(-1) != g["scales"].reshape(-1)
+    assert np.all(near_sb[blk_diff])
+    sbv = e4[osc.reshape(-1)].repeat(16)
+    same_blk = np.repeat(~blk_diff, 16)
+    diff = np.nonzero((oracle.unpack_codes(oc) != oracle.unpack_codes(g["codes"])) & same_blk)[0]
+    if diff.size:
+        scale = sbv[diff] * ot
+        a = np.abs(oy.reshape(-1)[diff].astype(np.float64)) / scale
+        mids = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0])
+        dist = np.min(np.abs(a[:, None] - mids[None, :]), axis=1)
+        assert np.all(dist <= np.repeat(tol_y, 16)[diff] / scale * 1.01 + 1e-6 * a)
+    return g
+
+
+@pytest.mark.parametrize("shape", [(1, 32), (5, 96), (64, 1024), (131, 2048)])
+@pytest.mark.parametrize("kind", ["normal", "outlier", "heavy", "zeros"])
+def test_rht_matches_oracle(shape, kind):
+    _rht_check(syn.random_case(shape, 5000 + shape[0], kind), 3)
+
+
+def test_rht_without_y_out_gives_same_codes():
+    x = syn.random_case((64, 512), 9, "heavy")
+    a = gpu_rht(x, 11, want_y=True)
+    b = gpu_rht(x, 11, want_y=False)
+    assert np.array_equal(a["codes"], b["codes"]) and np.array_equal(a["scales"], b["scales"])
+
+
+# ----------------------------------------------------------------- edge cases
+def test_empty_tensors():
+    b = lib()
+    x = torch.empty((0, 64), dtype=torch.bfloat16, device="cuda")
+    ts = torch.zeros(1, dtype=torch.float32, device="cuda")
+    ws = torch.zeros(4, dtype=torch.int32, device="cuda")
+    e = torch.empty(0, dtype=torch.uint8, device="cuda")
+    b.nvfp4_quantize_rtn(x, ws, e, e, ts, None, 0)
+    torch.cuda.synchronize()
+    assert ts.item() == 1.0
+    ts.zero_()
+    b.nvfp4_guided_requant(x, None, 2, ws, e, e, ts)
+    torch.cuda.synchronize()
+    assert ts.item() == 1.0
+    stats = torch.zeros(8, dtype=torch.int64, device="cuda")
+    b.nvfp4_mismatch_stats(e, e, ts, e, e, ts, 0, 64, stats)
+    b.nvfp4_emit_hint(e, 0, 2, e)
+    torch.cuda.synchronize()
+    assert not stats.any()
+
+
+def test_invalid_arguments_write_nothing():
+    b = lib()
+    x = dev_bf16(syn.random_case((4, 64), 1, "normal"))
+    codes = Buf(128)
+    scales = Buf(16)
+    ts = torch.zeros(1, dtype=torch.float32, device="cuda")
+    ws = torch.zeros(4, dtype=torch.int32, device="cuda")
+    raw = torch.zeros(4 * 64 + 16, dtype=torch.int16, device="cuda")
+    x_mis = raw[8:8 + 256].view(torch.bfloat16).view(4, 64)  # 16-byte aligned, not 32
+    cases = [
+        (lambda: b.nvfp4_quantize_rtn(x_mis, ws, codes.t, scales.t, ts), 2),
+        (lambda: b.nvfp4_quantize_rtn(x, ws, codes.t[1:], scales.t, ts), 2),
+        (lambda: b.nvfp4_quantize_rtn(x, ws, codes.t, scales.t, ts, codes.t, 3), 5),
+        (lambda: b.nvfp4_quantize_rtn(x, ws, codes.t, scales.t, ts, flags=8), 1),
+        (lambda: b.nvfp4_quantize_rtn(x[:, :40].contiguous(), ws, codes.t, scales.t, ts), 3),
+        (lambda: b.nvfp4_rht_quantize(x[:, :48].contiguous(), 1, ws, codes.t, scales.t, ts), 3),
+        (lambda: b.nvfp4_emit_hint(codes.t, 20, 2, scales.t), 3),
+    ]
+    for fn, status in cases:
+        with pytest.raises(b.Nvfp4Error) as ei:
+            fn()
+        assert ei.value.status == status
+    torch.cuda.synchronize()
+    assert np.all(codes.np() == 0xAB) and np.all(scales.np() == 0xAB) and ts.item() == 0.0
+
+
+def test_nonfinite_input_sets_warning_without_fault():
+    x = syn.random_case((8, 64), 2, "normal").copy()
+    x[3, 5] = 0x7F80  # +inf
+    x[6, 7] = 0x7FC1  # NaN
+    g = gpu_rtn(x, 2)
+    assert g["ws"][1] & 1
+    ok = syn.random_case((8, 64), 2, "normal")
+    assert gpu_rtn(ok, 2)["ws"][1] == 0

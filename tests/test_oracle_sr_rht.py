@@ -207,3 +207,15 @@ def test_rht_quantize_equals_quantize_of_rounded_transform():
     assert np.array_equal(y, yd.astype(np.float32))
     c2, s2, t2 = oracle.quantize_f32(y)
     assert np.array_equal(codes, c2) and np.array_equal(scales, s2) and ts == t2
+
+
+def test_sr_transpose_per_matrix_calls_match_whole_stack():
+    batch, rows, cols = 3, 16, 48
+    w = syn.random_case((batch, rows, cols), 29, "normal")
+    codes, scales, ts = _rtn_stack(w)
+    whole = oracle.sr_transpose_requant(codes, scales, ts, batch, rows, cols, 9, 4)
+    for e in range(batch):
+        part = oracle.sr_transpose_requant(codes[e:e + 1], scales[e:e + 1], ts[e:e + 1], 1, rows, cols,
+                                           9, 4, first=e)
+        assert np.array_equal(part[0][0], whole[0][e]) and np.array_equal(part[1][0], whole[1][e])
+        assert part[2][0] == whole[2][e]

@@ -1,0 +1,149 @@
+"""ctypes binding of libnvfp4trace.so: one Python function per C-ABI entry
+point, same names, argument marshalling only.
+
+Tensors are torch CUDA tensors (torch provides device memory and streams, the
+library does all the work).  Each function passes ``data_ptr()``s, sizes and
+the current CUDA stream, and raises ``Nvfp4Error`` on a non-zero status.  There
+is no CPU path: importing this module fails if the library is not built.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libnvfp4trace.so")
+if not os.path.exists(_LIB_PATH):
+    raise ImportError(
+        "libnvfp4trace.so is not built; run `python -m train_rollout_alignment_b200.build` "
+        "(nvcc, sm_100a).  There is no CPU fallback.")
+_lib = ctypes.CDLL(_LIB_PATH)
+
+_P = ctypes.c_void_p
+_I64 = ctypes.c_int64
+_I = ctypes.c_int
+_SIGS = {
+    "nvfp4_status_string": (ctypes.c_char_p, [_I]),
+    "nvfp4_tensor_amax": (_I, [_P, _I64, _P, _P]),
+    "nvfp4_quantize_rtn": (_I, [_P, _I64, _I64, _P, _I, _P, _P, _P, _P, _I, _P]),
+    "nvfp4_emit_hint": (_I, [_P, _I64, _I, _P, _P]),
+    "nvfp4_guided_requant": (_I, [_P, _I64, _I64, _P, _I, _P, _I, _P, _P, _P, _P, _P]),
+    "nvfp4_mismatch_stats": (_I, [_P, _P, _P, _P, _P, _P, _I64, _I64, _P, _P]),
+    "nvfp4_sr_transpose_requant": (
+        _I, [_P, _P, _P, _I64, _I64, _I64, ctypes.c_uint64, ctypes.c_uint32, _P, _P, _P, _P, _P]),
+    "nvfp4_rht_quantize": (_I, [_P, _I64, _I64, ctypes.c_uint64, _P, _P, _P, _P, _P, _P]),
+}
+for _name, (_res, _args) in _SIGS.items():
+    _fn = getattr(_lib, _name)
+    _fn.restype = _res
+    _fn.argtypes = _args
+
+# Constants mirrored from include/nvfp4_trace.h
+NVFP4_WS_WORDS = 4
+NVFP4_STATS8_WORDS = 8
+NVFP4_STATS4_WORDS = 4
+NVFP4_AMAX_PRECOMPUTED = 1
+NVFP4_WARN_NONFINITE = 1
+
+
+class Nvfp4Error(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        super().__init__("%s: %s (status %d)" % (fn, nvfp4_status_string(status), status))
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def nvfp4_status_string(status: int) -> str:
+    return _lib.nvfp4_status_string(int(status)).decode()
+
+
+def _ptr(t) -> int | None:
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("NVFP4 kernels take CUDA tensors")
+    if not t.is_contiguous():
+        raise ValueError("NVFP4 kernels take contiguous tensors")
+    return t.data_ptr()
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _check(fn: str, status: int):
+    if status != 0:
+        raise Nvfp4Error(fn, status)
+
+
+def _rows_cols(x):
+    if x.dim() != 2:
+        raise ValueError("expected a 2-D [rows, cols] tensor")
+    return int(x.shape[0]), int(x.shape[1])
+
+
+def nvfp4_tensor_amax(x, ws, stream=None):
+    _check("nvfp4_tensor_amax", _lib.nvfp4_tensor_amax(_ptr(x), x.numel(), _ptr(ws), _stream(stream)))
+
+
+def nvfp4_quantize_rtn(x, ws, codes, scales, tensor_scale, hints=None, hint_bits=0, flags=0,
+                       stream=None):
+    rows, cols = _rows_cols(x)
+    _check("nvfp4_quantize_rtn", _lib.nvfp4_quantize_rtn(
+        _ptr(x), rows, cols, _ptr(ws), int(flags), _ptr(codes), _ptr(scales), _ptr(tensor_scale),
+        _ptr(hints), int(hint_bits), _stream(stream)))
+
+
+def nvfp4_emit_hint(codes, n, hint_bits, hints, stream=None):
+    _check("nvfp4_emit_hint", _lib.nvfp4_emit_hint(_ptr(codes), int(n), int(hint_bits), _ptr(hints),
+                                                   _stream(stream)))
+
+
+def nvfp4_guided_requant(x, hints, hint_bits, ws, codes, scales, tensor_scale, stats4=None, flags=0,
+                         stream=None):
+    rows, cols = _rows_cols(x)
+    _check("nvfp4_guided_requant", _lib.nvfp4_guided_requant(
+        _ptr(x), rows, cols, _ptr(hints), int(hint_bits), _ptr(ws), int(flags), _ptr(codes),
+        _ptr(scales), _ptr(tensor_scale), _ptr(stats4), _stream(stream)))
+
+
+def nvfp4_mismatch_stats(codes_a, scales_a, ts_a, codes_b, scales_b, ts_b, rows, cols, stats8,
+                         stream=None):
+    _check("nvfp4_mismatch_stats", _lib.nvfp4_mismatch_stats(
+        _ptr(codes_a), _ptr(scales_a), _ptr(ts_a), _ptr(codes_b), _ptr(scales_b), _ptr(ts_b),
+        int(rows), int(cols), _ptr(stats8), _stream(stream)))
+
+
+def nvfp4_sr_transpose_requant(codes, scales, tensor_scale, batch, rows, cols, seed, draw, ws,
+                               codes_t, scales_t, tensor_scale_t, stream=None):
+    _check("nvfp4_sr_transpose_requant", _lib.nvfp4_sr_transpose_requant(
+        _ptr(codes), _ptr(scales), _ptr(tensor_scale), int(batch), int(rows), int(cols),
+        int(seed) & 0xFFFFFFFFFFFFFFFF, int(draw) & 0xFFFFFFFF, _ptr(ws), _ptr(codes_t),
+        _ptr(scales_t), _ptr(tensor_scale_t), _stream(stream)))
+
+
+def nvfp4_rht_quantize(x, sign_seed, ws, codes, scales, tensor_scale, y_out=None, stream=None):
+    rows, cols = _rows_cols(x)
+    _check("nvfp4_rht_quantize", _lib.nvfp4_rht_quantize(
+        _ptr(x), rows, cols, int(sign_seed) & 0xFFFFFFFFFFFFFFFF, _ptr(ws), _ptr(codes), _ptr(scales),
+        _ptr(tensor_scale), _ptr(y_out), _stream(stream)))
+
+
+# ----------------------------------------------------------------- output buffers
+def empty_nvfp4(rows: int, cols: int, device, hint_bits: int = 0):
+    """Device buffers for one quantized [rows, cols] tensor: codes, scales,
+    tensor scale, scratch words and (optionally) hints."""
+    codes = torch.empty((rows, cols // 2), dtype=torch.uint8, device=device)
+    scales = torch.empty((rows, cols // 16), dtype=torch.uint8, device=device)
+    ts = torch.empty(1, dtype=torch.float32, device=device)
+    ws = torch.empty(NVFP4_WS_WORDS, dtype=torch.int32, device=device)
+    hints = None
+    if hint_bits:
+        hints = torch.empty(((rows * cols * hint_bits + 7) // 8,), dtype=torch.uint8, device=device)
+    return codes, scales, ts, ws, hints

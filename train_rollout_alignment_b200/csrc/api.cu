@@ -1,0 +1,190 @@
+// api.cu -- the C ABI of libnvfp4trace.so (declared in include/nvfp4_trace.h).
+// Validates every argument before anything is enqueued, then launches the
+// kernels on the caller's stream.  No allocation, no synchronisation, no host
+// copies of device data.
+#include <cstdint>
+
+#include "../../include/nvfp4_trace.h"
+#include "launch.h"
+
+namespace {
+
+constexpr int64_t kMaxElems = int64_t(1) << 40;
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+nvfp4_status from_cuda(cudaError_t e) { return e == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA; }
+
+// Shape checks shared by the [rows, cols] entry points.
+nvfp4_status check_shape(int64_t rows, int64_t cols, int64_t col_multiple) {
+  if (rows < 0 || cols < 0) return NVFP4_ERR_INVALID_ARG;
+  if (cols % col_multiple != 0) return NVFP4_ERR_SHAPE;
+  if (rows != 0 && cols > kMaxElems / rows) return NVFP4_ERR_SHAPE;
+  return NVFP4_OK;
+}
+
+nvfp4_status check_hint_bits(int hint_bits) {
+  return (hint_bits == 1 || hint_bits == 2 || hint_bits == 4) ? NVFP4_OK : NVFP4_ERR_UNSUPPORTED;
+}
+
+// Output buffers that every quantizing call writes.
+nvfp4_status check_quant_outputs(const uint32_t* ws, const uint8_t* codes, const uint8_t* scales,
+                                 const float* tensor_scale) {
+  if (!ws || !codes || !scales || !tensor_scale) return NVFP4_ERR_INVALID_ARG;
+  if (!aligned(ws, 16) || !aligned(codes, 16) || !aligned(scales, 16) || !aligned(tensor_scale, 4))
+    return NVFP4_ERR_MISALIGNED;
+  return NVFP4_OK;
+}
+
+// Empty tensor: A = 0, so s_t = 1 is the only output.
+nvfp4_status write_unit_scale(float* tensor_scale, void* stream) {
+  if (!tensor_scale) return NVFP4_ERR_INVALID_ARG;
+  if (!aligned(tensor_scale, 4)) return NVFP4_ERR_MISALIGNED;
+  return from_cuda(nvfp4::launch_set_f32(tensor_scale, 1.0f, static_cast<cudaStream_t>(stream)));
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* nvfp4_status_string(nvfp4_status status) {
+  switch (status) {
+    case NVFP4_OK: return "ok";
+    case NVFP4_ERR_INVALID_ARG: return "invalid argument (null pointer, negative size or bad flag)";
+    case NVFP4_ERR_MISALIGNED: return "misaligned pointer";
+    case NVFP4_ERR_SHAPE: return "unsupported shape";
+    case NVFP4_ERR_CUDA: return "CUDA launch failed";
+    case NVFP4_ERR_UNSUPPORTED: return "unsupported hint_bits (expected 1, 2 or 4)";
+    default: return "unknown status";
+  }
+}
+
+nvfp4_status nvfp4_tensor_amax(const uint16_t* x_bf16, int64_t n, uint32_t* ws, void* stream) {
+  if (!ws || (n > 0 && !x_bf16)) return NVFP4_ERR_INVALID_ARG;
+  if (n < 0) return NVFP4_ERR_INVALID_ARG;
+  if (n % 16 != 0 || n >= kMaxElems) return NVFP4_ERR_SHAPE;
+  if (!aligned(ws, 16) || !aligned(x_bf16, 32)) return NVFP4_ERR_MISALIGNED;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemsetAsync(ws, 0, NVFP4_WS_WORDS * sizeof(uint32_t), s);
+  if (e != cudaSuccess) return NVFP4_ERR_CUDA;
+  return from_cuda(nvfp4::launch_amax_bf16(x_bf16, n / 16, ws, s));
+}
+
+nvfp4_status nvfp4_quantize_rtn(const uint16_t* x_bf16, int64_t rows, int64_t cols, uint32_t* ws,
+                                int flags, uint8_t* codes, uint8_t* scales, float* tensor_scale,
+                                uint8_t* hints, int hint_bits, void* stream) {
+  nvfp4_status st = check_shape(rows, cols, 16);
+  if (st != NVFP4_OK) return st;
+  if ((flags & ~NVFP4_AMAX_PRECOMPUTED) != 0) return NVFP4_ERR_INVALID_ARG;
+  if (rows * cols == 0) return write_unit_scale(tensor_scale, stream);
+  if (!x_bf16) return NVFP4_ERR_INVALID_ARG;
+  if ((st = check_quant_outputs(ws, codes, scales, tensor_scale)) != NVFP4_OK) return st;
+  if (hints) {
+    if ((st = check_hint_bits(hint_bits)) != NVFP4_OK) return st;
+    if (!aligned(hints, 16)) return NVFP4_ERR_MISALIGNED;
+  }
+  if (!aligned(x_bf16, 32)) return NVFP4_ERR_MISALIGNED;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int64_t n = rows * cols;
+  if (!(flags & NVFP4_AMAX_PRECOMPUTED)) {
+    st = nvfp4_tensor_amax(x_bf16, n, ws, stream);
+    if (st != NVFP4_OK) return st;
+  }
+  return from_cuda(nvfp4::launch_quantize_rtn(x_bf16, n / 16, ws, codes, scales, tensor_scale,
+                                              hints, hints ? hint_bits : 0, s));
+}
+
+nvfp4_status nvfp4_emit_hint(const uint8_t* codes, int64_t n, int hint_bits, uint8_t* hints,
+                             void* stream) {
+  if (n < 0) return NVFP4_ERR_INVALID_ARG;
+  if (n > 0 && (!codes || !hints)) return NVFP4_ERR_INVALID_ARG;
+  nvfp4_status st = check_hint_bits(hint_bits);
+  if (st != NVFP4_OK) return st;
+  if (n % 16 != 0 || n >= kMaxElems) return NVFP4_ERR_SHAPE;
+  if (!aligned(codes, 16) || !aligned(hints, 16)) return NVFP4_ERR_MISALIGNED;
+  return from_cuda(nvfp4::launch_emit_hint(codes, n / 16, hint_bits, hints,
+                                           static_cast<cudaStream_t>(stream)));
+}
+
+nvfp4_status nvfp4_guided_requant(const uint16_t* x_train_bf16, int64_t rows, int64_t cols,
+                                  const uint8_t* hints, int hint_bits, uint32_t* ws, int flags,
+                                  uint8_t* codes, uint8_t* scales, float* tensor_scale,
+                                  uint64_t* stats4, void* stream) {
+  nvfp4_status st = check_shape(rows, cols, 16);
+  if (st != NVFP4_OK) return st;
+  if ((flags & ~NVFP4_AMAX_PRECOMPUTED) != 0) return NVFP4_ERR_INVALID_ARG;
+  if (rows * cols == 0) return write_unit_scale(tensor_scale, stream);
+  if (!x_train_bf16) return NVFP4_ERR_INVALID_ARG;
+  if ((st = check_quant_outputs(ws, codes, scales, tensor_scale)) != NVFP4_OK) return st;
+  if (hints) {
+    if ((st = check_hint_bits(hint_bits)) != NVFP4_OK) return st;
+    if (!aligned(hints, 16)) return NVFP4_ERR_MISALIGNED;
+  }
+  if (!aligned(x_train_bf16, 32)) return NVFP4_ERR_MISALIGNED;
+  if (stats4 && !aligned(stats4, 8)) return NVFP4_ERR_MISALIGNED;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int64_t n = rows * cols;
+  if (!(flags & NVFP4_AMAX_PRECOMPUTED)) {
+    st = nvfp4_tensor_amax(x_train_bf16, n, ws, stream);
+    if (st != NVFP4_OK) return st;
+  }
+  return from_cuda(nvfp4::launch_guided(x_train_bf16, n / 16, hints, hint_bits, ws, codes, scales,
+                                        tensor_scale,
+                                        reinterpret_cast<unsigned long long*>(stats4), s));
+}
+
+nvfp4_status nvfp4_mismatch_stats(const uint8_t* codes_a, const uint8_t* scales_a,
+                                  const float* ts_a, const uint8_t* codes_b,
+                                  const uint8_t* scales_b, const float* ts_b, int64_t rows,
+                                  int64_t cols, uint64_t* stats8, void* stream) {
+  nvfp4_status st = check_shape(rows, cols, 16);
+  if (st != NVFP4_OK) return st;
+  if (rows * cols == 0) return NVFP4_OK;
+  if (!codes_a || !scales_a || !ts_a || !codes_b || !scales_b || !ts_b || !stats8)
+    return NVFP4_ERR_INVALID_ARG;
+  if (!aligned(codes_a, 16) || !aligned(codes_b, 16) || !aligned(scales_a, 16) ||
+      !aligned(scales_b, 16) || !aligned(ts_a, 4) || !aligned(ts_b, 4) || !aligned(stats8, 8))
+    return NVFP4_ERR_MISALIGNED;
+  return from_cuda(nvfp4::launch_mismatch_stats(codes_a, scales_a, ts_a, codes_b, scales_b, ts_b,
+                                                rows * cols / 16,
+                                                reinterpret_cast<unsigned long long*>(stats8),
+                                                static_cast<cudaStream_t>(stream)));
+}
+
+nvfp4_status nvfp4_sr_transpose_requant(const uint8_t* codes, const uint8_t* scales,
+                                        const float* tensor_scale, int64_t batch, int64_t rows,
+                                        int64_t cols, uint64_t seed, uint32_t draw, uint32_t* ws,
+                                        uint8_t* codes_t, uint8_t* scales_t,
+                                        float* tensor_scale_t, void* stream) {
+  if (batch < 0 || rows < 0 || cols < 0) return NVFP4_ERR_INVALID_ARG;
+  if (rows % 16 != 0 || cols % 16 != 0) return NVFP4_ERR_SHAPE;
+  if (batch > 65535 || rows / 64 >= 65535) return NVFP4_ERR_SHAPE;
+  if (rows != 0 && cols > kMaxElems / rows) return NVFP4_ERR_SHAPE;
+  if (batch != 0 && rows * cols > kMaxElems / batch) return NVFP4_ERR_SHAPE;
+  if (batch == 0) return NVFP4_OK;
+  if (!codes || !scales || !tensor_scale || !ws || !codes_t || !scales_t || !tensor_scale_t)
+    return NVFP4_ERR_INVALID_ARG;
+  if (!aligned(codes, 16) || !aligned(scales, 16) || !aligned(codes_t, 16) ||
+      !aligned(scales_t, 16) || !aligned(ws, 16) || !aligned(tensor_scale, 4) ||
+      !aligned(tensor_scale_t, 4))
+    return NVFP4_ERR_MISALIGNED;
+  return from_cuda(nvfp4::launch_sr_transpose(codes, scales, tensor_scale, batch, rows, cols, seed,
+                                              draw, ws, codes_t, scales_t, tensor_scale_t,
+                                              static_cast<cudaStream_t>(stream)));
+}
+
+nvfp4_status nvfp4_rht_quantize(const uint16_t* x_bf16, int64_t rows, int64_t cols,
+                                uint64_t sign_seed, uint32_t* ws, uint8_t* codes, uint8_t* scales,
+                                float* tensor_scale, float* y_out, void* stream) {
+  nvfp4_status st = check_shape(rows, cols, 32);
+  if (st != NVFP4_OK) return st;
+  if (rows * cols == 0) return write_unit_scale(tensor_scale, stream);
+  if (!x_bf16) return NVFP4_ERR_INVALID_ARG;
+  if ((st = check_quant_outputs(ws, codes, scales, tensor_scale)) != NVFP4_OK) return st;
+  if (!aligned(x_bf16, 32) || (y_out && !aligned(y_out, 32))) return NVFP4_ERR_MISALIGNED;
+  return from_cuda(nvfp4::launch_rht_quantize(x_bf16, rows * cols / 16, sign_seed, ws, codes,
+                                              scales, tensor_scale, y_out,
+                                              static_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"

@@ -1,0 +1,36 @@
+// launch.h -- host-side launchers shared by the C-ABI layer (api.cu) and the
+// kernel translation units.  Every launcher enqueues on `s` and returns the
+// launch status (cudaGetLastError after the launch).
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace nvfp4 {
+
+// Streaming grid: `ctas_per_sm` resident CTAs on every SM, capped by the work.
+int grid_for(int64_t work_items, int items_per_cta, int ctas_per_sm);
+int sm_count();
+
+cudaError_t launch_amax_bf16(const uint16_t* x, int64_t nblk, uint32_t* ws, cudaStream_t s);
+cudaError_t launch_quantize_rtn(const uint16_t* x, int64_t nblk, const uint32_t* ws,
+                                uint8_t* codes, uint8_t* scales, float* tensor_scale,
+                                uint8_t* hints, int hint_bits, cudaStream_t s);
+cudaError_t launch_guided(const uint16_t* x, int64_t nblk, const uint8_t* hints, int hint_bits,
+                          const uint32_t* ws, uint8_t* codes, uint8_t* scales,
+                          float* tensor_scale, unsigned long long* stats4, cudaStream_t s);
+cudaError_t launch_emit_hint(const uint8_t* codes, int64_t nblk, int hint_bits, uint8_t* hints,
+                             cudaStream_t s);
+cudaError_t launch_mismatch_stats(const uint8_t* ca, const uint8_t* sa, const float* ta,
+                                  const uint8_t* cb, const uint8_t* sb, const float* tb,
+                                  int64_t nblk, unsigned long long* stats8, cudaStream_t s);
+cudaError_t launch_sr_transpose(const uint8_t* codes, const uint8_t* scales, const float* ts,
+                                int64_t batch, int64_t rows, int64_t cols, uint64_t seed,
+                                uint32_t draw, uint32_t* ws, uint8_t* codes_t,
+                                uint8_t* scales_t, float* ts_t, cudaStream_t s);
+cudaError_t launch_rht_quantize(const uint16_t* x, int64_t nblk, uint64_t seed, uint32_t* ws,
+                                uint8_t* codes, uint8_t* scales, float* tensor_scale,
+                                float* y_out, cudaStream_t s);
+cudaError_t launch_set_f32(float* dst, float value, cudaStream_t s);
+
+}  // namespace nvfp4

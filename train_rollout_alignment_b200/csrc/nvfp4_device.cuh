@@ -1,0 +1,204 @@
+// nvfp4_device.cuh -- device-side building blocks for the NVFP4 kernels
+// (sm_100a).  Everything here is bit-exact IEEE binary32: no FMA contraction
+// (built with -fmad=false), no flush-to-zero, divisions via __fdiv_rn.
+//
+// Format (E2M1 codes, E4M3 block scale per 16 values, FP32 tensor scale) and
+// scale recipe: see include/nvfp4_trace.h.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace nvfp4 {
+
+constexpr float kTensorScaleDiv = 2688.0f;   // 6 (E2M1 max) * 448 (E4M3 max)
+constexpr float kE2M1Max = 6.0f;
+constexpr int kThreads = 256;                 // threads per CTA for the streaming kernels
+
+// ----------------------------------------------------------------- loads/stores
+// One 16-value BF16 block is 32 contiguous bytes: a single 256-bit load.
+struct alignas(32) Block16 {
+  uint32_t w[8];
+};
+
+__device__ __forceinline__ Block16 ld_block(const uint16_t* p) {
+  Block16 b;
+  asm volatile("ld.global.nc.v8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : "=r"(b.w[0]), "=r"(b.w[1]), "=r"(b.w[2]), "=r"(b.w[3]),
+                 "=r"(b.w[4]), "=r"(b.w[5]), "=r"(b.w[6]), "=r"(b.w[7])
+               : "l"(p));
+  return b;
+}
+
+__device__ __forceinline__ void st_v8f(float* p, const float* v) {
+  asm volatile("st.global.v8.f32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(p), "f"(v[0]),
+               "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7])
+               : "memory");
+}
+
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+__device__ __forceinline__ void unpack_block(const Block16& b, float* x) {
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    x[2 * k] = bf16_lo(b.w[k]);
+    x[2 * k + 1] = bf16_hi(b.w[k]);
+  }
+}
+
+// ----------------------------------------------------------------- conversions
+// Two FP32 values -> one byte holding two E2M1 codes, `lo` in bits 0..3 and
+// `hi` in bits 4..7.  Hardware round-to-nearest-even with saturation to +-6;
+// the sign of the input is kept (also for results that round to zero).
+__device__ __forceinline__ uint32_t e2m1x2(float lo, float hi) {
+  uint32_t r;
+  asm("{\n\t.reg .b8 t;\n\tcvt.rn.satfinite.e2m1x2.f32 t, %1, %2;\n\tcvt.u32.u8 %0, t;\n\t}"
+      : "=r"(r)
+      : "f"(hi), "f"(lo));
+  return r;
+}
+
+// Byte of two E2M1 codes -> the two decoded values (sign included) as FP32.
+__device__ __forceinline__ void e2m1x2_decode(uint32_t byte, float& lo, float& hi) {
+  uint32_t h2;
+  asm("{\n\t.reg .b8 t;\n\tcvt.u8.u32 t, %1;\n\tcvt.rn.f16x2.e2m1x2 %0, t;\n\t}"
+      : "=r"(h2)
+      : "r"(byte));
+  asm("cvt.f32.f16 %0, %1;" : "=f"(lo) : "h"((unsigned short)(h2 & 0xFFFFu)));
+  asm("cvt.f32.f16 %0, %1;" : "=f"(hi) : "h"((unsigned short)(h2 >> 16)));
+}
+
+// FP32 >= 0 -> E4M3 byte, round-to-nearest-even, saturating at 448.
+__device__ __forceinline__ uint32_t e4m3_rn_satfinite(float f) {
+  unsigned short r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %1;" : "=h"(r) : "f"(f));
+  return r & 0xFFu;
+}
+
+// E4M3 byte (sign bit ignored) -> exact FP32: e = 0 is m * 2^-9, otherwise
+// (8 + m) * 2^(e - 10), i.e. the FP32 pattern with exponent e + 120.
+__device__ __forceinline__ float e4m3_value(uint32_t b) {
+  b &= 0x7Fu;
+  float sub = __int2float_rn((int)(b & 7u)) * 0x1p-9f;
+  float nrm = __uint_as_float((b << 20) + (120u << 23));
+  return (b >> 3) ? nrm : sub;
+}
+
+// ----------------------------------------------------------------- scale recipe
+// Tensor decode multiplier s_t = A / 2688 (A == 0 -> 1).
+__device__ __forceinline__ float tensor_scale_from_amax(float A) {
+  return (A == 0.0f) ? 1.0f : __fdiv_rn(A, kTensorScaleDiv);
+}
+
+struct BlockScale {
+  uint32_t sb;   // E4M3 byte
+  float inv;     // 1 / (sb * s_t); 0 when sb decodes to 0 (all codes become +-0)
+};
+
+// sb = E4M3((amax_b / 6) / s_t), two rounded divisions in that order;
+// inv = 1 / (sb * s_t).
+__device__ __forceinline__ BlockScale block_scale(float amax_b, float s_t) {
+  BlockScale r;
+  float q = __fdiv_rn(amax_b, kE2M1Max);
+  float sbf = __fdiv_rn(q, s_t);
+  r.sb = e4m3_rn_satfinite(sbf);
+  float sbv = e4m3_value(r.sb);
+  r.inv = (sbv == 0.0f) ? 0.0f : __fdiv_rn(1.0f, __fmul_rn(sbv, s_t));
+  return r;
+}
+
+// 16 FP32 values (already multiplied by inv) -> 8 bytes of packed codes.
+__device__ __forceinline__ uint2 pack_codes16(const float* v) {
+  uint2 c;
+  c.x = e2m1x2(v[0], v[1]) | (e2m1x2(v[2], v[3]) << 8) | (e2m1x2(v[4], v[5]) << 16) |
+        (e2m1x2(v[6], v[7]) << 24);
+  c.y = e2m1x2(v[8], v[9]) | (e2m1x2(v[10], v[11]) << 8) | (e2m1x2(v[12], v[13]) << 16) |
+        (e2m1x2(v[14], v[15]) << 24);
+  return c;
+}
+
+// ----------------------------------------------------------------- hints
+// Compact the low `bits` bits of each of the 8 nibbles of `w` (magnitude bits
+// only for 1 and 2) into 8*bits contiguous bits, element 0 first.
+__device__ __forceinline__ uint32_t compact2(uint32_t w) {  // 8 nibbles -> 16 bits
+  uint32_t y = w & 0x33333333u;
+  y = (y | (y >> 2)) & 0x0F0F0F0Fu;
+  y = (y | (y >> 4)) & 0x00FF00FFu;
+  y = (y | (y >> 8)) & 0x0000FFFFu;
+  return y;
+}
+__device__ __forceinline__ uint32_t compact1(uint32_t w) {  // 8 nibbles -> 8 bits
+  uint32_t y = w & 0x11111111u;
+  y = (y | (y >> 3)) & 0x03030303u;
+  y = (y | (y >> 6)) & 0x000F000Fu;
+  y = (y | (y >> 12)) & 0x000000FFu;
+  return y;
+}
+
+// ----------------------------------------------------------------- reductions
+__device__ __forceinline__ uint32_t warp_max_u32(uint32_t v) {
+  return __reduce_max_sync(0xFFFFFFFFu, v);
+}
+
+// Block-wide max of a u32, result valid in every thread (blockDim.x == kThreads).
+__device__ __forceinline__ uint32_t block_max_u32(uint32_t v, uint32_t* smem32) {
+  v = warp_max_u32(v);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (lane == 0) smem32[warp] = v;
+  __syncthreads();
+  v = (lane < (kThreads / 32)) ? smem32[lane] : 0u;
+  v = warp_max_u32(v);
+  __syncthreads();
+  return v;
+}
+
+__device__ __forceinline__ unsigned long long warp_sum_u64(unsigned long long v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+  return v;
+}
+
+// Adds the block-wide sums of `vals[0..N)` to the global counters `dst`.
+template <int N>
+__device__ __forceinline__ void block_add_u64(const unsigned long long* vals,
+                                              unsigned long long* dst,
+                                              unsigned long long* smem /*[N][8]*/) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+#pragma unroll
+  for (int k = 0; k < N; ++k) {
+    unsigned long long s = warp_sum_u64(vals[k]);
+    if (lane == 0) smem[k * 8 + warp] = s;
+  }
+  __syncthreads();
+  if (warp == 0) {
+#pragma unroll
+    for (int k = 0; k < N; ++k) {
+      unsigned long long s = (lane < kThreads / 32) ? smem[k * 8 + lane] : 0ull;
+      s = warp_sum_u64(s);
+      if (lane == 0 && s != 0ull) atomicAdd(dst + k, s);
+    }
+  }
+}
+
+// ----------------------------------------------------------------- Philox4x32-10
+// Salmon, Moraes, Dror, Shaw, "Parallel random numbers: as easy as 1, 2, 3",
+// SC'11.  Returns output word x0 only.
+__device__ __forceinline__ uint32_t philox4x32_10_x0(uint32_t c0, uint32_t c1, uint32_t c2,
+                                                     uint32_t c3, uint32_t k0, uint32_t k1) {
+#pragma unroll
+  for (int r = 0; r < 10; ++r) {
+    const uint32_t hi0 = __umulhi(0xD2511F53u, c0), lo0 = 0xD2511F53u * c0;
+    const uint32_t hi1 = __umulhi(0xCD9E8D57u, c2), lo1 = 0xCD9E8D57u * c2;
+    const uint32_t n0 = hi1 ^ c1 ^ k0, n2 = hi0 ^ c3 ^ k1;
+    c0 = n0;
+    c1 = lo1;
+    c2 = n2;
+    c3 = lo0;
+    k0 += 0x9E3779B9u;
+    k1 += 0xBB67AE85u;
+  }
+  return c0;
+}
+
+}  // namespace nvfp4

@@ -1,0 +1,323 @@
+// quantize.cu -- streaming NVFP4 kernels over BF16 tensors (sm_100a):
+//   * tensor amax                       (TRACE explainer: each side scales its own values)
+//   * round-to-nearest quantize + fused hint emit   (rollout side)
+//   * guided re-quantize + counters     (train side; TRACE explainer,
+//                                        prescription and compaction paragraphs)
+//   * standalone hint emit from codes
+//
+// Data layout: the tensor is a flat sequence of 16-value blocks (rows * cols / 16
+// of them, cols % 16 == 0), so every kernel streams blocks: one thread owns one
+// block, reads its 32 bytes with a single 256-bit load and writes 8 bytes of
+// codes, 1 scale byte and 2/4/8 bytes of hints.  A warp therefore moves 1 KiB of
+// input and 256 B of codes per step, fully coalesced.  Grids are persistent
+// (a fixed number of CTAs per SM, grid-stride), each thread keeps U blocks in
+// flight.  HBM-bound: no tensor cores.
+#include "launch.h"
+#include "nvfp4_device.cuh"
+
+namespace nvfp4 {
+
+constexpr int kCtasPerSm = 4;
+constexpr int kUnroll = 2;
+
+// ----------------------------------------------------------------- amax
+// Max of |x| over BF16 magnitudes: |x| is the 15 low bits, and for non-negative
+// values the bit patterns order like the numbers, so an unsigned max on packed
+// 16-bit halves is exact.  Result: FP32 bits of A in ws[0] (atomicMax), and
+// NVFP4_WARN_NONFINITE in ws[1] when an Inf/NaN pattern was seen.
+template <int U>
+__global__ void __launch_bounds__(kThreads, kCtasPerSm)
+    k_amax_bf16(const uint16_t* __restrict__ x, int64_t nblk, uint32_t* __restrict__ ws) {
+  __shared__ uint32_t red[kThreads / 32];
+  const int64_t stride = (int64_t)gridDim.x * kThreads;
+  int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x;
+  uint32_t m2 = 0;  // two packed 16-bit maxima
+  for (; i + (U - 1) * stride < nblk; i += U * stride) {
+    Block16 b[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) b[u] = ld_block(x + (i + u * stride) * 16);
+#pragma unroll
+    for (int u = 0; u < U; ++u)
+#pragma unroll
+      for (int k = 0; k < 8; ++k) m2 = __vmaxu2(m2, b[u].w[k] & 0x7FFF7FFFu);
+  }
+  for (; i < nblk; i += stride) {
+    Block16 b = ld_block(x + i * 16);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) m2 = __vmaxu2(m2, b.w[k] & 0x7FFF7FFFu);
+  }
+  uint32_t m = max(m2 & 0xFFFFu, m2 >> 16) << 16;  // FP32 bits of the max magnitude
+  m = block_max_u32(m, red);
+  if (threadIdx.x == 0) {
+    if (m) atomicMax(ws, m);
+    if (m >= 0x7F800000u) atomicOr(ws + 1, 1u);
+  }
+}
+
+// ----------------------------------------------------------------- RTN quantize
+template <int HB>
+__device__ __forceinline__ void rtn_block(const Block16& b, float s_t, int64_t blk,
+                                          uint8_t* __restrict__ codes,
+                                          uint8_t* __restrict__ scales,
+                                          uint8_t* __restrict__ hints) {
+  float x[16];
+  unpack_block(b, x);
+  float amax = 0.0f;
+#pragma unroll
+  for (int k = 0; k < 16; ++k) amax = fmaxf(amax, fabsf(x[k]));
+  const BlockScale bs = block_scale(amax, s_t);
+  float v[16];
+#pragma unroll
+  for (int k = 0; k < 16; ++k) v[k] = __fmul_rn(x[k], bs.inv);
+  const uint2 c = pack_codes16(v);
+  reinterpret_cast<uint2*>(codes)[blk] = c;
+  scales[blk] = (uint8_t)bs.sb;
+  if (HB == 1) reinterpret_cast<uint16_t*>(hints)[blk] = (uint16_t)(compact1(c.x) | (compact1(c.y) << 8));
+  if (HB == 2) reinterpret_cast<uint32_t*>(hints)[blk] = compact2(c.x) | (compact2(c.y) << 16);
+  if (HB == 4) reinterpret_cast<uint2*>(hints)[blk] = c;
+}
+
+// Blocks are visited from the END of the tensor backwards: the amax pass that
+// runs just before streams forwards, so the tail it read last is still in L2.
+template <int HB, int U>
+__global__ void __launch_bounds__(kThreads, kCtasPerSm)
+    k_quantize_rtn(const uint16_t* __restrict__ x, int64_t nblk, const uint32_t* __restrict__ ws,
+                   uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
+                   float* __restrict__ tensor_scale, uint8_t* __restrict__ hints) {
+  const float s_t = tensor_scale_from_amax(__uint_as_float(ws[0]));
+  if (blockIdx.x == 0 && threadIdx.x == 0) *tensor_scale = s_t;
+  const int64_t stride = (int64_t)gridDim.x * kThreads;
+  int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x;
+  for (; i + (U - 1) * stride < nblk; i += U * stride) {
+    Block16 b[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) b[u] = ld_block(x + (nblk - 1 - (i + u * stride)) * 16);
+#pragma unroll
+    for (int u = 0; u < U; ++u) rtn_block<HB>(b[u], s_t, nblk - 1 - (i + u * stride), codes, scales, hints);
+  }
+  for (; i < nblk; i += stride) rtn_block<HB>(ld_block(x + (nblk - 1 - i) * 16), s_t, nblk - 1 - i, codes, scales, hints);
+}
+
+// ----------------------------------------------------------------- guided
+// Per element, with a = |v| and m the round-to-nearest magnitude index:
+//   a > G[m]  -> v lies in (G[m], G[m+1]): bracket (lo, hi) = (m, m+1)
+//   a < G[m]  -> bracket (m-1, m)
+//   a == G[m] -> on the grid, no decision;  m == 7 and a > 6 -> saturated.
+// The "other" end of the bracket replaces m when the hint names it.
+// HB = 1, 2: magnitude bits modulo 2^HB.  HB = 4: signed grid positions.
+struct GuidedCounts {
+  unsigned long long consulted, changed, outside;
+};
+
+template <int HB>
+__device__ __forceinline__ uint32_t hint_field(const uint8_t* __restrict__ hints, int64_t blk,
+                                               uint2& h4) {
+  if (HB == 1) return reinterpret_cast<const uint16_t*>(hints)[blk];
+  if (HB == 2) return reinterpret_cast<const uint32_t*>(hints)[blk];
+  h4 = reinterpret_cast<const uint2*>(hints)[blk];
+  return 0;
+}
+
+template <int HB>
+__device__ __forceinline__ void guided_block(const Block16& b, uint32_t hw, uint2 h4, float s_t,
+                                             int64_t blk, uint8_t* __restrict__ codes,
+                                             uint8_t* __restrict__ scales, GuidedCounts& cnt) {
+  float x[16];
+  unpack_block(b, x);
+  float amax = 0.0f;
+#pragma unroll
+  for (int k = 0; k < 16; ++k) amax = fmaxf(amax, fabsf(x[k]));
+  const BlockScale bs = block_scale(amax, s_t);
+  float v[16];
+#pragma unroll
+  for (int k = 0; k < 16; ++k) v[k] = __fmul_rn(x[k], bs.inv);
+  const uint2 c = pack_codes16(v);
+  uint32_t out[2] = {0u, 0u};
+#pragma unroll
+  for (int half = 0; half < 2; ++half) {
+    const uint32_t cw = half ? c.y : c.x;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      float g[2];
+      e2m1x2_decode((cw >> (8 * j)) & 0x77u, g[0], g[1]);
+#pragma unroll
+      for (int t = 0; t < 2; ++t) {
+        const int k = half * 8 + 2 * j + t;      // element within the block
+        const uint32_t nib = (cw >> (4 * (2 * j + t))) & 0xFu;
+        const uint32_t m = nib & 7u, sgn = nib >> 3;
+        const float a = fabsf(v[k]);
+        const bool up = (a > g[t]) && (m != 7u);
+        const bool dn = a < g[t];
+        uint32_t mo = m;
+        if (up || dn) {
+          const uint32_t other = up ? m + 1u : m - 1u;
+          bool take_other, match_rtn;
+          if (HB == 4) {
+            const uint32_t h = ((k < 8 ? h4.x : h4.y) >> (4 * (k & 7))) & 0xFu;
+            const uint32_t hm = h & 7u, hs = h >> 3;
+            take_other = (hm == other) && (hs == sgn || other == 0u);
+            match_rtn = (hm == m) && (hs == sgn || m == 0u);
+          } else {
+            const uint32_t mask = (1u << HB) - 1u;
+            const uint32_t h = (hw >> (HB * k)) & mask;
+            take_other = ((h ^ other) & mask) == 0u;
+            match_rtn = ((h ^ m) & mask) == 0u;
+          }
+          cnt.consulted += 1;
+          if (take_other) {
+            mo = other;
+            cnt.changed += 1;
+          } else if (!match_rtn) {
+            cnt.outside += 1;
+          }
+        }
+        out[half] |= ((sgn << 3) | mo) << (4 * (2 * j + t));
+      }
+    }
+  }
+  reinterpret_cast<uint2*>(codes)[blk] = make_uint2(out[0], out[1]);
+  scales[blk] = (uint8_t)bs.sb;
+}
+
+template <int HB, int U>
+__global__ void __launch_bounds__(kThreads, kCtasPerSm)
+    k_guided(const uint16_t* __restrict__ x, int64_t nblk, const uint8_t* __restrict__ hints,
+             const uint32_t* __restrict__ ws, uint8_t* __restrict__ codes,
+             uint8_t* __restrict__ scales, float* __restrict__ tensor_scale,
+             unsigned long long* __restrict__ stats4) {
+  __shared__ unsigned long long red[3 * 8];
+  const float s_t = tensor_scale_from_amax(__uint_as_float(ws[0]));
+  if (blockIdx.x == 0 && threadIdx.x == 0) *tensor_scale = s_t;
+  GuidedCounts cnt{0ull, 0ull, 0ull};
+  const int64_t stride = (int64_t)gridDim.x * kThreads;
+  int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x;
+  for (; i + (U - 1) * stride < nblk; i += U * stride) {
+    Block16 b[U];
+    uint32_t hw[U];
+    uint2 h4[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int64_t blk = nblk - 1 - (i + u * stride);
+      b[u] = ld_block(x + blk * 16);
+      hw[u] = hint_field<HB>(hints, blk, h4[u]);
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u)
+      guided_block<HB>(b[u], hw[u], h4[u], s_t, nblk - 1 - (i + u * stride), codes, scales, cnt);
+  }
+  for (; i < nblk; i += stride) {
+    const int64_t blk = nblk - 1 - i;
+    uint2 h4;
+    const uint32_t hw = hint_field<HB>(hints, blk, h4);
+    guided_block<HB>(ld_block(x + blk * 16), hw, h4, s_t, blk, codes, scales, cnt);
+  }
+  if (stats4 != nullptr) {
+    const unsigned long long vals[3] = {cnt.consulted, cnt.changed, cnt.outside};
+    block_add_u64<3>(vals, stats4, red);
+  }
+}
+
+// ----------------------------------------------------------------- emit hint
+template <int HB, int U>
+__global__ void __launch_bounds__(kThreads, kCtasPerSm)
+    k_emit_hint(const uint8_t* __restrict__ codes, int64_t nblk, uint8_t* __restrict__ hints) {
+  const int64_t stride = (int64_t)gridDim.x * kThreads;
+  int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x;
+  const uint2* __restrict__ c2 = reinterpret_cast<const uint2*>(codes);
+  for (; i + (U - 1) * stride < nblk; i += U * stride) {
+    uint2 c[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) c[u] = __ldg(c2 + i + u * stride);
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int64_t blk = i + u * stride;
+      if (HB == 1) reinterpret_cast<uint16_t*>(hints)[blk] = (uint16_t)(compact1(c[u].x) | (compact1(c[u].y) << 8));
+      if (HB == 2) reinterpret_cast<uint32_t*>(hints)[blk] = compact2(c[u].x) | (compact2(c[u].y) << 16);
+      if (HB == 4) reinterpret_cast<uint2*>(hints)[blk] = c[u];
+    }
+  }
+  for (; i < nblk; i += stride) {
+    const uint2 c = __ldg(c2 + i);
+    if (HB == 1) reinterpret_cast<uint16_t*>(hints)[i] = (uint16_t)(compact1(c.x) | (compact1(c.y) << 8));
+    if (HB == 2) reinterpret_cast<uint32_t*>(hints)[i] = compact2(c.x) | (compact2(c.y) << 16);
+    if (HB == 4) reinterpret_cast<uint2*>(hints)[i] = c;
+  }
+}
+
+__global__ void k_set_f32(float* dst, float value) { *dst = value; }
+
+// ----------------------------------------------------------------- launchers
+int sm_count() {
+  static int cached[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) dev = 0;
+  if (cached[dev] == 0) {
+    int n = 0;
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    cached[dev] = n > 0 ? n : 1;
+  }
+  return cached[dev];
+}
+
+int grid_for(int64_t work_items, int items_per_cta, int ctas_per_sm) {
+  const int64_t need = (work_items + items_per_cta - 1) / items_per_cta;
+  const int64_t full = (int64_t)sm_count() * ctas_per_sm;
+  return (int)(need < full ? (need > 0 ? need : 1) : full);
+}
+
+cudaError_t launch_amax_bf16(const uint16_t* x, int64_t nblk, uint32_t* ws, cudaStream_t s) {
+  if (nblk == 0) return cudaSuccess;
+  k_amax_bf16<kUnroll><<<grid_for(nblk, kThreads, kCtasPerSm), kThreads, 0, s>>>(x, nblk, ws);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quantize_rtn(const uint16_t* x, int64_t nblk, const uint32_t* ws,
+                                uint8_t* codes, uint8_t* scales, float* tensor_scale,
+                                uint8_t* hints, int hint_bits, cudaStream_t s) {
+  const int g = grid_for(nblk, kThreads, kCtasPerSm);
+  const int hb = hints ? hint_bits : 0;
+  switch (hb) {
+    case 0: k_quantize_rtn<0, kUnroll><<<g, kThreads, 0, s>>>(x, nblk, ws, codes, scales, tensor_scale, hints); break;
+    case 1: k_quantize_rtn<1, kUnroll><<<g, kThreads, 0, s>>>(x, nblk, ws, codes, scales, tensor_scale, hints); break;
+    case 2: k_quantize_rtn<2, kUnroll><<<g, kThreads, 0, s>>>(x, nblk, ws, codes, scales, tensor_scale, hints); break;
+    case 4: k_quantize_rtn<4, kUnroll><<<g, kThreads, 0, s>>>(x, nblk, ws, codes, scales, tensor_scale, hints); break;
+    default: return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_guided(const uint16_t* x, int64_t nblk, const uint8_t* hints, int hint_bits,
+                          const uint32_t* ws, uint8_t* codes, uint8_t* scales,
+                          float* tensor_scale, unsigned long long* stats4, cudaStream_t s) {
+  if (hints == nullptr)
+    return launch_quantize_rtn(x, nblk, ws, codes, scales, tensor_scale, nullptr, 0, s);
+  const int g = grid_for(nblk, kThreads, kCtasPerSm);
+  switch (hint_bits) {
+    case 1: k_guided<1, kUnroll><<<g, kThreads, 0, s>>>(x, nblk, hints, ws, codes, scales, tensor_scale, stats4); break;
+    case 2: k_guided<2, kUnroll><<<g, kThreads, 0, s>>>(x, nblk, hints, ws, codes, scales, tensor_scale, stats4); break;
+    case 4: k_guided<4, kUnroll><<<g, kThreads, 0, s>>>(x, nblk, hints, ws, codes, scales, tensor_scale, stats4); break;
+    default: return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_emit_hint(const uint8_t* codes, int64_t nblk, int hint_bits, uint8_t* hints,
+                             cudaStream_t s) {
+  if (nblk == 0) return cudaSuccess;
+  const int g = grid_for(nblk, kThreads, kCtasPerSm);
+  switch (hint_bits) {
+    case 1: k_emit_hint<1, 4><<<g, kThreads, 0, s>>>(codes, nblk, hints); break;
+    case 2: k_emit_hint<2, 4><<<g, kThreads, 0, s>>>(codes, nblk, hints); break;
+    case 4: k_emit_hint<4, 4><<<g, kThreads, 0, s>>>(codes, nblk, hints); break;
+    default: return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_set_f32(float* dst, float value, cudaStream_t s) {
+  k_set_f32<<<1, 1, 0, s>>>(dst, value);
+  return cudaGetLastError();
+}
+
+}  // namespace nvfp4
