@@ -161,8 +161,11 @@ def _rht_check(x, seed):
     assert np.all(near_sb[blk_diff])
     sbv = e4[osc.reshape(-1)].repeat(16)
     same_blk = np.repeat(~blk_diff, 16)
-    diff = np.nonzero((oracle.unpack_codes(oc) != oracle.unpack_codes(g["codes"])) & same_blk)[0]
+    # +0 and -0 are one value: an all-zero group may come out as either sign
+    pos = lambda c: np.where(c & 8, -(c & 7).astype(np.int64), (c & 7).astype(np.int64))
+    diff = np.nonzero((pos(oracle.unpack_codes(oc)) != pos(oracle.unpack_codes(g["codes"]))) & same_blk)[0]
     if diff.size:
+        assert np.all(sbv[diff] > 0)
         scale = sbv[diff] * ot
         a = np.abs(oy.reshape(-1)[diff].astype(np.float64)) / scale
         mids = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0])
