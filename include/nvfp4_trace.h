@@ -69,6 +69,7 @@ typedef int nvfp4_status;
 #define NVFP4_ERR_SHAPE         3   /* cols % 16 (RHT: % 32), rows % 16 (SR), size >= 2^40 */
 #define NVFP4_ERR_CUDA          4   /* a kernel launch failed */
 #define NVFP4_ERR_UNSUPPORTED   5   /* hint_bits not in {1, 2, 4} */
+#define NVFP4_ERR_SCRATCH_LIMIT 6   /* batch above NVFP4_SR_NOALLOC_MAX_BATCH (no-allocation entry point) */
 
 /* Scratch words written by the amax pass and read by the quantize pass. */
 #define NVFP4_WS_WORDS          4   /* ws[0] = bits of A (FP32), ws[1] = warning bits */
@@ -220,6 +221,39 @@ nvfp4_status nvfp4_rht_quantize(const uint16_t* x_bf16, int64_t rows, int64_t co
                                 uint64_t sign_seed, uint32_t* ws,
                                 uint8_t* codes, uint8_t* scales, float* tensor_scale,
                                 float* y_out, void* stream);
+
+/*
+ * nvfp4_sr_transpose_requant_noalloc -- nvfp4_sr_transpose_requant for callers
+ * that cannot allocate device memory.  (The pages have no counterpart: this is
+ * an interface variant, not a step of the method.)
+ *   Who needs it: callers that may not call cudaMalloc at this point -- e.g. a
+ *   rollout/serving engine that reserved nearly all HBM for its weight and
+ *   KV-cache pools at start-up and forbids later allocations, or C code with no
+ *   caching allocator that cannot afford the device synchronisation a
+ *   cudaMalloc/cudaFree may cause mid-step.  They cannot supply `ws`.
+ *   What it does: exactly what nvfp4_sr_transpose_requant does (same outputs,
+ *   bit for bit), with the per-matrix scratch words taken from a fixed array of
+ *   NVFP4_SR_NOALLOC_MAX_BATCH uint32 (16 KiB) inside the library.  Every GPU
+ *   that loads the library holds that array until the process exits.  Inputs
+ *   and outputs are still the caller's device buffers; nothing is allocated.
+ *   Limit: batch > NVFP4_SR_NOALLOC_MAX_BATCH returns NVFP4_ERR_SCRATCH_LIMIT
+ *   and enqueues nothing.
+ *   Set-up: the first call on a device looks up the array's device address
+ *   (cudaGetSymbolAddress, with that device current -- call with the stream's
+ *   device current) and caches it; make that first call before any stream
+ *   capture.
+ *   Sharing: all calls on a device share the one array; each call clears the
+ *   words it uses on `stream` before its kernels read them, and the array keeps
+ *   the last call's contents.  Calls whose work overlaps on the GPU (different
+ *   streams without ordering between them) race on the array: order them.
+ */
+#define NVFP4_SR_NOALLOC_MAX_BATCH 4096
+nvfp4_status nvfp4_sr_transpose_requant_noalloc(const uint8_t* codes, const uint8_t* scales,
+                                                const float* tensor_scale,
+                                                int64_t batch, int64_t rows, int64_t cols,
+                                                uint64_t seed, uint32_t draw,
+                                                uint8_t* codes_t, uint8_t* scales_t,
+                                                float* tensor_scale_t, void* stream);
 
 /* Human-readable name of a status code (static string, never NULL). */
 const char* nvfp4_status_string(nvfp4_status status);

@@ -33,6 +33,8 @@ _SIGS = {
     "nvfp4_sr_transpose_requant": (
         _I, [_P, _P, _P, _I64, _I64, _I64, ctypes.c_uint64, ctypes.c_uint32, _P, _P, _P, _P, _P]),
     "nvfp4_rht_quantize": (_I, [_P, _I64, _I64, ctypes.c_uint64, _P, _P, _P, _P, _P, _P]),
+    "nvfp4_sr_transpose_requant_noalloc": (
+        _I, [_P, _P, _P, _I64, _I64, _I64, ctypes.c_uint64, ctypes.c_uint32, _P, _P, _P, _P]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _fn = getattr(_lib, _name)
@@ -45,6 +47,8 @@ NVFP4_STATS8_WORDS = 8
 NVFP4_STATS4_WORDS = 4
 NVFP4_AMAX_PRECOMPUTED = 1
 NVFP4_WARN_NONFINITE = 1
+NVFP4_ERR_SCRATCH_LIMIT = 6
+NVFP4_SR_NOALLOC_MAX_BATCH = 4096
 
 
 class Nvfp4Error(RuntimeError):
@@ -126,6 +130,17 @@ def nvfp4_sr_transpose_requant(codes, scales, tensor_scale, batch, rows, cols, s
         _ptr(codes), _ptr(scales), _ptr(tensor_scale), int(batch), int(rows), int(cols),
         int(seed) & 0xFFFFFFFFFFFFFFFF, int(draw) & 0xFFFFFFFF, _ptr(ws), _ptr(codes_t),
         _ptr(scales_t), _ptr(tensor_scale_t), _stream(stream)))
+
+
+def nvfp4_sr_transpose_requant_noalloc(codes, scales, tensor_scale, batch, rows, cols, seed, draw,
+                                       codes_t, scales_t, tensor_scale_t, stream=None):
+    """SR transpose without a scratch argument, for callers that cannot
+    allocate device memory (the library keeps a fixed scratch array of
+    NVFP4_SR_NOALLOC_MAX_BATCH words per GPU; see include/nvfp4_trace.h)."""
+    _check("nvfp4_sr_transpose_requant_noalloc", _lib.nvfp4_sr_transpose_requant_noalloc(
+        _ptr(codes), _ptr(scales), _ptr(tensor_scale), int(batch), int(rows), int(cols),
+        int(seed) & 0xFFFFFFFFFFFFFFFF, int(draw) & 0xFFFFFFFF, _ptr(codes_t), _ptr(scales_t),
+        _ptr(tensor_scale_t), _stream(stream)))
 
 
 def nvfp4_rht_quantize(x, sign_seed, ws, codes, scales, tensor_scale, y_out=None, stream=None):

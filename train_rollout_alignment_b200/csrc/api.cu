@@ -55,6 +55,9 @@ const char* nvfp4_status_string(nvfp4_status status) {
     case NVFP4_ERR_SHAPE: return "unsupported shape";
     case NVFP4_ERR_CUDA: return "CUDA launch failed";
     case NVFP4_ERR_UNSUPPORTED: return "unsupported hint_bits (expected 1, 2 or 4)";
+    case NVFP4_ERR_SCRATCH_LIMIT:
+      return "batch exceeds the fixed scratch of the no-allocation entry point "
+             "(NVFP4_SR_NOALLOC_MAX_BATCH matrices)";
     default: return "unknown status";
   }
 }
