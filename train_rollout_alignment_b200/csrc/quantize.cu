@@ -19,6 +19,7 @@ namespace nvfp4 {
 
 constexpr int kCtasPerSm = 4;
 constexpr int kUnroll = 2;
+constexpr int kAmaxUnroll = 4;  // 128 bytes in flight per thread: the amax pass has no other work
 
 // ----------------------------------------------------------------- amax
 // Max of |x| over BF16 magnitudes: |x| is the 15 low bits, and for non-negative
@@ -105,6 +106,10 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 //   a == G[m] -> on the grid, no decision;  m == 7 and a > 6 -> saturated.
 // The "other" end of the bracket replaces m when the hint names it.
 // HB = 1, 2: magnitude bits modulo 2^HB.  HB = 4: signed grid positions.
+//
+// Only the up/down flags need per-element work (an exact FP32 comparison
+// of a with the decoded G[m], done on the bit patterns, which order like the
+// values for a >= 0).  Everything else runs on 8 packed nibbles at a time.
 struct GuidedCounts {
   unsigned long long consulted, changed, outside;
 };
@@ -116,6 +121,68 @@ __device__ __forceinline__ uint32_t hint_field(const uint8_t* __restrict__ hints
   if (HB == 2) return reinterpret_cast<const uint32_t*>(hints)[blk];
   h4 = reinterpret_cast<const uint2*>(hints)[blk];
   return 0;
+}
+
+// 8 one-bit (two-bit) fields -> bit 0 (bits 0..1) of 8 nibbles.
+__device__ __forceinline__ uint32_t expand1(uint32_t h8) {
+  uint32_t y = h8 & 0xFFu;
+  y = (y | (y << 12)) & 0x000F000Fu;
+  y = (y | (y << 6)) & 0x03030303u;
+  y = (y | (y << 3)) & 0x11111111u;
+  return y;
+}
+__device__ __forceinline__ uint32_t expand2(uint32_t h16) {
+  uint32_t y = h16 & 0xFFFFu;
+  y = (y | (y << 8)) & 0x00FF00FFu;
+  y = (y | (y << 4)) & 0x0F0F0F0Fu;
+  y = (y | (y << 2)) & 0x33333333u;
+  return y;
+}
+// bit 0 of each nibble: 1 iff the nibble of t is zero.
+__device__ __forceinline__ uint32_t nib_zero(uint32_t t) {
+  t |= t >> 1;
+  t |= t >> 2;
+  return ~t & 0x11111111u;
+}
+
+template <int HB>
+__device__ __forceinline__ uint32_t guided_word(uint32_t R, const float* v, uint32_t hword,
+                                                GuidedCounts& cnt) {
+  const uint32_t M = R & 0x77777777u;  // RTN magnitudes
+  const uint32_t S = R & 0x88888888u;  // signs (of x)
+  uint32_t UP = 0u, DN = 0u;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    float g[2];
+    e2m1x2_decode((M >> (8 * j)) & 0x77u, g[0], g[1]);
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+      const uint32_t ab = __float_as_uint(v[2 * j + t]) & 0x7FFFFFFFu;
+      const uint32_t gb = __float_as_uint(g[t]);
+      UP |= (uint32_t)(ab > gb) << (8 * j + 4 * t);
+      DN |= (uint32_t)(ab < gb) << (8 * j + 4 * t);
+    }
+  }
+  UP &= ~(M & (M >> 1) & (M >> 2));            // m == 7 and a > 6: saturated
+  const uint32_t OFF = UP | DN;                // a rounding decision exists
+  const uint32_t O = M + UP - DN;              // the other bracket end
+  uint32_t take, keep;
+  if (HB == 4) {
+    const uint32_t Hm = hword & 0x77777777u;
+    const uint32_t zh = nib_zero(Hm);
+    take = nib_zero(hword ^ (O | S)) | (nib_zero(O) & zh);
+    keep = nib_zero(hword ^ R) | (nib_zero(M) & zh);
+  } else {
+    const uint32_t mask = HB == 1 ? 0x11111111u : 0x33333333u;
+    const uint32_t H = HB == 1 ? expand1(hword) : expand2(hword);
+    take = nib_zero((H ^ O) & mask);
+    keep = nib_zero((H ^ M) & mask);
+  }
+  take &= OFF;
+  cnt.consulted += __popc(OFF);
+  cnt.changed += __popc(take);
+  cnt.outside += __popc(OFF & ~take & ~keep);
+  return (M + (take & UP) - (take & DN)) | S;
 }
 
 template <int HB>
@@ -132,50 +199,17 @@ __device__ __forceinline__ void guided_block(const Block16& b, uint32_t hw, uint
 #pragma unroll
   for (int k = 0; k < 16; ++k) v[k] = __fmul_rn(x[k], bs.inv);
   const uint2 c = pack_codes16(v);
-  uint32_t out[2] = {0u, 0u};
-#pragma unroll
-  for (int half = 0; half < 2; ++half) {
-    const uint32_t cw = half ? c.y : c.x;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      float g[2];
-      e2m1x2_decode((cw >> (8 * j)) & 0x77u, g[0], g[1]);
-#pragma unroll
-      for (int t = 0; t < 2; ++t) {
-        const int k = half * 8 + 2 * j + t;      // element within the block
-        const uint32_t nib = (cw >> (4 * (2 * j + t))) & 0xFu;
-        const uint32_t m = nib & 7u, sgn = nib >> 3;
-        const float a = fabsf(v[k]);
-        const bool up = (a > g[t]) && (m != 7u);
-        const bool dn = a < g[t];
-        uint32_t mo = m;
-        if (up || dn) {
-          const uint32_t other = up ? m + 1u : m - 1u;
-          bool take_other, match_rtn;
-          if (HB == 4) {
-            const uint32_t h = ((k < 8 ? h4.x : h4.y) >> (4 * (k & 7))) & 0xFu;
-            const uint32_t hm = h & 7u, hs = h >> 3;
-            take_other = (hm == other) && (hs == sgn || other == 0u);
-            match_rtn = (hm == m) && (hs == sgn || m == 0u);
-          } else {
-            const uint32_t mask = (1u << HB) - 1u;
-            const uint32_t h = (hw >> (HB * k)) & mask;
-            take_other = ((h ^ other) & mask) == 0u;
-            match_rtn = ((h ^ m) & mask) == 0u;
-          }
-          cnt.consulted += 1;
-          if (take_other) {
-            mo = other;
-            cnt.changed += 1;
-          } else if (!match_rtn) {
-            cnt.outside += 1;
-          }
-        }
-        out[half] |= ((sgn << 3) | mo) << (4 * (2 * j + t));
-      }
-    }
+  uint32_t h_lo, h_hi;
+  if (HB == 4) {
+    h_lo = h4.x;
+    h_hi = h4.y;
+  } else {
+    h_lo = hw;
+    h_hi = hw >> (8 * (HB & 3));
   }
-  reinterpret_cast<uint2*>(codes)[blk] = make_uint2(out[0], out[1]);
+  const uint32_t o0 = guided_word<HB>(c.x, v, h_lo, cnt);
+  const uint32_t o1 = guided_word<HB>(c.y, v + 8, h_hi, cnt);
+  reinterpret_cast<uint2*>(codes)[blk] = make_uint2(o0, o1);
   scales[blk] = (uint8_t)bs.sb;
 }
 
@@ -268,7 +302,7 @@ int grid_for(int64_t work_items, int items_per_cta, int ctas_per_sm) {
 
 cudaError_t launch_amax_bf16(const uint16_t* x, int64_t nblk, uint32_t* ws, cudaStream_t s) {
   if (nblk == 0) return cudaSuccess;
-  k_amax_bf16<kUnroll><<<grid_for(nblk, kThreads, kCtasPerSm), kThreads, 0, s>>>(x, nblk, ws);
+  k_amax_bf16<kAmaxUnroll><<<grid_for(nblk, kThreads, kCtasPerSm), kThreads, 0, s>>>(x, nblk, ws);
   return cudaGetLastError();
 }
 
