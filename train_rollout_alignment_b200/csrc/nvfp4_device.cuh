@@ -59,6 +59,26 @@ __device__ __forceinline__ uint32_t e2m1x2(float lo, float hi) {
   return r;
 }
 
+// Byte of two E2M1 codes -> the two decoded values as a packed f16x2 (code of
+// bits 0..3 in the low half); exact, sign included.
+__device__ __forceinline__ uint32_t e2m1x2_to_f16x2(uint32_t byte) {
+  uint32_t h2;
+  asm("{\n\t.reg .b8 t;\n\tcvt.u8.u32 t, %1;\n\tcvt.rn.f16x2.e2m1x2 %0, t;\n\t}"
+      : "=r"(h2)
+      : "r"(byte));
+  return h2;
+}
+
+// d0 = lo(h2) - a0, d1 = hi(h2) - a1: f16 minus f32 in one rounding to FP32
+// (exact whenever the two are within a factor of two, Sterbenz).
+__device__ __forceinline__ void f16x2_minus_f32(uint32_t h2, float a0, float a1, float& d0,
+                                                float& d1) {
+  asm("{\n\t.reg .f16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\tsub.rn.f32.f16 %0, lo, %3;\n\t"
+      "sub.rn.f32.f16 %1, hi, %4;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "r"(h2), "f"(a0), "f"(a1));
+}
+
 // Byte of two E2M1 codes -> the two decoded values (sign included) as FP32.
 __device__ __forceinline__ void e2m1x2_decode(uint32_t byte, float& lo, float& hi) {
   uint32_t h2;
@@ -108,6 +128,44 @@ __device__ __forceinline__ BlockScale block_scale(float amax_b, float s_t) {
   return r;
 }
 
+// Per-CTA tables for tensors whose block maxima are BF16 values (at most 8
+// significant bits), filled once per CTA from s_t:
+//   inv[b]  = 1 / (E4M3(b) * s_t)        (0 when E4M3(b) == 0), all 128 bytes;
+//   div6[m] = FP32 bits of RN((1 + m/128) / 6), one per BF16 mantissa.
+// RN(amax / 6) for amax = (1 + m/128) * 2^E is div6[m] with E added to its
+// exponent field whenever the result stays a normal float (scaling by a power
+// of two commutes with round-to-nearest there), so only sbf = q / s_t keeps a
+// division.  Results are bit-identical to block_scale().
+struct ScaleTables {
+  float inv[128];
+  uint32_t div6[128];
+};
+
+__device__ __forceinline__ void scale_tables_init(ScaleTables& t, float s_t) {
+  const int i = threadIdx.x;
+  if (i < 128) {
+    const float sbv = e4m3_value((uint32_t)i);
+    t.inv[i] = (sbv == 0.0f) ? 0.0f : __fdiv_rn(1.0f, __fmul_rn(sbv, s_t));
+    t.div6[i] = __float_as_uint(__fdiv_rn(__uint_as_float(0x3F800000u | ((uint32_t)i << 16)), kE2M1Max));
+  }
+  __syncthreads();
+}
+
+// block_scale() for a BF16-valued amax (bits of the FP32 value, low 16 zero).
+__device__ __forceinline__ BlockScale block_scale_bf16(uint32_t amax_bits, float s_t,
+                                                       const ScaleTables& t) {
+  const uint32_t e = amax_bits >> 23;  // biased exponent (amax >= 0)
+  float q;
+  if (e >= 4u && e < 255u)
+    q = __uint_as_float(t.div6[(amax_bits >> 16) & 0x7Fu] + ((e - 127u) << 23));
+  else
+    q = __fdiv_rn(__uint_as_float(amax_bits), kE2M1Max);
+  BlockScale r;
+  r.sb = e4m3_rn_satfinite(__fdiv_rn(q, s_t));
+  r.inv = t.inv[r.sb & 0x7Fu];
+  return r;
+}
+
 // 16 FP32 values (already multiplied by inv) -> 8 bytes of packed codes.
 __device__ __forceinline__ uint2 pack_codes16(const float* v) {
   uint2 c;
@@ -135,6 +193,21 @@ __device__ __forceinline__ uint32_t compact1(uint32_t w) {  // 8 nibbles -> 8 bi
   y = (y | (y >> 12)) & 0x000000FFu;
   return y;
 }
+
+// ----------------------------------------------------------------- nibble masks
+// Masks below use bit 0 of each nibble as the per-element flag.
+__device__ __forceinline__ uint32_t nib_nonzero(uint32_t t) {  // nibble != 0
+  t |= t >> 1;
+  t |= t >> 2;
+  return t & 0x11111111u;
+}
+__device__ __forceinline__ uint32_t nib_zero(uint32_t t) {  // nibble == 0
+  t |= t >> 1;
+  t |= t >> 2;
+  return ~t & 0x11111111u;
+}
+// Number of flags set (multiply-add instead of popc, which is a slow pipe).
+__device__ __forceinline__ uint32_t count_nib(uint32_t m) { return (m * 0x11111111u) >> 28; }
 
 // ----------------------------------------------------------------- reductions
 __device__ __forceinline__ uint32_t warp_max_u32(uint32_t v) {

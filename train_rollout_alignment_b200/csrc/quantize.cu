@@ -56,17 +56,22 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 }
 
 // ----------------------------------------------------------------- RTN quantize
+// Max |x| of a block as FP32 bits: packed 16-bit maxima of the BF16 magnitudes.
+__device__ __forceinline__ uint32_t block_amax_bits(const Block16& b) {
+  uint32_t m2 = 0u;
+#pragma unroll
+  for (int k = 0; k < 8; ++k) m2 = __vmaxu2(m2, b.w[k] & 0x7FFF7FFFu);
+  return max(m2 & 0xFFFFu, m2 >> 16) << 16;
+}
+
 template <int HB>
-__device__ __forceinline__ void rtn_block(const Block16& b, float s_t, int64_t blk,
-                                          uint8_t* __restrict__ codes,
+__device__ __forceinline__ void rtn_block(const Block16& b, float s_t, const ScaleTables& tab,
+                                          int64_t blk, uint8_t* __restrict__ codes,
                                           uint8_t* __restrict__ scales,
                                           uint8_t* __restrict__ hints) {
   float x[16];
   unpack_block(b, x);
-  float amax = 0.0f;
-#pragma unroll
-  for (int k = 0; k < 16; ++k) amax = fmaxf(amax, fabsf(x[k]));
-  const BlockScale bs = block_scale(amax, s_t);
+  const BlockScale bs = block_scale_bf16(block_amax_bits(b), s_t, tab);
   float v[16];
 #pragma unroll
   for (int k = 0; k < 16; ++k) v[k] = __fmul_rn(x[k], bs.inv);
@@ -85,8 +90,10 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     k_quantize_rtn(const uint16_t* __restrict__ x, int64_t nblk, const uint32_t* __restrict__ ws,
                    uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
                    float* __restrict__ tensor_scale, uint8_t* __restrict__ hints) {
+  __shared__ ScaleTables tab;
   const float s_t = tensor_scale_from_amax(__uint_as_float(ws[0]));
   if (blockIdx.x == 0 && threadIdx.x == 0) *tensor_scale = s_t;
+  scale_tables_init(tab, s_t);
   const int64_t stride = (int64_t)gridDim.x * kThreads;
   int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x;
   for (; i + (U - 1) * stride < nblk; i += U * stride) {
@@ -94,9 +101,11 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 #pragma unroll
     for (int u = 0; u < U; ++u) b[u] = ld_block(x + (nblk - 1 - (i + u * stride)) * 16);
 #pragma unroll
-    for (int u = 0; u < U; ++u) rtn_block<HB>(b[u], s_t, nblk - 1 - (i + u * stride), codes, scales, hints);
+    for (int u = 0; u < U; ++u)
+      rtn_block<HB>(b[u], s_t, tab, nblk - 1 - (i + u * stride), codes, scales, hints);
   }
-  for (; i < nblk; i += stride) rtn_block<HB>(ld_block(x + (nblk - 1 - i) * 16), s_t, nblk - 1 - i, codes, scales, hints);
+  for (; i < nblk; i += stride)
+    rtn_block<HB>(ld_block(x + (nblk - 1 - i) * 16), s_t, tab, nblk - 1 - i, codes, scales, hints);
 }
 
 // ----------------------------------------------------------------- guided
@@ -138,38 +147,21 @@ __device__ __forceinline__ uint32_t expand2(uint32_t h16) {
   y = (y | (y << 2)) & 0x33333333u;
   return y;
 }
-// bit 0 of each nibble: 1 iff the nibble of t is zero.
-__device__ __forceinline__ uint32_t nib_zero(uint32_t t) {
-  t |= t >> 1;
-  t |= t >> 2;
-  return ~t & 0x11111111u;
-}
 
+// Bracket, hint match and selection for 8 elements.  R: round-to-nearest
+// codes; DIR: per nibble the signed digit +1 (v above G[m]), -1 (below) or 0
+// (on the grid, or saturated), summed as sum_k dir_k * 16^k in modular
+// arithmetic, so M + DIR has the digits m_k + dir_k (all in 0..7).
 template <int HB>
-__device__ __forceinline__ uint32_t guided_word(uint32_t R, const float* v, uint32_t hword,
-                                                GuidedCounts& cnt) {
-  const uint32_t M = R & 0x77777777u;  // RTN magnitudes
+__device__ __forceinline__ uint32_t guided_select(uint32_t R, uint32_t DIR, uint32_t hword,
+                                                  GuidedCounts& cnt) {
+  const uint32_t M = R & 0x77777777u;  // round-to-nearest magnitudes
   const uint32_t S = R & 0x88888888u;  // signs (of x)
-  uint32_t UP = 0u, DN = 0u;
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    float g[2];
-    e2m1x2_decode((M >> (8 * j)) & 0x77u, g[0], g[1]);
-#pragma unroll
-    for (int t = 0; t < 2; ++t) {
-      const uint32_t ab = __float_as_uint(v[2 * j + t]) & 0x7FFFFFFFu;
-      const uint32_t gb = __float_as_uint(g[t]);
-      UP |= (uint32_t)(ab > gb) << (8 * j + 4 * t);
-      DN |= (uint32_t)(ab < gb) << (8 * j + 4 * t);
-    }
-  }
-  UP &= ~(M & (M >> 1) & (M >> 2));            // m == 7 and a > 6: saturated
-  const uint32_t OFF = UP | DN;                // a rounding decision exists
-  const uint32_t O = M + UP - DN;              // the other bracket end
+  const uint32_t O = M + DIR;          // the other end of each bracket
+  const uint32_t OFF = nib_nonzero(O ^ M);  // a rounding decision exists
   uint32_t take, keep;
   if (HB == 4) {
-    const uint32_t Hm = hword & 0x77777777u;
-    const uint32_t zh = nib_zero(Hm);
+    const uint32_t zh = nib_zero(hword & 0x77777777u);
     take = nib_zero(hword ^ (O | S)) | (nib_zero(O) & zh);
     keep = nib_zero(hword ^ R) | (nib_zero(M) & zh);
   } else {
@@ -179,37 +171,45 @@ __device__ __forceinline__ uint32_t guided_word(uint32_t R, const float* v, uint
     keep = nib_zero((H ^ M) & mask);
   }
   take &= OFF;
-  cnt.consulted += __popc(OFF);
-  cnt.changed += __popc(take);
-  cnt.outside += __popc(OFF & ~take & ~keep);
-  return (M + (take & UP) - (take & DN)) | S;
+  cnt.consulted += count_nib(OFF);
+  cnt.changed += count_nib(take);
+  cnt.outside += count_nib(OFF & ~take & ~keep);
+  const uint32_t T = take * 0xFu;  // whole-nibble select mask
+  return ((O & T) | (M & ~T)) | S;
 }
 
 template <int HB>
 __device__ __forceinline__ void guided_block(const Block16& b, uint32_t hw, uint2 h4, float s_t,
-                                             int64_t blk, uint8_t* __restrict__ codes,
+                                             const ScaleTables& tab, int64_t blk,
+                                             uint8_t* __restrict__ codes,
                                              uint8_t* __restrict__ scales, GuidedCounts& cnt) {
   float x[16];
   unpack_block(b, x);
-  float amax = 0.0f;
+  const BlockScale bs = block_scale_bf16(block_amax_bits(b), s_t, tab);
+  uint32_t out[2];
 #pragma unroll
-  for (int k = 0; k < 16; ++k) amax = fmaxf(amax, fabsf(x[k]));
-  const BlockScale bs = block_scale(amax, s_t);
-  float v[16];
+  for (int half = 0; half < 2; ++half) {
+    uint32_t R = 0u, DIR = 0u;
 #pragma unroll
-  for (int k = 0; k < 16; ++k) v[k] = __fmul_rn(x[k], bs.inv);
-  const uint2 c = pack_codes16(v);
-  uint32_t h_lo, h_hi;
-  if (HB == 4) {
-    h_lo = h4.x;
-    h_hi = h4.y;
-  } else {
-    h_lo = hw;
-    h_hi = hw >> (8 * (HB & 3));
+    for (int j = 0; j < 4; ++j) {
+      const int k = 8 * half + 2 * j;
+      const float v0 = __fmul_rn(x[k], bs.inv), v1 = __fmul_rn(x[k + 1], bs.inv);
+      const uint32_t byte = e2m1x2(v0, v1);  // round-to-nearest codes
+      R |= byte << (8 * j);
+      // G[m] - min(|v|, 6): exact; its sign is minus the direction of v
+      // from G[m] (min(|v|, 6) turns saturation into "on the grid")
+      float d0, d1;
+      f16x2_minus_f32(e2m1x2_to_f16x2(byte & 0x77u), fminf(fabsf(v0), kE2M1Max),
+                      fminf(fabsf(v1), kE2M1Max), d0, d1);
+      const int c0 = min(max(__float_as_int(d0), -1), 1), c1 = min(max(__float_as_int(d1), -1), 1);
+      DIR -= ((uint32_t)c0 << (8 * j)) + ((uint32_t)c1 << (8 * j + 4));
+    }
+    uint32_t hword;
+    if (HB == 4) hword = half ? h4.y : h4.x;
+    else hword = half ? (hw >> (8 * (HB & 3))) : hw;
+    out[half] = guided_select<HB>(R, DIR, hword, cnt);
   }
-  const uint32_t o0 = guided_word<HB>(c.x, v, h_lo, cnt);
-  const uint32_t o1 = guided_word<HB>(c.y, v + 8, h_hi, cnt);
-  reinterpret_cast<uint2*>(codes)[blk] = make_uint2(o0, o1);
+  reinterpret_cast<uint2*>(codes)[blk] = make_uint2(out[0], out[1]);
   scales[blk] = (uint8_t)bs.sb;
 }
 
@@ -220,8 +220,10 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
              uint8_t* __restrict__ scales, float* __restrict__ tensor_scale,
              unsigned long long* __restrict__ stats4) {
   __shared__ unsigned long long red[3 * 8];
+  __shared__ ScaleTables tab;
   const float s_t = tensor_scale_from_amax(__uint_as_float(ws[0]));
   if (blockIdx.x == 0 && threadIdx.x == 0) *tensor_scale = s_t;
+  scale_tables_init(tab, s_t);
   GuidedCounts cnt{0ull, 0ull, 0ull};
   const int64_t stride = (int64_t)gridDim.x * kThreads;
   int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x;
@@ -237,13 +239,13 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     }
 #pragma unroll
     for (int u = 0; u < U; ++u)
-      guided_block<HB>(b[u], hw[u], h4[u], s_t, nblk - 1 - (i + u * stride), codes, scales, cnt);
+      guided_block<HB>(b[u], hw[u], h4[u], s_t, tab, nblk - 1 - (i + u * stride), codes, scales, cnt);
   }
   for (; i < nblk; i += stride) {
     const int64_t blk = nblk - 1 - i;
     uint2 h4;
     const uint32_t hw = hint_field<HB>(hints, blk, h4);
-    guided_block<HB>(ld_block(x + blk * 16), hw, h4, s_t, blk, codes, scales, cnt);
+    guided_block<HB>(ld_block(x + blk * 16), hw, h4, s_t, tab, blk, codes, scales, cnt);
   }
   if (stats4 != nullptr) {
     const unsigned long long vals[3] = {cnt.consulted, cnt.changed, cnt.outside};

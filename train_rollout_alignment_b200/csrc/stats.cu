@@ -2,20 +2,27 @@
 // (TRACE explainer: the train/rollout distance is the quantity to shrink; the
 // compaction paragraph observes that >99% of mismatches are one cell apart).
 //
-// One thread per 16-value block: 8 code bytes and 1 scale byte from each side.
-// The kernel moves 1.125 bytes per element, so its integer work has to stay
-// near 6 instructions per element to keep pace with HBM: positions are handled
-// 8 nibbles at a time (SWAR) and |pos_a - pos_b| 4 bytes at a time.
+// One lane per 16-value block: 8 code bytes and 1 scale byte from each side,
+// 1.125 bytes per element.  On sm_100a the logic pipe (LOP3/SHF/PRMT/ISETP)
+// retires 64 lanes per clock per SM, so keeping pace with HBM leaves about 3
+// logic instructions per element.  Two ideas keep the kernel under that:
 //
-// Decoded-value mismatches, exactly (decoded value = (G[m] * sb) * s_t in FP32):
-//   * identical scales (same scale byte, same tensor scale) and all decoded
-//     magnitudes normal: values differ exactly where positions differ;
-//   * otherwise two nonzero values can only be equal if
-//     (sb_a * s_t_a) / (sb_b * s_t_b) lies within ~2^-22 of a ratio of two
-//     grid values, i.e. of 2^k, 3 * 2^k or 2^k / 3 (the grid is
-//     {2^k, 3 * 2^k}).  When the ratio's significand is far from 1, 4/3 and
-//     3/2, only zero/zero pairs are equal;
-//   * any other block falls back to the element-by-element FP32 comparison.
+//  * Position counters only need work where codes differ.  A block whose 16
+//    codes are identical on both sides contributes nothing, so each warp
+//    pushes its "dirty" blocks into a shared-memory queue (ballot + prefix
+//    rank) and processes them 32 at a time, one per lane, with the packed
+//    counting below.  The cost follows the mismatch rate, not the size.
+//  * Decoded-value mismatches (value = (G[m] * sb) * s_t in FP32) are decided
+//    per block with no per-element FP32 work:
+//      - same scale byte and same tensor scale, all products normal floats:
+//        values differ exactly where positions differ (taken from the queue);
+//      - otherwise two nonzero values can only be equal if
+//        (sb_a * s_t_a) / (sb_b * s_t_b) lies within ~2^-22 of a ratio of two
+//        grid values, i.e. of 2^k, 3 * 2^k or 2^k / 3 (the grid is
+//        {2^k, 3 * 2^k}).  The significand of that ratio depends only on the
+//        two scale significands (16 x 16 cases) given the tensor scales, so a
+//        per-CTA table says where only zero/zero pairs can be equal;
+//      - any other block compares the 16 values in FP32 (rare).
 #include "launch.h"
 #include "nvfp4_device.cuh"
 
@@ -23,10 +30,15 @@ namespace nvfp4 {
 
 constexpr int kStatsCtasPerSm = 4;
 constexpr int kStatsUnroll = 4;
+constexpr int kWarps = kThreads / 32;
+constexpr int kQueue = 64;  // dirty-block slots per warp (at most 31 + 32 are ever held)
 
 struct MismatchCounts {
   uint32_t mism, far, sumd, scale, value;
 };
+
+// Number of set bits of a mask that only uses bit 7 of each byte.
+__device__ __forceinline__ uint32_t count_byte_msb(uint32_t m) { return ((m >> 7) * 0x01010101u) >> 24; }
 
 // 8 codes -> 8 offset positions 8 + pos in [1, 15] (+0 and -0 both give 8).
 __device__ __forceinline__ uint32_t offset_pos(uint32_t w) {
@@ -35,39 +47,37 @@ __device__ __forceinline__ uint32_t offset_pos(uint32_t w) {
   return ((M ^ K) + 0x88888888u) - K;                // s ? 8 - m : 8 + m
 }
 
-// bit 0 of each nibble: nibble nonzero.
-__device__ __forceinline__ uint32_t nib_nonzero(uint32_t t) {
-  t |= t >> 1;
-  t |= t >> 2;
-  return t & 0x11111111u;
-}
-
 // |a - b| for 4 byte lanes holding values in [1, 15].
 __device__ __forceinline__ uint32_t absdiff_bytes(uint32_t a, uint32_t b) {
-  const uint32_t t = (a | 0x10101010u) - b;          // 16 + a - b in [2, 30]
+  const uint32_t t = (a | 0x10101010u) - b;                     // 16 + a - b in [2, 30]
   const uint32_t ng = ((t >> 4) & 0x01010101u) ^ 0x01010101u;  // a < b
   return ((t ^ (ng * 0x0Fu)) & 0x0F0F0F0Fu) + ng;
 }
 
-// Counts for one word of 8 elements; returns the nibble mask of positions
-// that differ (bit 0 per nibble).
-__device__ __forceinline__ uint32_t mismatch_word(uint32_t wa, uint32_t wb, MismatchCounts& c) {
+// Position counters of one word (8 elements); returns the number of
+// positions that differ.
+__device__ __forceinline__ uint32_t position_word(uint32_t wa, uint32_t wb, MismatchCounts& c) {
   const uint32_t pa = offset_pos(wa), pb = offset_pos(wb);
-  const uint32_t diff = nib_nonzero(pa ^ pb);
+  const uint32_t n = count_nib(nib_nonzero(pa ^ pb));
   const uint32_t d_even = absdiff_bytes(pa & 0x0F0F0F0Fu, pb & 0x0F0F0F0Fu);
   const uint32_t d_odd = absdiff_bytes((pa >> 4) & 0x0F0F0F0Fu, (pb >> 4) & 0x0F0F0F0Fu);
   c.sumd = __dp4a(d_even + d_odd, 0x01010101u, c.sumd);  // each byte sum <= 28
   const uint32_t far_e = ((d_even & 0x0E0E0E0Eu) + 0x7F7F7F7Fu) & 0x80808080u;
   const uint32_t far_o = ((d_odd & 0x0E0E0E0Eu) + 0x7F7F7F7Fu) & 0x80808080u;
-  c.far += __popc(far_e | (far_o >> 1));
-  c.mism += __popc(diff);
-  return diff;
+  c.far += count_byte_msb(far_e) + count_byte_msb(far_o);
+  c.mism += n;
+  return n;
 }
 
 __device__ __forceinline__ bool near_grid_ratio(float rho) {
   const int f = (int)(__float_as_uint(rho) & 0x7FFFFFu);  // significand bits
   const int tol = 64;                                      // 2^-17 relative
   return f < tol || f > 0x800000 - tol || abs(f - 0x2AAAAB) < tol || abs(f - 0x400000) < tol;
+}
+
+// Integer significand of an E4M3 byte: 8 + mantissa (normal) or mantissa.
+__device__ __forceinline__ uint32_t e4m3_significand(uint32_t b) {
+  return (b & 7u) | ((b & 0x78u) ? 8u : 0u);
 }
 
 __device__ __forceinline__ uint32_t value_mismatch_slow(uint2 a, uint2 b, float sva, float svb,
@@ -89,28 +99,32 @@ __device__ __forceinline__ uint32_t value_mismatch_slow(uint2 a, uint2 b, float 
   return n;
 }
 
-__device__ __forceinline__ void mismatch_block(uint2 a, uint2 b, uint32_t sba, uint32_t sbb,
-                                               float tsa, float tsb, bool same_ts,
-                                               MismatchCounts& c) {
-  c.scale += (sba != sbb) ? 1u : 0u;
-  const uint32_t d0 = mismatch_word(a.x, b.x, c);
-  const uint32_t d1 = mismatch_word(a.y, b.y, c);
-  const float sva = e4m3_value(sba), svb = e4m3_value(sbb);
-  const float xa = __fmul_rn(sva, tsa), xb = __fmul_rn(svb, tsb);
-  // every nonzero decoded value is a normal float (no underflow, no overflow)
-  const bool normal = xa >= 0x1p-124f && xb >= 0x1p-124f && xa <= 0x1p120f && xb <= 0x1p120f;
-  uint32_t value;
-  if (normal && same_ts && sba == sbb) {
-    value = __popc(d0) + __popc(d1);
-  } else if (normal && !near_grid_ratio(__fdividef(xa, xb))) {
-    // only zero/zero pairs can be equal
-    const uint32_t nz0 = nib_nonzero((a.x | b.x) & 0x77777777u);
-    const uint32_t nz1 = nib_nonzero((a.y | b.y) & 0x77777777u);
-    value = __popc(nz0) + __popc(nz1);
-  } else {
-    value = value_mismatch_slow(a, b, sva, svb, tsa, tsb);
+struct StatsShared {
+  uint4 queue[kWarps][kQueue];
+  uint8_t queue_same[kWarps][kQueue];  // value counter follows positions
+  uint8_t normal_a[128], normal_b[128];
+  uint8_t ratio_far[256];              // [sig_a * 16 + sig_b]: only zero pairs can be equal
+  unsigned long long red[6 * 8];
+};
+
+// Lane `lane` takes queue slot `lane` (if < n) and counts it; the slots
+// n..qn-1 then move to the front.  Returns the new queue length.
+__device__ __forceinline__ int flush_queue(StatsShared& sm, int warp, int lane, int qn, int n,
+                                           MismatchCounts& c) {
+  __syncwarp();
+  if (lane < n) {
+    const uint4 e = sm.queue[warp][lane];
+    const uint32_t mb = position_word(e.x, e.z, c) + position_word(e.y, e.w, c);
+    if (sm.queue_same[warp][lane]) c.value += mb;
   }
-  c.value += value;
+  __syncwarp();
+  const int rest = qn - n;
+  if (lane < rest) {
+    sm.queue[warp][lane] = sm.queue[warp][n + lane];
+    sm.queue_same[warp][lane] = sm.queue_same[warp][n + lane];
+  }
+  __syncwarp();
+  return rest;
 }
 
 template <int U>
@@ -119,33 +133,87 @@ __global__ void __launch_bounds__(kThreads, kStatsCtasPerSm)
                      const float* __restrict__ ta, const uint8_t* __restrict__ cb,
                      const uint8_t* __restrict__ sb, const float* __restrict__ tb, int64_t nblk,
                      unsigned long long* __restrict__ stats8) {
-  __shared__ unsigned long long red[6 * 8];
+  __shared__ StatsShared sm;
   const float tsa = *ta, tsb = *tb;
   const bool same_ts = __float_as_uint(tsa) == __float_as_uint(tsb);
+  const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+  if (t < 128) {
+    const float xa = __fmul_rn(e4m3_value(t), tsa), xb = __fmul_rn(e4m3_value(t), tsb);
+    // every nonzero decoded value of the block is a normal float
+    sm.normal_a[t] = xa >= 0x1p-124f && xa <= 0x1p120f;
+    sm.normal_b[t] = xb >= 0x1p-124f && xb <= 0x1p120f;
+  }
+  {
+    // significand of (sb_a * s_t_a) / (sb_b * s_t_b) for scale significands
+    // ma, mb (powers of two do not change it); approximate to a few ulps,
+    // far below the 2^-17 tolerance of near_grid_ratio
+    const uint32_t ma = (uint32_t)t >> 4, mb = (uint32_t)t & 15u;
+    const float tr = __fdiv_rn(tsa, tsb);
+    bool far_ratio = false;
+    if (ma != 0u && mb != 0u && tr >= 0x1p-120f && tr <= 0x1p120f)
+      far_ratio = !near_grid_ratio(__fmul_rn(__fdiv_rn((float)ma, (float)mb), tr));
+    sm.ratio_far[t] = far_ratio;
+  }
+  __syncthreads();
+
   MismatchCounts c{0u, 0u, 0u, 0u, 0u};
   const uint2* __restrict__ a2 = reinterpret_cast<const uint2*>(ca);
   const uint2* __restrict__ b2 = reinterpret_cast<const uint2*>(cb);
-  const int64_t stride = (int64_t)gridDim.x * kThreads;
-  int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x;
-  for (; i + (U - 1) * stride < nblk; i += U * stride) {
+  const uint32_t lt_mask = (1u << lane) - 1u;
+  const int64_t wstride = (int64_t)gridDim.x * kThreads;  // blocks per grid-wide step
+  int qn = 0;                                             // warp-uniform queue length
+  for (int64_t wb = (int64_t)blockIdx.x * kThreads + warp * 32; wb < nblk; wb += U * wstride) {
     uint2 va[U], vb[U];
     uint32_t xa[U], xb[U];
 #pragma unroll
     for (int u = 0; u < U; ++u) {
-      va[u] = __ldg(a2 + i + u * stride);
-      vb[u] = __ldg(b2 + i + u * stride);
-      xa[u] = __ldg(sa + i + u * stride);
-      xb[u] = __ldg(sb + i + u * stride);
+      const int64_t i = wb + u * wstride + lane;
+      if (i < nblk) {
+        va[u] = __ldg(a2 + i);
+        vb[u] = __ldg(b2 + i);
+        xa[u] = __ldg(sa + i);
+        xb[u] = __ldg(sb + i);
+      } else {
+        va[u] = vb[u] = make_uint2(0u, 0u);
+        xa[u] = xb[u] = 0u;
+      }
     }
 #pragma unroll
-    for (int u = 0; u < U; ++u) mismatch_block(va[u], vb[u], xa[u], xb[u], tsa, tsb, same_ts, c);
+    for (int u = 0; u < U; ++u) {
+      const bool valid = wb + u * wstride + lane < nblk;
+      const uint2 a = va[u], b = vb[u];
+      const bool same = same_ts && xa[u] == xb[u] && sm.normal_a[xa[u] & 0x7Fu];
+      const bool dirty = ((a.x ^ b.x) | (a.y ^ b.y)) != 0u;
+      const uint32_t m = __ballot_sync(0xFFFFFFFFu, dirty);
+      if (dirty) {
+        const int slot = qn + __popc(m & lt_mask);
+        sm.queue[warp][slot] = make_uint4(a.x, a.y, b.x, b.y);
+        sm.queue_same[warp][slot] = same;
+      }
+      qn += __popc(m);
+      if (qn >= 32) qn = flush_queue(sm, warp, lane, qn, 32, c);
+      if (valid) {
+        c.scale += (xa[u] != xb[u]) ? 1u : 0u;
+        if (!same) {
+          const uint32_t ia = xa[u] & 0x7Fu, ib = xb[u] & 0x7Fu;
+          if (sm.normal_a[ia] && sm.normal_b[ib] &&
+              sm.ratio_far[e4m3_significand(ia) * 16u + e4m3_significand(ib)]) {
+            // only zero/zero pairs are equal
+            c.value += count_nib(nib_nonzero((a.x | b.x) & 0x77777777u)) +
+                       count_nib(nib_nonzero((a.y | b.y) & 0x77777777u));
+          } else {
+            c.value += value_mismatch_slow(a, b, e4m3_value(xa[u]), e4m3_value(xb[u]), tsa, tsb);
+          }
+        }
+      }
+    }
   }
-  for (; i < nblk; i += stride)
-    mismatch_block(__ldg(a2 + i), __ldg(b2 + i), __ldg(sa + i), __ldg(sb + i), tsa, tsb, same_ts, c);
+  if (qn > 0) flush_queue(sm, warp, lane, qn, qn, c);
+
   const unsigned long long vals[6] = {c.mism, (unsigned long long)(c.mism - c.far), c.far, c.sumd,
                                       c.scale, c.value};
-  block_add_u64<6>(vals, stats8 + 1, red);
-  if (blockIdx.x == 0 && threadIdx.x == 0) atomicAdd(stats8, (unsigned long long)nblk * 16ull);
+  block_add_u64<6>(vals, stats8 + 1, sm.red);
+  if (blockIdx.x == 0 && t == 0) atomicAdd(stats8, (unsigned long long)nblk * 16ull);
 }
 
 cudaError_t launch_mismatch_stats(const uint8_t* ca, const uint8_t* sa, const float* ta,
