@@ -16,7 +16,7 @@ from _gpu_util import (Buf, assert_codes_equal, dev_bf16, f32_bits, gpu_emit_hin
 pytestmark = pytest.mark.gpu
 
 SHAPES = [(1, 16), (3, 48), (37, 528), (64, 1024), (257, 2080)]
-KINDS = ["normal", "heavy", "tiny", "outlier", "zeros", "ties"]
+KINDS = ["normal", "heavy", "tiny", "outlier", "zeros", "ties", "sparse"]
 
 
 @pytest.mark.parametrize("shape", SHAPES)
@@ -82,6 +82,25 @@ def test_guided_on_grid_values_ignore_hints():
         c, s, t, st = oracle.guided_requant(x, hints, bits)
         assert_codes_equal(g["codes"], c)
         assert list(g["stats"][:3]) == list(st[:3])
+
+
+@pytest.mark.parametrize("shape", [(3, 48), (64, 1024)])
+def test_guided_zeros_subnormals_adversarial_hints(shape):
+    """Exact zeros (+0 and -0) sit on the grid and must ignore the hint; BF16
+    subnormals are off the grid (bracket 0 / 0.5) and must follow it."""
+    x = syn.random_case(shape, 11, "sparse")
+    rng = np.random.default_rng(shape[0])
+    n = x.size
+    for bits in (1, 2, 4):
+        hints = rng.integers(0, 256, (n * bits + 7) // 8).astype(np.uint8)
+        g = gpu_guided(x, hints, bits)
+        c, s, t, st = oracle.guided_requant(x, hints, bits)
+        assert_codes_equal(g["scales"], s, "scales")
+        assert_codes_equal(g["codes"], c, "guided codes")
+        assert list(g["stats"][:3]) == list(st[:3])
+        r = gpu_rtn(x, bits)
+        oc, os_, ot, oh = oracle.quantize_rtn(x, hint_bits=bits)
+        assert_codes_equal(r["codes"], oc, "rtn codes")
 
 
 @pytest.mark.parametrize("n", [16, 48, 16 * 1001, 1 << 20])

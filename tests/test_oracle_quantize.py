@@ -139,6 +139,22 @@ def test_hint_pack_round_trip(bits):
     assert np.array_equal(vals, want)
 
 
+def test_sparse_case_zeros_are_on_grid():
+    """Exact zeros never consult the hint; BF16 subnormals next to a large
+    value quantize to zero magnitude but are off the grid (bracket 0 / 0.5)."""
+    x = syn.random_case((4, 64), 11, "sparse")
+    xf = syn.bf16_to_f32(x)
+    zero = xf.reshape(-1) == 0
+    assert zero.sum() > 64
+    for bits in (1, 2):
+        h_all = np.full(x.size * bits // 8, 0xFF, np.uint8)  # always names the odd cell
+        gc, _, _, st = oracle.guided_requant(x, h_all, bits)
+        c = _codes(gc, x.size)
+        assert np.all(c[zero] & 7 == 0)
+        assert np.array_equal(c[zero] >> 3, np.signbit(xf.reshape(-1)[zero]).astype(np.uint8))
+        assert st[0] <= x.size - zero.sum()
+
+
 @pytest.mark.parametrize("bits", [1, 2, 4])
 def test_guided_by_own_hints_is_rtn(bits):
     x = syn.random_case((16, 128), 7, "heavy")

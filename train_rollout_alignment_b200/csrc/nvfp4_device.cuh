@@ -59,24 +59,16 @@ __device__ __forceinline__ uint32_t e2m1x2(float lo, float hi) {
   return r;
 }
 
-// Byte of two E2M1 codes -> the two decoded values as a packed f16x2 (code of
-// bits 0..3 in the low half); exact, sign included.
-__device__ __forceinline__ uint32_t e2m1x2_to_f16x2(uint32_t byte) {
-  uint32_t h2;
-  asm("{\n\t.reg .b8 t;\n\tcvt.u8.u32 t, %1;\n\tcvt.rn.f16x2.e2m1x2 %0, t;\n\t}"
-      : "=r"(h2)
-      : "r"(byte));
-  return h2;
-}
-
-// d0 = lo(h2) - a0, d1 = hi(h2) - a1: f16 minus f32 in one rounding to FP32
-// (exact whenever the two are within a factor of two, Sterbenz).
-__device__ __forceinline__ void f16x2_minus_f32(uint32_t h2, float a0, float a1, float& d0,
-                                                float& d1) {
-  asm("{\n\t.reg .f16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\tsub.rn.f32.f16 %0, lo, %3;\n\t"
-      "sub.rn.f32.f16 %1, hi, %4;\n\t}"
-      : "=f"(d0), "=f"(d1)
-      : "r"(h2), "f"(a0), "f"(a1));
+// Four FP32 values -> four E2M1 codes (16 bits, a0 in bits 0..3) rounded
+// toward zero: the hardware stochastic-rounding conversion with all random bits
+// zero truncates, i.e. the magnitude index is floor onto the grid (saturating
+// at 6, sign kept).
+__device__ __forceinline__ uint32_t e2m1x4_rz(float a0, float a1, float a2, float a3) {
+  unsigned short r;
+  asm("cvt.rs.satfinite.e2m1x4.f32 %0, {%1, %2, %3, %4}, %5;"
+      : "=h"(r)
+      : "f"(a3), "f"(a2), "f"(a1), "f"(a0), "r"(0u));
+  return r;
 }
 
 // Byte of two E2M1 codes -> the two decoded values (sign included) as FP32.

@@ -148,34 +148,44 @@ __device__ __forceinline__ uint32_t expand2(uint32_t h16) {
   return y;
 }
 
-// Bracket, hint match and selection for 8 elements.  R: round-to-nearest
-// codes; DIR: per nibble the signed digit +1 (v above G[m]), -1 (below) or 0
-// (on the grid, or saturated), summed as sum_k dir_k * 16^k in modular
-// arithmetic, so M + DIR has the digits m_k + dir_k (all in 0..7).
+// Bracket, hint match and selection for 8 elements, all on packed nibbles.
+//   R: round-to-nearest codes of v (signs of x);
+//   Z: floor codes of a = |v| (the lower bracket end lo when a is off the grid);
+//   P: floor codes of a nudged down, (a - 2^-149) * (1 - 2^-24): equal to Z
+//      unless a sits exactly on a grid point (a grid value drops one cell, zero
+//      turns negative), so P != Z marks "no rounding decision".
+// Off the grid R is lo or lo + 1, so the other end of the bracket is
+// O = 2 * lo + 1 - m.  a > 6 gives Z = m = 7 and O = 8: saturated, no decision.
+// Per-element flags live in bit 3 of each nibble: a nibble value in 0..8 is
+// nonzero exactly when adding 7 sets its bit 3 (no carry leaves the nibble).
 template <int HB>
-__device__ __forceinline__ uint32_t guided_select(uint32_t R, uint32_t DIR, uint32_t hword,
-                                                  GuidedCounts& cnt) {
-  const uint32_t M = R & 0x77777777u;  // round-to-nearest magnitudes
-  const uint32_t S = R & 0x88888888u;  // signs (of x)
-  const uint32_t O = M + DIR;          // the other end of each bracket
-  const uint32_t OFF = nib_nonzero(O ^ M);  // a rounding decision exists
-  uint32_t take, keep;
+__device__ __forceinline__ uint32_t guided_select(uint32_t R, uint32_t Z, uint32_t P,
+                                                  uint32_t hword, GuidedCounts& cnt) {
+  constexpr uint32_t kB3 = 0x88888888u, kSeven = 0x77777777u;
+  const uint32_t M = R & kSeven;  // round-to-nearest magnitudes
+  const uint32_t S = R - M;       // signs (of x)
+  const uint32_t O = (Z << 1) + 0x11111111u - M;
+  // P ^ Z is 0 off the grid and 1, 3, 7 (a grid value) or 8 (zero) on it
+  const uint32_t off = ~(((P ^ Z) + kSeven) | O) & kB3;  // a rounding decision exists
+  uint32_t take, differs;  // differs: the hint does not name the round-to-nearest cell
   if (HB == 4) {
-    const uint32_t zh = nib_zero(hword & 0x77777777u);
-    take = nib_zero(hword ^ (O | S)) | (nib_zero(O) & zh);
-    keep = nib_zero(hword ^ R) | (nib_zero(M) & zh);
+    // signed positions: equal codes, or both magnitudes zero
+    const auto nz4 = [](uint32_t t) { return (((t & kSeven) + kSeven) | t) & kB3; };
+    const uint32_t zh = ~((hword & kSeven) + kSeven);
+    take = ~nz4(hword ^ (O | S)) | (~(O + kSeven) & zh);
+    differs = nz4(hword ^ R) & ((M + kSeven) | ~zh);
   } else {
     const uint32_t mask = HB == 1 ? 0x11111111u : 0x33333333u;
     const uint32_t H = HB == 1 ? expand1(hword) : expand2(hword);
-    take = nib_zero((H ^ O) & mask);
-    keep = nib_zero((H ^ M) & mask);
+    take = ~(((H ^ O) & mask) + kSeven);
+    differs = ((H ^ M) & mask) + kSeven;
   }
-  take &= OFF;
-  cnt.consulted += count_nib(OFF);
-  cnt.changed += count_nib(take);
-  cnt.outside += count_nib(OFF & ~take & ~keep);
-  const uint32_t T = take * 0xFu;  // whole-nibble select mask
-  return ((O & T) | (M & ~T)) | S;
+  take &= off;
+  cnt.consulted += __popc(off);
+  cnt.changed += __popc(take);
+  cnt.outside += __popc(off & ~take & differs);
+  const uint32_t T = (take >> 3) * 0xFu;  // whole-nibble select mask
+  return ((O & T) | (M & ~T)) + S;
 }
 
 template <int HB>
@@ -189,25 +199,24 @@ __device__ __forceinline__ void guided_block(const Block16& b, uint32_t hw, uint
   uint32_t out[2];
 #pragma unroll
   for (int half = 0; half < 2; ++half) {
-    uint32_t R = 0u, DIR = 0u;
+    float a[8], p[8];
+    uint32_t R = 0u;
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       const int k = 8 * half + 2 * j;
-      const float v0 = __fmul_rn(x[k], bs.inv), v1 = __fmul_rn(x[k + 1], bs.inv);
-      const uint32_t byte = e2m1x2(v0, v1);  // round-to-nearest codes
-      R |= byte << (8 * j);
-      // G[m] - min(|v|, 6): exact; its sign is minus the direction of v
-      // from G[m] (min(|v|, 6) turns saturation into "on the grid")
-      float d0, d1;
-      f16x2_minus_f32(e2m1x2_to_f16x2(byte & 0x77u), fminf(fabsf(v0), kE2M1Max),
-                      fminf(fabsf(v1), kE2M1Max), d0, d1);
-      const int c0 = min(max(__float_as_int(d0), -1), 1), c1 = min(max(__float_as_int(d1), -1), 1);
-      DIR -= ((uint32_t)c0 << (8 * j)) + ((uint32_t)c1 << (8 * j + 4));
+      R += e2m1x2(__fmul_rn(x[k], bs.inv), __fmul_rn(x[k + 1], bs.inv)) << (8 * j);
     }
+#pragma unroll
+    for (int t = 0; t < 8; ++t) {
+      a[t] = __fmul_rn(fabsf(x[8 * half + t]), bs.inv);  // |v|, bit-identical to |x * inv|
+      p[t] = __fmul_rn(__fsub_rn(a[t], 0x1p-149f), 0x1.fffffep-1f);
+    }
+    const uint32_t Z = e2m1x4_rz(a[0], a[1], a[2], a[3]) + (e2m1x4_rz(a[4], a[5], a[6], a[7]) << 16);
+    const uint32_t P = e2m1x4_rz(p[0], p[1], p[2], p[3]) + (e2m1x4_rz(p[4], p[5], p[6], p[7]) << 16);
     uint32_t hword;
     if (HB == 4) hword = half ? h4.y : h4.x;
     else hword = half ? (hw >> (8 * (HB & 3))) : hw;
-    out[half] = guided_select<HB>(R, DIR, hword, cnt);
+    out[half] = guided_select<HB>(R, Z, P, hword, cnt);
   }
   reinterpret_cast<uint2*>(codes)[blk] = make_uint2(out[0], out[1]);
   scales[blk] = (uint8_t)bs.sb;

@@ -98,7 +98,7 @@ CFG2_SR_SEED = 2
 def random_case(shape, seed: int, kind: str = "normal") -> np.ndarray:
     """Small edge-case inputs: 'normal', 'tiny' (subnormal block scales),
     'outlier' (one huge value), 'zeros', 'ties' (values near grid midpoints),
-    'heavy' (Student-t nu=2)."""
+    'heavy' (Student-t nu=2), 'sparse' (half exact zeros, BF16 subnormals)."""
     rng = np.random.Generator(np.random.PCG64(seed))
     if kind == "normal":
         x = rng.standard_normal(shape, dtype=np.float32)
@@ -118,6 +118,19 @@ def random_case(shape, seed: int, kind: str = "normal") -> np.ndarray:
         x.reshape(-1)[::16] = 6.0  # block max 6 -> scale close to 1 so ties survive
     elif kind == "heavy":
         x = rng.standard_t(2.0, size=shape).astype(np.float32)
+    elif kind == "sparse":
+        # half exact zeros (some -0), BF16 subnormals, normal values, one outlier
+        x = rng.standard_normal(shape, dtype=np.float32)
+        flat = x.reshape(-1)
+        u = rng.random(flat.size)
+        flat[u < 0.5] = 0.0
+        flat[(u >= 0.5) & (u < 0.55)] = -0.0
+        sub = (u >= 0.55) & (u < 0.65)
+        bits = bf16_bits(x).reshape(-1)
+        bits[sub] = rng.integers(1, 0x80, int(sub.sum())).astype(np.uint16) | \
+            (rng.integers(0, 2, int(sub.sum())).astype(np.uint16) << 15)
+        bits[rng.integers(0, bits.size)] = bf16_bits(np.float32([4.0e5]))[0]
+        return bits.reshape(shape)
     else:
         raise ValueError(kind)
     return bf16_bits(x)
