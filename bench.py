@@ -60,13 +60,6 @@ def _peaks():
     return 6650.0, "fallback"
 
 
-def _dist():
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    return world, rank, local
-
-
 # --------------------------------------------------------------------------- clocks
 CLOCK_QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
                "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -236,7 +229,8 @@ def main():
     ap.add_argument("--layers", type=int, default=48)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     args = ap.parse_args()
-    world, rank, local = _dist()
+    from train_rollout_alignment_b200 import dist as tdist
+    world, rank, local = tdist.world()
     if args.impl == "reference":
         return run_reference(args, world, rank, local)
     return run_ours(args, world, rank, local)
@@ -253,11 +247,11 @@ def _config(layers):
 
 def run_ours(args, world, rank, local):
     from train_rollout_alignment_b200 import _binding as b
+    from train_rollout_alignment_b200 import dist as tdist
     torch.cuda.set_device(local)
     device = torch.device("cuda", local)
     if world > 1:
-        import datetime
-        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+        tdist.init("nccl")
     peak, peak_kind = _peaks()
 
     stack = Stack(args.layers, args.layers // 2, device, rank)
@@ -269,14 +263,10 @@ def run_ours(args, world, rank, local):
         stack.step(b)
     torch.cuda.synchronize()
 
-    def barrier():
-        if world > 1:
-            torch.distributed.barrier()
-
     # ---- device-timed region: K steps, per-kernel events on the launching stream
     sampler = ClockSampler(local)
     time.sleep(0.3)
-    barrier()
+    tdist.barrier()
     torch.cuda.synchronize()
     events = []
     t_start = torch.cuda.Event(enable_timing=True)
@@ -286,13 +276,9 @@ def run_ours(args, world, rank, local):
         stack.step(b, events)
     t_end.record()
     torch.cuda.synchronize()
-    barrier()
+    tdist.barrier()
     clocks = sampler.stop()
-    elapsed = t_start.elapsed_time(t_end) / 1e3
-    t_max = torch.tensor([elapsed], dtype=torch.float64, device=device)
-    if world > 1:
-        torch.distributed.all_reduce(t_max, op=torch.distributed.ReduceOp.MAX)
-    t_max = float(t_max.item())
+    t_max = tdist.max_over_ranks(t_start.elapsed_time(t_end) / 1e3, device)
 
     # per-kernel durations (average over launches in the timed region)
     labels = [lab for l in range(args.layers) for lab, _ in stack.kernels_of_layer(l)] * args.steps
@@ -315,8 +301,11 @@ def run_ours(args, world, rank, local):
     dom_gbs = per[dom]["bytes"] / (per[dom]["ms"] / 1e3) / 1e9
     traffic = _ncu_traffic(dom)
 
-    value = world * args.steps * step_bytes / t_max / 1e9
-    elems = world * args.steps * step_elems / t_max
+    value = tdist.aggregate_rate(args.steps * step_bytes, world, t_max) / 1e9
+    elems = tdist.aggregate_rate(args.steps * step_elems, world, t_max)
+
+    # ---- the other rows of the path, each timed alone (rank-local)
+    other = time_other_kernels(b, stack, device, peak)
 
     # ---- end to end through the C ABI with host buffers (rank-local)
     e2e = run_e2e(b, stack, device, steps=min(args.steps, 2))
@@ -347,14 +336,13 @@ def run_ours(args, world, rank, local):
                      "peak_kind": peak_kind, "unit": "GB/s", "frac": round(dom_gbs / peak, 4),
                      "bytes_per_launch": dom_bytes_per_launch, "traffic": traffic},
         "kernels": kernels,
+        "other_kernels": other,
         "cpu_baseline": cpu,
         "e2e": e2e,
         "gpu_launches": launches,
         "clocks": clocks,
     }
-    if world > 1:
-        torch.distributed.barrier()
-        torch.distributed.destroy_process_group()
+    tdist.finish()
     if rank == 0:
         print(json.dumps(out))
 
@@ -378,6 +366,78 @@ def _ncu_traffic(kernel_label):
         if kv.get("label") == kernel_label and kv.get("src_sha") == src:
             return float(kv["dram_bytes_per_launch"])
     return None
+
+
+def _flush_l2(buf):
+    buf.add_(1)  # a write of 256 MiB evicts the 126 MB L2
+
+
+def _timed(fn, reps, flush):
+    """Average device time of fn over reps launches, L2 flushed before each."""
+    total = 0.0
+    for r in range(reps):
+        _flush_l2(flush)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record()
+        fn(r)
+        e1.record()
+        torch.cuda.synchronize()
+        total += e0.elapsed_time(e1)
+    return total / reps / 1e3
+
+
+def time_other_kernels(b, stack, device, peak, reps=10):
+    """Standalone hint emit (throughput stack, layer 24), SR transpose
+    re-quantize (128 x 512 x 2048 expert stack) and RHT32 + quantize
+    (16384 x 4096 activation with outliers): seconds per call and algorithmic
+    GB/s, L2 flushed before every call."""
+    from train_rollout_alignment_b200 import synthetic as syn
+    flush = torch.zeros(64 << 20, dtype=torch.float32, device=device)
+    out = {}
+    # hint emit from the codes of a hinted layer
+    l = stack.hint_from
+    h = torch.empty(stack.n * HINT_BITS // 8, dtype=torch.uint8, device=device)
+    t = _timed(lambda r: b.nvfp4_emit_hint(stack.cr[l], stack.n, HINT_BITS, h), reps, flush)
+    gbs = BYTES["emit_hint"] * stack.n / t / 1e9
+    out["emit_hint"] = {"workload": "%dx%d codes, 2-bit hints" % (ROWS, COLS), "avg_us": round(t * 1e6, 2),
+                        "GB/s": round(gbs, 1), "frac": round(gbs / peak, 4), "bytes_per_elem": BYTES["emit_hint"]}
+    # SR transpose: the expert stack quantized by the library's own RTN path
+    batch, er, ec = syn.CFG2_SHAPE
+    w = torch.from_numpy(syn.cfg2().view(np.int16)).view(torch.bfloat16).to(device)
+    ne = er * ec
+    codes = torch.empty(batch * ne // 2, dtype=torch.uint8, device=device)
+    scales = torch.empty(batch * ne // 16, dtype=torch.uint8, device=device)
+    ts = torch.empty(batch, dtype=torch.float32, device=device)
+    ws = torch.zeros(max(batch, 4), dtype=torch.int32, device=device)
+    for e in range(batch):
+        b.nvfp4_quantize_rtn(w[e], ws, codes[e * ne // 2:(e + 1) * ne // 2],
+                             scales[e * ne // 16:(e + 1) * ne // 16], ts[e:e + 1])
+    del w
+    ct, st, tst = torch.empty_like(codes), torch.empty_like(scales), torch.empty_like(ts)
+    t = _timed(lambda r: b.nvfp4_sr_transpose_requant(codes, scales, ts, batch, er, ec, syn.CFG2_SR_SEED, r,
+                                                      ws, ct, st, tst), reps, flush)
+    n = batch * ne
+    sr_bytes = 3 * (0.5 + 1 / 16)  # amax pre-pass reads codes+scales, main pass reads and writes them
+    out["sr_transpose_requant"] = {
+        "workload": "%dx%dx%d expert stack, one Philox4x32-10 word per element" % (batch, er, ec),
+        "avg_us": round(t * 1e6, 2), "GB/s": round(sr_bytes * n / t / 1e9, 1),
+        "frac": round(sr_bytes * n / t / 1e9 / peak, 4), "bytes_per_elem": sr_bytes,
+        "elements_per_s": round(n / t, 1)}
+    del codes, scales, ct, st
+    # RHT32 + quantize
+    x = torch.from_numpy(syn.cfg3().view(np.int16)).view(torch.bfloat16).to(device)
+    rr, cc = x.shape
+    c3 = torch.empty((rr, cc // 2), dtype=torch.uint8, device=device)
+    s3 = torch.empty((rr, cc // 16), dtype=torch.uint8, device=device)
+    t3 = torch.empty(1, dtype=torch.float32, device=device)
+    t = _timed(lambda r: b.nvfp4_rht_quantize(x, syn.CFG3_SIGN_SEED, ws, c3, s3, t3), reps, flush)
+    n = rr * cc
+    rht_bytes = 2 + 2 + 0.5 + 1 / 16
+    out["rht_quantize"] = {"workload": "%dx%d activation, 0.1%% outliers x100" % (rr, cc),
+                           "avg_us": round(t * 1e6, 2), "GB/s": round(rht_bytes * n / t / 1e9, 1),
+                           "frac": round(rht_bytes * n / t / 1e9 / peak, 4), "bytes_per_elem": rht_bytes}
+    return out
 
 
 def run_e2e(b, stack, device, steps):

@@ -40,8 +40,10 @@
  *
  * Conventions for every call:
  *   * Pointers are DEVICE pointers unless stated; the library never allocates,
- *     frees or keeps them.  Every pointer must be 16-byte aligned
- *     (NVFP4_ERR_MISALIGNED otherwise).
+ *     frees or keeps them.  Alignment (NVFP4_ERR_MISALIGNED otherwise): BF16
+ *     inputs and y_out 32 bytes (one 16-value block is one 256-bit load),
+ *     codes/scales/hints/ws 16 bytes, tensor scales 4, counters 8.  Any
+ *     row-offset view of a [rows, cols] tensor keeps these (cols % 16 == 0).
  *   * `stream` is a cudaStream_t (NULL = legacy default stream).  Calls are
  *     asynchronous on it; they return once the kernels are enqueued.
  *   * Arguments are validated before anything is enqueued: a call that returns
@@ -65,7 +67,7 @@ typedef int nvfp4_status;
 
 #define NVFP4_OK                0
 #define NVFP4_ERR_INVALID_ARG   1   /* null pointer, negative size, bad flag */
-#define NVFP4_ERR_MISALIGNED    2   /* a pointer is not 16-byte aligned */
+#define NVFP4_ERR_MISALIGNED    2   /* a pointer breaks its alignment rule (see above) */
 #define NVFP4_ERR_SHAPE         3   /* cols % 16 (RHT: % 32), rows % 16 (SR), size >= 2^40 */
 #define NVFP4_ERR_CUDA          4   /* a kernel launch failed */
 #define NVFP4_ERR_UNSUPPORTED   5   /* hint_bits not in {1, 2, 4} */
@@ -87,13 +89,13 @@ typedef int nvfp4_status;
 #define NVFP4_STAT_SUM_ABS_DELTA 4  /* sum of |pos_a - pos_b| */
 #define NVFP4_STAT_SCALE_MISMATCH 5 /* 16-blocks whose E4M3 scale bytes differ */
 #define NVFP4_STAT_VALUE_MISMATCH 6 /* decoded FP32 values differ (-0 == +0) */
-#define NVFP4_STATS8_WORDS       8  /* word 7 is reserved (written 0) */
+#define NVFP4_STATS8_WORDS       8  /* word 7 is reserved (left unchanged) */
 
 /* stats4 indices (nvfp4_guided_requant) */
 #define NVFP4_GSTAT_CONSULTED    0  /* off-grid and |v| < 6: the hint decided */
 #define NVFP4_GSTAT_CHANGED      1  /* guided code != round-to-nearest code */
 #define NVFP4_GSTAT_OUTSIDE      2  /* hint matched neither bracket end: RTN kept */
-#define NVFP4_STATS4_WORDS       4  /* word 3 is reserved (written 0) */
+#define NVFP4_STATS4_WORDS       4  /* word 3 is reserved (left unchanged) */
 
 /*
  * nvfp4_tensor_amax -- A = max |x| over n BF16 values.

@@ -137,12 +137,12 @@ def random_case(shape, seed: int, kind: str = "normal") -> np.ndarray:
 
 
 # --------------------------------------------------------------------------- device
-def cfg4_layer_device(layer: int, device, rank: int = 0):
+def cfg4_layer_device(layer: int, device, rank: int = 0, shape=CFG4_SHAPE):
     """48-layer throughput stack, one layer on the GPU: 65536x4096, N(0,1) times
     per-column scales c_j = exp(U(ln 0.1, ln 10)); seed 4, layer and rank mixed
-    into the generator seed.  Returns (train, rollout) as torch.bfloat16 on
-    ``device``."""
-    rows, cols = CFG4_SHAPE
+    into the generator seed (every rank of a multi-GPU run gets its own stack).
+    Returns (train, rollout) as torch.bfloat16 on ``device``."""
+    rows, cols = shape
     g = torch.Generator(device=device)
     g.manual_seed((4 << 40) | (rank << 20) | layer)
     c = torch.empty(cols, device=device, dtype=torch.float32)
