@@ -248,18 +248,21 @@ __device__ __forceinline__ void block_add_u64(const unsigned long long* vals,
 
 // ----------------------------------------------------------------- Philox4x32-10
 // Salmon, Moraes, Dror, Shaw, "Parallel random numbers: as easy as 1, 2, 3",
-// SC'11.  Returns output word x0 only.
+// SC'11.  Returns output word x0 only.  Each 32x32 -> 64-bit product is one
+// wide multiply; with the key schedule and the shared counter words hoisted by
+// the compiler, consecutive counters share the first round's second product.
 __device__ __forceinline__ uint32_t philox4x32_10_x0(uint32_t c0, uint32_t c1, uint32_t c2,
                                                      uint32_t c3, uint32_t k0, uint32_t k1) {
 #pragma unroll
   for (int r = 0; r < 10; ++r) {
-    const uint32_t hi0 = __umulhi(0xD2511F53u, c0), lo0 = 0xD2511F53u * c0;
-    const uint32_t hi1 = __umulhi(0xCD9E8D57u, c2), lo1 = 0xCD9E8D57u * c2;
-    const uint32_t n0 = hi1 ^ c1 ^ k0, n2 = hi0 ^ c3 ^ k1;
+    const uint64_t p0 = (uint64_t)0xD2511F53u * c0;
+    const uint64_t p1 = (uint64_t)0xCD9E8D57u * c2;
+    const uint32_t n0 = (uint32_t)(p1 >> 32) ^ c1 ^ k0;
+    const uint32_t n2 = (uint32_t)(p0 >> 32) ^ c3 ^ k1;
+    c1 = (uint32_t)p1;
+    c3 = (uint32_t)p0;
     c0 = n0;
-    c1 = lo1;
     c2 = n2;
-    c3 = lo0;
     k0 += 0x9E3779B9u;
     k1 += 0xBB67AE85u;
   }

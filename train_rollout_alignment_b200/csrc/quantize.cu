@@ -55,6 +55,14 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
   }
 }
 
+// Hint bits of one block (16 codes) from its 8 code bytes.
+template <int HB>
+__device__ __forceinline__ void hint_store(uint8_t* __restrict__ hints, int64_t blk, uint2 c) {
+  if (HB == 1) reinterpret_cast<uint16_t*>(hints)[blk] = (uint16_t)(compact1(c.x) | (compact1(c.y) << 8));
+  if (HB == 2) reinterpret_cast<uint32_t*>(hints)[blk] = compact2(c.x) | (compact2(c.y) << 16);
+  if (HB == 4) reinterpret_cast<uint2*>(hints)[blk] = c;
+}
+
 // ----------------------------------------------------------------- RTN quantize
 // Max |x| of a block as FP32 bits: packed 16-bit maxima of the BF16 magnitudes.
 __device__ __forceinline__ uint32_t block_amax_bits(const Block16& b) {
@@ -78,9 +86,7 @@ __device__ __forceinline__ void rtn_block(const Block16& b, float s_t, const Sca
   const uint2 c = pack_codes16(v);
   reinterpret_cast<uint2*>(codes)[blk] = c;
   scales[blk] = (uint8_t)bs.sb;
-  if (HB == 1) reinterpret_cast<uint16_t*>(hints)[blk] = (uint16_t)(compact1(c.x) | (compact1(c.y) << 8));
-  if (HB == 2) reinterpret_cast<uint32_t*>(hints)[blk] = compact2(c.x) | (compact2(c.y) << 16);
-  if (HB == 4) reinterpret_cast<uint2*>(hints)[blk] = c;
+  hint_store<HB>(hints, blk, c);
 }
 
 // Blocks are visited from the END of the tensor backwards: the amax pass that
@@ -263,30 +269,36 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 }
 
 // ----------------------------------------------------------------- emit hint
+// Two blocks (16 bytes of codes) per load, U loads in flight per thread; a
+// trailing odd block is done by thread 0.
+template <int HB>
+__device__ __forceinline__ void hint_store_pair(uint8_t* __restrict__ hints, int64_t pair, uint4 c) {
+  if (HB == 1)
+    reinterpret_cast<uint32_t*>(hints)[pair] =
+        compact1(c.x) | (compact1(c.y) << 8) | (compact1(c.z) << 16) | (compact1(c.w) << 24);
+  if (HB == 2)
+    reinterpret_cast<uint2*>(hints)[pair] =
+        make_uint2(compact2(c.x) | (compact2(c.y) << 16), compact2(c.z) | (compact2(c.w) << 16));
+  if (HB == 4) reinterpret_cast<uint4*>(hints)[pair] = c;
+}
+
 template <int HB, int U>
 __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     k_emit_hint(const uint8_t* __restrict__ codes, int64_t nblk, uint8_t* __restrict__ hints) {
+  const int64_t npair = nblk >> 1;
   const int64_t stride = (int64_t)gridDim.x * kThreads;
   int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x;
-  const uint2* __restrict__ c2 = reinterpret_cast<const uint2*>(codes);
-  for (; i + (U - 1) * stride < nblk; i += U * stride) {
-    uint2 c[U];
+  const uint4* __restrict__ c4 = reinterpret_cast<const uint4*>(codes);
+  for (; i + (U - 1) * stride < npair; i += U * stride) {
+    uint4 c[U];
 #pragma unroll
-    for (int u = 0; u < U; ++u) c[u] = __ldg(c2 + i + u * stride);
+    for (int u = 0; u < U; ++u) c[u] = __ldg(c4 + i + u * stride);
 #pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const int64_t blk = i + u * stride;
-      if (HB == 1) reinterpret_cast<uint16_t*>(hints)[blk] = (uint16_t)(compact1(c[u].x) | (compact1(c[u].y) << 8));
-      if (HB == 2) reinterpret_cast<uint32_t*>(hints)[blk] = compact2(c[u].x) | (compact2(c[u].y) << 16);
-      if (HB == 4) reinterpret_cast<uint2*>(hints)[blk] = c[u];
-    }
+    for (int u = 0; u < U; ++u) hint_store_pair<HB>(hints, i + u * stride, c[u]);
   }
-  for (; i < nblk; i += stride) {
-    const uint2 c = __ldg(c2 + i);
-    if (HB == 1) reinterpret_cast<uint16_t*>(hints)[i] = (uint16_t)(compact1(c.x) | (compact1(c.y) << 8));
-    if (HB == 2) reinterpret_cast<uint32_t*>(hints)[i] = compact2(c.x) | (compact2(c.y) << 16);
-    if (HB == 4) reinterpret_cast<uint2*>(hints)[i] = c;
-  }
+  for (; i < npair; i += stride) hint_store_pair<HB>(hints, i, __ldg(c4 + i));
+  if ((nblk & 1) && blockIdx.x == 0 && threadIdx.x == 0)
+    hint_store<HB>(hints, nblk - 1, __ldg(reinterpret_cast<const uint2*>(codes) + nblk - 1));
 }
 
 __global__ void k_set_f32(float* dst, float value) { *dst = value; }

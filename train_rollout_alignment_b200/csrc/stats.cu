@@ -29,7 +29,7 @@
 namespace nvfp4 {
 
 constexpr int kStatsCtasPerSm = 4;
-constexpr int kStatsUnroll = 4;
+constexpr int kStatsUnroll = 2;  // two pairs (four blocks) in flight per lane
 constexpr int kWarps = kThreads / 32;
 constexpr int kQueue = 64;  // dirty-block slots per warp (at most 31 + 32 are ever held)
 
@@ -102,8 +102,10 @@ __device__ __forceinline__ uint32_t value_mismatch_slow(uint2 a, uint2 b, float 
 struct StatsShared {
   uint4 queue[kWarps][kQueue];
   uint8_t queue_same[kWarps][kQueue];  // value counter follows positions
-  uint8_t normal_a[128], normal_b[128];
-  uint8_t ratio_far[256];              // [sig_a * 16 + sig_b]: only zero pairs can be equal
+  // per scale byte: 16 * significand (side a) / significand (side b) when every
+  // nonzero decoded value of such a block is a normal float, else 0x100
+  uint16_t key_a[128], key_b[128];
+  uint8_t ratio_far[256];  // [key_a + key_b]: only zero/zero pairs can be equal
   unsigned long long red[6 * 8];
 };
 
@@ -127,6 +129,45 @@ __device__ __forceinline__ int flush_queue(StatsShared& sm, int warp, int lane, 
   return rest;
 }
 
+// Elements of a word whose magnitudes are not both zero (bit 3 per nibble:
+// a nibble value in 0..7 plus 7 sets bit 3 iff it is nonzero).
+__device__ __forceinline__ uint32_t not_both_zero(uint32_t wa, uint32_t wb) {
+  return __popc((((wa | wb) & 0x77777777u) + 0x77777777u) & 0x88888888u);
+}
+
+// One block of the stream: queue it if its codes differ; count its scale and
+// (unless positions decide it) its decoded-value mismatches.
+__device__ __forceinline__ void count_block(StatsShared& sm, uint32_t ax, uint32_t ay, uint32_t bx,
+                                            uint32_t by, uint32_t sa, uint32_t sb, bool valid,
+                                            bool same_ts, float tsa, float tsb, int warp, int lane,
+                                            uint32_t lt_mask, int& qn, MismatchCounts& c) {
+  sa &= 0x7Fu;
+  sb &= 0x7Fu;
+  const uint32_t ka = sm.key_a[sa], kb = sm.key_b[sb];
+  const bool same = same_ts && sa == sb && ka < 0x100u;
+  const bool dirty = ((ax ^ bx) | (ay ^ by)) != 0u;
+  const uint32_t m = __ballot_sync(0xFFFFFFFFu, dirty);
+  if (dirty) {
+    const int slot = qn + __popc(m & lt_mask);
+    sm.queue[warp][slot] = make_uint4(ax, ay, bx, by);
+    sm.queue_same[warp][slot] = same;
+  }
+  qn += __popc(m);
+  if (qn >= 32) qn = flush_queue(sm, warp, lane, qn, 32, c);
+  if (valid) {
+    c.scale += (sa != sb) ? 1u : 0u;
+    if (!same) {
+      const uint32_t k = ka + kb;
+      if (k < 0x100u && sm.ratio_far[k]) {
+        c.value += not_both_zero(ax, bx) + not_both_zero(ay, by);  // only zero pairs are equal
+      } else {
+        c.value += value_mismatch_slow(make_uint2(ax, ay), make_uint2(bx, by), e4m3_value(sa),
+                                       e4m3_value(sb), tsa, tsb);
+      }
+    }
+  }
+}
+
 template <int U>
 __global__ void __launch_bounds__(kThreads, kStatsCtasPerSm)
     k_mismatch_stats(const uint8_t* __restrict__ ca, const uint8_t* __restrict__ sa,
@@ -138,10 +179,12 @@ __global__ void __launch_bounds__(kThreads, kStatsCtasPerSm)
   const bool same_ts = __float_as_uint(tsa) == __float_as_uint(tsb);
   const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
   if (t < 128) {
-    const float xa = __fmul_rn(e4m3_value(t), tsa), xb = __fmul_rn(e4m3_value(t), tsb);
+    const float sv = e4m3_value(t);
+    const float xa = __fmul_rn(sv, tsa), xb = __fmul_rn(sv, tsb);
     // every nonzero decoded value of the block is a normal float
-    sm.normal_a[t] = xa >= 0x1p-124f && xa <= 0x1p120f;
-    sm.normal_b[t] = xb >= 0x1p-124f && xb <= 0x1p120f;
+    const uint32_t sig = e4m3_significand(t);
+    sm.key_a[t] = (xa >= 0x1p-124f && xa <= 0x1p120f) ? (uint16_t)(sig << 4) : (uint16_t)0x100;
+    sm.key_b[t] = (xb >= 0x1p-124f && xb <= 0x1p120f) ? (uint16_t)sig : (uint16_t)0x100;
   }
   {
     // significand of (sb_a * s_t_a) / (sb_b * s_t_b) for scale significands
@@ -157,55 +200,52 @@ __global__ void __launch_bounds__(kThreads, kStatsCtasPerSm)
   __syncthreads();
 
   MismatchCounts c{0u, 0u, 0u, 0u, 0u};
-  const uint2* __restrict__ a2 = reinterpret_cast<const uint2*>(ca);
-  const uint2* __restrict__ b2 = reinterpret_cast<const uint2*>(cb);
+  const uint4* __restrict__ a4 = reinterpret_cast<const uint4*>(ca);
+  const uint4* __restrict__ b4 = reinterpret_cast<const uint4*>(cb);
+  const uint16_t* __restrict__ sa2 = reinterpret_cast<const uint16_t*>(sa);
+  const uint16_t* __restrict__ sb2 = reinterpret_cast<const uint16_t*>(sb);
   const uint32_t lt_mask = (1u << lane) - 1u;
-  const int64_t wstride = (int64_t)gridDim.x * kThreads;  // blocks per grid-wide step
-  int qn = 0;                                             // warp-uniform queue length
-  for (int64_t wb = (int64_t)blockIdx.x * kThreads + warp * 32; wb < nblk; wb += U * wstride) {
-    uint2 va[U], vb[U];
+  const int64_t npair = nblk >> 1;                       // two blocks per lane per load
+  const int64_t wstride = (int64_t)gridDim.x * kThreads;
+  int qn = 0;                                            // warp-uniform queue length
+  for (int64_t wb = (int64_t)blockIdx.x * kThreads + warp * 32; wb < npair; wb += U * wstride) {
+    uint4 va[U], vb[U];
     uint32_t xa[U], xb[U];
 #pragma unroll
     for (int u = 0; u < U; ++u) {
-      const int64_t i = wb + u * wstride + lane;
-      if (i < nblk) {
-        va[u] = __ldg(a2 + i);
-        vb[u] = __ldg(b2 + i);
-        xa[u] = __ldg(sa + i);
-        xb[u] = __ldg(sb + i);
+      const int64_t p = wb + u * wstride + lane;
+      if (p < npair) {
+        va[u] = __ldg(a4 + p);
+        vb[u] = __ldg(b4 + p);
+        xa[u] = __ldg(sa2 + p);
+        xb[u] = __ldg(sb2 + p);
       } else {
-        va[u] = vb[u] = make_uint2(0u, 0u);
+        va[u] = vb[u] = make_uint4(0u, 0u, 0u, 0u);
         xa[u] = xb[u] = 0u;
       }
     }
 #pragma unroll
     for (int u = 0; u < U; ++u) {
-      const bool valid = wb + u * wstride + lane < nblk;
-      const uint2 a = va[u], b = vb[u];
-      const bool same = same_ts && xa[u] == xb[u] && sm.normal_a[xa[u] & 0x7Fu];
-      const bool dirty = ((a.x ^ b.x) | (a.y ^ b.y)) != 0u;
-      const uint32_t m = __ballot_sync(0xFFFFFFFFu, dirty);
-      if (dirty) {
-        const int slot = qn + __popc(m & lt_mask);
-        sm.queue[warp][slot] = make_uint4(a.x, a.y, b.x, b.y);
-        sm.queue_same[warp][slot] = same;
+      const bool valid = wb + u * wstride + lane < npair;
+      count_block(sm, va[u].x, va[u].y, vb[u].x, vb[u].y, xa[u] & 0xFFu, xb[u] & 0xFFu, valid,
+                  same_ts, tsa, tsb, warp, lane, lt_mask, qn, c);
+      count_block(sm, va[u].z, va[u].w, vb[u].z, vb[u].w, xa[u] >> 8, xb[u] >> 8, valid, same_ts,
+                  tsa, tsb, warp, lane, lt_mask, qn, c);
+    }
+  }
+  if (nblk & 1) {  // a trailing odd block: warp 0 of CTA 0, lane 0
+    if (blockIdx.x == 0 && warp == 0) {
+      const int64_t i = nblk - 1;
+      uint2 a = make_uint2(0u, 0u), b = make_uint2(0u, 0u);
+      uint32_t x = 0u, y = 0u;
+      if (lane == 0) {
+        a = __ldg(reinterpret_cast<const uint2*>(ca) + i);
+        b = __ldg(reinterpret_cast<const uint2*>(cb) + i);
+        x = __ldg(sa + i);
+        y = __ldg(sb + i);
       }
-      qn += __popc(m);
-      if (qn >= 32) qn = flush_queue(sm, warp, lane, qn, 32, c);
-      if (valid) {
-        c.scale += (xa[u] != xb[u]) ? 1u : 0u;
-        if (!same) {
-          const uint32_t ia = xa[u] & 0x7Fu, ib = xb[u] & 0x7Fu;
-          if (sm.normal_a[ia] && sm.normal_b[ib] &&
-              sm.ratio_far[e4m3_significand(ia) * 16u + e4m3_significand(ib)]) {
-            // only zero/zero pairs are equal
-            c.value += count_nib(nib_nonzero((a.x | b.x) & 0x77777777u)) +
-                       count_nib(nib_nonzero((a.y | b.y) & 0x77777777u));
-          } else {
-            c.value += value_mismatch_slow(a, b, e4m3_value(xa[u]), e4m3_value(xb[u]), tsa, tsb);
-          }
-        }
-      }
+      count_block(sm, a.x, a.y, b.x, b.y, x, y, lane == 0, same_ts, tsa, tsb, warp, lane, lt_mask,
+                  qn, c);
     }
   }
   if (qn > 0) flush_queue(sm, warp, lane, qn, qn, c);
