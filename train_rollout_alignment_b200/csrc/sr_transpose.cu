@@ -7,42 +7,27 @@
 // Two kernels:
 //   1. k_sr_amax: per matrix, max over blocks of G[max m] * sb (exact in FP32);
 //      A' = that max times s_t (one rounding, which commutes with the max).
-//   2. k_sr_transpose: one CTA per 64x64 tile of a matrix.  The tile's codes
-//      (2 KiB) and scales (256 B) are staged in shared memory; thread t owns
-//      output block (column c = t/4, rows 16*(t%4)..+15), dequantizes its 16
-//      values, derives the new block scale, draws one Philox4x32-10 word per
-//      element (counter = output element index, draw) and writes 8 code bytes
-//      and one scale byte; the four threads of a column write 32 contiguous
-//      bytes.  Integer-ALU bound (10 Philox rounds per element).
+//   2. k_sr_transpose: one CTA per 64x64 tile of a matrix.  Each thread
+//      dequantizes one source block (16 values, one scale decode) into a
+//      padded FP32 tile in shared memory; then warp w takes 16 rows of 32
+//      consecutive columns (conflict-free column reads), derives the new block
+//      scale, draws one Philox4x32-10 word per element (counter = output
+//      element index, draw) and writes 8 code bytes and one scale byte.
+//      The lower grid point comes from the truncating E2M1 conversion; the
+//      round-up test is one exact product comparison.  Integer-ALU bound
+//      (10 Philox rounds per element).
 #include "launch.h"
 #include "nvfp4_device.cuh"
 
 namespace nvfp4 {
 
 constexpr int kTile = 64;
+constexpr int kYStride = kTile + 1;  // padded FP32 row of the staged tile
 
 __device__ __forceinline__ float grid_value(uint32_t m) {
   float lo, hi;
   e2m1x2_decode(m & 7u, lo, hi);
   return lo;
-}
-
-// Stochastic rounding of a = |v| with the 32-bit word r: on-grid values stay,
-// a >= 6 gives 6, otherwise round up iff (r >> 8) < p * 2^24 with
-// p = (a - G[lo]) / (G[hi] - G[lo]); both products are exact in FP32.
-__device__ __forceinline__ uint32_t sr_magnitude(float a, uint32_t r) {
-  if (a >= 6.0f) return 7u;
-  if (a != a) return 0u;
-  const uint32_t m = e2m1x2(a, 0.0f) & 7u;          // nearest grid index
-  const uint32_t lo = (grid_value(m) > a) ? m - 1u : m;
-  float glo, ghi;
-  e2m1x2_decode(lo | ((lo + 1u) << 4), glo, ghi);
-  if (glo == a) return lo;
-  const float w = __fsub_rn(ghi, glo);               // 0.5, 1 or 2
-  const float inv_w = (w == 0.5f) ? 2.0f : ((w == 1.0f) ? 1.0f : 0.5f);
-  const float p = __fmul_rn(__fsub_rn(a, glo), inv_w);
-  const float thr = __fmul_rn(p, 16777216.0f);
-  return (__uint2float_rn(r >> 8) < thr) ? lo + 1u : lo;
 }
 
 __global__ void __launch_bounds__(kThreads)
@@ -67,65 +52,107 @@ __global__ void __launch_bounds__(kThreads)
   if (threadIdx.x == 0 && best) atomicMax(ws + e, best);
 }
 
+// Stochastic rounding of 8 values: a = |v| clamped to 6.  Z: their codes
+// truncated toward zero (the lower grid point lo; 7 for a = 6).  With
+// glo = G[lo], w = G[lo + 1] - G[lo] and d = a - glo (all exact), round up
+// iff (r >> 8) < (d / w) * 2^24, evaluated as (r >> 8) * w < d * 2^24 (both
+// products exact).  On the grid d = 0 and nothing moves; at 6, w is taken as
+// |G[8 as a code] - 6| = 6 > 0 so nothing moves either.  Returns the 8 codes
+// (magnitudes) with the round-up applied.
+__device__ __forceinline__ uint32_t sr_word(const float* a, const uint32_t* r, uint32_t Z) {
+  const uint32_t Zh = Z + 0x11111111u;  // codes of the upper grid points
+  uint32_t up = 0u;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    float glo[2], ghi[2];
+    e2m1x2_decode((Z >> (8 * j)) & 0xFFu, glo[0], glo[1]);
+    e2m1x2_decode((Zh >> (8 * j)) & 0xFFu, ghi[0], ghi[1]);
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+      const int k = 2 * j + t;
+      const float w = fabsf(__fsub_rn(ghi[t], glo[t]));
+      const float d = __fsub_rn(a[k], glo[t]);
+      const bool rnd = __fmul_rn(__uint2float_rn(r[k] >> 8), w) < __fmul_rn(d, 16777216.0f);
+      up |= (rnd ? 1u : 0u) << (4 * k);
+    }
+  }
+  return Z + up;
+}
+
 __global__ void __launch_bounds__(kThreads)
     k_sr_transpose(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ scales,
                    const float* __restrict__ ts, int64_t rows, int64_t cols, uint32_t seed_lo,
                    uint32_t seed_hi, uint32_t draw, const uint32_t* __restrict__ ws,
                    uint8_t* __restrict__ codes_t, uint8_t* __restrict__ scales_t,
                    float* __restrict__ ts_t) {
-  __shared__ __align__(16) uint8_t cs[kTile][kTile / 2];
-  __shared__ uint8_t ss[kTile][kTile / 16];
+  __shared__ float ys[kTile][kYStride];
   const int64_t e = blockIdx.z;
   const int64_t r0 = (int64_t)blockIdx.y * kTile, c0 = (int64_t)blockIdx.x * kTile;
   const int t = threadIdx.x;
+  const float s_in = __ldg(ts + e);
   {
+    // dequantize: thread t takes 16 values (one source block) of tile row t / 4
     const int row = t >> 2, chunk = t & 3;
     const int64_t r = r0 + row, c = c0 + chunk * 16;
-    uint2 v = make_uint2(0u, 0u);
-    uint8_t sv = 0;
+    float y[16];
+#pragma unroll
+    for (int k = 0; k < 16; ++k) y[k] = 0.0f;
     if (r < rows && c < cols) {
       const int64_t base = e * rows + r;
-      v = __ldg(reinterpret_cast<const uint2*>(codes + base * (cols / 2) + c / 2));
-      sv = __ldg(scales + base * (cols / 16) + c / 16);
+      const uint2 v = __ldg(reinterpret_cast<const uint2*>(codes + base * (cols / 2) + c / 2));
+      const float sbv = e4m3_value(__ldg(scales + base * (cols / 16) + c / 16));
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        float g0, g1;
+        e2m1x2_decode(((j < 4 ? v.x : v.y) >> (8 * (j & 3))) & 0xFFu, g0, g1);
+        y[2 * j] = __fmul_rn(__fmul_rn(g0, sbv), s_in);  // (G[m] * sb) exact, then * s_t
+        y[2 * j + 1] = __fmul_rn(__fmul_rn(g1, sbv), s_in);
+      }
     }
-    *reinterpret_cast<uint2*>(&cs[row][chunk * 8]) = v;
-    ss[row][chunk] = sv;
+#pragma unroll
+    for (int k = 0; k < 16; ++k) ys[row][chunk * 16 + k] = y[k];
   }
   __syncthreads();
 
-  const float s_in = __ldg(ts + e);
   const float A = __fmul_rn(__uint_as_float(ws[e]), s_in);
   const float s_t = tensor_scale_from_amax(A);
   if (blockIdx.x == 0 && blockIdx.y == 0 && t == 0) ts_t[e] = s_t;
 
-  const int cl = t >> 2, rb = t & 3;
+  // warp w: 16 rows (16 * (w % 4)) of 32 consecutive columns (32 * (w / 4))
+  const int warp = t >> 5, lane = t & 31;
+  const int rb = warp & 3, cl = (warp >> 2) * 32 + lane;
   const int64_t c = c0 + cl, rbase = r0 + rb * 16;
   if (c >= cols || rbase >= rows) return;
   float y[16];
   float amax = 0.0f;
 #pragma unroll
   for (int k = 0; k < 16; ++k) {
-    const int rl = rb * 16 + k;
-    const uint32_t nib = (cs[rl][cl >> 1] >> (4 * (cl & 1))) & 0xFu;
-    float g, unused;
-    e2m1x2_decode(nib, g, unused);
-    y[k] = __fmul_rn(__fmul_rn(g, e4m3_value(ss[rl][cl >> 4])), s_in);
+    y[k] = ys[rb * 16 + k][cl];
     amax = fmaxf(amax, fabsf(y[k]));
   }
   const BlockScale bs = block_scale(amax, s_t);
   const uint64_t obase = ((uint64_t)e * (uint64_t)cols + (uint64_t)c) * (uint64_t)rows + (uint64_t)rbase;
-  uint32_t out[2] = {0u, 0u};
+  const uint32_t ctr_hi = (uint32_t)(obase >> 32);  // obase % 16 == 0: the 16 counters share it
+  float a[16];
+  uint32_t r[16];
 #pragma unroll
   for (int k = 0; k < 16; ++k) {
-    const float v = __fmul_rn(y[k], bs.inv);
-    uint32_t m = 0u;
-    if (bs.inv != 0.0f) {
-      const uint64_t i = obase + (uint64_t)k;
-      const uint32_t r = philox4x32_10_x0((uint32_t)i, (uint32_t)(i >> 32), draw, 0u, seed_lo, seed_hi);
-      m = sr_magnitude(fabsf(v), r);
-    }
-    const uint32_t sgn = __float_as_uint(y[k]) >> 31;
-    out[k >> 3] |= ((sgn << 3) | m) << (4 * (k & 7));
+    a[k] = fminf(fabsf(__fmul_rn(y[k], bs.inv)), kE2M1Max);
+    r[k] = philox4x32_10_x0((uint32_t)obase + (uint32_t)k, ctr_hi, draw, 0u, seed_lo, seed_hi);
+  }
+  uint32_t out[2];
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const float* ah = a + 8 * h;
+    const uint32_t Z = e2m1x4_rz(ah[0], ah[1], ah[2], ah[3]) + (e2m1x4_rz(ah[4], ah[5], ah[6], ah[7]) << 16);
+    uint32_t S = 0u;  // signs of y
+#pragma unroll
+    for (int k = 0; k < 8; ++k) S |= (__float_as_uint(y[8 * h + k]) >> 31) << (4 * k + 3);
+    out[h] = sr_word(ah, r + 8 * h, Z) | S;
+  }
+  if (bs.inv == 0.0f) {  // zero block scale: every code is +-0
+    out[0] &= 0x88888888u;
+    out[1] &= 0x88888888u;
   }
   *reinterpret_cast<uint2*>(codes_t + obase / 2) = make_uint2(out[0], out[1]);
   scales_t[obase / 16] = (uint8_t)bs.sb;
