@@ -35,7 +35,10 @@
  *   x       [rows, cols]        BF16 bit patterns (uint16), cols % 16 == 0
  *   codes   [rows, cols/2]      bytes; element 2j in the low nibble of byte j
  *   scales  [rows, cols/16]     E4M3 bytes, block b covers elements 16b..16b+15
- *   hints   ceil(n*bits/8)      element i at byte (i*bits)>>3, bit (i*bits)&7
+ *   hints   n*bits/8 bytes      read LSB first.  bits 4: element i at bit 4i.
+ *                               bits 1, 2: block b (elements 16b..16b+15) owns
+ *                               bits 16*bits*b ..; its element k takes field
+ *                               2*(k%8) + k/8 (fields of k and k+8 adjacent)
  *   ws      NVFP4_WS_WORDS uint32 words of device scratch (see below)
  *
  * Conventions for every call:

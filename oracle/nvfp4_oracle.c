@@ -185,8 +185,25 @@ static float* bf16_rows_to_f32(const uint16_t* x, int64_t n)
 
 /* Step 4: compact hint ([TRACE], compaction paragraph).  bits 1 -> m & 1
  * (the E2M1 mantissa bit, enough to tell two adjacent cells apart), 2 ->
- * m & 3, 4 -> the whole code (the uncompacted guidance).  Element i occupies
- * bits (i*bits) .. (i*bits + bits - 1) of the byte stream, LSB first. */
+ * m & 3, 4 -> the whole code (the uncompacted guidance).
+ *
+ * Layout (the page fixes only that a few low bits are sent, not their order):
+ * the hint stream is read LSB first, byte by byte.  With 4 bits, element i
+ * takes bits 4i .. 4i+3, like the codes.  With 1 or 2 bits, each 16-element
+ * block owns 16*bits consecutive bits, and inside the block element k takes
+ * field 2*(k mod 8) + (k div 8): the fields of elements k and k + 8 sit next
+ * to each other.  (A reader holding the block's codes as two words of 8
+ * nibbles then finds the hint of nibble k of either word at bit 4k of one
+ * 32-bit word, shifted by 0 or 2, or at bit 2k of a 16-bit word, shifted by 0
+ * or 1.) */
+static int64_t hint_pos(int64_t i, int bits)
+{
+    if (bits == 4) return i * 4;
+    int64_t blk = i / 16;
+    int k = (int)(i % 16);
+    return blk * 16 * bits + (int64_t)bits * (2 * (k % 8) + k / 8);
+}
+
 void oracle_emit_hint(const uint8_t* codes, int64_t n, int bits, uint8_t* hints)
 {
     int64_t nbytes = (n * bits + 7) / 8;
@@ -194,14 +211,14 @@ void oracle_emit_hint(const uint8_t* codes, int64_t n, int bits, uint8_t* hints)
     for (int64_t i = 0; i < n; ++i) {
         int code = nibble_get(codes, i);
         int h = (bits == 4) ? code : ((code & 7) & ((1 << bits) - 1));
-        int64_t pos = i * bits;
+        int64_t pos = hint_pos(i, bits);
         hints[pos >> 3] |= (uint8_t)(h << (pos & 7));
     }
 }
 
 static int hint_get(const uint8_t* hints, int64_t i, int bits)
 {
-    int64_t pos = i * bits;
+    int64_t pos = hint_pos(i, bits);
     return (hints[pos >> 3] >> (pos & 7)) & ((1 << bits) - 1);
 }
 

@@ -9,7 +9,7 @@ What pins what (none of these re-types the oracle's FP32 chain):
   tensor gives s_t = 1 and zero scales;
 * TRACE explainer, rounding-analogy / prescription paragraphs: the 2.49 / 2.51
   example;
-* hints: unpacking with numpy's unpackbits;
+* hints: unpacking with numpy's unpackbits and the stated field order;
 * guided rounding: guiding a tensor by its own hints changes nothing; the
   distance guarantee of the prescription paragraph (never further from the
   rollout than round-to-nearest) for full codes everywhere, for 2-bit hints
@@ -136,6 +136,10 @@ def test_hint_pack_round_trip(bits):
     fields = np.unpackbits(h, bitorder="little")[: n * bits].reshape(n, bits)
     vals = (fields * (1 << np.arange(bits))).sum(1)
     want = c if bits == 4 else (c & 7) & ((1 << bits) - 1)
+    if bits != 4:
+        # inside each 16-element block, field f holds element (f >> 1) + 8 * (f & 1)
+        order = np.array([(f >> 1) + 8 * (f & 1) for f in range(16)])
+        want = want.reshape(-1, 16)[:, order].reshape(-1)
     assert np.array_equal(vals, want)
 
 

@@ -158,32 +158,62 @@ __device__ __forceinline__ BlockScale block_scale_bf16(uint32_t amax_bits, float
   return r;
 }
 
+// 8 FP32 values -> 8 round-to-nearest codes, v[0] in bits 0..3.  The four
+// conversion bytes are joined by one vector move (no shifts or masks).
+__device__ __forceinline__ uint32_t pack_rn8(const float* v) {
+  uint32_t r;
+  asm("{\n\t.reg .b8 t0, t1, t2, t3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 t0, %2, %1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 t1, %4, %3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 t2, %6, %5;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 t3, %8, %7;\n\t"
+      "mov.b32 %0, {t0, t1, t2, t3};\n\t}"
+      : "=r"(r)
+      : "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7]));
+  return r;
+}
+
+// 8 FP32 values -> 8 codes rounded toward zero (sign kept), v[0] in bits
+// 0..3; see e2m1x4_rz.  NaN inputs give code 7 (magnitude 6).
+__device__ __forceinline__ uint32_t pack_rz8(const float* v) {
+  uint32_t r;
+  asm("{\n\t.reg .b16 l, h;\n\t"
+      "cvt.rs.satfinite.e2m1x4.f32 l, {%4, %3, %2, %1}, %9;\n\t"
+      "cvt.rs.satfinite.e2m1x4.f32 h, {%8, %7, %6, %5}, %9;\n\t"
+      "mov.b32 %0, {l, h};\n\t}"
+      : "=r"(r)
+      : "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7]),
+        "r"(0u));
+  return r;
+}
+
 // 16 FP32 values (already multiplied by inv) -> 8 bytes of packed codes.
 __device__ __forceinline__ uint2 pack_codes16(const float* v) {
-  uint2 c;
-  c.x = e2m1x2(v[0], v[1]) | (e2m1x2(v[2], v[3]) << 8) | (e2m1x2(v[4], v[5]) << 16) |
-        (e2m1x2(v[6], v[7]) << 24);
-  c.y = e2m1x2(v[8], v[9]) | (e2m1x2(v[10], v[11]) << 8) | (e2m1x2(v[12], v[13]) << 16) |
-        (e2m1x2(v[14], v[15]) << 24);
-  return c;
+  return make_uint2(pack_rn8(v), pack_rn8(v + 8));
 }
 
 // ----------------------------------------------------------------- hints
-// Compact the low `bits` bits of each of the 8 nibbles of `w` (magnitude bits
-// only for 1 and 2) into 8*bits contiguous bits, element 0 first.
-__device__ __forceinline__ uint32_t compact2(uint32_t w) {  // 8 nibbles -> 16 bits
-  uint32_t y = w & 0x33333333u;
+// Hint field of one block from its codes (c.x: elements 0..7, c.y: 8..15).
+// 1 and 2 bits keep the low magnitude bits, and the fields of elements k and
+// k + 8 are adjacent: field 2*(k%8) + k/8 of the block.
+//   2 bits: nibble k of the 32-bit result = (m_{k+8} & 3) << 2 | (m_k & 3)
+//   1 bit:  bits 2k, 2k+1 of the 16-bit result = m_k & 1, m_{k+8} & 1
+__device__ __forceinline__ uint32_t hint_field2(uint2 c) {
+  return (c.x & 0x33333333u) | ((c.y << 2) & 0xCCCCCCCCu);
+}
+__device__ __forceinline__ uint32_t hint_field1(uint2 c) {
+  uint32_t y = (c.x & 0x11111111u) | ((c.y << 1) & 0x22222222u);  // 2 bits per nibble
   y = (y | (y >> 2)) & 0x0F0F0F0Fu;
   y = (y | (y >> 4)) & 0x00FF00FFu;
-  y = (y | (y >> 8)) & 0x0000FFFFu;
-  return y;
+  return (y | (y >> 8)) & 0x0000FFFFu;
 }
-__device__ __forceinline__ uint32_t compact1(uint32_t w) {  // 8 nibbles -> 8 bits
-  uint32_t y = w & 0x11111111u;
-  y = (y | (y >> 3)) & 0x03030303u;
-  y = (y | (y >> 6)) & 0x000F000Fu;
-  y = (y | (y >> 12)) & 0x000000FFu;
-  return y;
+// Inverse spreading for 1-bit hints: the 16-bit field -> bits 0 (element k)
+// and 1 (element k + 8) of nibble k.
+__device__ __forceinline__ uint32_t hint_spread1(uint32_t h16) {
+  uint32_t y = h16 & 0xFFFFu;
+  y = (y | (y << 8)) & 0x00FF00FFu;
+  y = (y | (y << 4)) & 0x0F0F0F0Fu;
+  return (y | (y << 2)) & 0x33333333u;
 }
 
 // ----------------------------------------------------------------- nibble masks

@@ -58,8 +58,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 // Hint bits of one block (16 codes) from its 8 code bytes.
 template <int HB>
 __device__ __forceinline__ void hint_store(uint8_t* __restrict__ hints, int64_t blk, uint2 c) {
-  if (HB == 1) reinterpret_cast<uint16_t*>(hints)[blk] = (uint16_t)(compact1(c.x) | (compact1(c.y) << 8));
-  if (HB == 2) reinterpret_cast<uint32_t*>(hints)[blk] = compact2(c.x) | (compact2(c.y) << 16);
+  if (HB == 1) reinterpret_cast<uint16_t*>(hints)[blk] = (uint16_t)hint_field1(c);
+  if (HB == 2) reinterpret_cast<uint32_t*>(hints)[blk] = hint_field2(c);
   if (HB == 4) reinterpret_cast<uint2*>(hints)[blk] = c;
 }
 
@@ -115,19 +115,57 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 }
 
 // ----------------------------------------------------------------- guided
-// Per element, with a = |v| and m the round-to-nearest magnitude index:
-//   a > G[m]  -> v lies in (G[m], G[m+1]): bracket (lo, hi) = (m, m+1)
-//   a < G[m]  -> bracket (m-1, m)
-//   a == G[m] -> on the grid, no decision;  m == 7 and a > 6 -> saturated.
-// The "other" end of the bracket replaces m when the hint names it.
+// Per element, with v = x * inv, a = |v| and m the round-to-nearest magnitude:
+//   a off the grid and below 6 -> it lies in (G[lo], G[lo+1]) with lo the
+//       floor index, and m is lo or lo + 1;  the other end of that bracket
+//       replaces m when the hint names it;
+//   a on the grid (zero included) or above 6 -> no decision, m stays.
 // HB = 1, 2: magnitude bits modulo 2^HB.  HB = 4: signed grid positions.
-//
-// Only the up/down flags need per-element work (an exact FP32 comparison
-// of a with the decoded G[m], done on the bit patterns, which order like the
-// values for a >= 0).  Everything else runs on 8 packed nibbles at a time.
+// Everything runs on packed words of 8 nibbles:
+//   R  = round-to-nearest codes of v (hardware conversion, sign of x);
+//   Zs = codes of v rounded toward zero: the floor index lo with the sign;
+//   P  = the same for v moved one ulp toward zero (its bit pattern minus 1).
+//        Off the grid that cannot cross a grid point, so P == Zs; on a grid
+//        point the magnitude drops one cell; v = +-0 turns into a NaN pattern,
+//        which converts to magnitude 7.  So P != Zs (in magnitude) marks "no
+//        decision" exactly where a is on the grid.
+// Off the grid the other bracket end is O = 2 * lo + 1 - m; a > 6 gives
+// lo = m = 7 and O = 8, which also means no decision.  Per-element flags live
+// in bit 3 of each nibble: a nibble value in 0..8 is nonzero exactly when
+// adding 7 sets its bit 3 (no carry leaves the nibble).
 struct GuidedCounts {
-  unsigned long long consulted, changed, outside;
+  uint32_t consulted, changed, outside;  // per thread: at most 16 per block visited
 };
+
+// hword: for HB = 1, 2 the hint fields of these 8 elements in the low bits of
+// each nibble (higher nibble bits are ignored); for HB = 4 their full codes.
+template <int HB>
+__device__ __forceinline__ uint32_t guided_select(uint32_t R, uint32_t Zm, uint32_t pz,
+                                                  uint32_t hword, GuidedCounts& cnt) {
+  constexpr uint32_t kB3 = 0x88888888u, kSeven = 0x77777777u;
+  const uint32_t M = R & kSeven;  // round-to-nearest magnitudes
+  const uint32_t S = R & kB3;     // signs (of x)
+  const uint32_t O = (Zm << 1) + 0x11111111u - M;
+  const uint32_t off = ~((pz + kSeven) | O) & kB3;  // a rounding decision exists
+  uint32_t take, differs;  // differs: the hint does not name the round-to-nearest cell
+  if (HB == 4) {
+    // signed positions: equal codes, or both magnitudes zero
+    const auto nz4 = [](uint32_t t) { return (((t & kSeven) + kSeven) | t) & kB3; };
+    const uint32_t zh = ~((hword & kSeven) + kSeven);
+    take = ~nz4(hword ^ (O | S)) | (~(O + kSeven) & zh);
+    differs = nz4(hword ^ R) & ((M + kSeven) | ~zh);
+  } else {
+    const uint32_t mask = HB == 1 ? 0x11111111u : 0x33333333u;
+    take = ~(((hword ^ O) & mask) + kSeven);
+    differs = ((hword ^ M) & mask) + kSeven;
+  }
+  take &= off;
+  cnt.consulted += __popc(off);
+  cnt.changed += __popc(take);
+  cnt.outside += __popc(off & ~take & differs);
+  const uint32_t T = (take >> 3) * 0xFu;  // whole-nibble select mask
+  return ((O & T) | (M & ~T)) | S;
+}
 
 template <int HB>
 __device__ __forceinline__ uint32_t hint_field(const uint8_t* __restrict__ hints, int64_t blk,
@@ -138,62 +176,6 @@ __device__ __forceinline__ uint32_t hint_field(const uint8_t* __restrict__ hints
   return 0;
 }
 
-// 8 one-bit (two-bit) fields -> bit 0 (bits 0..1) of 8 nibbles.
-__device__ __forceinline__ uint32_t expand1(uint32_t h8) {
-  uint32_t y = h8 & 0xFFu;
-  y = (y | (y << 12)) & 0x000F000Fu;
-  y = (y | (y << 6)) & 0x03030303u;
-  y = (y | (y << 3)) & 0x11111111u;
-  return y;
-}
-__device__ __forceinline__ uint32_t expand2(uint32_t h16) {
-  uint32_t y = h16 & 0xFFFFu;
-  y = (y | (y << 8)) & 0x00FF00FFu;
-  y = (y | (y << 4)) & 0x0F0F0F0Fu;
-  y = (y | (y << 2)) & 0x33333333u;
-  return y;
-}
-
-// Bracket, hint match and selection for 8 elements, all on packed nibbles.
-//   R: round-to-nearest codes of v (signs of x);
-//   Z: floor codes of a = |v| (the lower bracket end lo when a is off the grid);
-//   P: floor codes of a nudged down, (a - 2^-149) * (1 - 2^-24): equal to Z
-//      unless a sits exactly on a grid point (a grid value drops one cell, zero
-//      turns negative), so P != Z marks "no rounding decision".
-// Off the grid R is lo or lo + 1, so the other end of the bracket is
-// O = 2 * lo + 1 - m.  a > 6 gives Z = m = 7 and O = 8: saturated, no decision.
-// Per-element flags live in bit 3 of each nibble: a nibble value in 0..8 is
-// nonzero exactly when adding 7 sets its bit 3 (no carry leaves the nibble).
-template <int HB>
-__device__ __forceinline__ uint32_t guided_select(uint32_t R, uint32_t Z, uint32_t P,
-                                                  uint32_t hword, GuidedCounts& cnt) {
-  constexpr uint32_t kB3 = 0x88888888u, kSeven = 0x77777777u;
-  const uint32_t M = R & kSeven;  // round-to-nearest magnitudes
-  const uint32_t S = R - M;       // signs (of x)
-  const uint32_t O = (Z << 1) + 0x11111111u - M;
-  // P ^ Z is 0 off the grid and 1, 3, 7 (a grid value) or 8 (zero) on it
-  const uint32_t off = ~(((P ^ Z) + kSeven) | O) & kB3;  // a rounding decision exists
-  uint32_t take, differs;  // differs: the hint does not name the round-to-nearest cell
-  if (HB == 4) {
-    // signed positions: equal codes, or both magnitudes zero
-    const auto nz4 = [](uint32_t t) { return (((t & kSeven) + kSeven) | t) & kB3; };
-    const uint32_t zh = ~((hword & kSeven) + kSeven);
-    take = ~nz4(hword ^ (O | S)) | (~(O + kSeven) & zh);
-    differs = nz4(hword ^ R) & ((M + kSeven) | ~zh);
-  } else {
-    const uint32_t mask = HB == 1 ? 0x11111111u : 0x33333333u;
-    const uint32_t H = HB == 1 ? expand1(hword) : expand2(hword);
-    take = ~(((H ^ O) & mask) + kSeven);
-    differs = ((H ^ M) & mask) + kSeven;
-  }
-  take &= off;
-  cnt.consulted += __popc(off);
-  cnt.changed += __popc(take);
-  cnt.outside += __popc(off & ~take & differs);
-  const uint32_t T = (take >> 3) * 0xFu;  // whole-nibble select mask
-  return ((O & T) | (M & ~T)) + S;
-}
-
 template <int HB>
 __device__ __forceinline__ void guided_block(const Block16& b, uint32_t hw, uint2 h4, float s_t,
                                              const ScaleTables& tab, int64_t blk,
@@ -202,27 +184,24 @@ __device__ __forceinline__ void guided_block(const Block16& b, uint32_t hw, uint
   float x[16];
   unpack_block(b, x);
   const BlockScale bs = block_scale_bf16(block_amax_bits(b), s_t, tab);
+  const uint32_t h1 = HB == 1 ? hint_spread1(hw) : 0u;
   uint32_t out[2];
 #pragma unroll
   for (int half = 0; half < 2; ++half) {
-    float a[8], p[8];
-    uint32_t R = 0u;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int k = 8 * half + 2 * j;
-      R += e2m1x2(__fmul_rn(x[k], bs.inv), __fmul_rn(x[k + 1], bs.inv)) << (8 * j);
-    }
+    float v[8], p[8];
 #pragma unroll
     for (int t = 0; t < 8; ++t) {
-      a[t] = __fmul_rn(fabsf(x[8 * half + t]), bs.inv);  // |v|, bit-identical to |x * inv|
-      p[t] = __fmul_rn(__fsub_rn(a[t], 0x1p-149f), 0x1.fffffep-1f);
+      v[t] = __fmul_rn(x[8 * half + t], bs.inv);
+      p[t] = __uint_as_float(__float_as_uint(v[t]) - 1u);  // one ulp toward zero
     }
-    const uint32_t Z = e2m1x4_rz(a[0], a[1], a[2], a[3]) + (e2m1x4_rz(a[4], a[5], a[6], a[7]) << 16);
-    const uint32_t P = e2m1x4_rz(p[0], p[1], p[2], p[3]) + (e2m1x4_rz(p[4], p[5], p[6], p[7]) << 16);
+    const uint32_t R = pack_rn8(v);
+    const uint32_t Zs = pack_rz8(v);
+    const uint32_t pz = (pack_rz8(p) ^ Zs) & 0x77777777u;
     uint32_t hword;
     if (HB == 4) hword = half ? h4.y : h4.x;
-    else hword = half ? (hw >> (8 * (HB & 3))) : hw;
-    out[half] = guided_select<HB>(R, Z, P, hword, cnt);
+    else if (HB == 2) hword = half ? (hw >> 2) : hw;
+    else hword = half ? (h1 >> 1) : h1;
+    out[half] = guided_select<HB>(R, Zs & 0x77777777u, pz, hword, cnt);
   }
   reinterpret_cast<uint2*>(codes)[blk] = make_uint2(out[0], out[1]);
   scales[blk] = (uint8_t)bs.sb;
@@ -239,7 +218,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
   const float s_t = tensor_scale_from_amax(__uint_as_float(ws[0]));
   if (blockIdx.x == 0 && threadIdx.x == 0) *tensor_scale = s_t;
   scale_tables_init(tab, s_t);
-  GuidedCounts cnt{0ull, 0ull, 0ull};
+  GuidedCounts cnt{0u, 0u, 0u};
   const int64_t stride = (int64_t)gridDim.x * kThreads;
   int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x;
   for (; i + (U - 1) * stride < nblk; i += U * stride) {
@@ -275,10 +254,10 @@ template <int HB>
 __device__ __forceinline__ void hint_store_pair(uint8_t* __restrict__ hints, int64_t pair, uint4 c) {
   if (HB == 1)
     reinterpret_cast<uint32_t*>(hints)[pair] =
-        compact1(c.x) | (compact1(c.y) << 8) | (compact1(c.z) << 16) | (compact1(c.w) << 24);
+        hint_field1(make_uint2(c.x, c.y)) | (hint_field1(make_uint2(c.z, c.w)) << 16);
   if (HB == 2)
     reinterpret_cast<uint2*>(hints)[pair] =
-        make_uint2(compact2(c.x) | (compact2(c.y) << 16), compact2(c.z) | (compact2(c.w) << 16));
+        make_uint2(hint_field2(make_uint2(c.x, c.y)), hint_field2(make_uint2(c.z, c.w)));
   if (HB == 4) reinterpret_cast<uint4*>(hints)[pair] = c;
 }
 

@@ -144,7 +144,7 @@ __global__ void __launch_bounds__(kThreads)
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
     const float* ah = a + 8 * h;
-    const uint32_t Z = e2m1x4_rz(ah[0], ah[1], ah[2], ah[3]) + (e2m1x4_rz(ah[4], ah[5], ah[6], ah[7]) << 16);
+    const uint32_t Z = pack_rz8(ah);
     uint32_t S = 0u;  // signs of y
 #pragma unroll
     for (int k = 0; k < 8; ++k) S |= (__float_as_uint(y[8 * h + k]) >> 31) << (4 * k + 3);
