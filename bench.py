@@ -25,6 +25,7 @@ same workload instead.
 from __future__ import annotations
 
 import argparse
+import gc
 import json
 import os
 import statistics
@@ -138,11 +139,12 @@ class Stack:
 
     def kernels_of_layer(self, l):
         """(kernel label, algorithmic bytes) in launch order for layer l."""
-        hinted = l >= self.hint_from
+        q = "quantize_rtn+hint" if l >= self.hint_from else "quantize_rtn"
+        g = "guided_requant+hint" if l >= self.hint_from else "guided_requant"
         return [("amax", BYTES["amax"] * self.n),
-                ("quantize_rtn", BYTES["quantize_rtn+hint" if hinted else "quantize_rtn"] * self.n),
+                (q, BYTES[q] * self.n),
                 ("amax", BYTES["amax"] * self.n),
-                ("guided_requant", BYTES["guided_requant+hint" if hinted else "guided_requant"] * self.n),
+                (g, BYTES[g] * self.n),
                 ("mismatch_stats", BYTES["mismatch_stats"] * self.n)]
 
     def step_bytes(self):
@@ -299,6 +301,8 @@ def run_ours(args, world, rank, local):
     step_elems = 2 * stack.n * args.layers
 
     s_roll, s_train = torch.cuda.Stream(device), torch.cuda.Stream(device)
+    gc.collect()
+    gc.disable()  # no collector pauses inside the timed regions
     for _ in range(args.warmup):
         stack.step_pipelined(b, s_roll, s_train)
     torch.cuda.synchronize()
@@ -365,6 +369,8 @@ def run_ours(args, world, rank, local):
     # ---- end to end through the C ABI with host buffers (rank-local)
     e2e = run_e2e(b, stack, device, steps=min(args.steps, 2))
 
+    gc.enable()
+
     # ---- CPU oracle baseline (rank 0, N = 1 only)
     cpu = None
     if world == 1:
@@ -427,32 +433,42 @@ def _ncu_traffic(kernel_label):
     return None
 
 
-def _flush_l2(buf):
-    buf.add_(1)  # a write of 256 MiB evicts the 126 MB L2
+def _flush_l2(bufs):
+    """Write 256 MiB, then read another 256 MiB: L2 (126 MB) ends up holding
+    clean lines only, so the timed call neither hits in L2 nor pays for
+    writing back the flush's dirty lines."""
+    w, r = bufs
+    w.add_(1)
+    torch.sum(r, dtype=torch.float32)
 
 
 def _timed(fn, reps, flush):
-    """Average device time of fn over reps launches, L2 flushed before each."""
-    total = 0.0
+    """Median device time of fn over reps calls, L2 flushed before each (outside
+    the events).  A short spin kernel ahead of the start event keeps the GPU
+    busy while the host enqueues the call, so host-side delays do not land
+    between the events."""
+    times = []
     for r in range(reps):
         _flush_l2(flush)
+        torch.cuda._sleep(100_000)
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
         e0.record()
         fn(r)
         e1.record()
         torch.cuda.synchronize()
-        total += e0.elapsed_time(e1)
-    return total / reps / 1e3
+        times.append(e0.elapsed_time(e1))
+    return statistics.median(times) / 1e3
 
 
 def time_other_kernels(b, stack, device, peak, reps=10):
     """Standalone hint emit (throughput stack, layer 24), SR transpose
     re-quantize (128 x 512 x 2048 expert stack) and RHT32 + quantize
     (16384 x 4096 activation with outliers): seconds per call and algorithmic
-    GB/s, L2 flushed before every call."""
+    GB/s (median of `reps` calls), L2 flushed before every call."""
     from train_rollout_alignment_b200 import synthetic as syn
-    flush = torch.zeros(64 << 20, dtype=torch.float32, device=device)
+    flush = (torch.zeros(64 << 20, dtype=torch.float32, device=device),
+             torch.ones(64 << 20, dtype=torch.float32, device=device))
     out = {}
     # hint emit from the codes of a hinted layer
     l = stack.hint_from

@@ -39,12 +39,36 @@ __device__ __forceinline__ void st_v8f(float* p, const float* v) {
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
+// BF16 -> FP32 with the mixed-precision add of sm_100 (x + -0 == x for every
+// x, signed zeros included), which runs on the FP pipes instead of the
+// integer/logic pipe.
 __device__ __forceinline__ void unpack_block(const Block16& b, float* x) {
 #pragma unroll
-  for (int k = 0; k < 8; ++k) {
-    x[2 * k] = bf16_lo(b.w[k]);
-    x[2 * k + 1] = bf16_hi(b.w[k]);
-  }
+  for (int k = 0; k < 8; ++k)
+    asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %2;\n\t"
+        "add.rn.f32.bf16 %0, l, 0f80000000;\n\tadd.rn.f32.bf16 %1, h, 0f80000000;\n\t}"
+        : "=f"(x[2 * k]), "=f"(x[2 * k + 1])
+        : "r"(b.w[k]));
+}
+
+// Max |x| of a 16-value block as FP32 bits (low 16 bits zero), from packed
+// BF16 maxima of magnitudes (max.xorsign.abs: the magnitude is the larger
+// |x|, exact; the sign bit is dropped at the end).  A NaN element is passed
+// over; the tensor amax pass flags non-finite inputs.
+__device__ __forceinline__ uint32_t block_amax_bits(const Block16& b) {
+  uint32_t m[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k)
+    asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(m[k]) : "r"(b.w[2 * k]), "r"(b.w[2 * k + 1]));
+  asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(m[0]) : "r"(m[0]), "r"(m[1]));
+  asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(m[2]) : "r"(m[2]), "r"(m[3]));
+  asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(m[0]) : "r"(m[0]), "r"(m[2]));
+  uint32_t r;
+  asm("{\n\t.reg .b16 l, h, q;\n\tmov.b32 {l, h}, %1;\n\t"
+      "max.xorsign.abs.bf16 q, l, h;\n\tmov.b32 %0, {0, q};\n\t}"
+      : "=r"(r)
+      : "r"(m[0]));
+  return r & 0x7FFF0000u;
 }
 
 // ----------------------------------------------------------------- conversions

@@ -64,14 +64,6 @@ __device__ __forceinline__ void hint_store(uint8_t* __restrict__ hints, int64_t 
 }
 
 // ----------------------------------------------------------------- RTN quantize
-// Max |x| of a block as FP32 bits: packed 16-bit maxima of the BF16 magnitudes.
-__device__ __forceinline__ uint32_t block_amax_bits(const Block16& b) {
-  uint32_t m2 = 0u;
-#pragma unroll
-  for (int k = 0; k < 8; ++k) m2 = __vmaxu2(m2, b.w[k] & 0x7FFF7FFFu);
-  return max(m2 & 0xFFFFu, m2 >> 16) << 16;
-}
-
 template <int HB>
 __device__ __forceinline__ void rtn_block(const Block16& b, float s_t, const ScaleTables& tab,
                                           int64_t blk, uint8_t* __restrict__ codes,
@@ -144,7 +136,6 @@ __device__ __forceinline__ uint32_t guided_select(uint32_t R, uint32_t Zm, uint3
                                                   uint32_t hword, GuidedCounts& cnt) {
   constexpr uint32_t kB3 = 0x88888888u, kSeven = 0x77777777u;
   const uint32_t M = R & kSeven;  // round-to-nearest magnitudes
-  const uint32_t S = R & kB3;     // signs (of x)
   const uint32_t O = (Zm << 1) + 0x11111111u - M;
   const uint32_t off = ~((pz + kSeven) | O) & kB3;  // a rounding decision exists
   uint32_t take, differs;  // differs: the hint does not name the round-to-nearest cell
@@ -152,7 +143,7 @@ __device__ __forceinline__ uint32_t guided_select(uint32_t R, uint32_t Zm, uint3
     // signed positions: equal codes, or both magnitudes zero
     const auto nz4 = [](uint32_t t) { return (((t & kSeven) + kSeven) | t) & kB3; };
     const uint32_t zh = ~((hword & kSeven) + kSeven);
-    take = ~nz4(hword ^ (O | S)) | (~(O + kSeven) & zh);
+    take = ~nz4(hword ^ (O | (R & kB3))) | (~(O + kSeven) & zh);
     differs = nz4(hword ^ R) & ((M + kSeven) | ~zh);
   } else {
     const uint32_t mask = HB == 1 ? 0x11111111u : 0x33333333u;
@@ -163,8 +154,10 @@ __device__ __forceinline__ uint32_t guided_select(uint32_t R, uint32_t Zm, uint3
   cnt.consulted += __popc(off);
   cnt.changed += __popc(take);
   cnt.outside += __popc(off & ~take & differs);
-  const uint32_t T = (take >> 3) * 0xFu;  // whole-nibble select mask
-  return ((O & T) | (M & ~T)) | S;
+  // magnitude-bit select mask: 7 in every nibble whose bit 3 is set in take,
+  // (take * 7) >> 3 taken from the high word of take * (7 << 29)
+  const uint32_t T = __umulhi(take, 0xE0000000u);
+  return (R & ~T) | (O & T);  // the sign bits of R stay
 }
 
 template <int HB>
@@ -180,7 +173,8 @@ template <int HB>
 __device__ __forceinline__ void guided_block(const Block16& b, uint32_t hw, uint2 h4, float s_t,
                                              const ScaleTables& tab, int64_t blk,
                                              uint8_t* __restrict__ codes,
-                                             uint8_t* __restrict__ scales, GuidedCounts& cnt) {
+                                             uint8_t* __restrict__ scales, GuidedCounts& cnt,
+                                             uint32_t one) {
   float x[16];
   unpack_block(b, x);
   const BlockScale bs = block_scale_bf16(block_amax_bits(b), s_t, tab);
@@ -192,7 +186,9 @@ __device__ __forceinline__ void guided_block(const Block16& b, uint32_t hw, uint
 #pragma unroll
     for (int t = 0; t < 8; ++t) {
       v[t] = __fmul_rn(x[8 * half + t], bs.inv);
-      p[t] = __uint_as_float(__float_as_uint(v[t]) - 1u);  // one ulp toward zero
+      // one ulp toward zero: bits * one - 1 with one == 1 known only at run
+      // time, so it issues as a multiply-add on the FP pipe
+      p[t] = __uint_as_float(__float_as_uint(v[t]) * one + 0xFFFFFFFFu);
     }
     const uint32_t R = pack_rn8(v);
     const uint32_t Zs = pack_rz8(v);
@@ -212,7 +208,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     k_guided(const uint16_t* __restrict__ x, int64_t nblk, const uint8_t* __restrict__ hints,
              const uint32_t* __restrict__ ws, uint8_t* __restrict__ codes,
              uint8_t* __restrict__ scales, float* __restrict__ tensor_scale,
-             unsigned long long* __restrict__ stats4) {
+             unsigned long long* __restrict__ stats4, uint32_t one) {
   __shared__ unsigned long long red[3 * 8];
   __shared__ ScaleTables tab;
   const float s_t = tensor_scale_from_amax(__uint_as_float(ws[0]));
@@ -233,13 +229,14 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     }
 #pragma unroll
     for (int u = 0; u < U; ++u)
-      guided_block<HB>(b[u], hw[u], h4[u], s_t, tab, nblk - 1 - (i + u * stride), codes, scales, cnt);
+      guided_block<HB>(b[u], hw[u], h4[u], s_t, tab, nblk - 1 - (i + u * stride), codes, scales, cnt,
+                       one);
   }
   for (; i < nblk; i += stride) {
     const int64_t blk = nblk - 1 - i;
     uint2 h4;
     const uint32_t hw = hint_field<HB>(hints, blk, h4);
-    guided_block<HB>(ld_block(x + blk * 16), hw, h4, s_t, tab, blk, codes, scales, cnt);
+    guided_block<HB>(ld_block(x + blk * 16), hw, h4, s_t, tab, blk, codes, scales, cnt, one);
   }
   if (stats4 != nullptr) {
     const unsigned long long vals[3] = {cnt.consulted, cnt.changed, cnt.outside};
@@ -330,9 +327,9 @@ cudaError_t launch_guided(const uint16_t* x, int64_t nblk, const uint8_t* hints,
     return launch_quantize_rtn(x, nblk, ws, codes, scales, tensor_scale, nullptr, 0, s);
   const int g = grid_for(nblk, kThreads, kCtasPerSm);
   switch (hint_bits) {
-    case 1: k_guided<1, kUnroll><<<g, kThreads, 0, s>>>(x, nblk, hints, ws, codes, scales, tensor_scale, stats4); break;
-    case 2: k_guided<2, kUnroll><<<g, kThreads, 0, s>>>(x, nblk, hints, ws, codes, scales, tensor_scale, stats4); break;
-    case 4: k_guided<4, kUnroll><<<g, kThreads, 0, s>>>(x, nblk, hints, ws, codes, scales, tensor_scale, stats4); break;
+    case 1: k_guided<1, kUnroll><<<g, kThreads, 0, s>>>(x, nblk, hints, ws, codes, scales, tensor_scale, stats4, 1u); break;
+    case 2: k_guided<2, kUnroll><<<g, kThreads, 0, s>>>(x, nblk, hints, ws, codes, scales, tensor_scale, stats4, 1u); break;
+    case 4: k_guided<4, kUnroll><<<g, kThreads, 0, s>>>(x, nblk, hints, ws, codes, scales, tensor_scale, stats4, 1u); break;
     default: return cudaErrorInvalidValue;
   }
   return cudaGetLastError();
