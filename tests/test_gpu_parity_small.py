@@ -130,6 +130,32 @@ def test_mismatch_stats_matches_oracle(shape):
         assert g[7] == 0
 
 
+@pytest.mark.parametrize("ratio", [1.001, 1.0 + 2.0 ** -20, 0.75, 1.0])
+def test_mismatch_stats_arbitrary_codes_and_scale_ratios(ratio):
+    """Random code bytes and scale bytes (zero scales with nonzero codes, E4M3
+    subnormal scales) under tensor-scale ratios that are far from every grid
+    ratio (1.001), within 2^-17 of one (1 + 2^-20), exactly one (0.75), or
+    equal (1.0): every path of the value counter, against the oracle."""
+    rng = np.random.default_rng(int(ratio * 1e6))
+    rows, cols = 96, 4096
+    n = rows * cols
+    ca = rng.integers(0, 256, n // 2).astype(np.uint8)
+    cb = ca.copy()
+    flip = rng.random(n // 2) < 0.3
+    cb[flip] = rng.integers(0, 256, int(flip.sum())).astype(np.uint8)
+    sa = rng.integers(0, 127, n // 16).astype(np.uint8)
+    sa[rng.random(n // 16) < 0.05] = 0
+    sa[rng.random(n // 16) < 0.05] = rng.integers(1, 8)  # subnormal scales
+    sb = sa.copy()
+    move = rng.random(n // 16) < 0.2
+    sb[move] = rng.integers(0, 127, int(move.sum())).astype(np.uint8)
+    ta = np.float32(0.0123)
+    tb = np.float32(ta * np.float32(ratio))
+    g = gpu_stats(ca, sa, ta, cb, sb, tb, rows, cols)
+    o = oracle.mismatch_stats(ca, sa, ta, cb, sb, tb, rows, cols)
+    assert list(g[:7]) == list(o[:7])
+
+
 def _rtn_stack(w):
     batch = w.shape[0]
     outs = [oracle.quantize_rtn(w[e]) for e in range(batch)]

@@ -23,6 +23,11 @@
 //        two scale significands (16 x 16 cases) given the tensor scales, so a
 //        per-CTA table says where only zero/zero pairs can be equal;
 //      - any other block compares the 16 values in FP32 (rare).
+//    When the two tensor scales differ and no pair of nonzero scale
+//    significands gives a ratio near a grid ratio (checked once per CTA over
+//    all 15 x 15 pairs, together with the normal-float condition for every
+//    nonzero scale byte), every block with two nonzero scales takes the
+//    zero/zero rule without table lookups.
 #include "launch.h"
 #include "nvfp4_device.cuh"
 
@@ -137,14 +142,22 @@ __device__ __forceinline__ uint32_t not_both_zero(uint32_t wa, uint32_t wb) {
 
 // One block of the stream: queue it if its codes differ; count its scale and
 // (unless positions decide it) its decoded-value mismatches.
+// far_all: CTA-uniform, the tensor scales differ and every pair of nonzero
+// scale bytes is regular and far from a grid ratio.
 __device__ __forceinline__ void count_block(StatsShared& sm, uint32_t ax, uint32_t ay, uint32_t bx,
                                             uint32_t by, uint32_t sa, uint32_t sb, bool valid,
-                                            bool same_ts, float tsa, float tsb, int warp, int lane,
-                                            uint32_t lt_mask, int& qn, MismatchCounts& c) {
+                                            bool same_ts, bool far_all, float tsa, float tsb,
+                                            int warp, int lane, uint32_t lt_mask, int& qn,
+                                            MismatchCounts& c) {
   sa &= 0x7Fu;
   sb &= 0x7Fu;
-  const uint32_t ka = sm.key_a[sa], kb = sm.key_b[sb];
-  const bool same = same_ts && sa == sb && ka < 0x100u;
+  const bool fast = far_all && sa != 0u && sb != 0u;
+  uint32_t ka = 0u, kb = 0u;
+  if (!fast) {
+    ka = sm.key_a[sa];
+    kb = sm.key_b[sb];
+  }
+  const bool same = !fast && same_ts && sa == sb && ka < 0x100u;
   const bool dirty = ((ax ^ bx) | (ay ^ by)) != 0u;
   const uint32_t m = __ballot_sync(0xFFFFFFFFu, dirty);
   if (dirty) {
@@ -156,10 +169,12 @@ __device__ __forceinline__ void count_block(StatsShared& sm, uint32_t ax, uint32
   if (qn >= 32) qn = flush_queue(sm, warp, lane, qn, 32, c);
   if (valid) {
     c.scale += (sa != sb) ? 1u : 0u;
-    if (!same) {
+    if (fast) {
+      c.value += not_both_zero(ax, bx) + not_both_zero(ay, by);  // only zero pairs are equal
+    } else if (!same) {
       const uint32_t k = ka + kb;
       if (k < 0x100u && sm.ratio_far[k]) {
-        c.value += not_both_zero(ax, bx) + not_both_zero(ay, by);  // only zero pairs are equal
+        c.value += not_both_zero(ax, bx) + not_both_zero(ay, by);
       } else {
         c.value += value_mismatch_slow(make_uint2(ax, ay), make_uint2(bx, by), e4m3_value(sa),
                                        e4m3_value(sb), tsa, tsb);
@@ -186,6 +201,7 @@ __global__ void __launch_bounds__(kThreads, kStatsCtasPerSm)
     sm.key_a[t] = (xa >= 0x1p-124f && xa <= 0x1p120f) ? (uint16_t)(sig << 4) : (uint16_t)0x100;
     sm.key_b[t] = (xb >= 0x1p-124f && xb <= 0x1p120f) ? (uint16_t)sig : (uint16_t)0x100;
   }
+  bool ok = true;
   {
     // significand of (sb_a * s_t_a) / (sb_b * s_t_b) for scale significands
     // ma, mb (powers of two do not change it); approximate to a few ulps,
@@ -196,8 +212,16 @@ __global__ void __launch_bounds__(kThreads, kStatsCtasPerSm)
     if (ma != 0u && mb != 0u && tr >= 0x1p-120f && tr <= 0x1p120f)
       far_ratio = !near_grid_ratio(__fmul_rn(__fdiv_rn((float)ma, (float)mb), tr));
     sm.ratio_far[t] = far_ratio;
+    // the CTA-wide shortcut: every nonzero significand pair far, every
+    // nonzero scale byte regular on both sides
+    ok = (ma == 0u || mb == 0u || far_ratio);
   }
-  __syncthreads();
+  if (t < 128 && t != 0) {
+    const float sv = e4m3_value(t);
+    const float xa = __fmul_rn(sv, tsa), xb = __fmul_rn(sv, tsb);
+    ok = ok && xa >= 0x1p-124f && xa <= 0x1p120f && xb >= 0x1p-124f && xb <= 0x1p120f;
+  }
+  const bool far_all = __syncthreads_and(ok && !same_ts) != 0;
 
   MismatchCounts c{0u, 0u, 0u, 0u, 0u};
   const uint4* __restrict__ a4 = reinterpret_cast<const uint4*>(ca);
@@ -228,9 +252,9 @@ __global__ void __launch_bounds__(kThreads, kStatsCtasPerSm)
     for (int u = 0; u < U; ++u) {
       const bool valid = wb + u * wstride + lane < npair;
       count_block(sm, va[u].x, va[u].y, vb[u].x, vb[u].y, xa[u] & 0xFFu, xb[u] & 0xFFu, valid,
-                  same_ts, tsa, tsb, warp, lane, lt_mask, qn, c);
+                  same_ts, far_all, tsa, tsb, warp, lane, lt_mask, qn, c);
       count_block(sm, va[u].z, va[u].w, vb[u].z, vb[u].w, xa[u] >> 8, xb[u] >> 8, valid, same_ts,
-                  tsa, tsb, warp, lane, lt_mask, qn, c);
+                  far_all, tsa, tsb, warp, lane, lt_mask, qn, c);
     }
   }
   if (nblk & 1) {  // a trailing odd block: warp 0 of CTA 0, lane 0
@@ -244,8 +268,8 @@ __global__ void __launch_bounds__(kThreads, kStatsCtasPerSm)
         x = __ldg(sa + i);
         y = __ldg(sb + i);
       }
-      count_block(sm, a.x, a.y, b.x, b.y, x, y, lane == 0, same_ts, tsa, tsb, warp, lane, lt_mask,
-                  qn, c);
+      count_block(sm, a.x, a.y, b.x, b.y, x, y, lane == 0, same_ts, far_all, tsa, tsb, warp, lane,
+                  lt_mask, qn, c);
     }
   }
   if (qn > 0) flush_queue(sm, warp, lane, qn, qn, c);
