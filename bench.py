@@ -56,6 +56,9 @@ BYTES = {
 }
 
 
+SPEC_HBM_GBS = 8000.0  # B200 HBM3e data-sheet bandwidth, reported beside the measured peak
+
+
 def _peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -399,6 +402,7 @@ def run_ours(args, world, rank, local):
                        "note": "one stream, events around every launch; source of the kernels table"},
         "roofline": {"bound": "hbm", "kernel": dom, "achieved": round(dom_gbs, 1), "peak": peak,
                      "peak_kind": peak_kind, "unit": "GB/s", "frac": round(dom_gbs / peak, 4),
+                     "frac_of_spec": round(dom_gbs / SPEC_HBM_GBS, 4),
                      "bytes_per_launch": dom_bytes_per_launch, "traffic": traffic},
         "kernels": kernels,
         "other_kernels": other,

@@ -73,6 +73,14 @@ def _load():
                     None, [P, P, P, I64, I64, I64, ctypes.c_uint64, ctypes.c_uint32, P, P, P]),
                 "oracle_sr_transpose_requant_from": (
                     None, [P, P, P, I64, I64, I64, I64, ctypes.c_uint64, ctypes.c_uint32, P, P, P]),
+                "oracle_quantize_tile16_bf16": (None, [P, I64, I64, F, P, P, P]),
+                "oracle_transpose_tile16": (None, [P, P, I64, I64, I64, P, P]),
+                "oracle_dequant_tile16": (None, [P, P, F, I64, I64, P]),
+                "oracle_e8m0_exponent": (ctypes.c_int, [F]),
+                "oracle_e4m3_sr": (ctypes.c_int, [F, ctypes.c_uint32]),
+                "oracle_mxfp8_sr_transpose_requant": (
+                    None, [P, P, P, I64, I64, I64, ctypes.c_uint64, ctypes.c_uint32, P, P]),
+                "oracle_mxfp8_dequant": (None, [P, P, I64, P]),
                 "oracle_rht_signs": (None, [ctypes.c_uint64, P]),
                 "oracle_rht32_f64": (None, [P, I64, I64, ctypes.c_uint64, P]),
                 "oracle_rht_quantize": (None, [P, I64, I64, ctypes.c_uint64, P, P, P, P]),
@@ -249,6 +257,71 @@ def sr_transpose_requant(codes, scales, ts, batch, rows, cols, seed, draw, first
                                              int(batch), int(rows), int(cols), int(seed),
                                              int(draw) & 0xFFFFFFFF, _ptr(ct), _ptr(st), _ptr(tst))
     return ct, st, tst
+
+
+def quantize_tile16(x, A: float | None = None):
+    """BF16 [rows, cols] -> (codes [rows, cols/2], tile scales [rows/16, cols/16], s_t)."""
+    x = _u16(x)
+    rows, cols = x.shape
+    if A is None:
+        A = amax_bf16(x)
+    codes = np.zeros((rows, cols // 2), np.uint8)
+    tscales = np.zeros((rows // 16, cols // 16), np.uint8)
+    ts = np.zeros(1, np.float32)
+    _load().oracle_quantize_tile16_bf16(_ptr(x), rows, cols, float(A), _ptr(codes), _ptr(tscales),
+                                        _ptr(ts))
+    return codes, tscales, float(ts[0])
+
+
+def transpose_tile16(codes, tscales, batch, rows, cols):
+    """[batch, rows, cols] tile-scaled codes -> [batch, cols, rows] (lossless)."""
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    tscales = np.ascontiguousarray(tscales, dtype=np.uint8)
+    ct = np.zeros((batch, cols, rows // 2), np.uint8)
+    st = np.zeros((batch, cols // 16, rows // 16), np.uint8)
+    _load().oracle_transpose_tile16(_ptr(codes), _ptr(tscales), int(batch), int(rows), int(cols),
+                                    _ptr(ct), _ptr(st))
+    return ct, st
+
+
+def dequant_tile16(codes, tscales, s_t: float, rows: int, cols: int) -> np.ndarray:
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    tscales = np.ascontiguousarray(tscales, dtype=np.uint8)
+    out = np.zeros((rows, cols), np.float32)
+    _load().oracle_dequant_tile16(_ptr(codes), _ptr(tscales), float(s_t), int(rows), int(cols),
+                                  _ptr(out))
+    return out
+
+
+def e8m0_exponent(amax: float) -> int:
+    return _load().oracle_e8m0_exponent(float(amax))
+
+
+def e4m3_sr(a: float, r: int) -> int:
+    return _load().oracle_e4m3_sr(float(a), int(r) & 0xFFFFFFFF)
+
+
+def mxfp8_sr_transpose_requant(codes, scales, ts, batch, rows, cols, seed, draw):
+    """[batch, rows, cols] NVFP4 -> (E4M3 bytes [batch, cols, rows],
+    E8M0 bytes [batch, cols, rows/32]) by dequantize, transpose and SR."""
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    scales = np.ascontiguousarray(scales, dtype=np.uint8)
+    ts = np.ascontiguousarray(ts, dtype=np.float32)
+    q = np.zeros((batch, cols, rows), np.uint8)
+    e8 = np.zeros((batch, cols, rows // 32), np.uint8)
+    _load().oracle_mxfp8_sr_transpose_requant(_ptr(codes), _ptr(scales), _ptr(ts), int(batch),
+                                              int(rows), int(cols), int(seed),
+                                              int(draw) & 0xFFFFFFFF, _ptr(q), _ptr(e8))
+    return q, e8
+
+
+def mxfp8_dequant(q, e8) -> np.ndarray:
+    """MXFP8 -> FP32, flat; blocks of 32 consecutive elements."""
+    q = np.ascontiguousarray(q, dtype=np.uint8)
+    e8 = np.ascontiguousarray(e8, dtype=np.uint8)
+    out = np.zeros(q.size, np.float32)
+    _load().oracle_mxfp8_dequant(_ptr(q), _ptr(e8), int(q.size), _ptr(out))
+    return out
 
 
 def rht32_f64(x, seed: int) -> np.ndarray:

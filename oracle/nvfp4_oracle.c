@@ -465,6 +465,163 @@ void oracle_sr_transpose_requant_from(const uint8_t* codes, const uint8_t* scale
 }
 
 /* ------------------------------------------------------------------------ */
+/* Alternative to step 7, A: 16x16-tile scaling ([TML4], forward/backward
+ * mismatch paragraph: NVIDIA's proposal enlarges the group sharing a scale to a
+ * 16 x 16 tile of 256 values, which a transpose maps onto itself, at the price
+ * of one large value flattening the rest of its tile).  Reading: the tile
+ * scale follows the same recipe as the 16-value block scale (E4M3 of
+ * (amax_tile / 6) / s_t with the FP32 tensor scale s_t = A / 2688), codes are
+ * round-to-nearest as in step 3.  Layout: codes [rows, cols/2] as for blocks,
+ * tile scales [rows/16, cols/16] row-major; rows % 16 == cols % 16 == 0. */
+void oracle_quantize_tile16_bf16(const uint16_t* x, int64_t rows, int64_t cols, float A,
+                                 uint8_t* codes, uint8_t* tscales, float* tensor_scale)
+{
+    float s_t = oracle_tensor_scale(A);
+    *tensor_scale = s_t;
+    int64_t tr = rows / 16, tc = cols / 16;
+    for (int64_t ti = 0; ti < tr; ++ti) {
+        for (int64_t tj = 0; tj < tc; ++tj) {
+            float amax_t = 0.0f;
+            for (int64_t r = 16 * ti; r < 16 * ti + 16; ++r)
+                for (int64_t c = 16 * tj; c < 16 * tj + 16; ++c) {
+                    float a = fabsf(oracle_bf16_to_f32(x[r * cols + c]));
+                    if (a > amax_t) amax_t = a;
+                }
+            int sb = oracle_block_scale(amax_t, s_t);
+            tscales[ti * tc + tj] = (uint8_t)sb;
+            float sbv = (float)oracle_e4m3_value(sb);
+            for (int64_t r = 16 * ti; r < 16 * ti + 16; ++r)
+                for (int64_t c = 16 * tj; c < 16 * tj + 16; ++c) {
+                    float xv = oracle_bf16_to_f32(x[r * cols + c]);
+                    int m = 0;
+                    if (sbv != 0.0f) m = oracle_e2m1_rne(fabsf(scaled_value(xv, sbv, s_t)));
+                    nibble_put(codes, r * cols + c, (sign_of(xv) << 3) | m);
+                }
+        }
+    }
+}
+
+/* Transpose of tile-scaled matrices: code (r, c) moves to (c, r) and tile
+ * scale (ti, tj) to (tj, ti); the tensor scale is unchanged.  Nothing is
+ * re-rounded: the result is the tile quantization of the transposed input. */
+void oracle_transpose_tile16(const uint8_t* codes, const uint8_t* tscales, int64_t batch,
+                             int64_t rows, int64_t cols, uint8_t* codes_t, uint8_t* tscales_t)
+{
+    int64_t n = rows * cols, tr = rows / 16, tc = cols / 16;
+    for (int64_t e = 0; e < batch; ++e) {
+        const uint8_t* ce = codes + e * n / 2;
+        uint8_t* cte = codes_t + e * n / 2;
+        for (int64_t r = 0; r < rows; ++r)
+            for (int64_t c = 0; c < cols; ++c) nibble_put(cte, c * rows + r, nibble_get(ce, r * cols + c));
+        for (int64_t ti = 0; ti < tr; ++ti)
+            for (int64_t tj = 0; tj < tc; ++tj)
+                tscales_t[e * tr * tc + tj * tr + ti] = tscales[e * tr * tc + ti * tc + tj];
+    }
+}
+
+/* Decoded values of a tile-scaled matrix (same per-element rule as blocks). */
+void oracle_dequant_tile16(const uint8_t* codes, const uint8_t* tscales, float s_t, int64_t rows,
+                           int64_t cols, float* out)
+{
+    int64_t tc = cols / 16;
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t c = 0; c < cols; ++c)
+            out[r * cols + c] = oracle_dequant_one(nibble_get(codes, r * cols + c),
+                                                   tscales[(r / 16) * tc + c / 16], s_t);
+}
+
+/* ------------------------------------------------------------------------ */
+/* Alternative to step 7, B: the backward in MXFP8 with stochastic rounding
+ * ([TML4]: the backward runs in MXFP8 with stochastic rounding after the
+ * dequantize -> transpose step; MXFP8 costs 8.25 bits per value, i.e. 8-bit
+ * elements and one 8-bit scale per 32 values).  Readings (OCP MX): elements
+ * E4M3 "fn", one E8M0 scale 2^e per 32 consecutive values along the new rows,
+ * e = floor(log2(amax_32)) - 8 (8 = exponent of the largest E4M3 binade),
+ * clamped to [-127, 127], e = -127 for an all-zero block; byte = e + 127.
+ * Element: v = y * 2^-e, stochastic rounding of |v| onto the E4M3 values with
+ * the same rule and random word as step 7 (the same Philox counter: the
+ * element's row-major index in the [batch, cols, rows] output stack),
+ * saturating at 448; sign from y. */
+int oracle_e8m0_exponent(float amax)
+{
+    if (!(amax > 0.0f)) return -127;
+    int ex;
+    frexp((double)amax, &ex);   /* amax = f * 2^ex, f in [0.5, 1) */
+    int e = (ex - 1) - 8;
+    if (e < -127) e = -127;
+    if (e > 127) e = 127;
+    return e;
+}
+
+/* Stochastic rounding of a >= 0 onto the non-negative E4M3 values (a byte
+ * 0x00..0x7E): lo = the largest value <= a (exhaustive search), hi the next
+ * one; p = (a - lo) / (hi - lo); round up iff (r >> 8) < p * 2^24.  Values on
+ * the grid stay, a >= 448 gives 448. */
+int oracle_e4m3_sr(float a, uint32_t r)
+{
+    if (a != a) return 0x7F;
+    if (a >= 448.0f) return 0x7E;
+    int lo = 0;
+    for (int b = 1; b <= 0x7E; ++b)
+        if (oracle_e4m3_value(b) <= (double)a) lo = b;
+    double vlo = oracle_e4m3_value(lo);
+    if ((double)a == vlo) return lo;
+    double vhi = oracle_e4m3_value(lo + 1);
+    double p = ((double)a - vlo) / (vhi - vlo);
+    return ((double)(r >> 8) < p * 16777216.0) ? lo + 1 : lo;
+}
+
+/* codes/scales/tensor_scale: a stack of NVFP4 matrices [batch, rows, cols]
+ * (16-value blocks along cols).  Output: E4M3 bytes [batch, cols, rows] and
+ * E8M0 bytes [batch, cols, rows / 32]. */
+void oracle_mxfp8_sr_transpose_requant(const uint8_t* codes, const uint8_t* scales,
+                                       const float* tensor_scale, int64_t batch, int64_t rows,
+                                       int64_t cols, uint64_t seed, uint32_t draw, uint8_t* q_t,
+                                       uint8_t* e8_t)
+{
+    int64_t n = rows * cols;
+    float* y = (float*)malloc((size_t)(n > 0 ? n : 1) * sizeof(float));
+    float* yt = (float*)malloc((size_t)(n > 0 ? n : 1) * sizeof(float));
+    uint32_t key[2] = {(uint32_t)seed, (uint32_t)(seed >> 32)};
+    int64_t nb = rows / 32;
+    for (int64_t e = 0; e < batch; ++e) {
+        oracle_dequant(codes + e * n / 2, scales + e * n / 16, tensor_scale[e], n, y);
+        for (int64_t r = 0; r < rows; ++r)
+            for (int64_t c = 0; c < cols; ++c) yt[c * rows + r] = y[r * cols + c];
+        for (int64_t c = 0; c < cols; ++c) {
+            for (int64_t b = 0; b < nb; ++b) {
+                const float* blk = yt + c * rows + b * 32;
+                float amax_b = oracle_amax_f32(blk, 32);
+                int ex = oracle_e8m0_exponent(amax_b);
+                e8_t[e * cols * nb + c * nb + b] = (uint8_t)(ex + 127);
+                float down = ldexpf(1.0f, -ex);  /* exact: 2^-127 .. 2^127 are floats */
+                for (int k = 0; k < 32; ++k) {
+                    int64_t local = c * rows + b * 32 + k;
+                    int64_t gi = e * n + local;
+                    uint32_t ctr[4] = {(uint32_t)gi, (uint32_t)((uint64_t)gi >> 32), draw, 0u};
+                    uint32_t out[4];
+                    oracle_philox4x32_10(ctr, key, out);
+                    float v = blk[k] * down;
+                    q_t[gi] = (uint8_t)((sign_of(blk[k]) << 7) | oracle_e4m3_sr(fabsf(v), out[0]));
+                }
+            }
+        }
+    }
+    free(y);
+    free(yt);
+}
+
+/* Decoded MXFP8 values, blocks of 32 consecutive elements: E4M3 value times
+ * 2^(byte - 127), one FP32 multiply (exact unless it overflows). */
+void oracle_mxfp8_dequant(const uint8_t* q, const uint8_t* e8, int64_t n, float* out)
+{
+    for (int64_t i = 0; i < n; ++i) {
+        float v = (float)oracle_e4m3_value(q[i]);
+        out[i] = v * ldexpf(1.0f, (int)e8[i / 32] - 127);
+    }
+}
+
+/* ------------------------------------------------------------------------ */
 /* Step 8: 32-point random Hadamard transform ([TML4], communication
  * paragraph).  Signs: sigma_j = -1 iff bit 0 of Philox4x32-10(key = (seed lo32,
  * seed hi32), counter = (j, 0, 0, 0)).x0 is set.  The transform is the plain
