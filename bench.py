@@ -492,7 +492,6 @@ def time_other_kernels(b, stack, device, peak, reps=10):
     for e in range(batch):
         b.nvfp4_quantize_rtn(w[e], ws, codes[e * ne // 2:(e + 1) * ne // 2],
                              scales[e * ne // 16:(e + 1) * ne // 16], ts[e:e + 1])
-    del w
     ct, st, tst = torch.empty_like(codes), torch.empty_like(scales), torch.empty_like(ts)
     t = _timed(lambda r: b.nvfp4_sr_transpose_requant(codes, scales, ts, batch, er, ec, syn.CFG2_SR_SEED, r,
                                                       ws, ct, st, tst), reps, flush)
@@ -503,7 +502,10 @@ def time_other_kernels(b, stack, device, peak, reps=10):
         "avg_us": round(t * 1e6, 2), "GB/s": round(sr_bytes * n / t / 1e9, 1),
         "frac": round(sr_bytes * n / t / 1e9 / peak, 4), "bytes_per_elem": sr_bytes,
         "elements_per_s": round(n / t, 1)}
-    del codes, scales, ct, st
+    b.nvfp4_sr_transpose_requant(codes, scales, ts, batch, er, ec, syn.CFG2_SR_SEED, 0, ws, ct, st, tst)
+    out.update(time_transpose_alternatives(b, stack, w, codes, scales, ts, (ct, st, tst), device, peak, reps,
+                                           flush))
+    del w, codes, scales, ct, st
     # RHT32 + quantize
     x = torch.from_numpy(syn.cfg3().view(np.int16)).view(torch.bfloat16).to(device)
     rr, cc = x.shape
@@ -516,6 +518,90 @@ def time_other_kernels(b, stack, device, peak, reps=10):
     out["rht_quantize"] = {"workload": "%dx%d activation, 0.1%% outliers x100" % (rr, cc),
                            "avg_us": round(t * 1e6, 2), "GB/s": round(rht_bytes * n / t / 1e9, 1),
                            "frac": round(rht_bytes * n / t / 1e9 / peak, 4), "bytes_per_elem": rht_bytes}
+    return out
+
+
+def time_transpose_alternatives(b, stack, w, codes, scales, ts, sr_out, device, peak, reps, flush):
+    """The two alternatives to the SR transpose on the expert stack: 16x16-tile
+    NVFP4 (tile quantize timed on a 65536x4096 layer, lossless transpose of the
+    stack) and MXFP8 SR transpose re-quantize; then the error of each way of
+    getting a quantized W^T, against the BF16 W^T (relative squared error,
+    relative bias, share of nonzero values decoded as 0)."""
+    batch, er, ec = w.shape
+    ne, n = er * ec, batch * er * ec
+    out = {}
+    # tile quantize, streaming: the train input of a hinted layer, its amax precomputed
+    l = stack.hint_from
+    ct16 = torch.empty((ROWS, COLS // 2), dtype=torch.uint8, device=device)
+    tt16 = torch.empty((ROWS // 16, COLS // 16), dtype=torch.uint8, device=device)
+    ts16 = torch.empty(1, dtype=torch.float32, device=device)
+    wsl = stack.ws[l, 1]
+    b.nvfp4_tensor_amax(stack.xt[l], wsl)
+    t = _timed(lambda r: b.nvfp4_quantize_tile16(stack.xt[l], wsl, ct16, tt16, ts16, flags=b.NVFP4_AMAX_PRECOMPUTED),
+               reps, flush)
+    qb = 2 + 0.5 + 1 / 256
+    out["quantize_tile16"] = {"workload": "%dx%d BF16 layer, amax precomputed" % (ROWS, COLS),
+                              "avg_us": round(t * 1e6, 2), "GB/s": round(qb * stack.n / t / 1e9, 1),
+                              "frac": round(qb * stack.n / t / 1e9 / peak, 4), "bytes_per_elem": qb}
+    del ct16, tt16
+    # tile codes of the expert stack, then the lossless transpose
+    tc = torch.empty(n // 2, dtype=torch.uint8, device=device)
+    tt = torch.empty(n // 256, dtype=torch.uint8, device=device)
+    tts = torch.empty(batch, dtype=torch.float32, device=device)
+    wse = torch.zeros(4, dtype=torch.int32, device=device)
+    for e in range(batch):
+        b.nvfp4_quantize_tile16(w[e], wse, tc[e * ne // 2:(e + 1) * ne // 2], tt[e * ne // 256:(e + 1) * ne // 256],
+                                tts[e:e + 1])
+    tct, ttt = torch.empty_like(tc), torch.empty_like(tt)
+    t = _timed(lambda r: b.nvfp4_transpose_tile16(tc, tt, batch, er, ec, tct, ttt), reps, flush)
+    tb = 0.5 + 0.5 + 2 / 256
+    out["transpose_tile16"] = {"workload": "%dx%dx%d expert stack" % (batch, er, ec), "avg_us": round(t * 1e6, 2),
+                               "GB/s": round(tb * n / t / 1e9, 1), "frac": round(tb * n / t / 1e9 / peak, 4),
+                               "bytes_per_elem": tb}
+    # MXFP8 SR transpose from the 16-value NVFP4 codes
+    q = torch.empty(n, dtype=torch.uint8, device=device)
+    e8 = torch.empty(n // 32, dtype=torch.uint8, device=device)
+    t = _timed(lambda r: b.mxfp8_sr_transpose_requant(codes, scales, ts, batch, er, ec, 2, r, q, e8), reps, flush)
+    mb = 0.5 + 1 / 16 + 1 + 1 / 32
+    out["mxfp8_sr_transpose_requant"] = {
+        "workload": "%dx%dx%d expert stack, one Philox4x32-10 word per element" % (batch, er, ec),
+        "avg_us": round(t * 1e6, 2), "GB/s": round(mb * n / t / 1e9, 1), "frac": round(mb * n / t / 1e9 / peak, 4),
+        "bytes_per_elem": mb, "elements_per_s": round(n / t, 1)}
+    b.mxfp8_sr_transpose_requant(codes, scales, ts, batch, er, ec, 2, 0, q, e8)
+    # quality of each quantized W^T against the BF16 W^T
+    wt = w.float().transpose(1, 2).contiguous()
+    deq = torch.empty((batch, ec, er), dtype=torch.float32, device=device)
+
+    def err(y):
+        d = (y - wt).double()
+        nz = wt != 0
+        return {"rel_sq_err": float((d * d).sum() / (wt.double() ** 2).sum()),
+                "rel_bias": float(d.sum() / wt.double().abs().sum()),
+                "nonzero_to_zero": float(((y == 0) & nz).sum() / nz.sum())}
+
+    quality = {}
+    ct_, st_, tst_ = sr_out
+    for e in range(batch):
+        b.nvfp4_dequantize(ct_[e * ne // 2:(e + 1) * ne // 2], st_[e * ne // 16:(e + 1) * ne // 16], tst_[e:e + 1],
+                           ec, er, b.NVFP4_SCALES_BLOCK16, deq[e])
+    quality["nvfp4_16_sr_transpose"] = err(deq)
+    for e in range(batch):
+        b.nvfp4_dequantize(tct[e * ne // 2:(e + 1) * ne // 2], ttt[e * ne // 256:(e + 1) * ne // 256], tts[e:e + 1],
+                           ec, er, b.NVFP4_SCALES_TILE16, deq[e])
+    quality["nvfp4_tile16_transpose"] = err(deq)
+    b.mxfp8_dequantize(q, e8, n, deq)
+    quality["mxfp8_sr_transpose"] = err(deq)
+    cd = torch.empty(ne // 2, dtype=torch.uint8, device=device)
+    sd = torch.empty(ne // 16, dtype=torch.uint8, device=device)
+    td = torch.empty(1, dtype=torch.float32, device=device)
+    for e in range(batch):
+        b.nvfp4_quantize_rtn(w[e].t().contiguous(), wse, cd, sd, td)
+        b.nvfp4_dequantize(cd, sd, td, ec, er, b.NVFP4_SCALES_BLOCK16, deq[e])
+    quality["nvfp4_16_rtn_of_transposed_bf16"] = err(deq)
+    quality["note"] = ("W^T of the %dx%dx%d expert stack; each row is one way to obtain a quantized W^T from "
+                       "the forward's quantized W (the last row quantizes the BF16 W^T directly, for reference)"
+                       % (batch, er, ec))
+    out["transpose_quality"] = quality
     return out
 
 

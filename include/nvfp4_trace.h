@@ -260,6 +260,93 @@ nvfp4_status nvfp4_sr_transpose_requant_noalloc(const uint8_t* codes, const uint
                                                 uint8_t* codes_t, uint8_t* scales_t,
                                                 float* tensor_scale_t, void* stream);
 
+/* ======================================================================
+ * Alternatives to nvfp4_sr_transpose_requant that [TML4] weighs
+ * (forward/backward mismatch paragraph and format table).
+ * ====================================================================== */
+
+#define NVFP4_SCALES_BLOCK16  0   /* one scale per 16 consecutive values of a row */
+#define NVFP4_SCALES_TILE16   1   /* one scale per 16 x 16 tile */
+
+/*
+ * nvfp4_quantize_tile16 -- NVFP4 with one E4M3 scale per 16 x 16 tile.
+ *   [TML4], forward/backward mismatch paragraph: NVIDIA's proposal enlarges
+ *   the group that shares a scale to a 256-value tile, which a transpose maps
+ *   onto itself (so no re-quantization is needed after transposing), at the
+ *   price of one large value flattening the rest of its tile.
+ *   Recipe as nvfp4_quantize_rtn with the block amax replaced by the tile
+ *   amax: sb = RNE_E4M3_satfinite((amax_tile / 6) / s_t), inv = 1/(sb * s_t),
+ *   codes round-to-nearest, sign from x.
+ *   x_bf16 [rows, cols], rows % 16 == cols % 16 == 0 (NVFP4_ERR_SHAPE).
+ *   codes [rows, cols/2] (same layout as blocks), tile_scales [rows/16,
+ *   cols/16] row-major E4M3 bytes, tensor_scale: 1 float.  ws and flags as in
+ *   nvfp4_quantize_rtn.
+ */
+nvfp4_status nvfp4_quantize_tile16(const uint16_t* x_bf16, int64_t rows, int64_t cols,
+                                   uint32_t* ws, int flags, uint8_t* codes,
+                                   uint8_t* tile_scales, float* tensor_scale, void* stream);
+
+/*
+ * nvfp4_transpose_tile16 -- transpose a stack of tile-scaled NVFP4 matrices
+ * without re-rounding: code (r, c) moves to (c, r), tile scale (i, j) to
+ * (j, i); each matrix keeps its tensor scale (the caller reuses it).  The
+ * result equals nvfp4_quantize_tile16 of the transposed input, bit for bit.
+ *   codes [batch, rows, cols/2], tile_scales [batch, rows/16, cols/16] ->
+ *   codes_t [batch, cols, rows/2], tile_scales_t [batch, cols/16, rows/16].
+ *   rows % 16 == cols % 16 == 0, batch <= 65535 (NVFP4_ERR_SHAPE).
+ */
+nvfp4_status nvfp4_transpose_tile16(const uint8_t* codes, const uint8_t* tile_scales,
+                                    int64_t batch, int64_t rows, int64_t cols,
+                                    uint8_t* codes_t, uint8_t* tile_scales_t, void* stream);
+
+/*
+ * mxfp8_sr_transpose_requant -- dequantize a stack of NVFP4 matrices,
+ * transpose, and re-quantize to MXFP8 with stochastic rounding.
+ *   [TML4]: the backward runs in MXFP8 with stochastic rounding after the
+ *   dequantize -> transpose step; MXFP8 costs 8.25 bits per value (format
+ *   table): 8-bit E4M3 elements and one 8-bit E8M0 scale per 32 values.
+ *   Per matrix e: y = (G[m] * sb) * s_t[e] as in nvfp4_sr_transpose_requant,
+ *   y^T is [cols, rows]; each 32 consecutive values of a row of y^T share
+ *   2^x, x = floor(log2(amax_32)) - 8 clamped to [-127, 127] (-127 for an
+ *   all-zero block; OCP MX: 8 is the exponent of E4M3's top binade), stored
+ *   as the byte x + 127.  v = y * 2^-x; with a = |v|: a >= 448 -> 448; lo =
+ *   the largest E4M3 value <= a, hi the next one;
+ *     round up iff (r >> 8) < ((a - lo) / (hi - lo)) * 2^24,
+ *   r the same Philox4x32-10 word as in nvfp4_sr_transpose_requant (counter
+ *   = row-major index i in the OUTPUT stack [batch, cols, rows], draw).
+ *   Element byte = sign(y) << 7 | E4M3 bits of the magnitude.
+ *   codes [batch, rows, cols/2], scales [batch, rows, cols/16],
+ *   tensor_scale [batch] -> q_t [batch, cols, rows] bytes,
+ *   e8_t [batch, cols, rows/32] bytes.  rows % 32 == 0, cols % 16 == 0,
+ *   batch <= 65535 (NVFP4_ERR_SHAPE).  No scratch: every scale is per block.
+ */
+nvfp4_status mxfp8_sr_transpose_requant(const uint8_t* codes, const uint8_t* scales,
+                                        const float* tensor_scale,
+                                        int64_t batch, int64_t rows, int64_t cols,
+                                        uint64_t seed, uint32_t draw,
+                                        uint8_t* q_t, uint8_t* e8_t, void* stream);
+
+/*
+ * nvfp4_dequantize -- NVFP4 -> FP32: value = sign * ((G[m] * sb) * s_t) in
+ * FP32 (the first product is exact).  [RLQ]: a decoded value is the code's
+ * value times the scale.
+ *   scale_layout NVFP4_SCALES_BLOCK16: scales [rows, cols/16];
+ *   NVFP4_SCALES_TILE16: scales [rows/16, cols/16] (rows % 16 == 0).
+ *   tensor_scale: device pointer to 1 float.  out [rows, cols] FP32, 32-byte
+ *   aligned.  cols % 16 == 0.
+ */
+nvfp4_status nvfp4_dequantize(const uint8_t* codes, const uint8_t* scales,
+                              const float* tensor_scale, int64_t rows, int64_t cols,
+                              int scale_layout, float* out, void* stream);
+
+/*
+ * mxfp8_dequantize -- MXFP8 -> FP32: E4M3 value of q[i] times
+ * 2^(e8[i / 32] - 127), one FP32 multiply (infinite if it overflows).
+ *   n % 32 == 0; q, e8 16-byte aligned, out 32-byte aligned.
+ */
+nvfp4_status mxfp8_dequantize(const uint8_t* q, const uint8_t* e8, int64_t n, float* out,
+                              void* stream);
+
 /* Human-readable name of a status code (static string, never NULL). */
 const char* nvfp4_status_string(nvfp4_status status);
 

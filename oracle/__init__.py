@@ -80,6 +80,8 @@ def _load():
                 "oracle_e4m3_sr": (ctypes.c_int, [F, ctypes.c_uint32]),
                 "oracle_mxfp8_sr_transpose_requant": (
                     None, [P, P, P, I64, I64, I64, ctypes.c_uint64, ctypes.c_uint32, P, P]),
+                "oracle_mxfp8_sr_transpose_requant_from": (
+                    None, [P, P, P, I64, I64, I64, I64, ctypes.c_uint64, ctypes.c_uint32, P, P]),
                 "oracle_mxfp8_dequant": (None, [P, P, I64, P]),
                 "oracle_rht_signs": (None, [ctypes.c_uint64, P]),
                 "oracle_rht32_f64": (None, [P, I64, I64, ctypes.c_uint64, P]),
@@ -301,17 +303,20 @@ def e4m3_sr(a: float, r: int) -> int:
     return _load().oracle_e4m3_sr(float(a), int(r) & 0xFFFFFFFF)
 
 
-def mxfp8_sr_transpose_requant(codes, scales, ts, batch, rows, cols, seed, draw):
+def mxfp8_sr_transpose_requant(codes, scales, ts, batch, rows, cols, seed, draw, first: int = 0):
     """[batch, rows, cols] NVFP4 -> (E4M3 bytes [batch, cols, rows],
-    E8M0 bytes [batch, cols, rows/32]) by dequantize, transpose and SR."""
+    E8M0 bytes [batch, cols, rows/32]) by dequantize, transpose and SR.
+
+    ``first``: index of the first given matrix within the whole stack (the
+    random counter is the element's index in the whole output stack)."""
     codes = np.ascontiguousarray(codes, dtype=np.uint8)
     scales = np.ascontiguousarray(scales, dtype=np.uint8)
     ts = np.ascontiguousarray(ts, dtype=np.float32)
     q = np.zeros((batch, cols, rows), np.uint8)
     e8 = np.zeros((batch, cols, rows // 32), np.uint8)
-    _load().oracle_mxfp8_sr_transpose_requant(_ptr(codes), _ptr(scales), _ptr(ts), int(batch),
-                                              int(rows), int(cols), int(seed),
-                                              int(draw) & 0xFFFFFFFF, _ptr(q), _ptr(e8))
+    _load().oracle_mxfp8_sr_transpose_requant_from(_ptr(codes), _ptr(scales), _ptr(ts), int(first),
+                                                   int(batch), int(rows), int(cols), int(seed),
+                                                   int(draw) & 0xFFFFFFFF, _ptr(q), _ptr(e8))
     return q, e8
 
 

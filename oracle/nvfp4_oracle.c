@@ -574,10 +574,28 @@ int oracle_e4m3_sr(float a, uint32_t r)
 /* codes/scales/tensor_scale: a stack of NVFP4 matrices [batch, rows, cols]
  * (16-value blocks along cols).  Output: E4M3 bytes [batch, cols, rows] and
  * E8M0 bytes [batch, cols, rows / 32]. */
+void oracle_mxfp8_sr_transpose_requant_from(const uint8_t* codes, const uint8_t* scales,
+                                            const float* tensor_scale, int64_t first,
+                                            int64_t batch, int64_t rows, int64_t cols,
+                                            uint64_t seed, uint32_t draw, uint8_t* q_t,
+                                            uint8_t* e8_t);
+
 void oracle_mxfp8_sr_transpose_requant(const uint8_t* codes, const uint8_t* scales,
                                        const float* tensor_scale, int64_t batch, int64_t rows,
                                        int64_t cols, uint64_t seed, uint32_t draw, uint8_t* q_t,
                                        uint8_t* e8_t)
+{
+    oracle_mxfp8_sr_transpose_requant_from(codes, scales, tensor_scale, 0, batch, rows, cols, seed,
+                                           draw, q_t, e8_t);
+}
+
+/* The same for matrices first .. first+batch-1 of a larger stack whose data
+ * starts at the given pointers (the counter keeps the whole stack's index). */
+void oracle_mxfp8_sr_transpose_requant_from(const uint8_t* codes, const uint8_t* scales,
+                                            const float* tensor_scale, int64_t first,
+                                            int64_t batch, int64_t rows, int64_t cols,
+                                            uint64_t seed, uint32_t draw, uint8_t* q_t,
+                                            uint8_t* e8_t)
 {
     int64_t n = rows * cols;
     float* y = (float*)malloc((size_t)(n > 0 ? n : 1) * sizeof(float));
@@ -597,12 +615,13 @@ void oracle_mxfp8_sr_transpose_requant(const uint8_t* codes, const uint8_t* scal
                 float down = ldexpf(1.0f, -ex);  /* exact: 2^-127 .. 2^127 are floats */
                 for (int k = 0; k < 32; ++k) {
                     int64_t local = c * rows + b * 32 + k;
-                    int64_t gi = e * n + local;
+                    int64_t gi = (first + e) * n + local;
                     uint32_t ctr[4] = {(uint32_t)gi, (uint32_t)((uint64_t)gi >> 32), draw, 0u};
                     uint32_t out[4];
                     oracle_philox4x32_10(ctr, key, out);
                     float v = blk[k] * down;
-                    q_t[gi] = (uint8_t)((sign_of(blk[k]) << 7) | oracle_e4m3_sr(fabsf(v), out[0]));
+                    q_t[e * n + local] =
+                        (uint8_t)((sign_of(blk[k]) << 7) | oracle_e4m3_sr(fabsf(v), out[0]));
                 }
             }
         }

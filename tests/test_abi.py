@@ -20,14 +20,16 @@ def _declared():
     for fname in os.listdir(os.path.join(ROOT, "include")):
         if fname.endswith(".h"):
             text = open(os.path.join(ROOT, "include", fname)).read()
-            names += re.findall(r"^\s*(?:nvfp4_status|const char\*)\s+(nvfp4_\w+)\s*\(", text, re.M)
+            names += re.findall(r"^\s*(?:nvfp4_status|const char\*)\s+((?:nvfp4|mxfp8)_\w+)\s*\(", text, re.M)
     return sorted(set(names))
 
 
 def test_header_declares_the_boundary():
     want = {"nvfp4_quantize_rtn", "nvfp4_emit_hint", "nvfp4_guided_requant",
             "nvfp4_sr_transpose_requant", "nvfp4_rht_quantize", "nvfp4_mismatch_stats",
-            "nvfp4_tensor_amax", "nvfp4_status_string"}
+            "nvfp4_tensor_amax", "nvfp4_status_string", "nvfp4_quantize_tile16",
+            "nvfp4_transpose_tile16", "mxfp8_sr_transpose_requant", "nvfp4_dequantize",
+            "mxfp8_dequantize"}
     assert want <= set(_declared())
 
 
@@ -76,3 +78,43 @@ def test_validation_rejects_bad_arguments_without_a_gpu():
     assert e(fake, 32, 3, fake, None) == 5
     assert e(fake, 24, 2, fake, None) == 3
     assert e(fake, 32, 2, fake + 4, None) == 2
+
+
+def test_validation_of_the_tile_and_mxfp8_entry_points_without_a_gpu():
+    lib = ctypes.CDLL(_lib_path())
+    P, I64, I, U64, U32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_uint64, ctypes.c_uint32
+    fake = 1 << 20
+    q = lib.nvfp4_quantize_tile16
+    q.restype = I
+    q.argtypes = [P, I64, I64, P, I, P, P, P, P]
+    assert q(fake, 24, 32, fake, 0, fake, fake, fake, None) == 3      # rows % 16
+    assert q(fake, 32, 40, fake, 0, fake, fake, fake, None) == 3      # cols % 16
+    assert q(None, 32, 32, fake, 0, fake, fake, fake, None) == 1
+    assert q(fake + 16, 32, 32, fake, 0, fake, fake, fake, None) == 2
+    assert q(fake, 32, 32, fake, 4, fake, fake, fake, None) == 1      # unknown flag
+    t = lib.nvfp4_transpose_tile16
+    t.restype = I
+    t.argtypes = [P, P, I64, I64, I64, P, P, P]
+    assert t(fake, fake, 1, 16, 24, fake, fake, None) == 3
+    assert t(fake, fake, 70000, 16, 16, fake, fake, None) == 3
+    assert t(fake, fake, 0, 16, 16, None, None, None) == 0            # empty stack
+    assert t(fake, fake, 1, 16, 16, fake + 8, fake, None) == 2
+    m = lib.mxfp8_sr_transpose_requant
+    m.restype = I
+    m.argtypes = [P, P, P, I64, I64, I64, U64, U32, P, P, P]
+    assert m(fake, fake, fake, 1, 48, 32, 2, 0, fake, fake, None) == 3  # rows % 32
+    assert m(fake, fake, fake, 1, 64, 24, 2, 0, fake, fake, None) == 3  # cols % 16
+    assert m(fake, fake, None, 1, 64, 32, 2, 0, fake, fake, None) == 1
+    assert m(fake, fake, fake, 1, 64, 32, 2, 0, fake + 4, fake, None) == 2
+    d = lib.nvfp4_dequantize
+    d.restype = I
+    d.argtypes = [P, P, P, I64, I64, I, P, P]
+    assert d(fake, fake, fake, 4, 32, 2, fake, None) == 1              # unknown layout
+    assert d(fake, fake, fake, 8, 32, 1, fake, None) == 3              # tiles need rows % 16
+    assert d(fake, fake, fake, 4, 32, 0, fake + 16, None) == 2         # out 32-B aligned
+    x = lib.mxfp8_dequantize
+    x.restype = I
+    x.argtypes = [P, P, I64, P, P]
+    assert x(fake, fake, 48, fake, None) == 3
+    assert x(fake, fake, 64, fake + 16, None) == 2
+    assert x(fake, fake, 0, None, None) == 0

@@ -270,3 +270,14 @@ def test_mxfp8_on_grid_values_transpose_losslessly():
         q, e8 = oracle.mxfp8_sr_transpose_requant(codes, scales, ts, 1, rows, cols, 2, draw)
         yt = oracle.mxfp8_dequant(q[0], e8[0])
         assert np.array_equal(yt.view(np.uint32), y.view(np.uint32)) or np.array_equal(yt, y)
+
+
+def test_mxfp8_per_matrix_calls_match_whole_stack():
+    batch, rows, cols = 3, 32, 32
+    w = syn.random_case((batch, rows, cols), 47, "normal")
+    codes, scales, ts = _nvfp4_stack(w)
+    q, e8 = oracle.mxfp8_sr_transpose_requant(codes, scales, ts, batch, rows, cols, 4, 2)
+    for e in range(batch):
+        qe, e8e = oracle.mxfp8_sr_transpose_requant(codes[e:e + 1], scales[e:e + 1], ts[e:e + 1], 1, rows,
+                                                    cols, 4, 2, first=e)
+        assert np.array_equal(qe[0], q[e]) and np.array_equal(e8e[0], e8[e])

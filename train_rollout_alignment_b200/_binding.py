@@ -35,6 +35,12 @@ _SIGS = {
     "nvfp4_rht_quantize": (_I, [_P, _I64, _I64, ctypes.c_uint64, _P, _P, _P, _P, _P, _P]),
     "nvfp4_sr_transpose_requant_noalloc": (
         _I, [_P, _P, _P, _I64, _I64, _I64, ctypes.c_uint64, ctypes.c_uint32, _P, _P, _P, _P]),
+    "nvfp4_quantize_tile16": (_I, [_P, _I64, _I64, _P, _I, _P, _P, _P, _P]),
+    "nvfp4_transpose_tile16": (_I, [_P, _P, _I64, _I64, _I64, _P, _P, _P]),
+    "mxfp8_sr_transpose_requant": (
+        _I, [_P, _P, _P, _I64, _I64, _I64, ctypes.c_uint64, ctypes.c_uint32, _P, _P, _P]),
+    "nvfp4_dequantize": (_I, [_P, _P, _P, _I64, _I64, _I, _P, _P]),
+    "mxfp8_dequantize": (_I, [_P, _P, _I64, _P, _P]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _fn = getattr(_lib, _name)
@@ -49,6 +55,8 @@ NVFP4_AMAX_PRECOMPUTED = 1
 NVFP4_WARN_NONFINITE = 1
 NVFP4_ERR_SCRATCH_LIMIT = 6
 NVFP4_SR_NOALLOC_MAX_BATCH = 4096
+NVFP4_SCALES_BLOCK16 = 0
+NVFP4_SCALES_TILE16 = 1
 
 
 class Nvfp4Error(RuntimeError):
@@ -162,3 +170,34 @@ def empty_nvfp4(rows: int, cols: int, device, hint_bits: int = 0):
     if hint_bits:
         hints = torch.empty(((rows * cols * hint_bits + 7) // 8,), dtype=torch.uint8, device=device)
     return codes, scales, ts, ws, hints
+
+
+# ----------------------------------------------------------------- alternatives to SR transpose
+def nvfp4_quantize_tile16(x, ws, codes, tile_scales, tensor_scale, flags=0, stream=None):
+    rows, cols = _rows_cols(x)
+    _check("nvfp4_quantize_tile16", _lib.nvfp4_quantize_tile16(
+        _ptr(x), rows, cols, _ptr(ws), int(flags), _ptr(codes), _ptr(tile_scales), _ptr(tensor_scale),
+        _stream(stream)))
+
+
+def nvfp4_transpose_tile16(codes, tile_scales, batch, rows, cols, codes_t, tile_scales_t, stream=None):
+    _check("nvfp4_transpose_tile16", _lib.nvfp4_transpose_tile16(
+        _ptr(codes), _ptr(tile_scales), int(batch), int(rows), int(cols), _ptr(codes_t),
+        _ptr(tile_scales_t), _stream(stream)))
+
+
+def mxfp8_sr_transpose_requant(codes, scales, tensor_scale, batch, rows, cols, seed, draw, q_t, e8_t,
+                               stream=None):
+    _check("mxfp8_sr_transpose_requant", _lib.mxfp8_sr_transpose_requant(
+        _ptr(codes), _ptr(scales), _ptr(tensor_scale), int(batch), int(rows), int(cols),
+        int(seed) & 0xFFFFFFFFFFFFFFFF, int(draw) & 0xFFFFFFFF, _ptr(q_t), _ptr(e8_t), _stream(stream)))
+
+
+def nvfp4_dequantize(codes, scales, tensor_scale, rows, cols, scale_layout, out, stream=None):
+    _check("nvfp4_dequantize", _lib.nvfp4_dequantize(
+        _ptr(codes), _ptr(scales), _ptr(tensor_scale), int(rows), int(cols), int(scale_layout), _ptr(out),
+        _stream(stream)))
+
+
+def mxfp8_dequantize(q, e8, n, out, stream=None):
+    _check("mxfp8_dequantize", _lib.mxfp8_dequantize(_ptr(q), _ptr(e8), int(n), _ptr(out), _stream(stream)))

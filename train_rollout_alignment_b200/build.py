@@ -15,7 +15,8 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libnvfp4trace.so")
-SOURCES = ["api.cu", "quantize.cu", "stats.cu", "sr_transpose.cu", "rht.cu", "noalloc.cu"]
+SOURCES = ["api.cu", "quantize.cu", "stats.cu", "sr_transpose.cu", "rht.cu", "noalloc.cu",
+           "next_formats.cu"]
 HEADERS = ["nvfp4_device.cuh", "launch.h"]
 
 NVCC_FLAGS = [

@@ -190,4 +190,90 @@ nvfp4_status nvfp4_rht_quantize(const uint16_t* x_bf16, int64_t rows, int64_t co
                                               static_cast<cudaStream_t>(stream)));
 }
 
+// ----------------------------------------------------------------- alternatives to SR transpose
+nvfp4_status nvfp4_quantize_tile16(const uint16_t* x_bf16, int64_t rows, int64_t cols, uint32_t* ws,
+                                   int flags, uint8_t* codes, uint8_t* tile_scales,
+                                   float* tensor_scale, void* stream) {
+  nvfp4_status st = check_shape(rows, cols, 16);
+  if (st != NVFP4_OK) return st;
+  if (rows % 16 != 0) return NVFP4_ERR_SHAPE;
+  if (flags & ~NVFP4_AMAX_PRECOMPUTED) return NVFP4_ERR_INVALID_ARG;
+  if (rows * cols == 0) return write_unit_scale(tensor_scale, stream);
+  if (!x_bf16) return NVFP4_ERR_INVALID_ARG;
+  if ((st = check_quant_outputs(ws, codes, tile_scales, tensor_scale)) != NVFP4_OK) return st;
+  if (!aligned(x_bf16, 32)) return NVFP4_ERR_MISALIGNED;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (!(flags & NVFP4_AMAX_PRECOMPUTED)) {
+    if (cudaMemsetAsync(ws, 0, NVFP4_WS_WORDS * sizeof(uint32_t), s) != cudaSuccess)
+      return NVFP4_ERR_CUDA;
+    if ((st = from_cuda(nvfp4::launch_amax_bf16(x_bf16, rows * cols / 16, ws, s))) != NVFP4_OK)
+      return st;
+  }
+  return from_cuda(nvfp4::launch_quantize_tile16(x_bf16, rows, cols, ws, codes, tile_scales,
+                                                 tensor_scale, s));
+}
+
+nvfp4_status nvfp4_transpose_tile16(const uint8_t* codes, const uint8_t* tile_scales, int64_t batch,
+                                    int64_t rows, int64_t cols, uint8_t* codes_t,
+                                    uint8_t* tile_scales_t, void* stream) {
+  if (batch < 0 || rows < 0 || cols < 0) return NVFP4_ERR_INVALID_ARG;
+  if (rows % 16 != 0 || cols % 16 != 0) return NVFP4_ERR_SHAPE;
+  if (batch > 65535 || rows / 64 >= 65535) return NVFP4_ERR_SHAPE;
+  if (rows != 0 && cols > kMaxElems / rows) return NVFP4_ERR_SHAPE;
+  if (batch != 0 && rows * cols > kMaxElems / batch) return NVFP4_ERR_SHAPE;
+  if (batch == 0 || rows == 0 || cols == 0) return NVFP4_OK;
+  if (!codes || !tile_scales || !codes_t || !tile_scales_t) return NVFP4_ERR_INVALID_ARG;
+  if (!aligned(codes, 16) || !aligned(tile_scales, 16) || !aligned(codes_t, 16) ||
+      !aligned(tile_scales_t, 16))
+    return NVFP4_ERR_MISALIGNED;
+  return from_cuda(nvfp4::launch_transpose_tile16(codes, tile_scales, batch, rows, cols, codes_t,
+                                                  tile_scales_t, static_cast<cudaStream_t>(stream)));
+}
+
+nvfp4_status mxfp8_sr_transpose_requant(const uint8_t* codes, const uint8_t* scales,
+                                        const float* tensor_scale, int64_t batch, int64_t rows,
+                                        int64_t cols, uint64_t seed, uint32_t draw, uint8_t* q_t,
+                                        uint8_t* e8_t, void* stream) {
+  if (batch < 0 || rows < 0 || cols < 0) return NVFP4_ERR_INVALID_ARG;
+  if (rows % 32 != 0 || cols % 16 != 0) return NVFP4_ERR_SHAPE;
+  if (batch > 65535 || rows / 128 >= 65535) return NVFP4_ERR_SHAPE;
+  if (rows != 0 && cols > kMaxElems / rows) return NVFP4_ERR_SHAPE;
+  if (batch != 0 && rows * cols > kMaxElems / batch) return NVFP4_ERR_SHAPE;
+  if (batch == 0 || rows == 0 || cols == 0) return NVFP4_OK;
+  if (!codes || !scales || !tensor_scale || !q_t || !e8_t) return NVFP4_ERR_INVALID_ARG;
+  if (!aligned(codes, 16) || !aligned(scales, 16) || !aligned(q_t, 16) || !aligned(e8_t, 16) ||
+      !aligned(tensor_scale, 4))
+    return NVFP4_ERR_MISALIGNED;
+  return from_cuda(nvfp4::launch_mxfp8_sr_transpose(codes, scales, tensor_scale, batch, rows, cols,
+                                                    seed, draw, q_t, e8_t,
+                                                    static_cast<cudaStream_t>(stream)));
+}
+
+nvfp4_status nvfp4_dequantize(const uint8_t* codes, const uint8_t* scales, const float* tensor_scale,
+                              int64_t rows, int64_t cols, int scale_layout, float* out,
+                              void* stream) {
+  nvfp4_status st = check_shape(rows, cols, 16);
+  if (st != NVFP4_OK) return st;
+  if (scale_layout != NVFP4_SCALES_BLOCK16 && scale_layout != NVFP4_SCALES_TILE16)
+    return NVFP4_ERR_INVALID_ARG;
+  if (scale_layout == NVFP4_SCALES_TILE16 && rows % 16 != 0) return NVFP4_ERR_SHAPE;
+  if (rows * cols == 0) return NVFP4_OK;
+  if (!codes || !scales || !tensor_scale || !out) return NVFP4_ERR_INVALID_ARG;
+  if (!aligned(codes, 16) || !aligned(scales, 16) || !aligned(tensor_scale, 4) || !aligned(out, 32))
+    return NVFP4_ERR_MISALIGNED;
+  return from_cuda(nvfp4::launch_dequant_nvfp4(codes, scales, tensor_scale, rows, cols,
+                                               scale_layout == NVFP4_SCALES_TILE16, out,
+                                               static_cast<cudaStream_t>(stream)));
+}
+
+nvfp4_status mxfp8_dequantize(const uint8_t* q, const uint8_t* e8, int64_t n, float* out,
+                              void* stream) {
+  if (n < 0) return NVFP4_ERR_INVALID_ARG;
+  if (n % 32 != 0 || n >= kMaxElems) return NVFP4_ERR_SHAPE;
+  if (n == 0) return NVFP4_OK;
+  if (!q || !e8 || !out) return NVFP4_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(e8, 16) || !aligned(out, 32)) return NVFP4_ERR_MISALIGNED;
+  return from_cuda(nvfp4::launch_dequant_mxfp8(q, e8, n, out, static_cast<cudaStream_t>(stream)));
+}
+
 }  // extern "C"

@@ -31,6 +31,20 @@ cudaError_t launch_sr_transpose(const uint8_t* codes, const uint8_t* scales, con
 cudaError_t launch_rht_quantize(const uint16_t* x, int64_t nblk, uint64_t seed, uint32_t* ws,
                                 uint8_t* codes, uint8_t* scales, float* tensor_scale,
                                 float* y_out, cudaStream_t s);
+cudaError_t launch_quantize_tile16(const uint16_t* x, int64_t rows, int64_t cols, const uint32_t* ws,
+                                   uint8_t* codes, uint8_t* tscales, float* tensor_scale,
+                                   cudaStream_t s);
+cudaError_t launch_transpose_tile16(const uint8_t* codes, const uint8_t* tscales, int64_t batch,
+                                    int64_t rows, int64_t cols, uint8_t* codes_t,
+                                    uint8_t* tscales_t, cudaStream_t s);
+cudaError_t launch_mxfp8_sr_transpose(const uint8_t* codes, const uint8_t* scales, const float* ts,
+                                      int64_t batch, int64_t rows, int64_t cols, uint64_t seed,
+                                      uint32_t draw, uint8_t* q_t, uint8_t* e8_t, cudaStream_t s);
+cudaError_t launch_dequant_nvfp4(const uint8_t* codes, const uint8_t* scales, const float* ts,
+                                 int64_t rows, int64_t cols, int tile16, float* out,
+                                 cudaStream_t s);
+cudaError_t launch_dequant_mxfp8(const uint8_t* q, const uint8_t* e8, int64_t n, float* out,
+                                 cudaStream_t s);
 cudaError_t launch_set_f32(float* dst, float value, cudaStream_t s);
 
 }  // namespace nvfp4
