@@ -218,7 +218,7 @@ nvfp4_status nvfp4_transpose_tile16(const uint8_t* codes, const uint8_t* tile_sc
                                     uint8_t* tile_scales_t, void* stream) {
   if (batch < 0 || rows < 0 || cols < 0) return NVFP4_ERR_INVALID_ARG;
   if (rows % 16 != 0 || cols % 16 != 0) return NVFP4_ERR_SHAPE;
-  if (batch > 65535 || rows / 64 >= 65535) return NVFP4_ERR_SHAPE;
+  if (batch > 65535 || rows / 128 >= 65535) return NVFP4_ERR_SHAPE;
   if (rows != 0 && cols > kMaxElems / rows) return NVFP4_ERR_SHAPE;
   if (batch != 0 && rows * cols > kMaxElems / batch) return NVFP4_ERR_SHAPE;
   if (batch == 0 || rows == 0 || cols == 0) return NVFP4_OK;

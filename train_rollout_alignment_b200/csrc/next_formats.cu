@@ -13,45 +13,17 @@
 namespace nvfp4 {
 
 // ----------------------------------------------------------------- tile-16 quantize
-// A warp owns two horizontally adjacent tiles per step: lane r of each half
-// holds row r of its tile (one 16-value block, one 256-bit load), so the two
-// halves read 64 contiguous bytes per row.  The tile amax is a 16-lane
-// shuffle reduction; then every lane quantizes its own block with the tile
-// scale.  Tile pairs are visited from the end of the tensor backwards (the
-// amax pass that runs just before streams forwards, so its tail is in L2).
-constexpr int kTileUnroll = 2;
+// A warp owns 32 horizontally adjacent tiles of one 16-row band (lane j: tile
+// column 32 s + j, i.e. block 32 s + j of each of the 16 rows).  Pass 1
+// streams the band -- each row is read as 1 KiB contiguous across the warp --
+// and keeps each lane's tile maximum in a register (no shuffles).  Pass 2
+// reads the same 16 KiB again, from L2 where pass 1 just left it, and writes
+// the codes (256 contiguous bytes per row) and one scale byte per lane.
+// Bands are visited from the end of the tensor backwards (the amax pass that
+// runs just before streams forwards, so its tail is still in L2).
+constexpr int kTileRowsInFlight = 8;
 
-__device__ __forceinline__ void tile16_item(const uint16_t* __restrict__ x, int64_t cols, int64_t tc,
-                                            int64_t ppr, int64_t item, int lane, float s_t,
-                                            const ScaleTables& tab, const Block16& b,
-                                            uint8_t* __restrict__ codes,
-                                            uint8_t* __restrict__ tscales) {
-  const int64_t ti = item / ppr;
-  const int64_t tj = 2 * (item % ppr) + (lane >> 4);
-  const bool valid = tj < tc;
-  uint32_t m = valid ? block_amax_bits(b) : 0u;
-#pragma unroll
-  for (int o = 1; o < 16; o <<= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
-  const BlockScale bs = block_scale_bf16(m, s_t, tab);
-  if (!valid) return;
-  float xf[16], v[16];
-  unpack_block(b, xf);
-#pragma unroll
-  for (int k = 0; k < 16; ++k) v[k] = __fmul_rn(xf[k], bs.inv);
-  const int64_t row = 16 * ti + (lane & 15);
-  reinterpret_cast<uint2*>(codes + row * (cols / 2))[tj] = pack_codes16(v);
-  if ((lane & 15) == 0) tscales[ti * tc + tj] = (uint8_t)bs.sb;
-}
-
-__device__ __forceinline__ Block16 tile16_load(const uint16_t* __restrict__ x, int64_t cols,
-                                               int64_t tc, int64_t ppr, int64_t item, int lane) {
-  const int64_t ti = item / ppr;
-  const int64_t tj = 2 * (item % ppr) + (lane >> 4);
-  if (tj >= tc) return Block16{};
-  return ld_block(x + (16 * ti + (lane & 15)) * cols + 16 * tj);
-}
-
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, 4)
     k_quantize_tile16(const uint16_t* __restrict__ x, int64_t rows, int64_t cols,
                       const uint32_t* __restrict__ ws, uint8_t* __restrict__ codes,
                       uint8_t* __restrict__ tscales, float* __restrict__ tensor_scale) {
@@ -60,68 +32,122 @@ __global__ void __launch_bounds__(kThreads)
   if (blockIdx.x == 0 && threadIdx.x == 0) *tensor_scale = s_t;
   scale_tables_init(tab, s_t);
   const int lane = threadIdx.x & 31;
-  const int64_t tc = cols / 16, ppr = (tc + 1) / 2, nitems = (rows / 16) * ppr;
+  const int64_t tc = cols / 16, segs = (tc + 31) / 32, nitems = (rows / 16) * segs;
   const int64_t wstride = (int64_t)gridDim.x * (kThreads / 32);
-  int64_t w = (int64_t)blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5);
-  for (; w + (kTileUnroll - 1) * wstride < nitems; w += kTileUnroll * wstride) {
-    Block16 b[kTileUnroll];
+  for (int64_t w = (int64_t)blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5); w < nitems;
+       w += wstride) {
+    const int64_t item = nitems - 1 - w;
+    const int64_t ti = item / segs, tj = (item % segs) * 32 + lane;
+    if (tj >= tc) continue;  // only in the last segment of a band
+    const uint16_t* band = x + 16 * ti * cols + 16 * tj;
+    uint32_t m = 0u;
+#pragma unroll 1
+    for (int r0 = 0; r0 < 16; r0 += kTileRowsInFlight) {
+      Block16 b[kTileRowsInFlight];
 #pragma unroll
-    for (int u = 0; u < kTileUnroll; ++u)
-      b[u] = tile16_load(x, cols, tc, ppr, nitems - 1 - (w + u * wstride), lane);
+      for (int u = 0; u < kTileRowsInFlight; ++u) b[u] = ld_block(band + (r0 + u) * cols);
 #pragma unroll
-    for (int u = 0; u < kTileUnroll; ++u)
-      tile16_item(x, cols, tc, ppr, nitems - 1 - (w + u * wstride), lane, s_t, tab, b[u], codes,
-                  tscales);
-  }
-  for (; w < nitems; w += wstride) {
-    const Block16 b = tile16_load(x, cols, tc, ppr, nitems - 1 - w, lane);
-    tile16_item(x, cols, tc, ppr, nitems - 1 - w, lane, s_t, tab, b, codes, tscales);
+      for (int u = 0; u < kTileRowsInFlight; ++u) m = max(m, block_amax_bits(b[u]));
+    }
+    const BlockScale bs = block_scale_bf16(m, s_t, tab);
+    uint2* out = reinterpret_cast<uint2*>(codes + 16 * ti * (cols / 2)) + tj;
+#pragma unroll 1
+    for (int r0 = 0; r0 < 16; r0 += kTileRowsInFlight) {
+      Block16 b[kTileRowsInFlight];
+#pragma unroll
+      for (int u = 0; u < kTileRowsInFlight; ++u) b[u] = ld_block(band + (r0 + u) * cols);
+#pragma unroll
+      for (int u = 0; u < kTileRowsInFlight; ++u) {
+        float xf[16], v[16];
+        unpack_block(b[u], xf);
+#pragma unroll
+        for (int k = 0; k < 16; ++k) v[k] = __fmul_rn(xf[k], bs.inv);
+        out[(r0 + u) * (cols / 16)] = pack_codes16(v);
+      }
+    }
+    tscales[ti * tc + tj] = (uint8_t)bs.sb;
   }
 }
 
 // ----------------------------------------------------------------- tile-16 transpose
-// One CTA per 64 x 64 element square of one matrix: the codes are unpacked
-// into a byte per element in shared memory, read back column-wise and packed
-// again; the (up to) 4 x 4 tile scales of the square move to their transposed
-// places.  Nothing is re-rounded.
-constexpr int kSq = 64;
-constexpr int kSqStride = kSq + 4;
+// One CTA per 128 x 128 element square of one matrix.  The square's codes
+// (128 rows of 64 bytes) are staged in shared memory as 32-bit words of 8
+// nibbles; each thread then owns an 8 x 8 nibble block (8 rows x one word
+// column), transposes it in registers with three rounds of masked swaps
+// (4x4, 2x2 and single-nibble blocks) and writes 8 words, one per output
+// row.  The row stride of 17 words and the lane -> block mapping (8 word
+// columns x 4 row groups per warp) make the column reads conflict-free.  The
+// square's 8 x 8 tile scales move to their transposed places.  Nothing is
+// re-rounded.
+constexpr int kSq = 128;
+constexpr int kSqWords = kSq / 8;      // 32-bit words of codes per row of a square
+constexpr int kSqStride = kSqWords + 1;
+
+__device__ __forceinline__ void nib_swap(uint32_t& a, uint32_t& b, int shift, uint32_t mask) {
+  const uint32_t t = ((a >> shift) ^ b) & mask;
+  b ^= t;
+  a ^= t << shift;
+}
 
 __global__ void __launch_bounds__(kThreads)
     k_transpose_tile16(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ tscales,
                        int64_t rows, int64_t cols, uint8_t* __restrict__ codes_t,
                        uint8_t* __restrict__ tscales_t) {
-  __shared__ uint8_t el[kSq][kSqStride];
+  __shared__ uint32_t sq[kSq][kSqStride];
   const int64_t e = blockIdx.z;
   const int64_t r0 = (int64_t)blockIdx.y * kSq, c0 = (int64_t)blockIdx.x * kSq;
   const int64_t n = rows * cols, tr = rows / 16, tc = cols / 16;
   const int t = threadIdx.x;
-  {
-    const int row = t >> 2, q = t & 3;
-    const int64_t r = r0 + row, c = c0 + 16 * q;
-    if (r < rows && c < cols) {
-      const uint2 v = __ldg(reinterpret_cast<const uint2*>(codes + e * (n / 2) + r * (cols / 2) + c / 2));
+  const uint8_t* src = codes + e * (n / 2);
 #pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        const uint32_t byte = ((k < 4 ? v.x : v.y) >> (8 * (k & 3))) & 0xFFu;
-        el[row][16 * q + 2 * k] = (uint8_t)(byte & 15u);
-        el[row][16 * q + 2 * k + 1] = (uint8_t)(byte >> 4);
+  for (int h = 0; h < 2; ++h) {
+    // 32 elements (16 bytes) per thread, as two 8-byte loads: a row of codes is
+    // cols / 2 bytes, a multiple of 8 but not always of 16
+    const int row = (t >> 2) + 64 * h, q = t & 3;
+    const int64_t r = r0 + row, c = c0 + 32 * q;
+    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+    if (r < rows && c < cols) {
+      const uint2* p = reinterpret_cast<const uint2*>(src + r * (cols / 2) + c / 2);
+      const uint2 lo = __ldg(p);
+      v.x = lo.x;
+      v.y = lo.y;
+      if (c + 32 <= cols) {  // else cols % 32 == 16: the row ends after 16 elements
+        const uint2 hi = __ldg(p + 1);
+        v.z = hi.x;
+        v.w = hi.y;
       }
     }
+    sq[row][4 * q] = v.x;
+    sq[row][4 * q + 1] = v.y;
+    sq[row][4 * q + 2] = v.z;
+    sq[row][4 * q + 3] = v.w;
   }
-  if (t < 16) {
-    const int64_t ti = r0 / 16 + (t >> 2), tj = c0 / 16 + (t & 3);
-    if (ti < tr && tj < tc) tscales_t[e * tr * tc + tj * tr + ti] = tscales[e * tr * tc + ti * tc + tj];
+  if (t < 64) {
+    const int64_t ti = r0 / 16 + (t >> 3), tj = c0 / 16 + (t & 7);
+    if (ti < tr && tj < tc)
+      tscales_t[e * tr * tc + tj * tr + ti] = tscales[e * tr * tc + ti * tc + tj];
   }
   __syncthreads();
-  const int oc = t >> 2, q = t & 3;  // output row c0 + oc, input rows r0 + 16q ..
-  const int64_t c = c0 + oc, r = r0 + 16 * q;
-  if (c < cols && r < rows) {
-    uint32_t w[2] = {0u, 0u};
+  const int warp = t >> 5, lane = t & 31;
+  const int bc = (lane & 7) + 8 * (warp & 1);   // word column: input columns 8 bc ..
+  const int br = (lane >> 3) + 4 * (warp >> 1);  // row group: input rows 8 br ..
+  const int64_t cb = c0 + 8 * bc, rb = r0 + 8 * br;
+  if (cb >= cols || rb >= rows) return;  // (both are multiples of 8; cols, rows of 16)
+  uint32_t m[8];
 #pragma unroll
-    for (int k = 0; k < 16; ++k) w[k >> 3] |= (uint32_t)el[16 * q + k][oc] << (4 * (k & 7));
-    reinterpret_cast<uint2*>(codes_t + e * (n / 2) + c * (rows / 2) + r / 2)[0] = make_uint2(w[0], w[1]);
+  for (int i = 0; i < 8; ++i) m[i] = sq[8 * br + i][bc];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) nib_swap(m[i], m[i + 4], 16, 0x0000FFFFu);
+#pragma unroll
+  for (int i = 0; i < 8; i += 4) {
+    nib_swap(m[i], m[i + 2], 8, 0x00FF00FFu);
+    nib_swap(m[i + 1], m[i + 3], 8, 0x00FF00FFu);
   }
+#pragma unroll
+  for (int i = 0; i < 8; i += 2) nib_swap(m[i], m[i + 1], 4, 0x0F0F0F0Fu);
+  uint8_t* dst = codes_t + e * (n / 2) + rb / 2;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) *reinterpret_cast<uint32_t*>(dst + (cb + j) * (rows / 2)) = m[j];
 }
 
 // ----------------------------------------------------------------- MXFP8 SR transpose
@@ -298,7 +324,7 @@ __global__ void __launch_bounds__(kThreads)
 cudaError_t launch_quantize_tile16(const uint16_t* x, int64_t rows, int64_t cols, const uint32_t* ws,
                                    uint8_t* codes, uint8_t* tscales, float* tensor_scale,
                                    cudaStream_t s) {
-  const int64_t items = (rows / 16) * ((cols / 16 + 1) / 2);
+  const int64_t items = (rows / 16) * ((cols / 16 + 31) / 32);  // one warp each
   const int g = grid_for(items * 32, kThreads, 4);
   k_quantize_tile16<<<g, kThreads, 0, s>>>(x, rows, cols, ws, codes, tscales, tensor_scale);
   return cudaGetLastError();
