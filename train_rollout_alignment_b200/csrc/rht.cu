@@ -32,27 +32,69 @@ __device__ __forceinline__ void load_sign_masks(uint32_t* masks, uint32_t seed_l
   __syncthreads();
 }
 
-// z = H32 * (sigma (.) x) for the group at x (32 BF16 values), unnormalised;
+// Packed FP32 pairs (sm_100 f32x2 arithmetic: both lanes rounded to nearest,
+// exactly as two scalar operations).
+typedef unsigned long long f32x2;
+
+__device__ __forceinline__ f32x2 pack2(float lo, float hi) {
+  f32x2 r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void unpack2(f32x2 p, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(p));
+}
+__device__ __forceinline__ f32x2 add2(f32x2 a, f32x2 b) {
+  f32x2 d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ f32x2 sub2(f32x2 a, f32x2 b) {
+  f32x2 d;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ f32x2 mul2(f32x2 a, f32x2 b) {
+  f32x2 d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
+// First butterfly stage on one BF16 word (elements 2k, 2k+1 = lo, hi):
+// (lo + hi, lo - hi) in FP32, the BF16 operand converted exactly inside the
+// mixed-precision add and subtract.
+__device__ __forceinline__ f32x2 stage1(uint32_t w) {
+  const float hi = __uint_as_float(w & 0xFFFF0000u);
+  float s, d;
+  asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %2;\n\t"
+      "add.rn.f32.bf16 %0, l, %3;\n\tsub.rn.f32.bf16 %1, l, %3;\n\t}"
+      : "=f"(s), "=f"(d)
+      : "r"(w), "f"(hi));
+  return pack2(s, d);
+}
+
+// z = H32 * (sigma (.) x) for the group at x (32 BF16 values), unnormalised,
+// as 16 pairs P[m] = (z[2m], z[2m+1]).  Stage h = 1 pairs the two halves of a
+// BF16 word; stages h = 2, 4, 8, 16 pair element j with j + h, i.e. pair m
+// with pair m + h/2, half for half, so they run on packed pairs.  The
+// operations and their order are those of the scalar butterfly.
 // masks: the per-CTA sign masks in shared memory (broadcast reads).
 __device__ __forceinline__ void hadamard32(const uint16_t* __restrict__ x, const uint32_t* masks,
-                                           float* z) {
+                                           f32x2* P) {
   const Block16 b0 = ld_block(x), b1 = ld_block(x + 16);
 #pragma unroll
   for (int k = 0; k < 8; ++k) {
-    const uint32_t w0 = b0.w[k] ^ masks[k], w1 = b1.w[k] ^ masks[8 + k];
-    z[2 * k] = bf16_lo(w0);
-    z[2 * k + 1] = bf16_hi(w0);
-    z[16 + 2 * k] = bf16_lo(w1);
-    z[16 + 2 * k + 1] = bf16_hi(w1);
+    P[k] = stage1(b0.w[k] ^ masks[k]);
+    P[8 + k] = stage1(b1.w[k] ^ masks[8 + k]);
   }
 #pragma unroll
-  for (int h = 1; h < 32; h <<= 1) {
+  for (int h2 = 1; h2 < 16; h2 <<= 1) {
 #pragma unroll
-    for (int j = 0; j < 32; ++j) {
-      if (j & h) continue;
-      const float a = z[j], c = z[j + h];
-      z[j] = __fadd_rn(a, c);
-      z[j + h] = __fsub_rn(a, c);
+    for (int m = 0; m < 16; ++m) {
+      if (m & h2) continue;
+      const f32x2 a = P[m], c = P[m + h2];
+      P[m] = add2(a, c);
+      P[m + h2] = sub2(a, c);
     }
   }
 }
@@ -63,15 +105,21 @@ __global__ void __launch_bounds__(kThreads, kRhtCtasPerSm)
   __shared__ uint32_t masks[16];
   __shared__ uint32_t red[kThreads / 32];
   load_sign_masks(masks, seed_lo, seed_hi);
-  uint32_t zmax = 0u;  // bits of max |z| (integer max, so a NaN is not dropped)
+  float zmax = 0.0f;  // max |z|; a NaN propagates (max.NaN), so it is not dropped
   const int64_t stride = (int64_t)gridDim.x * kThreads;
   for (int64_t g = (int64_t)blockIdx.x * kThreads + threadIdx.x; g < ngroups; g += stride) {
-    float z[32];
-    hadamard32(x + g * 32, masks, z);
+    f32x2 P[16];
+    hadamard32(x + g * 32, masks, P);
 #pragma unroll
-    for (int k = 0; k < 32; ++k) zmax = max(zmax, __float_as_uint(z[k]) & 0x7FFFFFFFu);
+    for (int m = 0; m < 16; ++m) {
+      float a, b;
+      unpack2(P[m], a, b);
+      asm("max.NaN.f32 %0, %0, %1;" : "+f"(zmax) : "f"(fabsf(a)));
+      asm("max.NaN.f32 %0, %0, %1;" : "+f"(zmax) : "f"(fabsf(b)));
+    }
   }
-  uint32_t best = zmax >= 0x7F800000u ? zmax : __float_as_uint(__fmul_rn(__uint_as_float(zmax), kInvSqrt32));
+  const uint32_t zb = __float_as_uint(zmax);
+  uint32_t best = zb >= 0x7F800000u ? zb : __float_as_uint(__fmul_rn(zmax, kInvSqrt32));
   best = block_max_u32(best, red);
   if (threadIdx.x == 0) {
     if (best) atomicMax(ws, best);
@@ -79,16 +127,17 @@ __global__ void __launch_bounds__(kThreads, kRhtCtasPerSm)
   }
 }
 
-__device__ __forceinline__ void quantize_block_f32(const float* y, float s_t, int64_t blk,
-                                                   uint8_t* __restrict__ codes,
+__device__ __forceinline__ void quantize_block_f32(const float* y, float s_t, const ScaleTables& tab,
+                                                   int64_t blk, uint8_t* __restrict__ codes,
                                                    uint8_t* __restrict__ scales) {
   float amax = 0.0f;
 #pragma unroll
   for (int k = 0; k < 16; ++k) amax = fmaxf(amax, fabsf(y[k]));
-  const BlockScale bs = block_scale(amax, s_t);
+  const BlockScale bs = block_scale_f32(amax, s_t, tab);
+  const f32x2 inv2 = pack2(bs.inv, bs.inv);
   float v[16];
 #pragma unroll
-  for (int k = 0; k < 16; ++k) v[k] = __fmul_rn(y[k], bs.inv);
+  for (int k = 0; k < 8; ++k) unpack2(mul2(pack2(y[2 * k], y[2 * k + 1]), inv2), v[2 * k], v[2 * k + 1]);
   reinterpret_cast<uint2*>(codes)[blk] = pack_codes16(v);
   scales[blk] = (uint8_t)bs.sb;
 }
@@ -99,21 +148,25 @@ __global__ void __launch_bounds__(kThreads, kRhtCtasPerSm)
                    uint8_t* __restrict__ scales, float* __restrict__ tensor_scale,
                    float* __restrict__ y_out) {
   __shared__ uint32_t masks[16];
+  __shared__ ScaleTables tab;
   load_sign_masks(masks, seed_lo, seed_hi);
   const float s_t = tensor_scale_from_amax(__uint_as_float(ws[0]));
   if (blockIdx.x == 0 && threadIdx.x == 0) *tensor_scale = s_t;
+  scale_tables_init_f32(tab, s_t);
+  const f32x2 c2 = pack2(kInvSqrt32, kInvSqrt32);
   const int64_t stride = (int64_t)gridDim.x * kThreads;
   for (int64_t g = (int64_t)blockIdx.x * kThreads + threadIdx.x; g < ngroups; g += stride) {
+    f32x2 P[16];
+    hadamard32(x + g * 32, masks, P);
     float z[32];
-    hadamard32(x + g * 32, masks, z);
 #pragma unroll
-    for (int k = 0; k < 32; ++k) z[k] = __fmul_rn(z[k], kInvSqrt32);
+    for (int m = 0; m < 16; ++m) unpack2(mul2(P[m], c2), z[2 * m], z[2 * m + 1]);
     if (y_out != nullptr) {
 #pragma unroll
       for (int q = 0; q < 4; ++q) st_v8f(y_out + g * 32 + 8 * q, z + 8 * q);
     }
-    quantize_block_f32(z, s_t, 2 * g, codes, scales);
-    quantize_block_f32(z + 16, s_t, 2 * g + 1, codes, scales);
+    quantize_block_f32(z, s_t, tab, 2 * g, codes, scales);
+    quantize_block_f32(z + 16, s_t, tab, 2 * g + 1, codes, scales);
   }
 }
 

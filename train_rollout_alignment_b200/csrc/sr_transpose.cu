@@ -86,10 +86,14 @@ __global__ void __launch_bounds__(kThreads)
                    uint8_t* __restrict__ codes_t, uint8_t* __restrict__ scales_t,
                    float* __restrict__ ts_t) {
   __shared__ float ys[kTile][kYStride];
+  __shared__ ScaleTables tab;
   const int64_t e = blockIdx.z;
   const int64_t r0 = (int64_t)blockIdx.y * kTile, c0 = (int64_t)blockIdx.x * kTile;
   const int t = threadIdx.x;
   const float s_in = __ldg(ts + e);
+  const float A = __fmul_rn(__uint_as_float(ws[e]), s_in);
+  const float s_t = tensor_scale_from_amax(A);
+  scale_tables_init_f32(tab, s_t);
   {
     // dequantize: thread t takes 16 values (one source block) of tile row t / 4
     const int row = t >> 2, chunk = t & 3;
@@ -114,8 +118,6 @@ __global__ void __launch_bounds__(kThreads)
   }
   __syncthreads();
 
-  const float A = __fmul_rn(__uint_as_float(ws[e]), s_in);
-  const float s_t = tensor_scale_from_amax(A);
   if (blockIdx.x == 0 && blockIdx.y == 0 && t == 0) ts_t[e] = s_t;
 
   // warp w: 16 rows (16 * (w % 4)) of 32 consecutive columns (32 * (w / 4))
@@ -130,7 +132,7 @@ __global__ void __launch_bounds__(kThreads)
     y[k] = ys[rb * 16 + k][cl];
     amax = fmaxf(amax, fabsf(y[k]));
   }
-  const BlockScale bs = block_scale(amax, s_t);
+  const BlockScale bs = block_scale_f32(amax, s_t, tab);
   const uint64_t obase = ((uint64_t)e * (uint64_t)cols + (uint64_t)c) * (uint64_t)rows + (uint64_t)rbase;
   const uint32_t ctr_hi = (uint32_t)(obase >> 32);  // obase % 16 == 0: the 16 counters share it
   float a[16];
