@@ -57,6 +57,21 @@ BYTES = {
 
 
 SPEC_HBM_GBS = 8000.0  # B200 HBM3e data-sheet bandwidth, reported beside the measured peak
+# Philox-bound kernels: each random word costs 18 32x32->64-bit multiplies per
+# element (10 rounds of 2; the first round's product of the shared draw word is
+# computed once, the last round needs one), and a B200 SM retires such
+# multiplies for 32 lanes per clock (measured with an instruction-throughput
+# probe: mul.wide.u32 30.6, mul.hi.u32 31.8 lanes/clk/SM).
+PHILOX_MULS_PER_ELEM = 18
+WIDE_MUL_LANES_PER_CLK = 32
+
+
+def _philox_roofline(elems_per_s, sms, sm_mhz):
+    peak = sms * sm_mhz * 1e6 * WIDE_MUL_LANES_PER_CLK / PHILOX_MULS_PER_ELEM
+    return {"bound": "alu", "unit": "elements/s", "achieved": round(elems_per_s, 1), "peak": round(peak, 1),
+            "frac": round(elems_per_s / peak, 4),
+            "basis": "%d Philox wide multiplies per element at %d lanes/clk/SM, %d SMs, %.0f MHz"
+                     % (PHILOX_MULS_PER_ELEM, WIDE_MUL_LANES_PER_CLK, sms, sm_mhz)}
 
 
 def _peaks():
@@ -367,7 +382,8 @@ def run_ours(args, world, rank, local):
     elems = tdist.aggregate_rate(args.steps * step_elems, world, t_max)
 
     # ---- the other rows of the path, each timed alone (rank-local)
-    other = time_other_kernels(b, stack, device, peak)
+    sm_mhz = clocks["sm_max_mhz"] if clocks else 1965.0
+    other = time_other_kernels(b, stack, device, peak, sm_mhz)
 
     # ---- end to end through the C ABI with host buffers (rank-local)
     e2e = run_e2e(b, stack, device, steps=min(args.steps, 2))
@@ -465,7 +481,7 @@ def _timed(fn, reps, flush):
     return statistics.median(times) / 1e3
 
 
-def time_other_kernels(b, stack, device, peak, reps=10):
+def time_other_kernels(b, stack, device, peak, sm_mhz, reps=10):
     """Standalone hint emit (throughput stack, layer 24), SR transpose
     re-quantize (128 x 512 x 2048 expert stack) and RHT32 + quantize
     (16384 x 4096 activation with outliers): seconds per call and algorithmic
@@ -501,10 +517,14 @@ def time_other_kernels(b, stack, device, peak, reps=10):
         "workload": "%dx%dx%d expert stack, one Philox4x32-10 word per element" % (batch, er, ec),
         "avg_us": round(t * 1e6, 2), "GB/s": round(sr_bytes * n / t / 1e9, 1),
         "frac": round(sr_bytes * n / t / 1e9 / peak, 4), "bytes_per_elem": sr_bytes,
-        "elements_per_s": round(n / t, 1)}
+        "elements_per_s": round(n / t, 1),
+        "alu_roofline": _philox_roofline(n / t, torch.cuda.get_device_properties(device).multi_processor_count, sm_mhz)}
     b.nvfp4_sr_transpose_requant(codes, scales, ts, batch, er, ec, syn.CFG2_SR_SEED, 0, ws, ct, st, tst)
     out.update(time_transpose_alternatives(b, stack, w, codes, scales, ts, (ct, st, tst), device, peak, reps,
                                            flush))
+    out["mxfp8_sr_transpose_requant"]["alu_roofline"] = _philox_roofline(
+        out["mxfp8_sr_transpose_requant"]["elements_per_s"], torch.cuda.get_device_properties(device).multi_processor_count,
+        sm_mhz)
     del w, codes, scales, ct, st
     # RHT32 + quantize
     x = torch.from_numpy(syn.cfg3().view(np.int16)).view(torch.bfloat16).to(device)

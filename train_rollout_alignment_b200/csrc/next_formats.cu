@@ -14,16 +14,18 @@ namespace nvfp4 {
 
 // ----------------------------------------------------------------- tile-16 quantize
 // A warp owns 32 horizontally adjacent tiles of one 16-row band (lane j: tile
-// column 32 s + j, i.e. block 32 s + j of each of the 16 rows).  Pass 1
-// streams the band -- each row is read as 1 KiB contiguous across the warp --
-// and keeps each lane's tile maximum in a register (no shuffles).  Pass 2
-// reads the same 16 KiB again, from L2 where pass 1 just left it, and writes
-// the codes (256 contiguous bytes per row) and one scale byte per lane.
+// column 32 s + j, i.e. block 32 s + j of each of the 16 rows).  Each lane
+// loads its 16 blocks (16 x 256-bit loads; every row is read as 1 KiB
+// contiguous across the warp) and keeps them in registers: the tile maximum
+// comes from all 16, then the same registers are quantized -- the band is
+// read from memory once.  128 registers of data per thread, so CTAs are
+// small (128 threads, 3 per SM: 12 warps with 16 KiB each in flight).
 // Bands are visited from the end of the tensor backwards (the amax pass that
 // runs just before streams forwards, so its tail is still in L2).
-constexpr int kTileRowsInFlight = 8;
+constexpr int kTileThreads = 128;
+constexpr int kTileCtasPerSm = 3;
 
-__global__ void __launch_bounds__(kThreads, 4)
+__global__ void __launch_bounds__(kTileThreads, kTileCtasPerSm)
     k_quantize_tile16(const uint16_t* __restrict__ x, int64_t rows, int64_t cols,
                       const uint32_t* __restrict__ ws, uint8_t* __restrict__ codes,
                       uint8_t* __restrict__ tscales, float* __restrict__ tensor_scale) {
@@ -33,37 +35,28 @@ __global__ void __launch_bounds__(kThreads, 4)
   scale_tables_init(tab, s_t);
   const int lane = threadIdx.x & 31;
   const int64_t tc = cols / 16, segs = (tc + 31) / 32, nitems = (rows / 16) * segs;
-  const int64_t wstride = (int64_t)gridDim.x * (kThreads / 32);
-  for (int64_t w = (int64_t)blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5); w < nitems;
+  const int64_t wstride = (int64_t)gridDim.x * (kTileThreads / 32);
+  for (int64_t w = (int64_t)blockIdx.x * (kTileThreads / 32) + (threadIdx.x >> 5); w < nitems;
        w += wstride) {
     const int64_t item = nitems - 1 - w;
     const int64_t ti = item / segs, tj = (item % segs) * 32 + lane;
     if (tj >= tc) continue;  // only in the last segment of a band
     const uint16_t* band = x + 16 * ti * cols + 16 * tj;
+    Block16 b[16];
+#pragma unroll
+    for (int r = 0; r < 16; ++r) b[r] = ld_block(band + r * cols);
     uint32_t m = 0u;
-#pragma unroll 1
-    for (int r0 = 0; r0 < 16; r0 += kTileRowsInFlight) {
-      Block16 b[kTileRowsInFlight];
 #pragma unroll
-      for (int u = 0; u < kTileRowsInFlight; ++u) b[u] = ld_block(band + (r0 + u) * cols);
-#pragma unroll
-      for (int u = 0; u < kTileRowsInFlight; ++u) m = max(m, block_amax_bits(b[u]));
-    }
+    for (int r = 0; r < 16; ++r) m = max(m, block_amax_bits(b[r]));
     const BlockScale bs = block_scale_bf16(m, s_t, tab);
     uint2* out = reinterpret_cast<uint2*>(codes + 16 * ti * (cols / 2)) + tj;
-#pragma unroll 1
-    for (int r0 = 0; r0 < 16; r0 += kTileRowsInFlight) {
-      Block16 b[kTileRowsInFlight];
 #pragma unroll
-      for (int u = 0; u < kTileRowsInFlight; ++u) b[u] = ld_block(band + (r0 + u) * cols);
+    for (int r = 0; r < 16; ++r) {
+      float xf[16], v[16];
+      unpack_block(b[r], xf);
 #pragma unroll
-      for (int u = 0; u < kTileRowsInFlight; ++u) {
-        float xf[16], v[16];
-        unpack_block(b[u], xf);
-#pragma unroll
-        for (int k = 0; k < 16; ++k) v[k] = __fmul_rn(xf[k], bs.inv);
-        out[(r0 + u) * (cols / 16)] = pack_codes16(v);
-      }
+      for (int k = 0; k < 16; ++k) v[k] = __fmul_rn(xf[k], bs.inv);
+      out[r * (cols / 16)] = pack_codes16(v);
     }
     tscales[ti * tc + tj] = (uint8_t)bs.sb;
   }
@@ -131,8 +124,6 @@ __global__ void __launch_bounds__(kThreads)
   const int warp = t >> 5, lane = t & 31;
   const int bc = (lane & 7) + 8 * (warp & 1);   // word column: input columns 8 bc ..
   const int br = (lane >> 3) + 4 * (warp >> 1);  // row group: input rows 8 br ..
-  const int64_t cb = c0 + 8 * bc, rb = r0 + 8 * br;
-  if (cb >= cols || rb >= rows) return;  // (both are multiples of 8; cols, rows of 16)
   uint32_t m[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) m[i] = sq[8 * br + i][bc];
@@ -145,9 +136,21 @@ __global__ void __launch_bounds__(kThreads)
   }
 #pragma unroll
   for (int i = 0; i < 8; i += 2) nib_swap(m[i], m[i + 1], 4, 0x0F0F0F0Fu);
-  uint8_t* dst = codes_t + e * (n / 2) + rb / 2;
+  // stage the square transposed (row 8 bc + j = output row, word br), then
+  // write whole output rows with 8-byte stores (a row of codes_t is rows / 2
+  // bytes: a multiple of 8)
+  __syncthreads();
 #pragma unroll
-  for (int j = 0; j < 8; ++j) *reinterpret_cast<uint32_t*>(dst + (cb + j) * (rows / 2)) = m[j];
+  for (int j = 0; j < 8; ++j) sq[8 * bc + j][br] = m[j];
+  __syncthreads();
+  uint8_t* dst = codes_t + e * (n / 2);
+#pragma unroll
+  for (int h = 0; h < 4; ++h) {
+    const int idx = t + kThreads * h, orow = idx >> 3, q = idx & 7;  // 8 bytes = 16 elements
+    const int64_t c = c0 + orow, r = r0 + 16 * q;
+    if (c < cols && r < rows)
+      *reinterpret_cast<uint2*>(dst + c * (rows / 2) + r / 2) = make_uint2(sq[orow][2 * q], sq[orow][2 * q + 1]);
+  }
 }
 
 // ----------------------------------------------------------------- MXFP8 SR transpose
@@ -325,8 +328,8 @@ cudaError_t launch_quantize_tile16(const uint16_t* x, int64_t rows, int64_t cols
                                    uint8_t* codes, uint8_t* tscales, float* tensor_scale,
                                    cudaStream_t s) {
   const int64_t items = (rows / 16) * ((cols / 16 + 31) / 32);  // one warp each
-  const int g = grid_for(items * 32, kThreads, 4);
-  k_quantize_tile16<<<g, kThreads, 0, s>>>(x, rows, cols, ws, codes, tscales, tensor_scale);
+  const int g = grid_for(items * 32, kTileThreads, kTileCtasPerSm);
+  k_quantize_tile16<<<g, kTileThreads, 0, s>>>(x, rows, cols, ws, codes, tscales, tensor_scale);
   return cudaGetLastError();
 }
 

@@ -132,33 +132,6 @@ struct BlockScale {
   float inv;     // 1 / (sb * s_t); 0 when sb decodes to 0 (all codes become +-0)
 };
 
-// a / b rounded to nearest-even (IEEE binary32), for a >= 0 and b > 0, given
-// y = RN(1 / b).  One correction step in the manner of P. Markstein
-// ("Computation of elementary functions on the IBM RISC System/6000
-// processor", IBM J. Res. Dev. 34(1), 1990) brings q within an ulp of a / b;
-// r = RN(a - b q) is then computed with one FMA.  If |r| is below half the
-// spacing of the floats around q, times b, q is the unique nearest float to
-// a / b (RN is monotone and that threshold is itself a float, so a rounded r
-// cannot hide a larger true remainder).  Below a power of two the spacing
-// halves.  Anything else -- a tie, the ends of the exponent range, non-finite
-// operands -- takes the full division.
-__device__ __forceinline__ float div_rn_checked(float a, float b, float y) {
-  if (a == 0.0f) return 0.0f;
-  float q = __fmul_rn(a, y);
-  float r = __fmaf_rn(-q, b, a);
-  q = __fmaf_rn(r, y, q);
-  r = __fmaf_rn(-q, b, a);
-  const uint32_t qb = __float_as_uint(q);
-  const uint32_t qe = qb & 0x7F800000u;
-  float h = __fmul_rn(__uint_as_float(qe - (24u << 23)), b);  // (ulp above q) / 2 * b
-  if ((qb & 0x7FFFFFu) == 0u && r < 0.0f) h = __fmul_rn(h, 0.5f);
-  if (qe > (26u << 23) && qe < (254u << 23) && h >= 0x1p-125f && h <= 0x1p125f && fabsf(r) < h)
-    return q;
-  return __fdiv_rn(a, b);
-}
-
-constexpr float kRcp6 = 1.0f / 6.0f;  // RN(1/6), folded at compile time
-
 // Per-CTA tables for tensors whose block maxima are BF16 values (at most 8
 // significant bits), filled once per CTA from s_t:
 //   inv[b]  = 1 / (E4M3(b) * s_t)        (0 when E4M3(b) == 0), all 128 bytes;
@@ -170,7 +143,6 @@ constexpr float kRcp6 = 1.0f / 6.0f;  // RN(1/6), folded at compile time
 struct ScaleTables {
   float inv[128];
   uint32_t div6[128];
-  float rcp_st;  // RN(1 / s_t)
 };
 
 __device__ __forceinline__ void scale_tables_init(ScaleTables& t, float s_t) {
@@ -180,18 +152,16 @@ __device__ __forceinline__ void scale_tables_init(ScaleTables& t, float s_t) {
     t.inv[i] = (sbv == 0.0f) ? 0.0f : __fdiv_rn(1.0f, __fmul_rn(sbv, s_t));
     t.div6[i] = __float_as_uint(__fdiv_rn(__uint_as_float(0x3F800000u | ((uint32_t)i << 16)), kE2M1Max));
   }
-  if (i == 0) t.rcp_st = __fdiv_rn(1.0f, s_t);
   __syncthreads();
 }
 
-// The part of the tables that FP32 block maxima need (inv and 1 / s_t).
+// The part of the tables that FP32 block maxima need (inv only).
 __device__ __forceinline__ void scale_tables_init_f32(ScaleTables& t, float s_t) {
   const int i = threadIdx.x;
   if (i < 128) {
     const float sbv = e4m3_value((uint32_t)i);
     t.inv[i] = (sbv == 0.0f) ? 0.0f : __fdiv_rn(1.0f, __fmul_rn(sbv, s_t));
   }
-  if (i == 0) t.rcp_st = __fdiv_rn(1.0f, s_t);
   __syncthreads();
 }
 
@@ -212,12 +182,12 @@ __device__ __forceinline__ BlockScale block_scale_bf16(uint32_t amax_bits, float
   return r;
 }
 
-// The same block scale for any FP32 amax (both divisions by div_rn_checked).
+// The same block scale for any FP32 amax (two divisions; inv from the table).
 __device__ __forceinline__ BlockScale block_scale_f32(float amax_b, float s_t,
                                                       const ScaleTables& t) {
   BlockScale r;
-  const float q = div_rn_checked(amax_b, kE2M1Max, kRcp6);
-  r.sb = e4m3_rn_satfinite(div_rn_checked(q, s_t, t.rcp_st));
+  const float q = __fdiv_rn(amax_b, kE2M1Max);
+  r.sb = e4m3_rn_satfinite(__fdiv_rn(q, s_t));
   r.inv = t.inv[r.sb & 0x7Fu];
   return r;
 }
