@@ -36,8 +36,6 @@ __device__ __forceinline__ void st_v8f(float* p, const float* v) {
                : "memory");
 }
 
-__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
-__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
 // BF16 -> FP32 with the mixed-precision add of sm_100 (x + -0 == x for every
 // x, signed zeros included), which runs on the FP pipes instead of the
@@ -256,11 +254,6 @@ __device__ __forceinline__ uint32_t nib_nonzero(uint32_t t) {  // nibble != 0
   t |= t >> 1;
   t |= t >> 2;
   return t & 0x11111111u;
-}
-__device__ __forceinline__ uint32_t nib_zero(uint32_t t) {  // nibble == 0
-  t |= t >> 1;
-  t |= t >> 2;
-  return ~t & 0x11111111u;
 }
 // Number of flags set (multiply-add instead of popc, which is a slow pipe).
 __device__ __forceinline__ uint32_t count_nib(uint32_t m) { return (m * 0x11111111u) >> 28; }
