@@ -385,6 +385,8 @@ def run_ours(args, world, rank, local):
     sm_mhz = clocks["sm_max_mhz"] if clocks else 1965.0
     other = time_other_kernels(b, stack, device, peak, sm_mhz)
 
+    other["hint_transport"] = time_hint_transport(stack, device)
+
     # ---- end to end through the C ABI with host buffers (rank-local)
     e2e = run_e2e(b, stack, device, steps=min(args.steps, 2))
 
@@ -623,6 +625,39 @@ def time_transpose_alternatives(b, stack, w, codes, scales, ts, sr_out, device, 
                        % (batch, er, ec))
     out["transpose_quality"] = quality
     return out
+
+
+def time_hint_transport(stack, device, reps=5):
+    """The guidance that leaves the GPU in one step: the back-half layers'
+    hints copied to pinned host memory on a copy stream (one copy per layer),
+    median of `reps` transfers; with its size against the uncompacted NVFP4 of
+    the same layers (4 + 0.5 bits per element)."""
+    hinted = [l for l in range(stack.layers) if stack.hints[l] is not None]
+    nbytes = sum(stack.hints[l].numel() for l in hinted)
+    host = torch.empty(nbytes, dtype=torch.uint8).pin_memory()
+    copy = torch.cuda.Stream(device)
+    times = []
+    for _ in range(reps):
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(copy):
+            e0.record(copy)
+            off = 0
+            for l in hinted:
+                n = stack.hints[l].numel()
+                host[off:off + n].copy_(stack.hints[l], non_blocking=True)
+                off += n
+            e1.record(copy)
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1) / 1e3)
+    t = statistics.median(times)
+    uncompacted = stack.n * len(hinted) * 4.5 / 8
+    return {"layers": "%d-%d" % (hinted[0], hinted[-1]), "hint_bits": HINT_BITS, "bytes_per_step": nbytes,
+            "seconds": round(t, 5), "d2h_GB/s": round(nbytes / t / 1e9, 2),
+            "uncompacted_nvfp4_bytes": int(uncompacted), "compaction": round(nbytes / uncompacted, 4),
+            "context": "the TRACE explainer sizes guidance transport at 300 GB/s GPU->CPU (GB200); "
+                       "this is the B200 host link with pinned memory"}
 
 
 def run_e2e(b, stack, device, steps):
