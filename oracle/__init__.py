@@ -83,6 +83,8 @@ def _load():
                 "oracle_mxfp8_sr_transpose_requant_from": (
                     None, [P, P, P, I64, I64, I64, I64, ctypes.c_uint64, ctypes.c_uint32, P, P]),
                 "oracle_mxfp8_dequant": (None, [P, P, I64, P]),
+                "oracle_quantize_rtn_rows_bf16": (None, [P, I64, I64, P, P, P, P, ctypes.c_int]),
+                "oracle_guided_rows_bf16": (None, [P, I64, I64, P, ctypes.c_int, P, P, P, P]),
                 "oracle_rht_signs": (None, [ctypes.c_uint64, P]),
                 "oracle_rht32_f64": (None, [P, I64, I64, ctypes.c_uint64, P]),
                 "oracle_rht_quantize": (None, [P, I64, I64, ctypes.c_uint64, P, P, P, P]),
@@ -218,6 +220,37 @@ def guided_requant(x, hints, hint_bits: int, A: float | None = None):
     _load().oracle_guided_bf16(_ptr(x), rows, cols, float(A), hp, int(hint_bits), _ptr(codes),
                                _ptr(scales), _ptr(ts), _ptr(stats))
     return codes, scales, float(ts[0]), stats
+
+
+def quantize_rtn_rows(x, hint_bits: int = 0):
+    """KV-cache layout: every row of BF16 [rows, cols] is its own tensor ->
+    (codes, scales, row_scales [rows], hints or None)."""
+    x = _u16(x)
+    rows, cols = x.shape
+    codes = np.zeros((rows, cols // 2), np.uint8)
+    scales = np.zeros((rows, cols // 16), np.uint8)
+    rs = np.zeros(rows, np.float32)
+    hints = np.zeros((rows * cols * hint_bits + 7) // 8, np.uint8) if hint_bits else None
+    _load().oracle_quantize_rtn_rows_bf16(_ptr(x), rows, cols, _ptr(codes), _ptr(scales), _ptr(rs),
+                                          _ptr(hints) if hints is not None else None, int(hint_bits))
+    return codes, scales, rs, hints
+
+
+def guided_requant_rows(x, hints, hint_bits: int):
+    """KV-cache layout, train side -> (codes, scales, row_scales, stats4)."""
+    x = _u16(x)
+    rows, cols = x.shape
+    codes = np.zeros((rows, cols // 2), np.uint8)
+    scales = np.zeros((rows, cols // 16), np.uint8)
+    rs = np.zeros(rows, np.float32)
+    stats = np.zeros(4, np.uint64)
+    hp = None
+    if hints is not None:
+        hints = np.ascontiguousarray(hints, dtype=np.uint8)
+        hp = _ptr(hints)
+    _load().oracle_guided_rows_bf16(_ptr(x), rows, cols, hp, int(hint_bits), _ptr(codes), _ptr(scales),
+                                    _ptr(rs), _ptr(stats))
+    return codes, scales, rs, stats
 
 
 def dequant_one(code: int, scale_byte: int, s_t: float) -> float:

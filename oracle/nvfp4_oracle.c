@@ -306,6 +306,39 @@ void oracle_guided_bf16(const uint16_t* x, int64_t rows, int64_t cols, float A,
     }
 }
 
+/* KV-cache layout ([TRACE], hyper-parameter table: the rollout keeps the KV
+ * cache in FP4 as well).  Reading: a cache entry is written one token at a
+ * time, so no tensor-wide amax exists when it is quantized; each row of the
+ * [tokens x heads, head_dim] cache (one token's vector for one head) is its
+ * own tensor, with its own FP32 scale amax_row / 2688 and blocks of 16 along
+ * head_dim.  So these are the tensor quantizers applied row by row; the hints
+ * of row r start at byte r * cols * bits / 8 of the stream (blocks never
+ * straddle rows).  row_scales: one float per row. */
+void oracle_quantize_rtn_rows_bf16(const uint16_t* x, int64_t rows, int64_t cols, uint8_t* codes,
+                                   uint8_t* scales, float* row_scales, uint8_t* hints,
+                                   int hint_bits)
+{
+    for (int64_t r = 0; r < rows; ++r) {
+        const uint16_t* xr = x + r * cols;
+        float A = oracle_amax_bf16(xr, cols);
+        oracle_quantize_rtn_bf16(xr, 1, cols, A, codes + r * cols / 2, scales + r * cols / 16,
+                                 row_scales + r, hints ? hints + r * cols * hint_bits / 8 : NULL,
+                                 hint_bits);
+    }
+}
+
+void oracle_guided_rows_bf16(const uint16_t* x, int64_t rows, int64_t cols, const uint8_t* hints,
+                             int hint_bits, uint8_t* codes, uint8_t* scales, float* row_scales,
+                             uint64_t* stats4)
+{
+    for (int64_t r = 0; r < rows; ++r) {
+        const uint16_t* xr = x + r * cols;
+        float A = oracle_amax_bf16(xr, cols);
+        oracle_guided_bf16(xr, 1, cols, A, hints ? hints + r * cols * hint_bits / 8 : NULL, hint_bits,
+                           codes + r * cols / 2, scales + r * cols / 16, row_scales + r, stats4);
+    }
+}
+
 /* Decoded value of element i: sign * ((G[m] * sb) * s_t) in FP32; the first
  * product is exact (2 x 4 significant bits).  [RLQ], shared-convention
  * paragraph: a code means code value times scale (code 3 with scale 0.1 is
