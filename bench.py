@@ -386,6 +386,7 @@ def run_ours(args, world, rank, local):
     other = time_other_kernels(b, stack, device, peak, sm_mhz)
 
     other["hint_transport"] = time_hint_transport(stack, device)
+    other.update(time_kv_rows(b, device, peak))
 
     # ---- end to end through the C ABI with host buffers (rank-local)
     e2e = run_e2e(b, stack, device, steps=min(args.steps, 2))
@@ -624,6 +625,38 @@ def time_transpose_alternatives(b, stack, w, codes, scales, ts, sr_out, device, 
                        "the forward's quantized W (the last row quantizes the BF16 W^T directly, for reference)"
                        % (batch, er, ec))
     out["transpose_quality"] = quality
+    return out
+
+
+def time_kv_rows(b, device, peak, reps=10):
+    """KV-cache layout (one FP32 scale per (token, head) row): a cache of
+    65536 tokens x 16 heads x 128 (head_dim), the rollout's RTN + 2-bit hints
+    and the train side's guided re-quantization, each the median of `reps`
+    calls with an L2 flush before each."""
+    tokens, heads, dim = 65536, 16, 128
+    rows = tokens * heads
+    n = rows * dim
+    gen = torch.Generator(device=device).manual_seed(6)
+    xt = (torch.randn((rows, dim), device=device, generator=gen)
+          * torch.exp(torch.empty((1, dim), device=device).uniform_(np.log(0.1), np.log(10.0), generator=gen)))
+    xt = xt.to(torch.bfloat16)
+    xr = (xt.float() * (1 + torch.randn(xt.shape, device=device, generator=gen) * 2.0 ** -8)).to(torch.bfloat16)
+    u8 = dict(dtype=torch.uint8, device=device)
+    cr, sr_, rr = torch.empty(n // 2, **u8), torch.empty(n // 16, **u8), torch.empty(rows, dtype=torch.float32, device=device)
+    ct, st_, rt = torch.empty(n // 2, **u8), torch.empty(n // 16, **u8), torch.empty(rows, dtype=torch.float32, device=device)
+    h = torch.empty(n * HINT_BITS // 8, **u8)
+    s4 = torch.zeros(4, dtype=torch.int64, device=device)
+    flush = (torch.zeros(64 << 20, dtype=torch.float32, device=device),
+             torch.ones(64 << 20, dtype=torch.float32, device=device))
+    t_r = _timed(lambda r: b.nvfp4_quantize_rtn_rows(xr, cr, sr_, rr, h, HINT_BITS), reps, flush)
+    t_t = _timed(lambda r: b.nvfp4_guided_requant_rows(xt, h, HINT_BITS, ct, st_, rt, s4), reps, flush)
+    nb = 2 + 0.5 + 1 / 16 + HINT_BITS / 8 + 4 / dim  # BF16 in; codes, scales, hints, row scale
+    work = "KV cache %d tokens x %d heads x %d, one FP32 scale per row, 2-bit hints" % (tokens, heads, dim)
+    out = {}
+    for name, t in (("kv_rows_rollout_rtn+hint", t_r), ("kv_rows_train_guided+hint", t_t)):
+        gbs = nb * n / t / 1e9
+        out[name] = {"workload": work, "avg_us": round(t * 1e6, 2), "GB/s": round(gbs, 1),
+                     "frac": round(gbs / peak, 4), "bytes_per_elem": nb, "elements_per_s": round(n / t, 1)}
     return out
 
 

@@ -261,6 +261,36 @@ nvfp4_status nvfp4_sr_transpose_requant_noalloc(const uint8_t* codes, const uint
                                                 float* tensor_scale_t, void* stream);
 
 /* ======================================================================
+ * KV-cache layout: one FP32 scale per row.
+ * ====================================================================== */
+
+/*
+ * nvfp4_quantize_rtn_rows / nvfp4_guided_requant_rows -- the rollout and
+ * train quantizers for a KV cache [tokens x heads, head_dim].
+ *   [TRACE], hyper-parameter table: the rollout keeps the KV cache in FP4 as
+ *   well.  A cache entry is written one token at a time, so no tensor-wide
+ *   amax exists when it is quantized: every row (one token's vector for one
+ *   head) is its own tensor, with its own FP32 scale s_row = amax_row / 2688
+ *   (1 for an all-zero row) and 16-value blocks along head_dim, quantized
+ *   exactly as nvfp4_quantize_rtn / nvfp4_guided_requant quantize a
+ *   one-row tensor (same rounding, hints and guidance rules).
+ *   x_bf16 [rows, cols], cols = head_dim in {16, 32, 64, 128, 256, 512}
+ *   (NVFP4_ERR_SHAPE otherwise); codes [rows, cols/2], scales [rows, cols/16],
+ *   row_scales [rows] floats; hints laid out as for the tensor calls (the
+ *   hints of row r start at byte r * cols * bits / 8).  No scratch: the row
+ *   amax is reduced inside the kernel.  stats4 as in nvfp4_guided_requant
+ *   (added to).  Non-finite inputs: outputs unspecified (there is no warning
+ *   word on this path).
+ */
+nvfp4_status nvfp4_quantize_rtn_rows(const uint16_t* x_bf16, int64_t rows, int64_t cols,
+                                     uint8_t* codes, uint8_t* scales, float* row_scales,
+                                     uint8_t* hints, int hint_bits, void* stream);
+nvfp4_status nvfp4_guided_requant_rows(const uint16_t* x_bf16, int64_t rows, int64_t cols,
+                                       const uint8_t* hints, int hint_bits, uint8_t* codes,
+                                       uint8_t* scales, float* row_scales, uint64_t* stats4,
+                                       void* stream);
+
+/* ======================================================================
  * Alternatives to nvfp4_sr_transpose_requant that [TML4] weighs
  * (forward/backward mismatch paragraph and format table).
  * ====================================================================== */

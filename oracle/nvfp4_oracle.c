@@ -141,7 +141,10 @@ int oracle_block_scale(float amax_block, float s_t)
 }
 
 /* Step 3: the per-element scaled value v = x * (1 / (sb * s_t)), three
- * rounded FP32 operations in that order. */
+ * rounded FP32 operations in that order.  When s_t lies deep in the subnormal
+ * range, 1 / (sb * s_t) overflows to +inf: every nonzero x then scales to
+ * +-inf and saturates, and x = +-0 keeps magnitude 0 (0 * inf would be a
+ * NaN; zero sits on the grid).  Callers skip the product for x == 0. */
 static float scaled_value(float x, float sbv, float s_t)
 {
     float denom = sbv * s_t;
@@ -169,7 +172,8 @@ void oracle_quantize_f32(const float* y, int64_t rows, int64_t cols, float A,
             float sbv = (float)oracle_e4m3_value(sb);
             for (int k = 0; k < 16; ++k) {
                 int m = 0;
-                if (sbv != 0.0f) m = oracle_e2m1_rne(fabsf(scaled_value(blk[k], sbv, s_t)));
+                if (sbv != 0.0f && blk[k] != 0.0f)
+                    m = oracle_e2m1_rne(fabsf(scaled_value(blk[k], sbv, s_t)));
                 nibble_put(codes, r * cols + b * 16 + k, (sign_of(blk[k]) << 3) | m);
             }
         }
@@ -264,7 +268,7 @@ void oracle_guided_bf16(const uint16_t* x, int64_t rows, int64_t cols, float A,
                 int64_t i = r * cols + b * 16 + k;
                 int sgn = sign_of(blk[k]);
                 int m = 0;
-                if (sbv != 0.0f) {
+                if (sbv != 0.0f && blk[k] != 0.0f) {
                     float a = fabsf(scaled_value(blk[k], sbv, s_t));
                     int m_rtn = oracle_e2m1_rne(a);
                     m = m_rtn;
@@ -482,7 +486,7 @@ void oracle_sr_transpose_requant_from(const uint8_t* codes, const uint8_t* scale
                     int64_t local = c * rows + b * 16 + k;
                     int64_t gi = (first + e) * n + local;
                     int m = 0;
-                    if (sbv != 0.0f) {
+                    if (sbv != 0.0f && blk[k] != 0.0f) {
                         uint32_t ctr[4] = {(uint32_t)gi, (uint32_t)((uint64_t)gi >> 32), draw, 0u};
                         uint32_t out[4];
                         oracle_philox4x32_10(ctr, key, out);
@@ -527,7 +531,7 @@ void oracle_quantize_tile16_bf16(const uint16_t* x, int64_t rows, int64_t cols, 
                 for (int64_t c = 16 * tj; c < 16 * tj + 16; ++c) {
                     float xv = oracle_bf16_to_f32(x[r * cols + c]);
                     int m = 0;
-                    if (sbv != 0.0f) m = oracle_e2m1_rne(fabsf(scaled_value(xv, sbv, s_t)));
+                    if (sbv != 0.0f && xv != 0.0f) m = oracle_e2m1_rne(fabsf(scaled_value(xv, sbv, s_t)));
                     nibble_put(codes, r * cols + c, (sign_of(xv) << 3) | m);
                 }
         }

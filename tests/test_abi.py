@@ -29,7 +29,7 @@ def test_header_declares_the_boundary():
             "nvfp4_sr_transpose_requant", "nvfp4_rht_quantize", "nvfp4_mismatch_stats",
             "nvfp4_tensor_amax", "nvfp4_status_string", "nvfp4_quantize_tile16",
             "nvfp4_transpose_tile16", "mxfp8_sr_transpose_requant", "nvfp4_dequantize",
-            "mxfp8_dequantize"}
+            "mxfp8_dequantize", "nvfp4_quantize_rtn_rows", "nvfp4_guided_requant_rows"}
     assert want <= set(_declared())
 
 
@@ -118,3 +118,25 @@ def test_validation_of_the_tile_and_mxfp8_entry_points_without_a_gpu():
     assert x(fake, fake, 48, fake, None) == 3
     assert x(fake, fake, 64, fake + 16, None) == 2
     assert x(fake, fake, 0, None, None) == 0
+
+
+def test_validation_of_the_kv_row_entry_points_without_a_gpu():
+    lib = ctypes.CDLL(_lib_path())
+    P, I64, I = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
+    fake = 1 << 20
+    q = lib.nvfp4_quantize_rtn_rows
+    q.restype = I
+    q.argtypes = [P, I64, I64, P, P, P, P, I, P]
+    assert q(fake, 8, 96, fake, fake, fake, None, 0, None) == 3        # head_dim not a power of two
+    assert q(fake, 8, 1024, fake, fake, fake, None, 0, None) == 3      # head_dim > 512
+    assert q(fake, -1, 128, fake, fake, fake, None, 0, None) == 1
+    assert q(None, 8, 128, fake, fake, fake, None, 0, None) == 1
+    assert q(fake + 16, 8, 128, fake, fake, fake, None, 0, None) == 2
+    assert q(fake, 8, 128, fake, fake, fake + 2, None, 0, None) == 2   # row scales 4-B aligned
+    assert q(fake, 8, 128, fake, fake, fake, fake, 3, None) == 5
+    assert q(fake, 0, 128, None, None, None, None, 0, None) == 0       # empty cache
+    g = lib.nvfp4_guided_requant_rows
+    g.restype = I
+    g.argtypes = [P, I64, I64, P, I, P, P, P, P, P]
+    assert g(fake, 8, 128, fake, 3, fake, fake, fake, None, None) == 5
+    assert g(fake, 8, 128, fake, 2, fake, fake, fake, fake + 4, None) == 2  # stats 8-B aligned

@@ -287,3 +287,52 @@ def test_nonfinite_input_sets_warning_without_fault():
     assert g["ws"][1] & 1
     ok = syn.random_case((8, 64), 2, "normal")
     assert gpu_rtn(ok, 2)["ws"][1] == 0
+
+
+def test_subnormal_tensor_scales_every_path():
+    """Inputs so small that the tensor (or row) scale is an FP32 subnormal and
+    1 / (sb * s_t) overflows to +inf: RTN, hints, guided, the KV rows, the
+    tile quantizer, RHT and SR must all give the oracle's codes (nonzero ->
+    saturated, zero -> +-0)."""
+    b = lib()
+    rng = np.random.default_rng(22)
+    xf = (rng.standard_normal((64, 256)) * 1e-39).astype(np.float32)
+    xf[rng.random(xf.shape) < 0.3] = 0.0
+    xf[1, :3] = [-0.0, 0.0, 1e-40]
+    x = syn.bf16_bits(xf)
+    g = gpu_rtn(x, 2)
+    oc, os_, ot, oh = oracle.quantize_rtn(x, hint_bits=2)
+    assert f32_bits(g["ts"]) == f32_bits(ot) and 0 < ot < 2.0 ** -126
+    assert_codes_equal(g["scales"], os_, "scales")
+    assert_codes_equal(g["codes"], oc, "codes")
+    assert_codes_equal(g["hints"], oh, "hints")
+    gg = gpu_guided(x, oh, 2)
+    gc, gs, gt, gst = oracle.guided_requant(x, oh, 2)
+    assert_codes_equal(gg["codes"], gc, "guided codes")
+    assert list(gg["stats"][:3]) == list(gst[:3])
+    # KV rows: every row its own tensor, each with a subnormal scale
+    xt = dev_bf16(x)
+    rows, cols = x.shape
+    codes, scales, rs = Buf(rows * cols // 2), Buf(rows * cols // 16), Buf(4 * rows, torch.float32)
+    b.nvfp4_quantize_rtn_rows(xt, codes.t, scales.t, rs.t)
+    torch.cuda.synchronize()
+    rc, rsc, rr, _ = oracle.quantize_rtn_rows(x)
+    assert_codes_equal(codes.np(), rc.reshape(-1), "row codes")
+    # tile quantizer
+    tcodes, tsc, tts = Buf(rows * cols // 2), Buf(rows * cols // 256), Buf(4, torch.float32)
+    b.nvfp4_quantize_tile16(xt, torch.zeros(4, dtype=torch.int32, device="cuda"), tcodes.t, tsc.t, tts.t)
+    torch.cuda.synchronize()
+    tc, tt, tst = oracle.quantize_tile16(x)
+    assert_codes_equal(tcodes.np(), tc.reshape(-1), "tile codes")
+    # RHT: the transform of tiny inputs stays tiny
+    gr = gpu_rht(x, 3)
+    qc, qs, qt = oracle.quantize_f32(gr["y"])
+    assert_codes_equal(gr["codes"], qc, "rht codes")
+    # SR transpose with a subnormal tensor scale on the input stack
+    w = syn.random_case((2, 32, 64), 23, "normal")
+    codes2, scales2, ts2 = _rtn_stack(w)
+    ts2 = np.array([1e-44, 2e-45], np.float32)
+    ct, st, tst2 = gpu_sr(codes2, scales2, ts2, 2, 32, 64, 2, 0)
+    oc2, osc2, ots2 = oracle.sr_transpose_requant(codes2, scales2, ts2, 2, 32, 64, 2, 0)
+    assert_codes_equal(st, osc2, "sr scales")
+    assert_codes_equal(ct, oc2, "sr codes")

@@ -312,3 +312,22 @@ def test_mismatch_stats_identity_and_constructed_pairs():
     packed = (b[0::2] | (b[1::2] << 4)).astype(np.uint8)
     st = oracle.mismatch_stats(c, s, t, packed, s, t, 8, 128)
     assert list(st[1:5]) == [1, 0, 1, 6]
+
+
+def test_subnormal_tensor_scale_saturates_nonzero_and_keeps_zeros():
+    """A tensor of BF16 subnormals: s_t = A / 2688 is deep in the FP32
+    subnormal range and 1 / (sb * s_t) overflows to +inf; every nonzero value
+    then takes the top code and zeros keep code sign << 3 (closed form)."""
+    rng = np.random.default_rng(21)
+    xf = (rng.standard_normal((4, 64)) * 1e-39).astype(np.float32)
+    xf[rng.random(xf.shape) < 0.3] = 0.0
+    xf[0, :4] = [-0.0, 0.0, 1e-40, -1e-40]
+    x = syn.bf16_bits(xf)
+    codes, scales, s_t, hints = oracle.quantize_rtn(x, hint_bits=2)
+    assert 0 < s_t < 2.0 ** -126
+    c = _codes(codes, x.size)
+    xb = syn.bf16_to_f32(x).reshape(-1)
+    sign = np.signbit(xb).astype(np.uint8) << 3
+    assert np.array_equal(c, np.where(xb != 0, sign | 7, sign))
+    gc, gs, gt, st = oracle.guided_requant(x, hints, 2)
+    assert np.array_equal(gc, codes) and st[0] == 0  # no rounding decisions

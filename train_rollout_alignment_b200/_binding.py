@@ -36,6 +36,8 @@ _SIGS = {
     "nvfp4_sr_transpose_requant_noalloc": (
         _I, [_P, _P, _P, _I64, _I64, _I64, ctypes.c_uint64, ctypes.c_uint32, _P, _P, _P, _P]),
     "nvfp4_quantize_tile16": (_I, [_P, _I64, _I64, _P, _I, _P, _P, _P, _P]),
+    "nvfp4_quantize_rtn_rows": (_I, [_P, _I64, _I64, _P, _P, _P, _P, _I, _P]),
+    "nvfp4_guided_requant_rows": (_I, [_P, _I64, _I64, _P, _I, _P, _P, _P, _P, _P]),
     "nvfp4_transpose_tile16": (_I, [_P, _P, _I64, _I64, _I64, _P, _P, _P]),
     "mxfp8_sr_transpose_requant": (
         _I, [_P, _P, _P, _I64, _I64, _I64, ctypes.c_uint64, ctypes.c_uint32, _P, _P, _P]),
@@ -201,3 +203,18 @@ def nvfp4_dequantize(codes, scales, tensor_scale, rows, cols, scale_layout, out,
 
 def mxfp8_dequantize(q, e8, n, out, stream=None):
     _check("mxfp8_dequantize", _lib.mxfp8_dequantize(_ptr(q), _ptr(e8), int(n), _ptr(out), _stream(stream)))
+
+
+# ----------------------------------------------------------------- KV-cache rows
+def nvfp4_quantize_rtn_rows(x, codes, scales, row_scales, hints=None, hint_bits=0, stream=None):
+    rows, cols = _rows_cols(x)
+    _check("nvfp4_quantize_rtn_rows", _lib.nvfp4_quantize_rtn_rows(
+        _ptr(x), rows, cols, _ptr(codes), _ptr(scales), _ptr(row_scales), _ptr(hints), int(hint_bits),
+        _stream(stream)))
+
+
+def nvfp4_guided_requant_rows(x, hints, hint_bits, codes, scales, row_scales, stats4=None, stream=None):
+    rows, cols = _rows_cols(x)
+    _check("nvfp4_guided_requant_rows", _lib.nvfp4_guided_requant_rows(
+        _ptr(x), rows, cols, _ptr(hints), int(hint_bits), _ptr(codes), _ptr(scales), _ptr(row_scales),
+        _ptr(stats4), _stream(stream)))

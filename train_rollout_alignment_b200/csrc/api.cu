@@ -190,6 +190,56 @@ nvfp4_status nvfp4_rht_quantize(const uint16_t* x_bf16, int64_t rows, int64_t co
                                               static_cast<cudaStream_t>(stream)));
 }
 
+// ----------------------------------------------------------------- KV-cache rows
+namespace {
+nvfp4_status check_rows(const uint16_t* x, int64_t rows, int64_t cols, const uint8_t* codes,
+                        const uint8_t* scales, const float* row_scales) {
+  if (rows < 0 || cols < 0) return NVFP4_ERR_INVALID_ARG;
+  if (cols != 16 && cols != 32 && cols != 64 && cols != 128 && cols != 256 && cols != 512)
+    return NVFP4_ERR_SHAPE;
+  if (rows > kMaxElems / cols) return NVFP4_ERR_SHAPE;
+  if (rows == 0) return NVFP4_OK;
+  if (!x || !codes || !scales || !row_scales) return NVFP4_ERR_INVALID_ARG;
+  if (!aligned(x, 32) || !aligned(codes, 16) || !aligned(scales, 16) || !aligned(row_scales, 4))
+    return NVFP4_ERR_MISALIGNED;
+  return NVFP4_OK;
+}
+}  // namespace
+
+nvfp4_status nvfp4_quantize_rtn_rows(const uint16_t* x_bf16, int64_t rows, int64_t cols,
+                                     uint8_t* codes, uint8_t* scales, float* row_scales,
+                                     uint8_t* hints, int hint_bits, void* stream) {
+  nvfp4_status st = check_rows(x_bf16, rows, cols, codes, scales, row_scales);
+  if (st != NVFP4_OK || rows == 0) return st;
+  if (hints) {
+    if ((st = check_hint_bits(hint_bits)) != NVFP4_OK) return st;
+    if (!aligned(hints, 16)) return NVFP4_ERR_MISALIGNED;
+  }
+  return from_cuda(nvfp4::launch_quantize_rows(x_bf16, rows, cols, nullptr, hint_bits, false, codes,
+                                               scales, row_scales, hints, nullptr,
+                                               static_cast<cudaStream_t>(stream)));
+}
+
+nvfp4_status nvfp4_guided_requant_rows(const uint16_t* x_bf16, int64_t rows, int64_t cols,
+                                       const uint8_t* hints, int hint_bits, uint8_t* codes,
+                                       uint8_t* scales, float* row_scales, uint64_t* stats4,
+                                       void* stream) {
+  nvfp4_status st = check_rows(x_bf16, rows, cols, codes, scales, row_scales);
+  if (st != NVFP4_OK || rows == 0) return st;
+  if (hints) {
+    if ((st = check_hint_bits(hint_bits)) != NVFP4_OK) return st;
+    if (!aligned(hints, 16)) return NVFP4_ERR_MISALIGNED;
+  }
+  if (stats4 && !aligned(stats4, 8)) return NVFP4_ERR_MISALIGNED;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (!hints)  // no guidance: round-to-nearest
+    return from_cuda(nvfp4::launch_quantize_rows(x_bf16, rows, cols, nullptr, 0, false, codes, scales,
+                                                 row_scales, nullptr, nullptr, s));
+  return from_cuda(nvfp4::launch_quantize_rows(x_bf16, rows, cols, hints, hint_bits, true, codes,
+                                               scales, row_scales, nullptr,
+                                               reinterpret_cast<unsigned long long*>(stats4), s));
+}
+
 // ----------------------------------------------------------------- alternatives to SR transpose
 nvfp4_status nvfp4_quantize_tile16(const uint16_t* x_bf16, int64_t rows, int64_t cols, uint32_t* ws,
                                    int flags, uint8_t* codes, uint8_t* tile_scales,

@@ -45,6 +45,10 @@ cudaError_t launch_dequant_nvfp4(const uint8_t* codes, const uint8_t* scales, co
                                  cudaStream_t s);
 cudaError_t launch_dequant_mxfp8(const uint8_t* q, const uint8_t* e8, int64_t n, float* out,
                                  cudaStream_t s);
+cudaError_t launch_quantize_rows(const uint16_t* x, int64_t rows, int64_t cols, const uint8_t* hints_in,
+                                 int hint_bits, bool guided, uint8_t* codes, uint8_t* scales,
+                                 float* row_scales, uint8_t* hints_out,
+                                 unsigned long long* stats4, cudaStream_t s);
 cudaError_t launch_set_f32(float* dst, float value, cudaStream_t s);
 
 }  // namespace nvfp4

@@ -50,13 +50,18 @@ __global__ void __launch_bounds__(kTileThreads, kTileCtasPerSm)
     for (int r = 0; r < 16; ++r) m = max(m, block_amax_bits(b[r]));
     const BlockScale bs = block_scale_bf16(m, s_t, tab);
     uint2* out = reinterpret_cast<uint2*>(codes + 16 * ti * (cols / 2)) + tj;
+    if (inv_overflowed(bs.inv)) {
 #pragma unroll
-    for (int r = 0; r < 16; ++r) {
-      float xf[16], v[16];
-      unpack_block(b[r], xf);
+      for (int r = 0; r < 16; ++r) out[r * (cols / 16)] = overflow_codes_bf16(b[r]);
+    } else {
 #pragma unroll
-      for (int k = 0; k < 16; ++k) v[k] = __fmul_rn(xf[k], bs.inv);
-      out[r * (cols / 16)] = pack_codes16(v);
+      for (int r = 0; r < 16; ++r) {
+        float xf[16], v[16];
+        unpack_block(b[r], xf);
+#pragma unroll
+        for (int k = 0; k < 16; ++k) v[k] = __fmul_rn(xf[k], bs.inv);
+        out[r * (cols / 16)] = pack_codes16(v);
+      }
     }
     tscales[ti * tc + tj] = (uint8_t)bs.sb;
   }

@@ -219,6 +219,36 @@ __device__ __forceinline__ uint32_t pack_rz8(const float* v) {
   return r;
 }
 
+// A block whose inv = 1 / (sb * s_t) overflowed to +inf (a tensor or row
+// scale deep in the subnormal range): every nonzero x scales to +-inf and
+// saturates (code 7); a zero stays zero (0 * inf would be a NaN, and zero
+// sits on the grid).  Sign from x.  Rare; not on the fast path.
+__device__ __forceinline__ bool inv_overflowed(float inv) { return inv > 3.40282347e38f; }
+
+__device__ __forceinline__ uint32_t overflow_code(uint32_t mag_nonzero, uint32_t sign) {
+  return (sign << 3) | (mag_nonzero ? 7u : 0u);
+}
+__device__ __forceinline__ uint2 overflow_codes_bf16(const Block16& b) {
+  uint32_t out[2] = {0u, 0u};
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const uint32_t w = b.w[k];
+    const uint32_t lo = overflow_code(w & 0x7FFFu, (w >> 15) & 1u);
+    const uint32_t hi = overflow_code(w & 0x7FFF0000u, w >> 31);
+    out[k >> 2] |= (lo | (hi << 4)) << (8 * (k & 3));
+  }
+  return make_uint2(out[0], out[1]);
+}
+__device__ __forceinline__ uint2 overflow_codes_f32(const float* y) {
+  uint32_t out[2] = {0u, 0u};
+#pragma unroll
+  for (int k = 0; k < 16; ++k) {
+    const uint32_t u = __float_as_uint(y[k]);
+    out[k >> 3] |= overflow_code(u & 0x7FFFFFFFu, u >> 31) << (4 * (k & 7));
+  }
+  return make_uint2(out[0], out[1]);
+}
+
 // 16 FP32 values (already multiplied by inv) -> 8 bytes of packed codes.
 __device__ __forceinline__ uint2 pack_codes16(const float* v) {
   return make_uint2(pack_rn8(v), pack_rn8(v + 8));

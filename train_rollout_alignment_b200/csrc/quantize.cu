@@ -65,20 +65,32 @@ __device__ __forceinline__ void hint_store(uint8_t* __restrict__ hints, int64_t 
 
 // ----------------------------------------------------------------- RTN quantize
 template <int HB>
+__device__ __forceinline__ void rtn_block_scaled(const Block16& b, BlockScale bs, int64_t blk,
+                                                 uint8_t* __restrict__ codes,
+                                                 uint8_t* __restrict__ scales,
+                                                 uint8_t* __restrict__ hints) {
+  uint2 c;
+  if (inv_overflowed(bs.inv)) {
+    c = overflow_codes_bf16(b);
+  } else {
+    float x[16];
+    unpack_block(b, x);
+    float v[16];
+#pragma unroll
+    for (int k = 0; k < 16; ++k) v[k] = __fmul_rn(x[k], bs.inv);
+    c = pack_codes16(v);
+  }
+  reinterpret_cast<uint2*>(codes)[blk] = c;
+  scales[blk] = (uint8_t)bs.sb;
+  hint_store<HB>(hints, blk, c);
+}
+
+template <int HB>
 __device__ __forceinline__ void rtn_block(const Block16& b, float s_t, const ScaleTables& tab,
                                           int64_t blk, uint8_t* __restrict__ codes,
                                           uint8_t* __restrict__ scales,
                                           uint8_t* __restrict__ hints) {
-  float x[16];
-  unpack_block(b, x);
-  const BlockScale bs = block_scale_bf16(block_amax_bits(b), s_t, tab);
-  float v[16];
-#pragma unroll
-  for (int k = 0; k < 16; ++k) v[k] = __fmul_rn(x[k], bs.inv);
-  const uint2 c = pack_codes16(v);
-  reinterpret_cast<uint2*>(codes)[blk] = c;
-  scales[blk] = (uint8_t)bs.sb;
-  hint_store<HB>(hints, blk, c);
+  rtn_block_scaled<HB>(b, block_scale_bf16(block_amax_bits(b), s_t, tab), blk, codes, scales, hints);
 }
 
 // Blocks are visited from the END of the tensor backwards: the amax pass that
@@ -170,14 +182,18 @@ __device__ __forceinline__ uint32_t hint_field(const uint8_t* __restrict__ hints
 }
 
 template <int HB>
-__device__ __forceinline__ void guided_block(const Block16& b, uint32_t hw, uint2 h4, float s_t,
-                                             const ScaleTables& tab, int64_t blk,
-                                             uint8_t* __restrict__ codes,
-                                             uint8_t* __restrict__ scales, GuidedCounts& cnt,
-                                             uint32_t one) {
+__device__ __forceinline__ void guided_block_scaled(const Block16& b, uint32_t hw, uint2 h4,
+                                                    BlockScale bs, int64_t blk,
+                                                    uint8_t* __restrict__ codes,
+                                                    uint8_t* __restrict__ scales, GuidedCounts& cnt,
+                                                    uint32_t one) {
+  if (inv_overflowed(bs.inv)) {  // every element saturated or zero: no decision
+    reinterpret_cast<uint2*>(codes)[blk] = overflow_codes_bf16(b);
+    scales[blk] = (uint8_t)bs.sb;
+    return;
+  }
   float x[16];
   unpack_block(b, x);
-  const BlockScale bs = block_scale_bf16(block_amax_bits(b), s_t, tab);
   const uint32_t h1 = HB == 1 ? hint_spread1(hw) : 0u;
   uint32_t out[2];
 #pragma unroll
@@ -201,6 +217,16 @@ __device__ __forceinline__ void guided_block(const Block16& b, uint32_t hw, uint
   }
   reinterpret_cast<uint2*>(codes)[blk] = make_uint2(out[0], out[1]);
   scales[blk] = (uint8_t)bs.sb;
+}
+
+template <int HB>
+__device__ __forceinline__ void guided_block(const Block16& b, uint32_t hw, uint2 h4, float s_t,
+                                             const ScaleTables& tab, int64_t blk,
+                                             uint8_t* __restrict__ codes,
+                                             uint8_t* __restrict__ scales, GuidedCounts& cnt,
+                                             uint32_t one) {
+  guided_block_scaled<HB>(b, hw, h4, block_scale_bf16(block_amax_bits(b), s_t, tab), blk, codes,
+                          scales, cnt, one);
 }
 
 template <int HB, int U>
@@ -241,6 +267,132 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
   if (stats4 != nullptr) {
     const unsigned long long vals[3] = {cnt.consulted, cnt.changed, cnt.outside};
     block_add_u64<3>(vals, stats4, red);
+  }
+}
+
+// ----------------------------------------------------------------- KV-cache rows
+// One FP32 scale per row of [rows, cols] (one token's vector for one head of a
+// KV cache, cols = head_dim), as if every row were its own tensor.  LPR =
+// cols / 16 lanes share a row (one 16-value block each), so a warp covers
+// 32 / LPR rows = 1 KiB of contiguous input per step; the row amax is a
+// shuffle reduction over those lanes.  The block scale takes RN(amax_b / 6)
+// from the per-CTA table of BF16 mantissas; q / s_row and 1 / (sb s_row) are
+// divisions (s_row changes from row to row).  The per-block work is the
+// tensor kernels' own.
+__device__ __forceinline__ BlockScale block_scale_row(uint32_t amax_bits, float s_row,
+                                                      const ScaleTables& t) {
+  const uint32_t e = amax_bits >> 23;
+  float q;
+  if (e >= 4u && e < 255u)
+    q = __uint_as_float(t.div6[(amax_bits >> 16) & 0x7Fu] + ((e - 127u) << 23));
+  else
+    q = __fdiv_rn(__uint_as_float(amax_bits), kE2M1Max);
+  BlockScale r;
+  r.sb = e4m3_rn_satfinite(__fdiv_rn(q, s_row));
+  const float sbv = e4m3_value(r.sb);
+  r.inv = (sbv == 0.0f) ? 0.0f : __fdiv_rn(1.0f, __fmul_rn(sbv, s_row));
+  return r;
+}
+
+
+constexpr int kRowsCtasPerSm = 3;  // 85 registers: two row groups in flight per warp
+
+template <int LPR, int HB, bool GUIDED>
+__global__ void __launch_bounds__(kThreads, kRowsCtasPerSm)
+    k_rows(const uint16_t* __restrict__ x, int64_t rows, const uint8_t* __restrict__ hints_in,
+           uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
+           float* __restrict__ row_scales, uint8_t* __restrict__ hints_out,
+           unsigned long long* __restrict__ stats4, uint32_t one) {
+  __shared__ ScaleTables tab;  // the RN(amax / 6) table; its inv part is not used
+  __shared__ unsigned long long red[3 * 8];
+  scale_tables_init(tab, 1.0f);
+  constexpr int kRpw = 32 / LPR;  // rows per warp step
+  constexpr int kRowsUnroll = 2;
+  const int lane = threadIdx.x & 31, sub = lane / LPR, j = lane % LPR;
+  const int64_t ngroups = (rows + kRpw - 1) / kRpw;
+  const int64_t wstride = (int64_t)gridDim.x * (kThreads / 32);
+  GuidedCounts cnt{0u, 0u, 0u};
+  for (int64_t g0 = (int64_t)blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5); g0 < ngroups;
+       g0 += kRowsUnroll * wstride) {
+    Block16 b[kRowsUnroll];
+    uint32_t hw[kRowsUnroll];
+    uint2 h4[kRowsUnroll];
+#pragma unroll
+    for (int u = 0; u < kRowsUnroll; ++u) {
+      const int64_t row = (g0 + u * wstride) * kRpw + sub;
+      const int64_t blk = row * LPR + j;
+      b[u] = Block16{};
+      hw[u] = 0u;
+      h4[u] = make_uint2(0u, 0u);
+      if (g0 + u * wstride < ngroups && row < rows) {
+        b[u] = ld_block(x + blk * 16);
+        if constexpr (GUIDED) hw[u] = hint_field<HB>(hints_in, blk, h4[u]);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kRowsUnroll; ++u) {
+      const int64_t row = (g0 + u * wstride) * kRpw + sub;
+      const int64_t blk = row * LPR + j;
+      const uint32_t own = block_amax_bits(b[u]);
+      uint32_t m = own;
+#pragma unroll
+      for (int o = 1; o < LPR; o <<= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+      if (g0 + u * wstride >= ngroups || row >= rows) continue;
+      const float s_row = tensor_scale_from_amax(__uint_as_float(m));
+      if (j == 0) row_scales[row] = s_row;
+      const BlockScale bs = block_scale_row(own, s_row, tab);
+      if constexpr (GUIDED)
+        guided_block_scaled<HB>(b[u], hw[u], h4[u], bs, blk, codes, scales, cnt, one);
+      else
+        rtn_block_scaled<HB>(b[u], bs, blk, codes, scales, hints_out);
+    }
+  }
+  if constexpr (GUIDED) {
+    if (stats4 != nullptr) {
+      const unsigned long long vals[3] = {cnt.consulted, cnt.changed, cnt.outside};
+      block_add_u64<3>(vals, stats4, red);
+    }
+  }
+}
+
+template <int LPR>
+cudaError_t launch_rows_lpr(const uint16_t* x, int64_t rows, const uint8_t* hints_in, int hint_bits,
+                            bool guided, uint8_t* codes, uint8_t* scales, float* row_scales,
+                            uint8_t* hints_out, unsigned long long* stats4, cudaStream_t s) {
+  const int64_t groups = (rows + 32 / LPR - 1) / (32 / LPR);
+  const int g = grid_for(groups * 32, kThreads, kRowsCtasPerSm);
+  if (guided) {
+    switch (hint_bits) {
+      case 1: k_rows<LPR, 1, true><<<g, kThreads, 0, s>>>(x, rows, hints_in, codes, scales, row_scales, nullptr, stats4, 1u); break;
+      case 2: k_rows<LPR, 2, true><<<g, kThreads, 0, s>>>(x, rows, hints_in, codes, scales, row_scales, nullptr, stats4, 1u); break;
+      case 4: k_rows<LPR, 4, true><<<g, kThreads, 0, s>>>(x, rows, hints_in, codes, scales, row_scales, nullptr, stats4, 1u); break;
+      default: return cudaErrorInvalidValue;
+    }
+  } else {
+    switch (hints_out ? hint_bits : 0) {
+      case 0: k_rows<LPR, 0, false><<<g, kThreads, 0, s>>>(x, rows, nullptr, codes, scales, row_scales, nullptr, nullptr, 1u); break;
+      case 1: k_rows<LPR, 1, false><<<g, kThreads, 0, s>>>(x, rows, nullptr, codes, scales, row_scales, hints_out, nullptr, 1u); break;
+      case 2: k_rows<LPR, 2, false><<<g, kThreads, 0, s>>>(x, rows, nullptr, codes, scales, row_scales, hints_out, nullptr, 1u); break;
+      case 4: k_rows<LPR, 4, false><<<g, kThreads, 0, s>>>(x, rows, nullptr, codes, scales, row_scales, hints_out, nullptr, 1u); break;
+      default: return cudaErrorInvalidValue;
+    }
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quantize_rows(const uint16_t* x, int64_t rows, int64_t cols, const uint8_t* hints_in,
+                                 int hint_bits, bool guided, uint8_t* codes, uint8_t* scales,
+                                 float* row_scales, uint8_t* hints_out,
+                                 unsigned long long* stats4, cudaStream_t s) {
+  if (rows == 0) return cudaSuccess;
+  switch (cols) {
+    case 16: return launch_rows_lpr<1>(x, rows, hints_in, hint_bits, guided, codes, scales, row_scales, hints_out, stats4, s);
+    case 32: return launch_rows_lpr<2>(x, rows, hints_in, hint_bits, guided, codes, scales, row_scales, hints_out, stats4, s);
+    case 64: return launch_rows_lpr<4>(x, rows, hints_in, hint_bits, guided, codes, scales, row_scales, hints_out, stats4, s);
+    case 128: return launch_rows_lpr<8>(x, rows, hints_in, hint_bits, guided, codes, scales, row_scales, hints_out, stats4, s);
+    case 256: return launch_rows_lpr<16>(x, rows, hints_in, hint_bits, guided, codes, scales, row_scales, hints_out, stats4, s);
+    case 512: return launch_rows_lpr<32>(x, rows, hints_in, hint_bits, guided, codes, scales, row_scales, hints_out, stats4, s);
+    default: return cudaErrorInvalidValue;
   }
 }
 

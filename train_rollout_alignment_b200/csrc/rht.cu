@@ -134,11 +134,15 @@ __device__ __forceinline__ void quantize_block_f32(const float* y, float s_t, co
 #pragma unroll
   for (int k = 0; k < 16; ++k) amax = fmaxf(amax, fabsf(y[k]));
   const BlockScale bs = block_scale_f32(amax, s_t, tab);
-  const f32x2 inv2 = pack2(bs.inv, bs.inv);
-  float v[16];
+  if (inv_overflowed(bs.inv)) {
+    reinterpret_cast<uint2*>(codes)[blk] = overflow_codes_f32(y);
+  } else {
+    const f32x2 inv2 = pack2(bs.inv, bs.inv);
+    float v[16];
 #pragma unroll
-  for (int k = 0; k < 8; ++k) unpack2(mul2(pack2(y[2 * k], y[2 * k + 1]), inv2), v[2 * k], v[2 * k + 1]);
-  reinterpret_cast<uint2*>(codes)[blk] = pack_codes16(v);
+    for (int k = 0; k < 8; ++k) unpack2(mul2(pack2(y[2 * k], y[2 * k + 1]), inv2), v[2 * k], v[2 * k + 1]);
+    reinterpret_cast<uint2*>(codes)[blk] = pack_codes16(v);
+  }
   scales[blk] = (uint8_t)bs.sb;
 }
 

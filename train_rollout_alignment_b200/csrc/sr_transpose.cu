@@ -155,6 +155,10 @@ __global__ void __launch_bounds__(kThreads)
   if (bs.inv == 0.0f) {  // zero block scale: every code is +-0
     out[0] &= 0x88888888u;
     out[1] &= 0x88888888u;
+  } else if (inv_overflowed(bs.inv)) {  // every nonzero y saturates, zeros stay
+    const uint2 o = overflow_codes_f32(y);
+    out[0] = o.x;
+    out[1] = o.y;
   }
   *reinterpret_cast<uint2*>(codes_t + obase / 2) = make_uint2(out[0], out[1]);
   scales_t[obase / 16] = (uint8_t)bs.sb;
