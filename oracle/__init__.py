@@ -88,6 +88,8 @@ def _load():
                 "oracle_rht_signs": (None, [ctypes.c_uint64, P]),
                 "oracle_rht32_f64": (None, [P, I64, I64, ctypes.c_uint64, P]),
                 "oracle_rht_quantize": (None, [P, I64, I64, ctypes.c_uint64, P, P, P, P]),
+                "oracle_gemm_nvfp4": (None, [P, P, F, P, P, F, I64, I64, I64, P, P]),
+                "oracle_scales_to_mma": (None, [P, I64, I64, P]),
             }
             for name, (res, args) in sig.items():
                 fn = getattr(lib, name)
@@ -379,6 +381,38 @@ def rht_quantize(x, seed: int):
     _load().oracle_rht_quantize(_ptr(x), rows, cols, int(seed), _ptr(codes), _ptr(scales), _ptr(ts),
                                 _ptr(y))
     return codes, scales, float(ts[0]), y
+
+
+def gemm_nvfp4(a_codes, a_scales, a_ts: float, b_codes, b_scales, b_ts: float, m: int, n: int,
+               k: int):
+    """D = dec(A) @ dec(B)^T for NVFP4 A [m, k], B [n, k] (row-layout scales).
+
+    -> (d, dabs) float64 [m, n]: D (exact sum, one final rounding) and the
+    same sum of |terms|."""
+    a_codes = np.ascontiguousarray(a_codes, dtype=np.uint8).reshape(-1)
+    b_codes = np.ascontiguousarray(b_codes, dtype=np.uint8).reshape(-1)
+    a_scales = np.ascontiguousarray(a_scales, dtype=np.uint8).reshape(-1)
+    b_scales = np.ascontiguousarray(b_scales, dtype=np.uint8).reshape(-1)
+    assert a_codes.size == m * k // 2 and b_codes.size == n * k // 2
+    assert a_scales.size == m * k // 16 and b_scales.size == n * k // 16
+    d = np.zeros((m, n), np.float64)
+    dabs = np.zeros((m, n), np.float64)
+    _load().oracle_gemm_nvfp4(_ptr(a_codes), _ptr(a_scales), float(a_ts), _ptr(b_codes),
+                              _ptr(b_scales), float(b_ts), m, n, k, _ptr(d), _ptr(dabs))
+    return d, dabs
+
+
+def scales_to_mma(scales, rows: int, sf_cols: int) -> np.ndarray:
+    """Row-layout block scales [rows, sf_cols] -> the 128x4-tiled MMA layout."""
+    scales = np.ascontiguousarray(scales, dtype=np.uint8).reshape(-1)
+    assert scales.size == rows * sf_cols
+    out = np.zeros(mma_scale_bytes(rows, sf_cols), np.uint8)
+    _load().oracle_scales_to_mma(_ptr(scales), rows, sf_cols, _ptr(out))
+    return out
+
+
+def mma_scale_bytes(rows: int, sf_cols: int) -> int:
+    return ((rows + 127) // 128) * ((sf_cols + 3) // 4) * 512
 
 
 # --------------------------------------------------------------------------- helpers

@@ -733,3 +733,59 @@ void oracle_rht_quantize(const uint16_t* x, int64_t rows, int64_t cols, uint64_t
     float A = oracle_amax_f32(y_f32, n);
     oracle_quantize_f32(y_f32, rows, cols, A, codes, scales, tensor_scale);
 }
+
+/* ------------------------------------------------------------------------ */
+/* Rollout producer ([TML4], configuration paragraph and format table: the MoE
+ * forward GEMMs of pre-training and of rollout sampling run in NVFP4).
+ *
+ * D[i][j] = sum_k dec(A)[i][k] * dec(B)[j][k] for A [m, k] and B [n, k], both
+ * NVFP4 with 16-element blocks along k, dec = code value * E4M3(scale) * s_t.
+ * The sum is taken without s_t (each term G_a * sa * G_b * sb is a multiple
+ * of 2^-20 below 2^23 and has at most 12 significant bits) in long double,
+ * whose 64-bit mantissa holds every partial sum exactly for k <= 2^16; the
+ * exact sum is then multiplied once by s_a * s_b and rounded to double.
+ * dabs receives the same with |term|, the scale of any accumulation error. */
+void oracle_gemm_nvfp4(const uint8_t* a_codes, const uint8_t* a_scales, float a_ts,
+                       const uint8_t* b_codes, const uint8_t* b_scales, float b_ts,
+                       int64_t m, int64_t n, int64_t k, double* d, double* dabs)
+{
+    int64_t kb = k / 16;
+    long double st = (long double)a_ts * (long double)b_ts;
+    for (int64_t i = 0; i < m; ++i) {
+        for (int64_t j = 0; j < n; ++j) {
+            long double s = 0.0L, sa = 0.0L;
+            for (int64_t e = 0; e < k; ++e) {
+                int ca = nibble_get(a_codes, i * k + e), cb = nibble_get(b_codes, j * k + e);
+                long double va = (long double)GRID[ca & 7] *
+                                 (long double)oracle_e4m3_value(a_scales[i * kb + e / 16]);
+                long double vb = (long double)GRID[cb & 7] *
+                                 (long double)oracle_e4m3_value(b_scales[j * kb + e / 16]);
+                long double t = va * vb;
+                sa += t;
+                s += ((ca >> 3) ^ (cb >> 3)) ? -t : t;
+            }
+            d[i * n + j] = (double)(s * st);
+            dabs[i * n + j] = (double)(sa * fabsl(st));
+        }
+    }
+}
+
+/* Scale-factor layout read by the block-scaled tensor-core MMA of sm_100
+ * (NVIDIA PTX ISA, tcgen05 block scaling; cuBLAS documentation, 1D block
+ * scaling factors layout).  The [rows, sf_cols] scale matrix (sf_cols =
+ * cols / 16) is cut into tiles of 128 rows x 4 scale columns, 512 bytes each,
+ * tile (rt, kt) at byte (rt * ceil(sf_cols / 4) + kt) * 512; inside a tile the
+ * scale of row r, column c sits at (r % 32) * 16 + (r / 32) * 4 + c.  Rows
+ * padded to 128 and columns to 4 hold zero. */
+void oracle_scales_to_mma(const uint8_t* scales, int64_t rows, int64_t sf_cols, uint8_t* out)
+{
+    int64_t row_tiles = (rows + 127) / 128, col_tiles = (sf_cols + 3) / 4;
+    memset(out, 0, (size_t)(row_tiles * col_tiles * 512));
+    for (int64_t r = 0; r < rows; ++r) {
+        for (int64_t c = 0; c < sf_cols; ++c) {
+            int64_t tile = (r / 128) * col_tiles + c / 4;
+            int64_t rr = r % 128;
+            out[tile * 512 + (rr % 32) * 16 + (rr / 32) * 4 + c % 4] = scales[r * sf_cols + c];
+        }
+    }
+}
