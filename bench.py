@@ -82,6 +82,18 @@ def _peaks():
     return 6650.0, "fallback"
 
 
+# dense FP4 tensor-core peak = measured cuBLAS BF16 burst x the nominal FP4/BF16
+# ratio (9 / 2.25 PFLOP/s)
+FP4_PER_BF16 = 4.0
+
+
+def _fp4_peak_tflops():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        return float(json.load(open(path))["bf16_tflops"]) * FP4_PER_BF16, "measured bf16 burst x 4"
+    return 1590.0 * FP4_PER_BF16, "fallback bf16 x 4"
+
+
 # --------------------------------------------------------------------------- clocks
 CLOCK_QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
                "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -387,6 +399,7 @@ def run_ours(args, world, rank, local):
 
     other["hint_transport"] = time_hint_transport(stack, device)
     other.update(time_kv_rows(b, device, peak))
+    other["rollout_producer"] = time_producer(b, device)
 
     # ---- end to end through the C ABI with host buffers (rank-local)
     e2e = run_e2e(b, stack, device, steps=min(args.steps, 2))
@@ -658,6 +671,57 @@ def time_kv_rows(b, device, peak, reps=10):
         out[name] = {"workload": work, "avg_us": round(t * 1e6, 2), "GB/s": round(gbs, 1),
                      "frac": round(gbs / peak, 4), "bytes_per_elem": nb, "elements_per_s": round(n / t, 1)}
     return out
+
+
+def time_producer(b, device, reps=10, m=8192, n=4096, k=4096):
+    """The fused rollout producer: an NVFP4 activation [m tokens, k] times an
+    NVFP4 weight [n, k] on the tensor cores, the product quantized to NVFP4
+    with 2-bit hints and both scale layouts in the epilogue.  Operands come from
+    the library's own quantizer on synthetic N(0, 1) activations and N(0, 0.02^2)
+    weights; the output tensor scale uses the max |D| recorded by a previous
+    call (delayed scaling).  Median of `reps` calls, L2 flushed before each."""
+    gen = torch.Generator(device=device).manual_seed(8)
+    u8 = dict(dtype=torch.uint8, device=device)
+
+    def nvfp4_operand(rows, std):
+        x = (torch.randn((rows, k), device=device, generator=gen) * std).to(torch.bfloat16)
+        codes, scales, ts, ws, _ = b.empty_nvfp4(rows, k, device)
+        b.nvfp4_quantize_rtn(x, ws, codes, scales, ts)
+        smma = torch.empty(b.mma_scale_bytes(rows, k // 16), **u8)
+        b.nvfp4_scales_to_mma(scales, rows, k // 16, smma)
+        return codes, smma, ts
+
+    a_codes, a_sf, a_ts = nvfp4_operand(m, 1.0)
+    w_codes, w_sf, w_ts = nvfp4_operand(n, 0.02)
+    codes, scales, ts, ws, hints = b.empty_nvfp4(m, n, device, hint_bits=HINT_BITS)
+    smma = torch.empty(b.mma_scale_bytes(m, n // 16), **u8)
+    d = torch.empty((m, n), dtype=torch.float32, device=device)
+    ws.zero_()
+
+    def call(r, d_out=None):
+        b.nvfp4_gemm_quantize(a_codes, a_sf, a_ts, w_codes, w_sf, w_ts, m, n, k, ws, codes, scales, ts,
+                              scales_mma=smma, hints=hints, hint_bits=HINT_BITS, d_out=d_out)
+
+    call(0)
+    torch.cuda.synchronize()
+    ws[0] = ws[2]                       # delayed scaling: the amax this product just produced
+    flush = (torch.zeros(64 << 20, dtype=torch.float32, device=device),
+             torch.ones(64 << 20, dtype=torch.float32, device=device))
+    t = _timed(call, reps, flush)
+    t_d = _timed(lambda r: call(r, d), reps, flush)
+    warn = int(ws[1].item())
+    peak, basis = _fp4_peak_tflops()
+    flops = 2.0 * m * n * k
+    out_bytes = m * n * (0.5 + 1 / 16 + 1 / 16 + HINT_BITS / 8)
+    tf = flops / t / 1e12
+    return {"workload": "NVFP4 [%d tokens x %d] x NVFP4 weight [%d x %d]^T -> NVFP4 + %d-bit hints + "
+                        "tensor-core scale layout" % (m, k, n, k, HINT_BITS),
+            "avg_us": round(t * 1e6, 2), "TFLOP/s": round(tf, 1),
+            "roofline": {"bound": "tensor", "achieved": round(tf, 1), "peak": round(peak, 1),
+                         "unit": "TFLOP/s", "frac": round(tf / peak, 4), "peak_basis": basis},
+            "epilogue_out_bytes": int(out_bytes),
+            "with_fp32_D_written_us": round(t_d * 1e6, 2),
+            "warning_bits": warn}
 
 
 def time_hint_transport(stack, device, reps=5):

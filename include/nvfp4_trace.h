@@ -79,6 +79,8 @@ typedef int nvfp4_status;
 /* Scratch words written by the amax pass and read by the quantize pass. */
 #define NVFP4_WS_WORDS          4   /* ws[0] = bits of A (FP32), ws[1] = warning bits */
 #define NVFP4_WARN_NONFINITE    1u  /* ws[1]: an input was Inf or NaN */
+#define NVFP4_WARN_TIMEOUT      2u  /* ws[1]: a pipeline wait inside nvfp4_gemm_quantize gave
+                                       up (outputs unspecified; the GPU stays usable) */
 
 /* flags */
 #define NVFP4_AMAX_PRECOMPUTED  1   /* ws[0] already holds A (e.g. from nvfp4_tensor_amax) */
@@ -376,6 +378,63 @@ nvfp4_status nvfp4_dequantize(const uint8_t* codes, const uint8_t* scales,
  */
 nvfp4_status mxfp8_dequantize(const uint8_t* q, const uint8_t* e8, int64_t n, float* out,
                               void* stream);
+
+/* ======================================================================
+ * Rollout producer: NVFP4 GEMM on the tensor cores with a quantizing epilogue.
+ * ====================================================================== */
+
+/*
+ * nvfp4_scales_to_mma -- row-layout block scales -> the layout the block-
+ * scaled tensor-core MMA of sm_100 reads (NVIDIA PTX ISA, tcgen05 block
+ * scaling; cuBLAS documentation, 1D block scaling factors layout).
+ *   scales [rows, sf_cols] bytes (sf_cols = cols / 16 of the NVFP4 tensor).
+ *   scales_mma: ceil(rows / 128) * ceil(sf_cols / 4) tiles of 512 bytes; tile
+ *   (rt, kt) at byte (rt * ceil(sf_cols / 4) + kt) * 512 holds rows
+ *   128 rt .. 128 rt + 127 and scale columns 4 kt .. 4 kt + 3, the scale of
+ *   (row r, column c) at (r % 32) * 16 + ((r % 128) / 32) * 4 + c % 4; padding
+ *   (rows past `rows`, columns past `sf_cols`) is written as 0.  scales_mma
+ *   16-byte aligned.  Any rows, sf_cols >= 0.
+ */
+nvfp4_status nvfp4_scales_to_mma(const uint8_t* scales, int64_t rows, int64_t sf_cols,
+                                 uint8_t* scales_mma, void* stream);
+
+/*
+ * nvfp4_gemm_quantize -- D = s_a s_b (A B^T) on the tensor cores, quantized
+ * to NVFP4 in the epilogue, with the rollout hints of D.
+ *   [TML4], configuration paragraph and format table: the MoE forward GEMMs
+ *   (pre-training and rollout sampling) run in NVFP4, and what they produce
+ *   is sent on in NVFP4; [TRACE] (problem statement): the rollout records a
+ *   few low bits of each code for the trainer.  This is the producer of those
+ *   codes fused into the GEMM, so D never round-trips through HBM.
+ *   A: a_codes [m, k/2] (element 2j in the low nibble), a_scales_mma its block
+ *   scales in the MMA layout of nvfp4_scales_to_mma (rows m, sf_cols k/16),
+ *   a_tensor_scale 1 float (device); B likewise with n rows ([n, k]: the
+ *   weight of y = x W^T).
+ *   Product: the block-scaled MMA's FP32 accumulation of the exact products
+ *   (G_a sa)(G_b sb), then one FP32 multiply by fl(s_a * s_b).  The order and
+ *   internal precision of the accumulation are the hardware's: D is not
+ *   bit-reproducible against a CPU sum, its quantization of D is (same rules
+ *   as nvfp4_quantize_rtn applied to FP32 D).
+ *   Output tensor scale: one pass cannot know max |D| before quantizing, so
+ *   ws[0] must hold the FP32 bits of the amax A_out to use (the previous
+ *   step's, or a calibration); s_t = A_out / 2688 goes to tensor_scale, and
+ *   blocks above 6 * 448 * s_t saturate to scale 448 / code 7.  The call
+ *   clears ws[1..3], records the observed max |D| (FP32 bits) in ws[2] for the
+ *   next call, and sets NVFP4_WARN_TIMEOUT in ws[1] if a pipeline wait gave up.
+ *   Outputs: codes [m, n/2], scales [m, n/16] (row layout), scales_mma
+ *   (nullable: the same scales in the MMA layout, ready for the next GEMM),
+ *   hints (nullable; hint_bits 1, 2 or 4, laid out as nvfp4_emit_hint's),
+ *   d_out (nullable: FP32 D [m, n], for checking).
+ *   Shapes: m % 128 == 0, n % 128 == 0, k % 256 == 0 and k > 0
+ *   (NVFP4_ERR_SHAPE); m or n == 0 only writes tensor_scale.  d_out 32-byte
+ *   aligned, every other pointer 16 (tensor scales 4).  Runs on sm_100 only.
+ */
+nvfp4_status nvfp4_gemm_quantize(const uint8_t* a_codes, const uint8_t* a_scales_mma,
+                                 const float* a_tensor_scale, const uint8_t* b_codes,
+                                 const uint8_t* b_scales_mma, const float* b_tensor_scale,
+                                 int64_t m, int64_t n, int64_t k, uint32_t* ws, uint8_t* codes,
+                                 uint8_t* scales, uint8_t* scales_mma, float* tensor_scale,
+                                 uint8_t* hints, int hint_bits, float* d_out, void* stream);
 
 /* Human-readable name of a status code (static string, never NULL). */
 const char* nvfp4_status_string(nvfp4_status status);

@@ -29,7 +29,8 @@ def test_header_declares_the_boundary():
             "nvfp4_sr_transpose_requant", "nvfp4_rht_quantize", "nvfp4_mismatch_stats",
             "nvfp4_tensor_amax", "nvfp4_status_string", "nvfp4_quantize_tile16",
             "nvfp4_transpose_tile16", "mxfp8_sr_transpose_requant", "nvfp4_dequantize",
-            "mxfp8_dequantize", "nvfp4_quantize_rtn_rows", "nvfp4_guided_requant_rows"}
+            "mxfp8_dequantize", "nvfp4_quantize_rtn_rows", "nvfp4_guided_requant_rows",
+            "nvfp4_scales_to_mma", "nvfp4_gemm_quantize"}
     assert want <= set(_declared())
 
 
@@ -140,3 +141,34 @@ def test_validation_of_the_kv_row_entry_points_without_a_gpu():
     g.argtypes = [P, I64, I64, P, I, P, P, P, P, P]
     assert g(fake, 8, 128, fake, 3, fake, fake, fake, None, None) == 5
     assert g(fake, 8, 128, fake, 2, fake, fake, fake, fake + 4, None) == 2  # stats 8-B aligned
+
+
+def test_validation_of_the_producer_entry_points_without_a_gpu():
+    lib = ctypes.CDLL(_lib_path())
+    P, I64, I = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
+    g = lib.nvfp4_gemm_quantize
+    g.restype = I
+    g.argtypes = [P, P, P, P, P, P, I64, I64, I64, P, P, P, P, P, P, I, P, P]
+    f = 1 << 20  # never dereferenced: every call below fails validation first
+
+    def call(m=256, n=256, k=512, a=f, ws=f, codes=f, hints=None, hb=0, d_out=None, ts=f):
+        return g(a, f, f, f, f, f, m, n, k, ws, codes, f, None, ts, hints, hb, d_out, None)
+
+    assert call(m=200) == 3                       # m % 128
+    assert call(n=100) == 3                       # n % 128
+    assert call(k=384) == 3                       # k % 256
+    assert call(k=0) == 3                         # k > 0
+    assert call(m=-128) == 1                      # negative size
+    assert call(ws=None) == 1                     # no scratch
+    assert call(a=None) == 1                      # null operand
+    assert call(codes=f + 8) == 2                 # output codes not 16-B aligned
+    assert call(ws=f + 4) == 2                    # ws not 16-B aligned
+    assert call(d_out=f + 16) == 2                # D output not 32-B aligned
+    assert call(hints=f, hb=3) == 5               # hint_bits not in {1, 2, 4}
+    s2m = lib.nvfp4_scales_to_mma
+    s2m.restype = I
+    s2m.argtypes = [P, I64, I64, P, P]
+    assert s2m(f, -1, 4, f, None) == 1
+    assert s2m(f, 128, 4, f + 8, None) == 2
+    assert s2m(None, 128, 4, f, None) == 1
+    assert s2m(None, 0, 4, None, None) == 0       # empty: nothing to do

@@ -43,6 +43,9 @@ _SIGS = {
         _I, [_P, _P, _P, _I64, _I64, _I64, ctypes.c_uint64, ctypes.c_uint32, _P, _P, _P]),
     "nvfp4_dequantize": (_I, [_P, _P, _P, _I64, _I64, _I, _P, _P]),
     "mxfp8_dequantize": (_I, [_P, _P, _I64, _P, _P]),
+    "nvfp4_scales_to_mma": (_I, [_P, _I64, _I64, _P, _P]),
+    "nvfp4_gemm_quantize": (
+        _I, [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _P, _P, _P, _P, _P, _I, _P, _P]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _fn = getattr(_lib, _name)
@@ -55,6 +58,7 @@ NVFP4_STATS8_WORDS = 8
 NVFP4_STATS4_WORDS = 4
 NVFP4_AMAX_PRECOMPUTED = 1
 NVFP4_WARN_NONFINITE = 1
+NVFP4_WARN_TIMEOUT = 2
 NVFP4_ERR_SCRATCH_LIMIT = 6
 NVFP4_SR_NOALLOC_MAX_BATCH = 4096
 NVFP4_SCALES_BLOCK16 = 0
@@ -218,3 +222,23 @@ def nvfp4_guided_requant_rows(x, hints, hint_bits, codes, scales, row_scales, st
     _check("nvfp4_guided_requant_rows", _lib.nvfp4_guided_requant_rows(
         _ptr(x), rows, cols, _ptr(hints), int(hint_bits), _ptr(codes), _ptr(scales), _ptr(row_scales),
         _ptr(stats4), _stream(stream)))
+
+
+# ----------------------------------------------------------------- rollout producer
+def mma_scale_bytes(rows: int, sf_cols: int) -> int:
+    """Size of the 128x4-tiled tensor-core scale layout of [rows, sf_cols] scales."""
+    return ((rows + 127) // 128) * ((sf_cols + 3) // 4) * 512
+
+
+def nvfp4_scales_to_mma(scales, rows, sf_cols, scales_mma, stream=None):
+    _check("nvfp4_scales_to_mma", _lib.nvfp4_scales_to_mma(
+        _ptr(scales), int(rows), int(sf_cols), _ptr(scales_mma), _stream(stream)))
+
+
+def nvfp4_gemm_quantize(a_codes, a_scales_mma, a_ts, b_codes, b_scales_mma, b_ts, m, n, k, ws, codes,
+                        scales, tensor_scale, scales_mma=None, hints=None, hint_bits=0, d_out=None,
+                        stream=None):
+    _check("nvfp4_gemm_quantize", _lib.nvfp4_gemm_quantize(
+        _ptr(a_codes), _ptr(a_scales_mma), _ptr(a_ts), _ptr(b_codes), _ptr(b_scales_mma), _ptr(b_ts),
+        int(m), int(n), int(k), _ptr(ws), _ptr(codes), _ptr(scales), _ptr(scales_mma), _ptr(tensor_scale),
+        _ptr(hints), int(hint_bits), _ptr(d_out), _stream(stream)))

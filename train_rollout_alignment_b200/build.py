@@ -16,8 +16,8 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libnvfp4trace.so")
 SOURCES = ["api.cu", "quantize.cu", "stats.cu", "sr_transpose.cu", "rht.cu", "noalloc.cu",
-           "next_formats.cu"]
-HEADERS = ["nvfp4_device.cuh", "launch.h"]
+           "next_formats.cu", "producer.cu"]
+HEADERS = ["nvfp4_device.cuh", "launch.h", "umma.cuh"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

@@ -326,4 +326,52 @@ nvfp4_status mxfp8_dequantize(const uint8_t* q, const uint8_t* e8, int64_t n, fl
   return from_cuda(nvfp4::launch_dequant_mxfp8(q, e8, n, out, static_cast<cudaStream_t>(stream)));
 }
 
+nvfp4_status nvfp4_scales_to_mma(const uint8_t* scales, int64_t rows, int64_t sf_cols,
+                                 uint8_t* scales_mma, void* stream) {
+  if (rows < 0 || sf_cols < 0) return NVFP4_ERR_INVALID_ARG;
+  if (rows != 0 && sf_cols > kMaxElems / 16 / rows) return NVFP4_ERR_SHAPE;
+  if (rows == 0 || sf_cols == 0) return NVFP4_OK;
+  if (!scales || !scales_mma) return NVFP4_ERR_INVALID_ARG;
+  if (!aligned(scales_mma, 16)) return NVFP4_ERR_MISALIGNED;
+  return from_cuda(nvfp4::launch_scales_to_mma(scales, rows, sf_cols, scales_mma,
+                                               static_cast<cudaStream_t>(stream)));
+}
+
+nvfp4_status nvfp4_gemm_quantize(const uint8_t* a_codes, const uint8_t* a_scales_mma,
+                                 const float* a_tensor_scale, const uint8_t* b_codes,
+                                 const uint8_t* b_scales_mma, const float* b_tensor_scale,
+                                 int64_t m, int64_t n, int64_t k, uint32_t* ws, uint8_t* codes,
+                                 uint8_t* scales, uint8_t* scales_mma, float* tensor_scale,
+                                 uint8_t* hints, int hint_bits, float* d_out, void* stream) {
+  if (m < 0 || n < 0 || k < 0) return NVFP4_ERR_INVALID_ARG;
+  if (m % 128 != 0 || n % 128 != 0 || k % 256 != 0 || k == 0) return NVFP4_ERR_SHAPE;
+  if (m >= kMaxElems || n >= kMaxElems || k >= (int64_t(1) << 31) ||
+      (m != 0 && n > kMaxElems / m) || (m != 0 && k > kMaxElems / m) ||
+      (n != 0 && k > kMaxElems / n) || m / 128 >= 65536)
+    return NVFP4_ERR_SHAPE;
+  if (!ws || !tensor_scale) return NVFP4_ERR_INVALID_ARG;
+  if (!aligned(ws, 16) || !aligned(tensor_scale, 4)) return NVFP4_ERR_MISALIGNED;
+  if (hints != nullptr) {
+    nvfp4_status st = check_hint_bits(hint_bits);
+    if (st != NVFP4_OK) return st;
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (m == 0 || n == 0)
+    return from_cuda(nvfp4::launch_gemm_quantize(nullptr, nullptr, nullptr, nullptr, nullptr,
+                                                 nullptr, m, n, k, ws, nullptr, nullptr, nullptr,
+                                                 tensor_scale, nullptr, 0, nullptr, s));
+  if (!a_codes || !a_scales_mma || !a_tensor_scale || !b_codes || !b_scales_mma ||
+      !b_tensor_scale || !codes || !scales)
+    return NVFP4_ERR_INVALID_ARG;
+  if (!aligned(a_codes, 16) || !aligned(a_scales_mma, 16) || !aligned(a_tensor_scale, 4) ||
+      !aligned(b_codes, 16) || !aligned(b_scales_mma, 16) || !aligned(b_tensor_scale, 4) ||
+      !aligned(codes, 16) || !aligned(scales, 16) || !aligned(scales_mma, 16) ||
+      !aligned(hints, 16) || !aligned(d_out, 32))
+    return NVFP4_ERR_MISALIGNED;
+  return from_cuda(nvfp4::launch_gemm_quantize(a_codes, a_scales_mma, a_tensor_scale, b_codes,
+                                                b_scales_mma, b_tensor_scale, m, n, k, ws, codes,
+                                                scales, scales_mma, tensor_scale, hints,
+                                                hint_bits, d_out, s));
+}
+
 }  // extern "C"

@@ -1,0 +1,339 @@
+// producer.cu -- the fused rollout producer: an NVFP4 x NVFP4 GEMM on the
+// 5th-generation tensor cores whose epilogue quantizes its own output to
+// NVFP4 (and emits the rollout hints), so the next layer's NVFP4 GEMM reads it
+// directly ("Thinking Machines Lab releases 4-bit training": the MoE forward
+// GEMMs of pre-training and rollout sampling run in NVFP4, and tokens are sent
+// to the experts in NVFP4).
+//
+//   D = s_a s_b * (A B^T)      A [m, k], B [n, k], E2M1 codes with one E4M3
+//                              scale per 16 elements along k
+//   out = NVFP4(D)             codes, row-layout scales, MMA-layout scales,
+//                              hints; tensor scale from a given amax A_out
+//
+// One CTA per 128 x 128 output tile; 128 threads.  Thread 0 streams K-blocks
+// of 256 (A and B tiles by 128-byte-swizzled TMA, their scale tiles by bulk
+// copy) through a 3-stage shared-memory ring; thread 32 copies each stage's
+// scales into TMEM (tcgen05.cp) and issues four 128x128x64 block-scaled MMAs
+// into a 128-column FP32 accumulator in TMEM.  Then all four warps read the
+// accumulator back (warp w owns rows 32w..32w+31, one 16-column NVFP4 block
+// per tcgen05.ld), multiply by s_a s_b and quantize in registers.  Two CTAs
+// fit on an SM (shared memory 110 KB, TMEM 256 columns each), so one CTA's
+// epilogue overlaps the other's main loop.
+//
+// The tensor scale of the output cannot wait for the output's own amax in a
+// single pass; it comes from ws[0] (an amax known beforehand -- the previous
+// step's, or a calibration), and the call records the observed max |D| in
+// ws[2] for the next step.  Blocks above 6 * 448 * s_t saturate.
+#include <cstdint>
+#include <cudaTypedefs.h>
+
+#include "../../include/nvfp4_trace.h"
+#include "launch.h"
+#include "nvfp4_device.cuh"
+#include "umma.cuh"
+
+namespace nvfp4 {
+namespace {
+
+using namespace umma;
+
+constexpr int kBM = 128, kBN = 128;
+constexpr int kBK = 256;                             // elements per K-block (128 bytes)
+constexpr int kStages = 3;
+constexpr int kProducerThreads = 128;
+constexpr uint32_t kTileBytes = kBM * kBK / 2;       // 16 KB for A, same for B (kBN == kBM)
+constexpr uint32_t kScaleTile = 512;                 // 128 rows x 4 scales
+constexpr uint32_t kScaleBytes = (kBK / 64) * kScaleTile;  // 2 KB per operand per stage
+constexpr uint32_t kStageTx = 2 * kTileBytes + 2 * kScaleBytes;
+constexpr uint32_t kTmemCols = 256;  // 128 accumulator + 3 stages x (16 SFA + 16 SFB)
+
+constexpr uint32_t kOffA = 0;
+constexpr uint32_t kOffB = kOffA + kStages * kTileBytes;
+constexpr uint32_t kOffSfa = kOffB + kStages * kTileBytes;
+constexpr uint32_t kOffSfb = kOffSfa + kStages * kScaleBytes;
+constexpr uint32_t kOffBar = kOffSfb + kStages * kScaleBytes;   // full[S], empty[S], accum
+constexpr uint32_t kOffTmemSlot = kOffBar + 8 * (2 * kStages + 1);
+constexpr uint32_t kOffAbort = kOffTmemSlot + 4;
+constexpr uint32_t kOffTables = (kOffAbort + 4 + 15) / 16 * 16;
+constexpr uint32_t kSmemUsed = kOffTables + sizeof(ScaleTables);
+constexpr uint32_t kSmemBytes = kSmemUsed + 1024;    // slack to align the base to 1024
+static_assert(kOffB % 1024 == 0 && kOffSfa % 1024 == 0, "swizzled tiles need 1024-byte bases");
+static_assert(2 * (kSmemBytes + 1024) <= 228 * 1024, "two CTAs per SM");
+
+// Byte offset of scale (row r, scale column c) in the 128x4-tiled MMA layout of
+// a matrix with col_tiles = ceil(sf_cols / 4) scale tiles per 128 rows.
+__device__ __forceinline__ size_t mma_scale_offset(int64_t r, int64_t c, int64_t col_tiles) {
+  const int64_t rr = r & 127;
+  return (size_t)(((r >> 7) * col_tiles + (c >> 2)) * kScaleTile) + (size_t)((rr & 31) * 16) +
+         (size_t)((rr >> 5) * 4) + (size_t)(c & 3);
+}
+
+// ----------------------------------------------------------------- scale layout
+// One thread per 4-byte word (row r, scale tile kt) of the padded MMA layout.
+__global__ void __launch_bounds__(kThreads) k_scales_to_mma(const uint8_t* __restrict__ scales,
+                                                            int64_t rows, int64_t sf_cols,
+                                                            int64_t padded_rows, int64_t col_tiles,
+                                                            uint8_t* __restrict__ out) {
+  const int64_t words = padded_rows * col_tiles;
+  for (int64_t w = (int64_t)blockIdx.x * kThreads + threadIdx.x; w < words;
+       w += (int64_t)gridDim.x * kThreads) {
+    const int64_t r = w / col_tiles, kt = w - r * col_tiles;
+    uint32_t v = 0;
+    if (r < rows) {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int64_t c = kt * 4 + j;
+        if (c < sf_cols) v |= (uint32_t)scales[r * sf_cols + c] << (8 * j);
+      }
+    }
+    *reinterpret_cast<uint32_t*>(out + mma_scale_offset(r, kt * 4, col_tiles)) = v;
+  }
+}
+
+// ----------------------------------------------------------------- GEMM + quantize
+struct ProducerOut {
+  uint8_t* codes;       // [m, n/2]
+  uint8_t* scales;      // [m, n/16]
+  uint8_t* scales_mma;  // MMA layout of the same scales, or null
+  float* tensor_scale;
+  uint8_t* hints;       // null when HB == 0
+  float* d_out;         // FP32 D [m, n], or null
+};
+
+template <int HB>
+__device__ __forceinline__ void store_hint(uint8_t* __restrict__ hints, int64_t blk, uint2 c) {
+  if (HB == 1) reinterpret_cast<uint16_t*>(hints)[blk] = (uint16_t)hint_field1(c);
+  if (HB == 2) reinterpret_cast<uint32_t*>(hints)[blk] = hint_field2(c);
+  if (HB == 4) reinterpret_cast<uint2*>(hints)[blk] = c;
+}
+
+template <int HB>
+__global__ void __launch_bounds__(kProducerThreads, 2)
+    k_gemm_nvfp4_quantize(const __grid_constant__ CUtensorMap tm_a,
+                          const __grid_constant__ CUtensorMap tm_b,
+                          const uint8_t* __restrict__ a_sf, const uint8_t* __restrict__ b_sf,
+                          const float* __restrict__ a_ts, const float* __restrict__ b_ts, int n,
+                          int kblocks, uint32_t* __restrict__ ws, ProducerOut out) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nt = blockIdx.x, mt = blockIdx.y;
+  const uint32_t base = smem_u32(smem);
+  const uint32_t full = base + kOffBar, empty = full + 8 * kStages, accum = empty + 8 * kStages;
+  volatile int* abort = reinterpret_cast<volatile int*>(smem + kOffAbort);
+  ScaleTables& tab = *reinterpret_cast<ScaleTables*>(smem + kOffTables);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(full + 8 * s, 1);
+      mbar_init(empty + 8 * s, 1);
+    }
+    mbar_init(accum, 1);
+    *abort = 0;
+    fence_mbar_init();
+    prefetch_tensormap(&tm_a);
+    prefetch_tensormap(&tm_b);
+  }
+  if (warp == 1) {
+    tmem_alloc(base + kOffTmemSlot, kTmemCols);
+    tc_fence_before();
+  }
+  const float s_t = tensor_scale_from_amax(__uint_as_float(ws[0]));
+  scale_tables_init_f32(tab, s_t);  // ends with __syncthreads
+  tc_fence_after();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + kOffTmemSlot);
+  const int64_t col_tiles_k = (int64_t)kblocks * (kBK / 64);
+
+  if (threadIdx.x == 0) {
+    // ---------------- producer: TMA for the tiles, bulk copies for the scales
+    const uint8_t* sfa = a_sf + (size_t)mt * col_tiles_k * kScaleTile;
+    const uint8_t* sfb = b_sf + (size_t)nt * col_tiles_k * kScaleTile;
+    for (int kb = 0; kb < kblocks; ++kb) {
+      const int s = kb % kStages;
+      const uint32_t ph = (uint32_t)(kb / kStages) & 1u;
+      if (!mbar_wait(empty + 8 * s, ph ^ 1u, abort)) break;
+      const uint32_t bar = full + 8 * s;
+      mbar_arrive_expect_tx(bar, kStageTx);
+      tma_load_2d(base + kOffA + s * kTileBytes, &tm_a, bar, kb * (kBK / 2), mt * kBM);
+      tma_load_2d(base + kOffB + s * kTileBytes, &tm_b, bar, kb * (kBK / 2), nt * kBN);
+      bulk_load(base + kOffSfa + s * kScaleBytes, sfa + (size_t)kb * kScaleBytes, kScaleBytes, bar);
+      bulk_load(base + kOffSfb + s * kScaleBytes, sfb + (size_t)kb * kScaleBytes, kScaleBytes, bar);
+    }
+  } else if (threadIdx.x == 32) {
+    // ---------------- MMA issuer
+    constexpr uint32_t idesc = idesc_nvf4(kBM, kBN);
+    for (int kb = 0; kb < kblocks; ++kb) {
+      const int s = kb % kStages;
+      const uint32_t ph = (uint32_t)(kb / kStages) & 1u;
+      if (!mbar_wait(full + 8 * s, ph, abort)) break;
+      tc_fence_after();
+      const uint32_t sf_cols = tmem + 128u + 32u * (uint32_t)s;  // SFA at +0, SFB at +16
+#pragma unroll
+      for (int j = 0; j < kBK / 64; ++j) {
+        cp_32x128b_warpx4(sf_cols + 4 * j,
+                          desc_scale_chunk(base + kOffSfa + s * kScaleBytes + j * kScaleTile));
+        cp_32x128b_warpx4(sf_cols + 16 + 4 * j,
+                          desc_scale_chunk(base + kOffSfb + s * kScaleBytes + j * kScaleTile));
+      }
+      const uint64_t da = desc_kmajor_sw128(base + kOffA + s * kTileBytes);
+      const uint64_t db = desc_kmajor_sw128(base + kOffB + s * kTileBytes);
+#pragma unroll
+      for (int j = 0; j < kBK / 64; ++j)  // K = 64 = 32 bytes per MMA: start address + 2
+        mma_nvf4(tmem, da + 2 * j, db + 2 * j, idesc, sf_cols + 4 * j, sf_cols + 16 + 4 * j,
+                 (kb | j) != 0);
+      mma_commit(empty + 8 * s);
+    }
+    mma_commit(accum);
+  }
+  __syncwarp();
+
+  // ---------------- epilogue: TMEM -> D -> NVFP4
+  mbar_wait(accum, 0, abort);
+  __syncwarp();  // tcgen05.ld is warp-collective
+  tc_fence_after();
+  const int64_t row = (int64_t)mt * kBM + warp * 32 + lane;
+  const uint32_t t_row = tmem + ((uint32_t)(warp * 32) << 16);
+  const float alpha = __fmul_rn(*a_ts, *b_ts);
+  const int64_t sf_cols_out = n / 16;
+  const int64_t blk0 = row * sf_cols_out + (int64_t)nt * (kBN / 16);
+  if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) *out.tensor_scale = s_t;
+  float dmax = 0.0f;
+  uint64_t sc = 0;  // the tile row's 8 scale bytes, block c16 in byte c16
+#pragma unroll 1
+  for (int c16 = 0; c16 < kBN / 16; ++c16) {
+    float y[16];
+    tmem_ld16(t_row + 16 * c16, y);
+    float amax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      y[i] = __fmul_rn(y[i], alpha);
+      amax = fmaxf(amax, fabsf(y[i]));
+    }
+    dmax = fmaxf(dmax, amax);
+    if (out.d_out != nullptr) {
+      float* dp = out.d_out + row * n + (int64_t)nt * kBN + 16 * c16;
+#pragma unroll
+      for (int q = 0; q < 2; ++q) st_v8f(dp + 8 * q, y + 8 * q);
+    }
+    const BlockScale bs = block_scale_f32(amax, s_t, tab);
+    uint2 c;
+    if (inv_overflowed(bs.inv)) {
+      c = overflow_codes_f32(y);
+    } else {
+      float v[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) v[i] = __fmul_rn(y[i], bs.inv);
+      c = pack_codes16(v);
+    }
+    const int64_t blk = blk0 + c16;
+    reinterpret_cast<uint2*>(out.codes)[blk] = c;
+    sc |= (uint64_t)bs.sb << (8 * c16);
+    if (HB != 0) store_hint<HB>(out.hints, blk, c);
+  }
+  *reinterpret_cast<uint64_t*>(out.scales + blk0) = sc;
+  if (out.scales_mma != nullptr) {
+    const int64_t col_tiles_n = n / 64;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int64_t c = (int64_t)nt * (kBN / 16) + 4 * h;
+      *reinterpret_cast<uint32_t*>(out.scales_mma + mma_scale_offset(row, c, col_tiles_n)) =
+          (uint32_t)(sc >> (32 * h));
+    }
+  }
+  const uint32_t wmax = warp_max_u32(__float_as_uint(dmax));
+  if (lane == 0) atomicMax(ws + 2, wmax);
+
+  tc_fence_before();
+  __syncthreads();
+  if (*abort && threadIdx.x == 0) atomicOr(ws + 1, NVFP4_WARN_TIMEOUT);
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (fn == nullptr) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// [rows, k/2] bytes of packed codes, boxes of 128 rows x 128 bytes, 128-byte swizzle.
+bool codes_tensor_map(CUtensorMap* map, const uint8_t* codes, int64_t rows, int64_t k) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+  if (enc == nullptr) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)(k / 2), (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)(k / 2)};
+  cuuint32_t box[2] = {kBK / 2, kBM};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(codes), dims, strides,
+             box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int HB>
+cudaError_t launch_gemm_hb(const CUtensorMap& ta, const CUtensorMap& tb, const uint8_t* a_sf,
+                           const uint8_t* b_sf, const float* a_ts, const float* b_ts, int64_t m,
+                           int64_t n, int64_t k, uint32_t* ws, const ProducerOut& out,
+                           cudaStream_t s) {
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(k_gemm_nvfp4_quantize<HB>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  const dim3 grid((unsigned)(n / kBN), (unsigned)(m / kBM));
+  k_gemm_nvfp4_quantize<HB><<<grid, kProducerThreads, kSmemBytes, s>>>(
+      ta, tb, a_sf, b_sf, a_ts, b_ts, (int)n, (int)(k / kBK), ws, out);
+  return cudaGetLastError();
+}
+
+__global__ void k_tensor_scale_from_ws(const uint32_t* ws, float* tensor_scale) {
+  *tensor_scale = tensor_scale_from_amax(__uint_as_float(ws[0]));
+}
+
+}  // namespace
+
+cudaError_t launch_scales_to_mma(const uint8_t* scales, int64_t rows, int64_t sf_cols,
+                                 uint8_t* out, cudaStream_t s) {
+  const int64_t padded_rows = (rows + 127) / 128 * 128, col_tiles = (sf_cols + 3) / 4;
+  const int64_t words = padded_rows * col_tiles;
+  if (words == 0) return cudaSuccess;
+  k_scales_to_mma<<<grid_for(words, kThreads, 4), kThreads, 0, s>>>(scales, rows, sf_cols,
+                                                                   padded_rows, col_tiles, out);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gemm_quantize(const uint8_t* a_codes, const uint8_t* a_sf, const float* a_ts,
+                                 const uint8_t* b_codes, const uint8_t* b_sf, const float* b_ts,
+                                 int64_t m, int64_t n, int64_t k, uint32_t* ws, uint8_t* codes,
+                                 uint8_t* scales, uint8_t* scales_mma, float* tensor_scale,
+                                 uint8_t* hints, int hint_bits, float* d_out, cudaStream_t s) {
+  cudaError_t e = cudaMemsetAsync(ws + 1, 0, 3 * sizeof(uint32_t), s);
+  if (e != cudaSuccess) return e;
+  if (m == 0 || n == 0) {
+    k_tensor_scale_from_ws<<<1, 1, 0, s>>>(ws, tensor_scale);
+    return cudaGetLastError();
+  }
+  CUtensorMap ta, tb;
+  if (!codes_tensor_map(&ta, a_codes, m, k) || !codes_tensor_map(&tb, b_codes, n, k))
+    return cudaErrorInvalidValue;
+  const ProducerOut out{codes, scales, scales_mma, tensor_scale, hints, d_out};
+  switch (hints == nullptr ? 0 : hint_bits) {
+    case 1: return launch_gemm_hb<1>(ta, tb, a_sf, b_sf, a_ts, b_ts, m, n, k, ws, out, s);
+    case 2: return launch_gemm_hb<2>(ta, tb, a_sf, b_sf, a_ts, b_ts, m, n, k, ws, out, s);
+    case 4: return launch_gemm_hb<4>(ta, tb, a_sf, b_sf, a_ts, b_ts, m, n, k, ws, out, s);
+    default: return launch_gemm_hb<0>(ta, tb, a_sf, b_sf, a_ts, b_ts, m, n, k, ws, out, s);
+  }
+}
+
+}  // namespace nvfp4
