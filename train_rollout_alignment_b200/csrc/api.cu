@@ -347,7 +347,7 @@ nvfp4_status nvfp4_gemm_quantize(const uint8_t* a_codes, const uint8_t* a_scales
   if (m % 128 != 0 || n % 128 != 0 || k % 256 != 0 || k == 0) return NVFP4_ERR_SHAPE;
   if (m >= kMaxElems || n >= kMaxElems || k >= (int64_t(1) << 31) ||
       (m != 0 && n > kMaxElems / m) || (m != 0 && k > kMaxElems / m) ||
-      (n != 0 && k > kMaxElems / n) || m / 128 >= 65536)
+      (n != 0 && k > kMaxElems / n))
     return NVFP4_ERR_SHAPE;
   if (!ws || !tensor_scale) return NVFP4_ERR_INVALID_ARG;
   if (!aligned(ws, 16) || !aligned(tensor_scale, 4)) return NVFP4_ERR_MISALIGNED;

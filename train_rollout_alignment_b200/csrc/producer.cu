@@ -10,15 +10,17 @@
 //   out = NVFP4(D)             codes, row-layout scales, MMA-layout scales,
 //                              hints; tensor scale from a given amax A_out
 //
-// One CTA per 128 x 128 output tile; 128 threads.  Thread 0 streams K-blocks
-// of 256 (A and B tiles by 128-byte-swizzled TMA, their scale tiles by bulk
-// copy) through a 3-stage shared-memory ring; thread 32 copies each stage's
-// scales into TMEM (tcgen05.cp) and issues four 128x128x64 block-scaled MMAs
-// into a 128-column FP32 accumulator in TMEM.  Then all four warps read the
-// accumulator back (warp w owns rows 32w..32w+31, one 16-column NVFP4 block
-// per tcgen05.ld), multiply by s_a s_b and quantize in registers.  Two CTAs
-// fit on an SM (shared memory 110 KB, TMEM 256 columns each), so one CTA's
-// epilogue overlaps the other's main loop.
+// Persistent and warp-specialized: two CTAs per SM, each walking 128 x 128
+// output tiles.  In a CTA, warp 0 (one lane) streams K-blocks of 256 -- A and
+// B tiles by 128-byte-swizzled TMA, their scale tiles by bulk copy -- through
+// a 3-stage shared-memory ring that runs on across tile boundaries.  Warp 1
+// (one lane) copies each stage's scales into TMEM (tcgen05.cp) and issues four
+// 128x128x64 block-scaled MMAs into a 128-column FP32 accumulator.  Warps
+// 2..5 drain it: warp w owns TMEM lanes 32 (w % 4) .. + 31 (tile rows), one
+// 16-column NVFP4 block per tcgen05.ld, multiply by s_a s_b, quantize in
+// registers and store, handing the accumulator back as soon as its last
+// block is read.  While one CTA's epilogue runs, its producer keeps loading
+// the next tile and the SM's other CTA keeps the tensor core busy.
 //
 // The tensor scale of the output cannot wait for the output's own amax in a
 // single pass; it comes from ws[0] (an amax known beforehand -- the previous
@@ -37,28 +39,58 @@ namespace {
 
 using namespace umma;
 
+// Pipeline shape (compile-time).  Measured on B200 at 8192 x 4096 x 4096:
+// 2 CTAs per SM with 3 stages and one accumulator each (106 us) beat one CTA
+// with 6 stages and two accumulators (148 us) -- two independent
+// producer/MMA pipelines per SM keep more loads in flight than one deeper
+// ring.
+//   STAGES  shared-memory ring depth (K-blocks of 256 in flight per CTA)
+//   ACC     accumulator buffers per CTA (2: a CTA's epilogue overlaps its own
+//           next tile's MMAs; needs TMEM for 2 x 128 columns)
+//   CTAS    resident CTAs per SM
+#ifndef NVFP4_GEMM_STAGES
+#define NVFP4_GEMM_STAGES 3
+#endif
+#ifndef NVFP4_GEMM_ACC
+#define NVFP4_GEMM_ACC 1
+#endif
+#ifndef NVFP4_GEMM_CTAS
+#define NVFP4_GEMM_CTAS 2
+#endif
+
 constexpr int kBM = 128, kBN = 128;
 constexpr int kBK = 256;                             // elements per K-block (128 bytes)
-constexpr int kStages = 3;
-constexpr int kProducerThreads = 128;
+constexpr int kStages = NVFP4_GEMM_STAGES;
+constexpr int kAccBufs = NVFP4_GEMM_ACC;
+constexpr int kCtasPerSm = NVFP4_GEMM_CTAS;
+constexpr int kEpiWarps = 4;
+constexpr int kProducerThreads = 32 * (2 + kEpiWarps);
 constexpr uint32_t kTileBytes = kBM * kBK / 2;       // 16 KB for A, same for B (kBN == kBM)
 constexpr uint32_t kScaleTile = 512;                 // 128 rows x 4 scales
 constexpr uint32_t kScaleBytes = (kBK / 64) * kScaleTile;  // 2 KB per operand per stage
 constexpr uint32_t kStageTx = 2 * kTileBytes + 2 * kScaleBytes;
-constexpr uint32_t kTmemCols = 256;  // 128 accumulator + 3 stages x (16 SFA + 16 SFB)
+// TMEM: accumulator buffer b at column 128 b; then stage s scales at
+// kTmemSfBase + 32 s (SFA +0..15, SFB +16..31)
+constexpr uint32_t kTmemSfBase = kAccBufs * kBN;
+constexpr uint32_t kTmemNeed = kTmemSfBase + 32 * kStages;
+constexpr uint32_t kTmemCols = kTmemNeed <= 32 ? 32 : kTmemNeed <= 64 ? 64 : kTmemNeed <= 128 ? 128
+                               : kTmemNeed <= 256 ? 256 : 512;
+static_assert(kTmemNeed <= 512 && kCtasPerSm * kTmemCols <= 512, "TMEM budget");
 
 constexpr uint32_t kOffA = 0;
 constexpr uint32_t kOffB = kOffA + kStages * kTileBytes;
 constexpr uint32_t kOffSfa = kOffB + kStages * kTileBytes;
 constexpr uint32_t kOffSfb = kOffSfa + kStages * kScaleBytes;
-constexpr uint32_t kOffBar = kOffSfb + kStages * kScaleBytes;   // full[S], empty[S], accum
-constexpr uint32_t kOffTmemSlot = kOffBar + 8 * (2 * kStages + 1);
+// barriers: full[S], empty[S], acc_full[2], acc_empty[2]
+constexpr uint32_t kOffBar = kOffSfb + kStages * kScaleBytes;
+constexpr uint32_t kOffTmemSlot = kOffBar + 8 * (2 * kStages + 2 * kAccBufs);
 constexpr uint32_t kOffAbort = kOffTmemSlot + 4;
 constexpr uint32_t kOffTables = (kOffAbort + 4 + 15) / 16 * 16;
 constexpr uint32_t kSmemUsed = kOffTables + sizeof(ScaleTables);
 constexpr uint32_t kSmemBytes = kSmemUsed + 1024;    // slack to align the base to 1024
 static_assert(kOffB % 1024 == 0 && kOffSfa % 1024 == 0, "swizzled tiles need 1024-byte bases");
-static_assert(2 * (kSmemBytes + 1024) <= 228 * 1024, "two CTAs per SM");
+static_assert(kSmemBytes <= 227 * 1024 && kCtasPerSm * (kSmemBytes + 1024) <= 228 * 1024,
+              "shared memory per SM");
 
 // Byte offset of scale (row r, scale column c) in the 128x4-tiled MMA layout of
 // a matrix with col_tiles = ceil(sf_cols / 4) scale tiles per 128 rows.
@@ -108,19 +140,20 @@ __device__ __forceinline__ void store_hint(uint8_t* __restrict__ hints, int64_t 
 }
 
 template <int HB>
-__global__ void __launch_bounds__(kProducerThreads, 2)
+__global__ void __launch_bounds__(kProducerThreads, kCtasPerSm)
     k_gemm_nvfp4_quantize(const __grid_constant__ CUtensorMap tm_a,
                           const __grid_constant__ CUtensorMap tm_b,
                           const uint8_t* __restrict__ a_sf, const uint8_t* __restrict__ b_sf,
                           const float* __restrict__ a_ts, const float* __restrict__ b_ts, int n,
-                          int kblocks, uint32_t* __restrict__ ws, ProducerOut out) {
+                          int n_tiles_n, int tiles, int kblocks, uint32_t* __restrict__ ws,
+                          ProducerOut out) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int nt = blockIdx.x, mt = blockIdx.y;
   const uint32_t base = smem_u32(smem);
-  const uint32_t full = base + kOffBar, empty = full + 8 * kStages, accum = empty + 8 * kStages;
+  const uint32_t full = base + kOffBar, empty = full + 8 * kStages;
+  const uint32_t acc_full = empty + 8 * kStages, acc_empty = acc_full + 8 * kAccBufs;
   volatile int* abort = reinterpret_cast<volatile int*>(smem + kOffAbort);
   ScaleTables& tab = *reinterpret_cast<ScaleTables*>(smem + kOffTables);
 
@@ -129,7 +162,10 @@ __global__ void __launch_bounds__(kProducerThreads, 2)
       mbar_init(full + 8 * s, 1);
       mbar_init(empty + 8 * s, 1);
     }
-    mbar_init(accum, 1);
+    for (int b = 0; b < kAccBufs; ++b) {
+      mbar_init(acc_full + 8 * b, 1);
+      mbar_init(acc_empty + 8 * b, kEpiWarps);
+    }
     *abort = 0;
     fence_mbar_init();
     prefetch_tensormap(&tm_a);
@@ -145,104 +181,136 @@ __global__ void __launch_bounds__(kProducerThreads, 2)
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + kOffTmemSlot);
   const int64_t col_tiles_k = (int64_t)kblocks * (kBK / 64);
 
-  if (threadIdx.x == 0) {
+  if (warp == 0) {
     // ---------------- producer: TMA for the tiles, bulk copies for the scales
-    const uint8_t* sfa = a_sf + (size_t)mt * col_tiles_k * kScaleTile;
-    const uint8_t* sfb = b_sf + (size_t)nt * col_tiles_k * kScaleTile;
-    for (int kb = 0; kb < kblocks; ++kb) {
-      const int s = kb % kStages;
-      const uint32_t ph = (uint32_t)(kb / kStages) & 1u;
-      if (!mbar_wait(empty + 8 * s, ph ^ 1u, abort)) break;
-      const uint32_t bar = full + 8 * s;
-      mbar_arrive_expect_tx(bar, kStageTx);
-      tma_load_2d(base + kOffA + s * kTileBytes, &tm_a, bar, kb * (kBK / 2), mt * kBM);
-      tma_load_2d(base + kOffB + s * kTileBytes, &tm_b, bar, kb * (kBK / 2), nt * kBN);
-      bulk_load(base + kOffSfa + s * kScaleBytes, sfa + (size_t)kb * kScaleBytes, kScaleBytes, bar);
-      bulk_load(base + kOffSfb + s * kScaleBytes, sfb + (size_t)kb * kScaleBytes, kScaleBytes, bar);
-    }
-  } else if (threadIdx.x == 32) {
-    // ---------------- MMA issuer
-    constexpr uint32_t idesc = idesc_nvf4(kBM, kBN);
-    for (int kb = 0; kb < kblocks; ++kb) {
-      const int s = kb % kStages;
-      const uint32_t ph = (uint32_t)(kb / kStages) & 1u;
-      if (!mbar_wait(full + 8 * s, ph, abort)) break;
-      tc_fence_after();
-      const uint32_t sf_cols = tmem + 128u + 32u * (uint32_t)s;  // SFA at +0, SFB at +16
-#pragma unroll
-      for (int j = 0; j < kBK / 64; ++j) {
-        cp_32x128b_warpx4(sf_cols + 4 * j,
-                          desc_scale_chunk(base + kOffSfa + s * kScaleBytes + j * kScaleTile));
-        cp_32x128b_warpx4(sf_cols + 16 + 4 * j,
-                          desc_scale_chunk(base + kOffSfb + s * kScaleBytes + j * kScaleTile));
+    if (lane == 0) {
+      int it = 0;
+      for (int tile = blockIdx.x; tile < tiles && !*abort; tile += gridDim.x) {
+        const int mt = tile / n_tiles_n, nt = tile - mt * n_tiles_n;
+        const uint8_t* sfa = a_sf + (size_t)mt * col_tiles_k * kScaleTile;
+        const uint8_t* sfb = b_sf + (size_t)nt * col_tiles_k * kScaleTile;
+        for (int kb = 0; kb < kblocks; ++kb, ++it) {
+          const int s = it % kStages;
+          const uint32_t ph = (uint32_t)(it / kStages) & 1u;
+          if (!mbar_wait(empty + 8 * s, ph ^ 1u, abort)) break;
+          const uint32_t bar = full + 8 * s;
+          mbar_arrive_expect_tx(bar, kStageTx);
+          tma_load_2d(base + kOffA + s * kTileBytes, &tm_a, bar, kb * (kBK / 2), mt * kBM);
+          tma_load_2d(base + kOffB + s * kTileBytes, &tm_b, bar, kb * (kBK / 2), nt * kBN);
+          bulk_load(base + kOffSfa + s * kScaleBytes, sfa + (size_t)kb * kScaleBytes, kScaleBytes,
+                    bar);
+          bulk_load(base + kOffSfb + s * kScaleBytes, sfb + (size_t)kb * kScaleBytes, kScaleBytes,
+                    bar);
+        }
       }
-      const uint64_t da = desc_kmajor_sw128(base + kOffA + s * kTileBytes);
-      const uint64_t db = desc_kmajor_sw128(base + kOffB + s * kTileBytes);
-#pragma unroll
-      for (int j = 0; j < kBK / 64; ++j)  // K = 64 = 32 bytes per MMA: start address + 2
-        mma_nvf4(tmem, da + 2 * j, db + 2 * j, idesc, sf_cols + 4 * j, sf_cols + 16 + 4 * j,
-                 (kb | j) != 0);
-      mma_commit(empty + 8 * s);
     }
-    mma_commit(accum);
-  }
-  __syncwarp();
-
-  // ---------------- epilogue: TMEM -> D -> NVFP4
-  mbar_wait(accum, 0, abort);
-  __syncwarp();  // tcgen05.ld is warp-collective
-  tc_fence_after();
-  const int64_t row = (int64_t)mt * kBM + warp * 32 + lane;
-  const uint32_t t_row = tmem + ((uint32_t)(warp * 32) << 16);
-  const float alpha = __fmul_rn(*a_ts, *b_ts);
-  const int64_t sf_cols_out = n / 16;
-  const int64_t blk0 = row * sf_cols_out + (int64_t)nt * (kBN / 16);
-  if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) *out.tensor_scale = s_t;
-  float dmax = 0.0f;
-  uint64_t sc = 0;  // the tile row's 8 scale bytes, block c16 in byte c16
-#pragma unroll 1
-  for (int c16 = 0; c16 < kBN / 16; ++c16) {
-    float y[16];
-    tmem_ld16(t_row + 16 * c16, y);
-    float amax = 0.0f;
+    __syncwarp();
+  } else if (warp == 1) {
+    // ---------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_nvf4(kBM, kBN);
+      int it = 0, tc = 0;
+      for (int tile = blockIdx.x; tile < tiles && !*abort; tile += gridDim.x, ++tc) {
+        const int buf = tc % kAccBufs;
+        const uint32_t aph = (uint32_t)(tc / kAccBufs) & 1u;
+        if (!mbar_wait(acc_empty + 8 * buf, aph ^ 1u, abort)) break;
+        tc_fence_after();
+        const uint32_t d = tmem + (uint32_t)(buf * kBN);
+        for (int kb = 0; kb < kblocks; ++kb, ++it) {
+          const int s = it % kStages;
+          const uint32_t ph = (uint32_t)(it / kStages) & 1u;
+          if (!mbar_wait(full + 8 * s, ph, abort)) break;
+          tc_fence_after();
+          const uint32_t sf = tmem + kTmemSfBase + 32u * (uint32_t)s;  // SFA +0, SFB +16
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      y[i] = __fmul_rn(y[i], alpha);
-      amax = fmaxf(amax, fabsf(y[i]));
-    }
-    dmax = fmaxf(dmax, amax);
-    if (out.d_out != nullptr) {
-      float* dp = out.d_out + row * n + (int64_t)nt * kBN + 16 * c16;
+          for (int j = 0; j < kBK / 64; ++j) {
+            cp_32x128b_warpx4(sf + 4 * j,
+                              desc_scale_chunk(base + kOffSfa + s * kScaleBytes + j * kScaleTile));
+            cp_32x128b_warpx4(sf + 16 + 4 * j,
+                              desc_scale_chunk(base + kOffSfb + s * kScaleBytes + j * kScaleTile));
+          }
+          const uint64_t da = desc_kmajor_sw128(base + kOffA + s * kTileBytes);
+          const uint64_t db = desc_kmajor_sw128(base + kOffB + s * kTileBytes);
 #pragma unroll
-      for (int q = 0; q < 2; ++q) st_v8f(dp + 8 * q, y + 8 * q);
+          for (int j = 0; j < kBK / 64; ++j)  // K = 64 = 32 bytes per MMA: start address + 2
+            mma_nvf4(d, da + 2 * j, db + 2 * j, idesc, sf + 4 * j, sf + 16 + 4 * j,
+                     (kb | j) != 0);
+          mma_commit(empty + 8 * s);
+        }
+        mma_commit(acc_full + 8 * buf);
+      }
     }
-    const BlockScale bs = block_scale_f32(amax, s_t, tab);
-    uint2 c;
-    if (inv_overflowed(bs.inv)) {
-      c = overflow_codes_f32(y);
-    } else {
-      float v[16];
-#pragma unroll
-      for (int i = 0; i < 16; ++i) v[i] = __fmul_rn(y[i], bs.inv);
-      c = pack_codes16(v);
-    }
-    const int64_t blk = blk0 + c16;
-    reinterpret_cast<uint2*>(out.codes)[blk] = c;
-    sc |= (uint64_t)bs.sb << (8 * c16);
-    if (HB != 0) store_hint<HB>(out.hints, blk, c);
-  }
-  *reinterpret_cast<uint64_t*>(out.scales + blk0) = sc;
-  if (out.scales_mma != nullptr) {
+    __syncwarp();
+  } else {
+    // ---------------- epilogue: TMEM -> D -> NVFP4
+    const int q = warp & 3;  // TMEM lane quadrant this warp may read
+    const float alpha = __fmul_rn(*a_ts, *b_ts);
+    const int64_t sf_cols_out = n / 16;
     const int64_t col_tiles_n = n / 64;
+    if (blockIdx.x == 0 && warp == 2 && lane == 0) *out.tensor_scale = s_t;
+    float dmax = 0.0f;
+    int tc = 0;
+    for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x, ++tc) {
+      const int mt = tile / n_tiles_n, nt = tile - mt * n_tiles_n;
+      const int buf = tc % kAccBufs;
+      const uint32_t aph = (uint32_t)(tc / kAccBufs) & 1u;
+      const bool ok = mbar_wait(acc_full + 8 * buf, aph, abort);
+      __syncwarp();  // tcgen05.ld is warp-collective
+      if (!__all_sync(0xFFFFFFFFu, ok)) break;
+      tc_fence_after();
+      const int64_t row = (int64_t)mt * kBM + q * 32 + lane;
+      const uint32_t t_row = tmem + (uint32_t)(buf * kBN) + ((uint32_t)(q * 32) << 16);
+      const int64_t blk0 = row * sf_cols_out + (int64_t)nt * (kBN / 16);
+      uint64_t sc = 0;  // the tile row's 8 scale bytes, block c16 in byte c16
+#pragma unroll 1
+      for (int c16 = 0; c16 < kBN / 16; ++c16) {
+        float y[16];
+        tmem_ld16(t_row + 16 * c16, y);
+        if (c16 == kBN / 16 - 1) {  // accumulator fully read: hand it back to the MMA warp
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(acc_empty + 8 * buf);
+        }
+        float amax = 0.0f;
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const int64_t c = (int64_t)nt * (kBN / 16) + 4 * h;
-      *reinterpret_cast<uint32_t*>(out.scales_mma + mma_scale_offset(row, c, col_tiles_n)) =
-          (uint32_t)(sc >> (32 * h));
+        for (int i = 0; i < 16; ++i) {
+          y[i] = __fmul_rn(y[i], alpha);
+          amax = fmaxf(amax, fabsf(y[i]));
+        }
+        dmax = fmaxf(dmax, amax);
+        if (out.d_out != nullptr) {
+          float* dp = out.d_out + row * n + (int64_t)nt * kBN + 16 * c16;
+#pragma unroll
+          for (int h = 0; h < 2; ++h) st_v8f(dp + 8 * h, y + 8 * h);
+        }
+        const BlockScale bs = block_scale_f32(amax, s_t, tab);
+        uint2 c;
+        if (inv_overflowed(bs.inv)) {
+          c = overflow_codes_f32(y);
+        } else {
+          float v[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) v[i] = __fmul_rn(y[i], bs.inv);
+          c = pack_codes16(v);
+        }
+        const int64_t blk = blk0 + c16;
+        reinterpret_cast<uint2*>(out.codes)[blk] = c;
+        sc |= (uint64_t)bs.sb << (8 * c16);
+        if (HB != 0) store_hint<HB>(out.hints, blk, c);
+      }
+      *reinterpret_cast<uint64_t*>(out.scales + blk0) = sc;
+      if (out.scales_mma != nullptr) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int64_t c = (int64_t)nt * (kBN / 16) + 4 * h;
+          *reinterpret_cast<uint32_t*>(out.scales_mma + mma_scale_offset(row, c, col_tiles_n)) =
+              (uint32_t)(sc >> (32 * h));
+        }
+      }
     }
+    const uint32_t wmax = warp_max_u32(__float_as_uint(dmax));
+    if (lane == 0) atomicMax(ws + 2, wmax);
   }
-  const uint32_t wmax = warp_max_u32(__float_as_uint(dmax));
-  if (lane == 0) atomicMax(ws + 2, wmax);
 
   tc_fence_before();
   __syncthreads();
@@ -291,9 +359,11 @@ cudaError_t launch_gemm_hb(const CUtensorMap& ta, const CUtensorMap& tb, const u
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  const dim3 grid((unsigned)(n / kBN), (unsigned)(m / kBM));
+  const int64_t tiles = (m / kBM) * (n / kBN);
+  const int64_t slots = (int64_t)kCtasPerSm * sm_count();
+  const int grid = (int)(tiles < slots ? tiles : slots);
   k_gemm_nvfp4_quantize<HB><<<grid, kProducerThreads, kSmemBytes, s>>>(
-      ta, tb, a_sf, b_sf, a_ts, b_ts, (int)n, (int)(k / kBK), ws, out);
+      ta, tb, a_sf, b_sf, a_ts, b_ts, (int)n, (int)(n / kBN), (int)tiles, (int)(k / kBK), ws, out);
   return cudaGetLastError();
 }
 
