@@ -16,10 +16,10 @@
 // a 3-stage shared-memory ring that runs on across tile boundaries.  Warp 1
 // (one lane) copies each stage's scales into TMEM (tcgen05.cp) and issues four
 // 128x128x64 block-scaled MMAs into a 128-column FP32 accumulator.  Warps
-// 2..5 drain it: warp w owns TMEM lanes 32 (w % 4) .. + 31 (tile rows), one
-// 16-column NVFP4 block per tcgen05.ld, multiply by s_a s_b, quantize in
-// registers and store, handing the accumulator back as soon as its last
-// block is read.  While one CTA's epilogue runs, its producer keeps loading
+// 2..9 drain it: warp w owns TMEM lanes 32 (w % 4) .. + 31 (tile rows) and
+// one 64-column half of the tile, one 16-column NVFP4 block per tcgen05.ld,
+// multiply by s_a s_b, quantize in registers and store, handing the
+// accumulator back as soon as its last block is read.  While one CTA's epilogue runs, its producer keeps loading
 // the next tile and the SM's other CTA keeps the tensor core busy.
 //
 // The tensor scale of the output cannot wait for the output's own amax in a
@@ -40,14 +40,17 @@ namespace {
 using namespace umma;
 
 // Pipeline shape (compile-time).  Measured on B200 at 8192 x 4096 x 4096:
-// 2 CTAs per SM with 3 stages and one accumulator each (106 us) beat one CTA
+// 2 CTAs per SM with 3 stages and one accumulator each (108 us) beat one CTA
 // with 6 stages and two accumulators (148 us) -- two independent
 // producer/MMA pipelines per SM keep more loads in flight than one deeper
-// ring.
+// ring -- and 8 epilogue warps (100 us) beat 4, because the accumulator is
+// handed back twice as soon.
 //   STAGES  shared-memory ring depth (K-blocks of 256 in flight per CTA)
 //   ACC     accumulator buffers per CTA (2: a CTA's epilogue overlaps its own
 //           next tile's MMAs; needs TMEM for 2 x 128 columns)
 //   CTAS    resident CTAs per SM
+//   EPI_WARPS  epilogue warps (4: one per TMEM lane quadrant, all 128
+//           columns; 8: two per quadrant, 64 columns each)
 #ifndef NVFP4_GEMM_STAGES
 #define NVFP4_GEMM_STAGES 3
 #endif
@@ -57,13 +60,19 @@ using namespace umma;
 #ifndef NVFP4_GEMM_CTAS
 #define NVFP4_GEMM_CTAS 2
 #endif
+#ifndef NVFP4_GEMM_EPI_WARPS
+#define NVFP4_GEMM_EPI_WARPS 8
+#endif
 
 constexpr int kBM = 128, kBN = 128;
 constexpr int kBK = 256;                             // elements per K-block (128 bytes)
 constexpr int kStages = NVFP4_GEMM_STAGES;
 constexpr int kAccBufs = NVFP4_GEMM_ACC;
 constexpr int kCtasPerSm = NVFP4_GEMM_CTAS;
-constexpr int kEpiWarps = 4;
+constexpr int kEpiWarps = NVFP4_GEMM_EPI_WARPS;
+constexpr int kEpiColGroups = kEpiWarps / 4;         // column slices per lane quadrant
+constexpr int kEpiBlocks = kBN / 16 / kEpiColGroups; // 16-column blocks per epilogue thread
+static_assert(kEpiWarps == 4 || kEpiWarps == 8, "epilogue warps");
 constexpr int kProducerThreads = 32 * (2 + kEpiWarps);
 constexpr uint32_t kTileBytes = kBM * kBK / 2;       // 16 KB for A, same for B (kBN == kBM)
 constexpr uint32_t kScaleTile = 512;                 // 128 rows x 4 scales
@@ -244,6 +253,7 @@ __global__ void __launch_bounds__(kProducerThreads, kCtasPerSm)
   } else {
     // ---------------- epilogue: TMEM -> D -> NVFP4
     const int q = warp & 3;  // TMEM lane quadrant this warp may read
+    const int cg = (warp - 2) >> 2;  // column slice: blocks cg * kEpiBlocks ..
     const float alpha = __fmul_rn(*a_ts, *b_ts);
     const int64_t sf_cols_out = n / 16;
     const int64_t col_tiles_n = n / 64;
@@ -259,14 +269,15 @@ __global__ void __launch_bounds__(kProducerThreads, kCtasPerSm)
       if (!__all_sync(0xFFFFFFFFu, ok)) break;
       tc_fence_after();
       const int64_t row = (int64_t)mt * kBM + q * 32 + lane;
-      const uint32_t t_row = tmem + (uint32_t)(buf * kBN) + ((uint32_t)(q * 32) << 16);
-      const int64_t blk0 = row * sf_cols_out + (int64_t)nt * (kBN / 16);
-      uint64_t sc = 0;  // the tile row's 8 scale bytes, block c16 in byte c16
+      const int b0 = cg * kEpiBlocks;  // first 16-column block of this warp
+      const uint32_t t_row = tmem + (uint32_t)(buf * kBN + 16 * b0) + ((uint32_t)(q * 32) << 16);
+      const int64_t blk0 = row * sf_cols_out + (int64_t)nt * (kBN / 16) + b0;
+      uint64_t sc = 0;  // this thread's scale bytes, block c16 in byte c16
 #pragma unroll 1
-      for (int c16 = 0; c16 < kBN / 16; ++c16) {
+      for (int c16 = 0; c16 < kEpiBlocks; ++c16) {
         float y[16];
         tmem_ld16(t_row + 16 * c16, y);
-        if (c16 == kBN / 16 - 1) {  // accumulator fully read: hand it back to the MMA warp
+        if (c16 == kEpiBlocks - 1) {  // slice fully read: release it to the MMA warp
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(acc_empty + 8 * buf);
@@ -279,7 +290,7 @@ __global__ void __launch_bounds__(kProducerThreads, kCtasPerSm)
         }
         dmax = fmaxf(dmax, amax);
         if (out.d_out != nullptr) {
-          float* dp = out.d_out + row * n + (int64_t)nt * kBN + 16 * c16;
+          float* dp = out.d_out + row * n + (int64_t)nt * kBN + 16 * (b0 + c16);
 #pragma unroll
           for (int h = 0; h < 2; ++h) st_v8f(dp + 8 * h, y + 8 * h);
         }
@@ -298,11 +309,14 @@ __global__ void __launch_bounds__(kProducerThreads, kCtasPerSm)
         sc |= (uint64_t)bs.sb << (8 * c16);
         if (HB != 0) store_hint<HB>(out.hints, blk, c);
       }
-      *reinterpret_cast<uint64_t*>(out.scales + blk0) = sc;
+      if (kEpiBlocks == 8)
+        *reinterpret_cast<uint64_t*>(out.scales + blk0) = sc;
+      else
+        *reinterpret_cast<uint32_t*>(out.scales + blk0) = (uint32_t)sc;
       if (out.scales_mma != nullptr) {
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const int64_t c = (int64_t)nt * (kBN / 16) + 4 * h;
+        for (int h = 0; h < kEpiBlocks / 4; ++h) {
+          const int64_t c = (int64_t)nt * (kBN / 16) + b0 + 4 * h;
           *reinterpret_cast<uint32_t*>(out.scales_mma + mma_scale_offset(row, c, col_tiles_n)) =
               (uint32_t)(sc >> (32 * h));
         }
