@@ -448,23 +448,30 @@ def run_ours(args, world, rank, local):
         print(json.dumps(out))
 
 
+def _sources_sha(files):
+    """sha256 (first 16 hex digits) of the named kernel source files, in order."""
+    import hashlib
+    from train_rollout_alignment_b200 import build as bld
+    h = hashlib.sha256()
+    for f in files:
+        h.update(open(os.path.join(bld.CSRC, f), "rb").read())
+    return h.hexdigest()[:16]
+
+
 def _ncu_traffic(kernel_label):
     """DRAM bytes per launch of the dominant kernel from the committed ncu
-    summary, if it was taken on the current kernel sources (else None)."""
-    import hashlib
+    summary, if it was taken on the current sources of that kernel (the files
+    its line names; else None)."""
     path = os.path.join(ROOT, "profiles", "ncu_dram_traffic.txt")
     if not os.path.exists(path):
         return None
-    from train_rollout_alignment_b200 import build as bld
-    h = hashlib.sha256()
-    for f in bld.SOURCES + bld.HEADERS:
-        h.update(open(os.path.join(bld.CSRC, f), "rb").read())
-    src = h.hexdigest()[:16]
     for line in open(path):
         if line.startswith("#") or "=" not in line:
             continue
         kv = dict(tok.split("=", 1) for tok in line.split())
-        if kv.get("label") == kernel_label and kv.get("src_sha") == src:
+        if kv.get("label") != kernel_label or "files" not in kv:
+            continue
+        if kv.get("src_sha") == _sources_sha(kv["files"].split(",")):
             return float(kv["dram_bytes_per_launch"])
     return None
 

@@ -436,6 +436,16 @@ nvfp4_status nvfp4_gemm_quantize(const uint8_t* a_codes, const uint8_t* a_scales
                                  uint8_t* scales, uint8_t* scales_mma, float* tensor_scale,
                                  uint8_t* hints, int hint_bits, float* d_out, void* stream);
 
+/*
+ * nvfp4_wait_selftest -- failure detection of the producer pipeline, without
+ * a fault: runs the bounded mbarrier wait that nvfp4_gemm_quantize uses on a
+ * barrier that nothing completes.  After about 2 s the wait gives up and
+ * NVFP4_WARN_TIMEOUT is set in ws[1] (the call clears ws[1] first); the
+ * kernel returns normally and the context stays usable.  ws: NVFP4_WS_WORDS
+ * words, 16-byte aligned.
+ */
+nvfp4_status nvfp4_wait_selftest(uint32_t* ws, void* stream);
+
 /* Human-readable name of a status code (static string, never NULL). */
 const char* nvfp4_status_string(nvfp4_status status);
 

@@ -24,6 +24,10 @@
  * (test_oracle_*.py) against library casts, brute force, closed forms and the
  * pages' worked examples.  The per-tensor scale constants (2688 = 6 * 448) and
  * the order of the two block-scale divisions are readings, not pinned values.
+ * oracle_scales_to_mma: parity unpinned on the CPU beyond its structure (the
+ * byte positions are the tensor core's operand format, not the pages'); the
+ * GPU tests pin it through the tensor core, whose GEMM must match
+ * oracle_gemm_nvfp4.
  */
 #include <math.h>
 #include <stdint.h>

@@ -30,7 +30,7 @@ def test_header_declares_the_boundary():
             "nvfp4_tensor_amax", "nvfp4_status_string", "nvfp4_quantize_tile16",
             "nvfp4_transpose_tile16", "mxfp8_sr_transpose_requant", "nvfp4_dequantize",
             "mxfp8_dequantize", "nvfp4_quantize_rtn_rows", "nvfp4_guided_requant_rows",
-            "nvfp4_scales_to_mma", "nvfp4_gemm_quantize"}
+            "nvfp4_scales_to_mma", "nvfp4_gemm_quantize", "nvfp4_wait_selftest"}
     assert want <= set(_declared())
 
 

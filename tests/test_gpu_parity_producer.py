@@ -219,3 +219,20 @@ def test_gemm_quantize_full_size_sampled_rows():
     err = np.abs(D[rows].astype(np.float64) - d_ref)
     assert np.all(err <= _d_bound(d_ref, dabs, k))
     _check_against_own_d(got, m, n, a_out, 2)
+
+
+def test_bounded_wait_reports_timeout_and_the_gpu_stays_usable():
+    """Failure detection without a fault: the pipeline's bounded wait on a
+    barrier nothing completes gives up after ~2 s with NVFP4_WARN_TIMEOUT, and
+    a GEMM right after it still matches the oracle."""
+    import time
+    b = lib()
+    ws = torch.zeros(4, dtype=torch.int32, device="cuda")
+    torch.cuda.synchronize()
+    t0 = time.time()
+    b.nvfp4_wait_selftest(ws)
+    torch.cuda.synchronize()
+    dt = time.time() - t0
+    assert int(ws[1]) & b.NVFP4_WARN_TIMEOUT
+    assert 1.5 < dt < 30.0, dt
+    _run_case(128, 128, 256, 41)

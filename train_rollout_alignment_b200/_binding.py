@@ -44,6 +44,7 @@ _SIGS = {
     "nvfp4_dequantize": (_I, [_P, _P, _P, _I64, _I64, _I, _P, _P]),
     "mxfp8_dequantize": (_I, [_P, _P, _I64, _P, _P]),
     "nvfp4_scales_to_mma": (_I, [_P, _I64, _I64, _P, _P]),
+    "nvfp4_wait_selftest": (_I, [_P, _P]),
     "nvfp4_gemm_quantize": (
         _I, [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _P, _P, _P, _P, _P, _I, _P, _P]),
 }
@@ -242,3 +243,7 @@ def nvfp4_gemm_quantize(a_codes, a_scales_mma, a_ts, b_codes, b_scales_mma, b_ts
         _ptr(a_codes), _ptr(a_scales_mma), _ptr(a_ts), _ptr(b_codes), _ptr(b_scales_mma), _ptr(b_ts),
         int(m), int(n), int(k), _ptr(ws), _ptr(codes), _ptr(scales), _ptr(scales_mma), _ptr(tensor_scale),
         _ptr(hints), int(hint_bits), _ptr(d_out), _stream(stream)))
+
+
+def nvfp4_wait_selftest(ws, stream=None):
+    _check("nvfp4_wait_selftest", _lib.nvfp4_wait_selftest(_ptr(ws), _stream(stream)))

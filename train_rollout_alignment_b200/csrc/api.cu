@@ -374,4 +374,10 @@ nvfp4_status nvfp4_gemm_quantize(const uint8_t* a_codes, const uint8_t* a_scales
                                                 hint_bits, d_out, s));
 }
 
+nvfp4_status nvfp4_wait_selftest(uint32_t* ws, void* stream) {
+  if (!ws) return NVFP4_ERR_INVALID_ARG;
+  if (!aligned(ws, 16)) return NVFP4_ERR_MISALIGNED;
+  return from_cuda(nvfp4::launch_wait_selftest(ws, static_cast<cudaStream_t>(stream)));
+}
+
 }  // extern "C"

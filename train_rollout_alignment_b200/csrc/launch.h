@@ -56,6 +56,7 @@ cudaError_t launch_gemm_quantize(const uint8_t* a_codes, const uint8_t* a_sf, co
                                  int64_t m, int64_t n, int64_t k, uint32_t* ws, uint8_t* codes,
                                  uint8_t* scales, uint8_t* scales_mma, float* tensor_scale,
                                  uint8_t* hints, int hint_bits, float* d_out, cudaStream_t s);
+cudaError_t launch_wait_selftest(uint32_t* ws, cudaStream_t s);
 cudaError_t launch_set_f32(float* dst, float value, cudaStream_t s);
 
 }  // namespace nvfp4

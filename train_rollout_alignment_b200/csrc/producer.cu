@@ -381,6 +381,21 @@ cudaError_t launch_gemm_hb(const CUtensorMap& ta, const CUtensorMap& tb, const u
   return cudaGetLastError();
 }
 
+// The bounded wait of the GEMM pipeline on a barrier that nothing completes
+// (initialised for one arrival that never comes): it must give up after
+// kWaitLimitNs and report NVFP4_WARN_TIMEOUT, leaving the context usable.
+__global__ void k_wait_selftest(uint32_t* ws) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar), 1);
+    abort = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0 && !mbar_wait(smem_u32(&bar), 0, &abort)) atomicOr(ws + 1, NVFP4_WARN_TIMEOUT);
+}
+
 __global__ void k_tensor_scale_from_ws(const uint32_t* ws, float* tensor_scale) {
   *tensor_scale = tensor_scale_from_amax(__uint_as_float(ws[0]));
 }
@@ -394,6 +409,13 @@ cudaError_t launch_scales_to_mma(const uint8_t* scales, int64_t rows, int64_t sf
   if (words == 0) return cudaSuccess;
   k_scales_to_mma<<<grid_for(words, kThreads, 4), kThreads, 0, s>>>(scales, rows, sf_cols,
                                                                    padded_rows, col_tiles, out);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_wait_selftest(uint32_t* ws, cudaStream_t s) {
+  cudaError_t e = cudaMemsetAsync(ws + 1, 0, sizeof(uint32_t), s);
+  if (e != cudaSuccess) return e;
+  k_wait_selftest<<<1, 32, 0, s>>>(ws);
   return cudaGetLastError();
 }
 
