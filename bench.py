@@ -686,7 +686,9 @@ def time_producer(b, device, reps=10, m=8192, n=4096, k=4096):
     with 2-bit hints and both scale layouts in the epilogue.  Operands come from
     the library's own quantizer on synthetic N(0, 1) activations and N(0, 0.02^2)
     weights; the output tensor scale uses the max |D| recorded by a previous
-    call (delayed scaling).  Median of `reps` calls, L2 flushed before each."""
+    call (delayed scaling).  Also the MoE form (routed rows grouped by expert,
+    one weight per expert, one launch).  Median of `reps` calls, L2 flushed
+    before each."""
     gen = torch.Generator(device=device).manual_seed(8)
     u8 = dict(dtype=torch.uint8, device=device)
 
@@ -721,14 +723,44 @@ def time_producer(b, device, reps=10, m=8192, n=4096, k=4096):
     flops = 2.0 * m * n * k
     out_bytes = m * n * (0.5 + 1 / 16 + 1 / 16 + HINT_BITS / 8)
     tf = flops / t / 1e12
-    return {"workload": "NVFP4 [%d tokens x %d] x NVFP4 weight [%d x %d]^T -> NVFP4 + %d-bit hints + "
-                        "tensor-core scale layout" % (m, k, n, k, HINT_BITS),
-            "avg_us": round(t * 1e6, 2), "TFLOP/s": round(tf, 1),
-            "roofline": {"bound": "tensor", "achieved": round(tf, 1), "peak": round(peak, 1),
-                         "unit": "TFLOP/s", "frac": round(tf / peak, 4), "peak_basis": basis},
-            "epilogue_out_bytes": int(out_bytes),
-            "with_fp32_D_written_us": round(t_d * 1e6, 2),
-            "warning_bits": warn}
+    out = {"workload": "NVFP4 [%d tokens x %d] x NVFP4 weight [%d x %d]^T -> NVFP4 + %d-bit hints + "
+                       "tensor-core scale layout" % (m, k, n, k, HINT_BITS),
+           "avg_us": round(t * 1e6, 2), "TFLOP/s": round(tf, 1),
+           "roofline": {"bound": "tensor", "achieved": round(tf, 1), "peak": round(peak, 1),
+                        "unit": "TFLOP/s", "frac": round(tf / peak, 4), "peak_basis": basis},
+           "epilogue_out_bytes": int(out_bytes),
+           "with_fp32_D_written_us": round(t_d * 1e6, 2),
+           "warning_bits": warn}
+    del a_codes, a_sf, codes, scales, smma, d, hints
+
+    # MoE form: 8 experts x 2048 routed rows (8192 tokens, top-2), hidden k ->
+    # expert width n_e, one launch for all experts, each expert its own scale
+    E, rows_e, n_e = 8, 2048, 2048
+    mm = E * rows_e
+    a_codes, a_sf, a_ts = nvfp4_operand(mm, 1.0)
+    parts = [nvfp4_operand(n_e, 0.02) for _ in range(E)]
+    w_codes = torch.cat([p_[0] for p_ in parts])
+    w_sf = torch.cat([p_[1] for p_ in parts])
+    w_ts = torch.cat([p_[2] for p_ in parts])
+    offs = torch.arange(0, mm + 1, rows_e, dtype=torch.int32, device=device)
+    codes, scales, ts, ws, hints = b.empty_nvfp4(mm, n_e, device, hint_bits=HINT_BITS)
+    smma = torch.empty(b.mma_scale_bytes(mm, n_e // 16), **u8)
+    ws.zero_()
+
+    def moe(r):
+        b.nvfp4_moe_gemm_quantize(a_codes, a_sf, a_ts, w_codes, w_sf, w_ts, offs, E, mm, n_e, k, ws, codes,
+                                  scales, ts, scales_mma=smma, hints=hints, hint_bits=HINT_BITS)
+
+    moe(0)
+    torch.cuda.synchronize()
+    ws[0] = ws[2]
+    t_m = _timed(moe, reps, flush)
+    tf_m = 2.0 * mm * n_e * k / t_m / 1e12
+    out["moe"] = {"workload": "%d experts x %d routed rows, NVFP4 [%d x %d] x per-expert NVFP4 weight [%d x %d]^T "
+                              "-> NVFP4 + %d-bit hints, one launch" % (E, rows_e, mm, k, n_e, k, HINT_BITS),
+                  "avg_us": round(t_m * 1e6, 2), "TFLOP/s": round(tf_m, 1), "frac": round(tf_m / peak, 4),
+                  "warning_bits": int(ws[1].item())}
+    return out
 
 
 def time_hint_transport(stack, device, reps=5):

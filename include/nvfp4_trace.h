@@ -437,6 +437,35 @@ nvfp4_status nvfp4_gemm_quantize(const uint8_t* a_codes, const uint8_t* a_scales
                                  uint8_t* hints, int hint_bits, float* d_out, void* stream);
 
 /*
+ * nvfp4_moe_gemm_quantize -- nvfp4_gemm_quantize over the experts of an MoE
+ * layer: the routed tokens, grouped by expert, times each expert's weight,
+ * one launch for all experts.
+ *   [TML4], configuration paragraph: the MoE layers' forward runs in NVFP4,
+ *   and tokens reach the experts in NVFP4 (communication paragraph).  The
+ *   all-to-all that delivers them is not part of this call: A arrives
+ *   grouped, expert e owning rows expert_rows[e] .. expert_rows[e + 1] - 1.
+ *   expert_rows: device int32 [experts + 1], non-decreasing, expert_rows[0] =
+ *   0, expert_rows[experts] = m, every entry a multiple of 128 (pad each
+ *   expert's tokens to 128 rows); an entry breaking that gives wrong rows,
+ *   never an out-of-bounds read (every 128-row tile takes the weight of the
+ *   expert owning its first row).
+ *   w_codes [experts, n, k/2] and w_scales_mma (each expert's scales in the
+ *   MMA layout, concatenated, i.e. the MMA layout of [experts * n, k/16]);
+ *   w_tensor_scales [experts] floats (device).  D rows follow A's rows, row r
+ *   of expert e being s_a s_w[e] (A_r . W_e^T); everything else (one output
+ *   tensor scale from ws[0], hints, both scale layouts, ws[2], warnings,
+ *   shapes, alignment) as nvfp4_gemm_quantize, expert_rows 4-byte aligned.
+ *   1 <= experts <= 65536 (NVFP4_ERR_INVALID_ARG).
+ */
+nvfp4_status nvfp4_moe_gemm_quantize(const uint8_t* a_codes, const uint8_t* a_scales_mma,
+                                     const float* a_tensor_scale, const uint8_t* w_codes,
+                                     const uint8_t* w_scales_mma, const float* w_tensor_scales,
+                                     const int32_t* expert_rows, int64_t experts, int64_t m,
+                                     int64_t n, int64_t k, uint32_t* ws, uint8_t* codes,
+                                     uint8_t* scales, uint8_t* scales_mma, float* tensor_scale,
+                                     uint8_t* hints, int hint_bits, float* d_out, void* stream);
+
+/*
  * nvfp4_wait_selftest -- failure detection of the producer pipeline, without
  * a fault: runs the bounded mbarrier wait that nvfp4_gemm_quantize uses on a
  * barrier that nothing completes.  After about 2 s the wait gives up and

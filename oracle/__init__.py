@@ -402,6 +402,29 @@ def gemm_nvfp4(a_codes, a_scales, a_ts: float, b_codes, b_scales, b_ts: float, m
     return d, dabs
 
 
+def moe_gemm_nvfp4(a_codes, a_scales, a_ts: float, w_codes, w_scales, w_ts, expert_rows, n: int,
+                   k: int):
+    """The MoE form of gemm_nvfp4: A rows expert_rows[e] .. expert_rows[e+1]-1
+    times expert e's weight W_e [n, k] (w_* indexed by expert).  Each expert's
+    block is the plain GEMM of its rows ("Thinking Machines Lab releases 4-bit
+    training", configuration paragraph: the MoE forward runs in NVFP4).
+
+    -> (d, dabs) float64 [m, n]."""
+    rows = [int(r) for r in expert_rows]
+    m = rows[-1]
+    a_codes = np.ascontiguousarray(a_codes, dtype=np.uint8).reshape(m, k // 2)
+    a_scales = np.ascontiguousarray(a_scales, dtype=np.uint8).reshape(m, k // 16)
+    d = np.zeros((m, n), np.float64)
+    dabs = np.zeros((m, n), np.float64)
+    for e in range(len(rows) - 1):
+        r0, r1 = rows[e], rows[e + 1]
+        if r1 == r0:
+            continue
+        d[r0:r1], dabs[r0:r1] = gemm_nvfp4(a_codes[r0:r1], a_scales[r0:r1], a_ts, w_codes[e], w_scales[e],
+                                           float(w_ts[e]), r1 - r0, n, k)
+    return d, dabs
+
+
 def scales_to_mma(scales, rows: int, sf_cols: int) -> np.ndarray:
     """Row-layout block scales [rows, sf_cols] -> the 128x4-tiled MMA layout."""
     scales = np.ascontiguousarray(scales, dtype=np.uint8).reshape(-1)

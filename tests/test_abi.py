@@ -30,7 +30,8 @@ def test_header_declares_the_boundary():
             "nvfp4_tensor_amax", "nvfp4_status_string", "nvfp4_quantize_tile16",
             "nvfp4_transpose_tile16", "mxfp8_sr_transpose_requant", "nvfp4_dequantize",
             "mxfp8_dequantize", "nvfp4_quantize_rtn_rows", "nvfp4_guided_requant_rows",
-            "nvfp4_scales_to_mma", "nvfp4_gemm_quantize", "nvfp4_wait_selftest"}
+            "nvfp4_scales_to_mma", "nvfp4_gemm_quantize", "nvfp4_wait_selftest",
+            "nvfp4_moe_gemm_quantize"}
     assert want <= set(_declared())
 
 
@@ -172,3 +173,10 @@ def test_validation_of_the_producer_entry_points_without_a_gpu():
     assert s2m(f, 128, 4, f + 8, None) == 2
     assert s2m(None, 128, 4, f, None) == 1
     assert s2m(None, 0, 4, None, None) == 0       # empty: nothing to do
+    mg = lib.nvfp4_moe_gemm_quantize
+    mg.restype = I
+    mg.argtypes = [P, P, P, P, P, P, P, I64, I64, I64, I64, P, P, P, P, P, P, I, P, P]
+    assert mg(f, f, f, f, f, f, f, 0, 256, 256, 512, f, f, f, None, f, None, 0, None, None) == 1  # no experts
+    assert mg(f, f, f, f, f, f, None, 4, 256, 256, 512, f, f, f, None, f, None, 0, None, None) == 1  # no offsets
+    assert mg(f, f, f, f, f, f, f + 2, 4, 256, 256, 512, f, f, f, None, f, None, 0, None, None) == 2  # offsets align
+    assert mg(f, f, f, f, f, f, f, 4, 200, 256, 512, f, f, f, None, f, None, 0, None, None) == 3  # m % 128

@@ -236,3 +236,48 @@ def test_bounded_wait_reports_timeout_and_the_gpu_stays_usable():
     assert int(ws[1]) & b.NVFP4_WARN_TIMEOUT
     assert 1.5 < dt < 30.0, dt
     _run_case(128, 128, 256, 41)
+
+
+# ----------------------------------------------------------------- MoE form
+def gpu_moe(ca, sa, ta, experts, rows, n, k, a_out, hint_bits=2):
+    """experts: list of (codes [n, k/2], scales [n, k/16], s_t) per expert."""
+    b = lib()
+    m, E = rows[-1], len(experts)
+    sfa = _dev_mma_scales(sa, m, k // 16)
+    w_scales = np.concatenate([np.asarray(w[1]).reshape(n, k // 16) for w in experts])
+    sfw = _dev_mma_scales(w_scales, E * n, k // 16)       # = the experts' layouts, concatenated
+    w_codes = np.concatenate([np.asarray(w[0]).reshape(n, k // 2) for w in experts])
+    w_ts = np.array([w[2] for w in experts], np.float32)
+    offs = torch.tensor(rows, dtype=torch.int32, device="cuda")
+    ws = torch.zeros(4, dtype=torch.int32, device="cuda")
+    ws[0] = np.int32(np.uint32(f32_bits(a_out)).view(np.int32))
+    codes, scales = Buf(m * n // 2), Buf(m * n // 16)
+    smma = Buf(b.mma_scale_bytes(m, n // 16))
+    ts = Buf(4, torch.float32)
+    hints = Buf(m * n * hint_bits // 8) if hint_bits else None
+    d = Buf(4 * m * n, torch.float32)
+    b.nvfp4_moe_gemm_quantize(_dev(ca), sfa.t, _dev(np.array([ta], np.float32)), _dev(w_codes), sfw.t,
+                              _dev(w_ts), offs, E, m, n, k, ws, codes.t, scales.t, ts.t, scales_mma=smma.t,
+                              hints=hints.t if hints else None, hint_bits=hint_bits, d_out=d.t)
+    torch.cuda.synchronize()
+    return dict(codes=codes.np(), scales=scales.np(), smma=smma.np(), ts=ts.np(),
+                ws=ws.cpu().numpy().view(np.uint32), hints=hints.np() if hints else None,
+                d=d.np().reshape(m, n))
+
+
+@pytest.mark.parametrize("rows,n,k,kinds", [
+    ([0, 256, 256, 640, 768], 256, 512, ("normal", "heavy")),    # expert 1 gets no tokens
+    ([0, 128, 256, 384, 512, 640, 768, 896, 1024], 128, 1024, ("outlier", "normal")),
+])
+def test_moe_gemm_quantize(rows, n, k, kinds):
+    m, E = rows[-1], len(rows) - 1
+    ca, sa, ta = _operand(m, k, 90 + E, kinds[0])
+    experts = [_operand(n, k, 100 + e, kinds[1]) for e in range(E)]
+    d_ref, dabs = oracle.moe_gemm_nvfp4(ca, sa, ta, [w[0] for w in experts], [w[1] for w in experts],
+                                        [w[2] for w in experts], rows, n, k)
+    a_out = np.float32(np.abs(d_ref).max())
+    got = gpu_moe(ca, sa, ta, experts, rows, n, k, a_out)
+    err = np.abs(got["d"].astype(np.float64) - d_ref)
+    assert np.all(err <= _d_bound(d_ref, dabs, k))
+    _check_against_own_d(got, m, n, a_out, 2)
+    _check_against_oracle_d(got, d_ref, dabs, k, a_out)

@@ -140,3 +140,29 @@ def test_scale_layout_padding_is_zero():
     rows, sf_cols = 70, 3
     out = oracle.scales_to_mma(_labelled(rows, sf_cols), rows, sf_cols)
     assert out.size == 512 and np.count_nonzero(out) == rows * sf_cols
+
+
+# ----------------------------------------------------------------- MoE form
+def test_moe_gemm_is_the_plain_gemm_per_expert_block():
+    n, k = 24, 128
+    rows = [0, 16, 16, 48, 56]          # expert 1 has no tokens
+    m = rows[-1]
+    ca, sa, ta = _nvfp4(m, k, 51)
+    ws = [_nvfp4(n, k, 60 + e, "heavy") for e in range(4)]
+    d, dabs = oracle.moe_gemm_nvfp4(ca, sa, ta, [w[0] for w in ws], [w[1] for w in ws],
+                                    [w[2] for w in ws], rows, n, k)
+    A = _dequant_unit(ca, sa, m, k)
+    for e in range(4):
+        r0, r1 = rows[e], rows[e + 1]
+        B = _dequant_unit(ws[e][0], ws[e][1], n, k)
+        want = (A[r0:r1] @ B.T) * (float(ta) * float(ws[e][2]))
+        assert np.allclose(d[r0:r1], want, rtol=1e-15, atol=0.0)
+
+
+def test_moe_gemm_with_one_expert_is_the_plain_gemm():
+    m, n, k = 32, 16, 64
+    ca, sa, ta = _nvfp4(m, k, 71)
+    cb, sb, tb = _nvfp4(n, k, 72)
+    d1, a1 = oracle.gemm_nvfp4(ca, sa, ta, cb, sb, tb, m, n, k)
+    d2, a2 = oracle.moe_gemm_nvfp4(ca, sa, ta, [cb], [sb], [tb], [0, m], n, k)
+    assert np.array_equal(d1, d2) and np.array_equal(a1, a2)

@@ -45,6 +45,8 @@ _SIGS = {
     "mxfp8_dequantize": (_I, [_P, _P, _I64, _P, _P]),
     "nvfp4_scales_to_mma": (_I, [_P, _I64, _I64, _P, _P]),
     "nvfp4_wait_selftest": (_I, [_P, _P]),
+    "nvfp4_moe_gemm_quantize": (
+        _I, [_P, _P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _P, _P, _P, _P, _P, _P, _I, _P, _P]),
     "nvfp4_gemm_quantize": (
         _I, [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _P, _P, _P, _P, _P, _I, _P, _P]),
 }
@@ -243,6 +245,15 @@ def nvfp4_gemm_quantize(a_codes, a_scales_mma, a_ts, b_codes, b_scales_mma, b_ts
         _ptr(a_codes), _ptr(a_scales_mma), _ptr(a_ts), _ptr(b_codes), _ptr(b_scales_mma), _ptr(b_ts),
         int(m), int(n), int(k), _ptr(ws), _ptr(codes), _ptr(scales), _ptr(scales_mma), _ptr(tensor_scale),
         _ptr(hints), int(hint_bits), _ptr(d_out), _stream(stream)))
+
+
+def nvfp4_moe_gemm_quantize(a_codes, a_scales_mma, a_ts, w_codes, w_scales_mma, w_ts, expert_rows, experts, m,
+                            n, k, ws, codes, scales, tensor_scale, scales_mma=None, hints=None, hint_bits=0,
+                            d_out=None, stream=None):
+    _check("nvfp4_moe_gemm_quantize", _lib.nvfp4_moe_gemm_quantize(
+        _ptr(a_codes), _ptr(a_scales_mma), _ptr(a_ts), _ptr(w_codes), _ptr(w_scales_mma), _ptr(w_ts),
+        _ptr(expert_rows), int(experts), int(m), int(n), int(k), _ptr(ws), _ptr(codes), _ptr(scales),
+        _ptr(scales_mma), _ptr(tensor_scale), _ptr(hints), int(hint_bits), _ptr(d_out), _stream(stream)))
 
 
 def nvfp4_wait_selftest(ws, stream=None):

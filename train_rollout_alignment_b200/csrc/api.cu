@@ -337,17 +337,22 @@ nvfp4_status nvfp4_scales_to_mma(const uint8_t* scales, int64_t rows, int64_t sf
                                                static_cast<cudaStream_t>(stream)));
 }
 
-nvfp4_status nvfp4_gemm_quantize(const uint8_t* a_codes, const uint8_t* a_scales_mma,
-                                 const float* a_tensor_scale, const uint8_t* b_codes,
-                                 const uint8_t* b_scales_mma, const float* b_tensor_scale,
-                                 int64_t m, int64_t n, int64_t k, uint32_t* ws, uint8_t* codes,
-                                 uint8_t* scales, uint8_t* scales_mma, float* tensor_scale,
-                                 uint8_t* hints, int hint_bits, float* d_out, void* stream) {
+}  // extern "C"
+
+namespace {
+
+nvfp4_status gemm_quantize(const uint8_t* a_codes, const uint8_t* a_scales_mma,
+                           const float* a_tensor_scale, const uint8_t* b_codes,
+                           const uint8_t* b_scales_mma, const float* b_tensor_scales,
+                           const int32_t* group_rows, int64_t groups, int64_t m, int64_t n,
+                           int64_t k, uint32_t* ws, uint8_t* codes, uint8_t* scales,
+                           uint8_t* scales_mma, float* tensor_scale, uint8_t* hints,
+                           int hint_bits, float* d_out, void* stream) {
   if (m < 0 || n < 0 || k < 0) return NVFP4_ERR_INVALID_ARG;
   if (m % 128 != 0 || n % 128 != 0 || k % 256 != 0 || k == 0) return NVFP4_ERR_SHAPE;
   if (m >= kMaxElems || n >= kMaxElems || k >= (int64_t(1) << 31) ||
       (m != 0 && n > kMaxElems / m) || (m != 0 && k > kMaxElems / m) ||
-      (n != 0 && k > kMaxElems / n))
+      (n != 0 && k > kMaxElems / n) || (n != 0 && groups > kMaxElems / n / k))
     return NVFP4_ERR_SHAPE;
   if (!ws || !tensor_scale) return NVFP4_ERR_INVALID_ARG;
   if (!aligned(ws, 16) || !aligned(tensor_scale, 4)) return NVFP4_ERR_MISALIGNED;
@@ -358,20 +363,49 @@ nvfp4_status nvfp4_gemm_quantize(const uint8_t* a_codes, const uint8_t* a_scales
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (m == 0 || n == 0)
     return from_cuda(nvfp4::launch_gemm_quantize(nullptr, nullptr, nullptr, nullptr, nullptr,
-                                                 nullptr, m, n, k, ws, nullptr, nullptr, nullptr,
-                                                 tensor_scale, nullptr, 0, nullptr, s));
+                                                 nullptr, nullptr, 1, m, n, k, ws, nullptr,
+                                                 nullptr, nullptr, tensor_scale, nullptr, 0,
+                                                 nullptr, s));
   if (!a_codes || !a_scales_mma || !a_tensor_scale || !b_codes || !b_scales_mma ||
-      !b_tensor_scale || !codes || !scales)
+      !b_tensor_scales || !codes || !scales || (groups > 1 && !group_rows))
     return NVFP4_ERR_INVALID_ARG;
   if (!aligned(a_codes, 16) || !aligned(a_scales_mma, 16) || !aligned(a_tensor_scale, 4) ||
-      !aligned(b_codes, 16) || !aligned(b_scales_mma, 16) || !aligned(b_tensor_scale, 4) ||
-      !aligned(codes, 16) || !aligned(scales, 16) || !aligned(scales_mma, 16) ||
-      !aligned(hints, 16) || !aligned(d_out, 32))
+      !aligned(b_codes, 16) || !aligned(b_scales_mma, 16) || !aligned(b_tensor_scales, 4) ||
+      !aligned(group_rows, 4) || !aligned(codes, 16) || !aligned(scales, 16) ||
+      !aligned(scales_mma, 16) || !aligned(hints, 16) || !aligned(d_out, 32))
     return NVFP4_ERR_MISALIGNED;
-  return from_cuda(nvfp4::launch_gemm_quantize(a_codes, a_scales_mma, a_tensor_scale, b_codes,
-                                                b_scales_mma, b_tensor_scale, m, n, k, ws, codes,
-                                                scales, scales_mma, tensor_scale, hints,
-                                                hint_bits, d_out, s));
+  return from_cuda(nvfp4::launch_gemm_quantize(
+      a_codes, a_scales_mma, a_tensor_scale, b_codes, b_scales_mma, b_tensor_scales,
+      groups > 1 ? group_rows : nullptr, groups, m, n, k, ws, codes, scales, scales_mma,
+      tensor_scale, hints, hint_bits, d_out, s));
+}
+
+}  // namespace
+
+extern "C" {
+
+nvfp4_status nvfp4_gemm_quantize(const uint8_t* a_codes, const uint8_t* a_scales_mma,
+                                 const float* a_tensor_scale, const uint8_t* b_codes,
+                                 const uint8_t* b_scales_mma, const float* b_tensor_scale,
+                                 int64_t m, int64_t n, int64_t k, uint32_t* ws, uint8_t* codes,
+                                 uint8_t* scales, uint8_t* scales_mma, float* tensor_scale,
+                                 uint8_t* hints, int hint_bits, float* d_out, void* stream) {
+  return gemm_quantize(a_codes, a_scales_mma, a_tensor_scale, b_codes, b_scales_mma,
+                       b_tensor_scale, nullptr, 1, m, n, k, ws, codes, scales, scales_mma,
+                       tensor_scale, hints, hint_bits, d_out, stream);
+}
+
+nvfp4_status nvfp4_moe_gemm_quantize(const uint8_t* a_codes, const uint8_t* a_scales_mma,
+                                     const float* a_tensor_scale, const uint8_t* w_codes,
+                                     const uint8_t* w_scales_mma, const float* w_tensor_scales,
+                                     const int32_t* expert_rows, int64_t experts, int64_t m,
+                                     int64_t n, int64_t k, uint32_t* ws, uint8_t* codes,
+                                     uint8_t* scales, uint8_t* scales_mma, float* tensor_scale,
+                                     uint8_t* hints, int hint_bits, float* d_out, void* stream) {
+  if (experts < 1 || experts > 65536) return NVFP4_ERR_INVALID_ARG;
+  return gemm_quantize(a_codes, a_scales_mma, a_tensor_scale, w_codes, w_scales_mma,
+                       w_tensor_scales, expert_rows, experts, m, n, k, ws, codes, scales,
+                       scales_mma, tensor_scale, hints, hint_bits, d_out, stream);
 }
 
 nvfp4_status nvfp4_wait_selftest(uint32_t* ws, void* stream) {

@@ -51,11 +51,15 @@ cudaError_t launch_quantize_rows(const uint16_t* x, int64_t rows, int64_t cols, 
                                  unsigned long long* stats4, cudaStream_t s);
 cudaError_t launch_scales_to_mma(const uint8_t* scales, int64_t rows, int64_t sf_cols,
                                  uint8_t* out, cudaStream_t s);
+// group_rows: device prefix offsets [groups + 1] of the A rows of each group
+// (multiples of 128); null with groups == 1 for a plain GEMM.  B holds the
+// groups' weights stacked [groups * n, k], b_ts one tensor scale per group.
 cudaError_t launch_gemm_quantize(const uint8_t* a_codes, const uint8_t* a_sf, const float* a_ts,
                                  const uint8_t* b_codes, const uint8_t* b_sf, const float* b_ts,
-                                 int64_t m, int64_t n, int64_t k, uint32_t* ws, uint8_t* codes,
-                                 uint8_t* scales, uint8_t* scales_mma, float* tensor_scale,
-                                 uint8_t* hints, int hint_bits, float* d_out, cudaStream_t s);
+                                 const int32_t* group_rows, int64_t groups, int64_t m, int64_t n,
+                                 int64_t k, uint32_t* ws, uint8_t* codes, uint8_t* scales,
+                                 uint8_t* scales_mma, float* tensor_scale, uint8_t* hints,
+                                 int hint_bits, float* d_out, cudaStream_t s);
 cudaError_t launch_wait_selftest(uint32_t* ws, cudaStream_t s);
 cudaError_t launch_set_f32(float* dst, float value, cudaStream_t s);
 

@@ -141,6 +141,20 @@ struct ProducerOut {
   float* d_out;         // FP32 D [m, n], or null
 };
 
+// Group (expert) of the A rows starting at `row`: the last g with
+// group_rows[g] <= row (group_rows non-decreasing, group_rows[0] = 0).  The
+// result is in [0, groups - 1] whatever the array holds, so B reads stay
+// inside the stacked weights.  groups == 1 reads nothing.
+__device__ __forceinline__ int group_of(const int32_t* __restrict__ group_rows, int groups,
+                                        int64_t row) {
+  int lo = 0, hi = groups - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if ((int64_t)__ldg(group_rows + mid) <= row) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
 template <int HB>
 __device__ __forceinline__ void store_hint(uint8_t* __restrict__ hints, int64_t blk, uint2 c) {
   if (HB == 1) reinterpret_cast<uint16_t*>(hints)[blk] = (uint16_t)hint_field1(c);
@@ -153,7 +167,8 @@ __global__ void __launch_bounds__(kProducerThreads, kCtasPerSm)
     k_gemm_nvfp4_quantize(const __grid_constant__ CUtensorMap tm_a,
                           const __grid_constant__ CUtensorMap tm_b,
                           const uint8_t* __restrict__ a_sf, const uint8_t* __restrict__ b_sf,
-                          const float* __restrict__ a_ts, const float* __restrict__ b_ts, int n,
+                          const float* __restrict__ a_ts, const float* __restrict__ b_ts,
+                          const int32_t* __restrict__ group_rows, int groups, int n,
                           int n_tiles_n, int tiles, int kblocks, uint32_t* __restrict__ ws,
                           ProducerOut out) {
   extern __shared__ uint8_t smem_raw[];
@@ -196,8 +211,10 @@ __global__ void __launch_bounds__(kProducerThreads, kCtasPerSm)
       int it = 0;
       for (int tile = blockIdx.x; tile < tiles && !*abort; tile += gridDim.x) {
         const int mt = tile / n_tiles_n, nt = tile - mt * n_tiles_n;
+        // B is the groups' weights stacked [groups * n, k]: this tile's rows
+        const int bt = group_of(group_rows, groups, (int64_t)mt * kBM) * n_tiles_n + nt;
         const uint8_t* sfa = a_sf + (size_t)mt * col_tiles_k * kScaleTile;
-        const uint8_t* sfb = b_sf + (size_t)nt * col_tiles_k * kScaleTile;
+        const uint8_t* sfb = b_sf + (size_t)bt * col_tiles_k * kScaleTile;
         for (int kb = 0; kb < kblocks; ++kb, ++it) {
           const int s = it % kStages;
           const uint32_t ph = (uint32_t)(it / kStages) & 1u;
@@ -205,7 +222,7 @@ __global__ void __launch_bounds__(kProducerThreads, kCtasPerSm)
           const uint32_t bar = full + 8 * s;
           mbar_arrive_expect_tx(bar, kStageTx);
           tma_load_2d(base + kOffA + s * kTileBytes, &tm_a, bar, kb * (kBK / 2), mt * kBM);
-          tma_load_2d(base + kOffB + s * kTileBytes, &tm_b, bar, kb * (kBK / 2), nt * kBN);
+          tma_load_2d(base + kOffB + s * kTileBytes, &tm_b, bar, kb * (kBK / 2), bt * kBN);
           bulk_load(base + kOffSfa + s * kScaleBytes, sfa + (size_t)kb * kScaleBytes, kScaleBytes,
                     bar);
           bulk_load(base + kOffSfb + s * kScaleBytes, sfb + (size_t)kb * kScaleBytes, kScaleBytes,
@@ -254,7 +271,7 @@ __global__ void __launch_bounds__(kProducerThreads, kCtasPerSm)
     // ---------------- epilogue: TMEM -> D -> NVFP4
     const int q = warp & 3;  // TMEM lane quadrant this warp may read
     const int cg = (warp - 2) >> 2;  // column slice: blocks cg * kEpiBlocks ..
-    const float alpha = __fmul_rn(*a_ts, *b_ts);
+    const float a_scale = *a_ts;
     const int64_t sf_cols_out = n / 16;
     const int64_t col_tiles_n = n / 64;
     if (blockIdx.x == 0 && warp == 2 && lane == 0) *out.tensor_scale = s_t;
@@ -268,6 +285,7 @@ __global__ void __launch_bounds__(kProducerThreads, kCtasPerSm)
       __syncwarp();  // tcgen05.ld is warp-collective
       if (!__all_sync(0xFFFFFFFFu, ok)) break;
       tc_fence_after();
+      const float alpha = __fmul_rn(a_scale, b_ts[group_of(group_rows, groups, (int64_t)mt * kBM)]);
       const int64_t row = (int64_t)mt * kBM + q * 32 + lane;
       const int b0 = cg * kEpiBlocks;  // first 16-column block of this warp
       const uint32_t t_row = tmem + (uint32_t)(buf * kBN + 16 * b0) + ((uint32_t)(q * 32) << 16);
@@ -363,9 +381,9 @@ bool codes_tensor_map(CUtensorMap* map, const uint8_t* codes, int64_t rows, int6
 
 template <int HB>
 cudaError_t launch_gemm_hb(const CUtensorMap& ta, const CUtensorMap& tb, const uint8_t* a_sf,
-                           const uint8_t* b_sf, const float* a_ts, const float* b_ts, int64_t m,
-                           int64_t n, int64_t k, uint32_t* ws, const ProducerOut& out,
-                           cudaStream_t s) {
+                           const uint8_t* b_sf, const float* a_ts, const float* b_ts,
+                           const int32_t* group_rows, int groups, int64_t m, int64_t n, int64_t k,
+                           uint32_t* ws, const ProducerOut& out, cudaStream_t s) {
   static bool attr_set = false;
   if (!attr_set) {
     cudaError_t e = cudaFuncSetAttribute(k_gemm_nvfp4_quantize<HB>,
@@ -377,7 +395,8 @@ cudaError_t launch_gemm_hb(const CUtensorMap& ta, const CUtensorMap& tb, const u
   const int64_t slots = (int64_t)kCtasPerSm * sm_count();
   const int grid = (int)(tiles < slots ? tiles : slots);
   k_gemm_nvfp4_quantize<HB><<<grid, kProducerThreads, kSmemBytes, s>>>(
-      ta, tb, a_sf, b_sf, a_ts, b_ts, (int)n, (int)(n / kBN), (int)tiles, (int)(k / kBK), ws, out);
+      ta, tb, a_sf, b_sf, a_ts, b_ts, group_rows, groups, (int)n, (int)(n / kBN), (int)tiles,
+      (int)(k / kBK), ws, out);
   return cudaGetLastError();
 }
 
@@ -421,9 +440,10 @@ cudaError_t launch_wait_selftest(uint32_t* ws, cudaStream_t s) {
 
 cudaError_t launch_gemm_quantize(const uint8_t* a_codes, const uint8_t* a_sf, const float* a_ts,
                                  const uint8_t* b_codes, const uint8_t* b_sf, const float* b_ts,
-                                 int64_t m, int64_t n, int64_t k, uint32_t* ws, uint8_t* codes,
-                                 uint8_t* scales, uint8_t* scales_mma, float* tensor_scale,
-                                 uint8_t* hints, int hint_bits, float* d_out, cudaStream_t s) {
+                                 const int32_t* group_rows, int64_t groups, int64_t m, int64_t n,
+                                 int64_t k, uint32_t* ws, uint8_t* codes, uint8_t* scales,
+                                 uint8_t* scales_mma, float* tensor_scale, uint8_t* hints,
+                                 int hint_bits, float* d_out, cudaStream_t s) {
   cudaError_t e = cudaMemsetAsync(ws + 1, 0, 3 * sizeof(uint32_t), s);
   if (e != cudaSuccess) return e;
   if (m == 0 || n == 0) {
@@ -431,14 +451,15 @@ cudaError_t launch_gemm_quantize(const uint8_t* a_codes, const uint8_t* a_sf, co
     return cudaGetLastError();
   }
   CUtensorMap ta, tb;
-  if (!codes_tensor_map(&ta, a_codes, m, k) || !codes_tensor_map(&tb, b_codes, n, k))
+  if (!codes_tensor_map(&ta, a_codes, m, k) || !codes_tensor_map(&tb, b_codes, groups * n, k))
     return cudaErrorInvalidValue;
   const ProducerOut out{codes, scales, scales_mma, tensor_scale, hints, d_out};
+  const int g = (int)groups;
   switch (hints == nullptr ? 0 : hint_bits) {
-    case 1: return launch_gemm_hb<1>(ta, tb, a_sf, b_sf, a_ts, b_ts, m, n, k, ws, out, s);
-    case 2: return launch_gemm_hb<2>(ta, tb, a_sf, b_sf, a_ts, b_ts, m, n, k, ws, out, s);
-    case 4: return launch_gemm_hb<4>(ta, tb, a_sf, b_sf, a_ts, b_ts, m, n, k, ws, out, s);
-    default: return launch_gemm_hb<0>(ta, tb, a_sf, b_sf, a_ts, b_ts, m, n, k, ws, out, s);
+    case 1: return launch_gemm_hb<1>(ta, tb, a_sf, b_sf, a_ts, b_ts, group_rows, g, m, n, k, ws, out, s);
+    case 2: return launch_gemm_hb<2>(ta, tb, a_sf, b_sf, a_ts, b_ts, group_rows, g, m, n, k, ws, out, s);
+    case 4: return launch_gemm_hb<4>(ta, tb, a_sf, b_sf, a_ts, b_ts, group_rows, g, m, n, k, ws, out, s);
+    default: return launch_gemm_hb<0>(ta, tb, a_sf, b_sf, a_ts, b_ts, group_rows, g, m, n, k, ws, out, s);
   }
 }
 
