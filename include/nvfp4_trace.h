@@ -426,8 +426,9 @@ nvfp4_status nvfp4_scales_to_mma(const uint8_t* scales, int64_t rows, int64_t sf
  *   hints (nullable; hint_bits 1, 2 or 4, laid out as nvfp4_emit_hint's),
  *   d_out (nullable: FP32 D [m, n], for checking).
  *   Shapes: m % 128 == 0, n % 128 == 0, k % 256 == 0 and k > 0
- *   (NVFP4_ERR_SHAPE); m or n == 0 only writes tensor_scale.  d_out 32-byte
- *   aligned, every other pointer 16 (tensor scales 4).  Runs on sm_100 only.
+ *   (NVFP4_ERR_SHAPE); m or n == 0 only writes tensor_scale.  codes, hints and
+ *   d_out 32-byte aligned (each thread writes a whole 32-byte row segment),
+ *   every other pointer 16 (tensor scales 4).  Runs on sm_100 only.
  */
 nvfp4_status nvfp4_gemm_quantize(const uint8_t* a_codes, const uint8_t* a_scales_mma,
                                  const float* a_tensor_scale, const uint8_t* b_codes,

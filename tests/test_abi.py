@@ -162,7 +162,7 @@ def test_validation_of_the_producer_entry_points_without_a_gpu():
     assert call(m=-128) == 1                      # negative size
     assert call(ws=None) == 1                     # no scratch
     assert call(a=None) == 1                      # null operand
-    assert call(codes=f + 8) == 2                 # output codes not 16-B aligned
+    assert call(codes=f + 16) == 2                # output codes not 32-B aligned
     assert call(ws=f + 4) == 2                    # ws not 16-B aligned
     assert call(d_out=f + 16) == 2                # D output not 32-B aligned
     assert call(hints=f, hb=3) == 5               # hint_bits not in {1, 2, 4}

@@ -371,8 +371,8 @@ nvfp4_status gemm_quantize(const uint8_t* a_codes, const uint8_t* a_scales_mma,
     return NVFP4_ERR_INVALID_ARG;
   if (!aligned(a_codes, 16) || !aligned(a_scales_mma, 16) || !aligned(a_tensor_scale, 4) ||
       !aligned(b_codes, 16) || !aligned(b_scales_mma, 16) || !aligned(b_tensor_scales, 4) ||
-      !aligned(group_rows, 4) || !aligned(codes, 16) || !aligned(scales, 16) ||
-      !aligned(scales_mma, 16) || !aligned(hints, 16) || !aligned(d_out, 32))
+      !aligned(group_rows, 4) || !aligned(codes, 32) || !aligned(scales, 16) ||
+      !aligned(scales_mma, 16) || !aligned(hints, 32) || !aligned(d_out, 32))
     return NVFP4_ERR_MISALIGNED;
   return from_cuda(nvfp4::launch_gemm_quantize(
       a_codes, a_scales_mma, a_tensor_scale, b_codes, b_scales_mma, b_tensor_scales,

@@ -90,7 +90,7 @@ constexpr uint32_t kOffA = 0;
 constexpr uint32_t kOffB = kOffA + kStages * kTileBytes;
 constexpr uint32_t kOffSfa = kOffB + kStages * kTileBytes;
 constexpr uint32_t kOffSfb = kOffSfa + kStages * kScaleBytes;
-// barriers: full[S], empty[S], acc_full[2], acc_empty[2]
+// barriers: full[STAGES], empty[STAGES], acc_full[ACC], acc_empty[ACC]
 constexpr uint32_t kOffBar = kOffSfb + kStages * kScaleBytes;
 constexpr uint32_t kOffTmemSlot = kOffBar + 8 * (2 * kStages + 2 * kAccBufs);
 constexpr uint32_t kOffAbort = kOffTmemSlot + 4;
@@ -155,11 +155,37 @@ __device__ __forceinline__ int group_of(const int32_t* __restrict__ group_rows, 
   return lo;
 }
 
-template <int HB>
-__device__ __forceinline__ void store_hint(uint8_t* __restrict__ hints, int64_t blk, uint2 c) {
-  if (HB == 1) reinterpret_cast<uint16_t*>(hints)[blk] = (uint16_t)hint_field1(c);
-  if (HB == 2) reinterpret_cast<uint32_t*>(hints)[blk] = hint_field2(c);
-  if (HB == 4) reinterpret_cast<uint2*>(hints)[blk] = c;
+// Whole-sector stores of one thread's row segment (its blocks are adjacent
+// in the row): 32 bytes of codes for 4 blocks in one 256-bit store.
+template <int NB>
+__device__ __forceinline__ void store_row_segment(uint8_t* __restrict__ p, const uint2* c) {
+  static_assert(NB == 4 || NB == 8, "blocks per thread");
+#pragma unroll
+  for (int q = 0; q < NB / 4; ++q)
+    asm volatile("st.global.v8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(p + 32 * q),
+                 "r"(c[4 * q].x), "r"(c[4 * q].y), "r"(c[4 * q + 1].x), "r"(c[4 * q + 1].y),
+                 "r"(c[4 * q + 2].x), "r"(c[4 * q + 2].y), "r"(c[4 * q + 3].x),
+                 "r"(c[4 * q + 3].y)
+                 : "memory");
+}
+template <int HB, int NB>
+__device__ __forceinline__ void store_hints_segment(uint8_t* __restrict__ hints, int64_t blk0,
+                                                    const uint2* c) {
+  if (HB == 4) {
+    store_row_segment<NB>(hints + blk0 * 8, c);
+  } else if (HB == 2) {  // 4 bytes per block: 16-byte stores
+#pragma unroll
+    for (int q = 0; q < NB / 4; ++q)
+      reinterpret_cast<uint4*>(hints + blk0 * 4)[q] =
+          make_uint4(hint_field2(c[4 * q]), hint_field2(c[4 * q + 1]), hint_field2(c[4 * q + 2]),
+                     hint_field2(c[4 * q + 3]));
+  } else if (HB == 1) {  // 2 bytes per block: 8-byte stores
+#pragma unroll
+    for (int q = 0; q < NB / 4; ++q)
+      reinterpret_cast<uint2*>(hints + blk0 * 2)[q] =
+          make_uint2(hint_field1(c[4 * q]) | (hint_field1(c[4 * q + 1]) << 16),
+                     hint_field1(c[4 * q + 2]) | (hint_field1(c[4 * q + 3]) << 16));
+  }
 }
 
 template <int HB>
@@ -290,8 +316,9 @@ __global__ void __launch_bounds__(kProducerThreads, kCtasPerSm)
       const int b0 = cg * kEpiBlocks;  // first 16-column block of this warp
       const uint32_t t_row = tmem + (uint32_t)(buf * kBN + 16 * b0) + ((uint32_t)(q * 32) << 16);
       const int64_t blk0 = row * sf_cols_out + (int64_t)nt * (kBN / 16) + b0;
-      uint64_t sc = 0;  // this thread's scale bytes, block c16 in byte c16
-#pragma unroll 1
+      uint64_t sc = 0;     // this thread's scale bytes, block c16 in byte c16
+      uint2 cc[kEpiBlocks];  // its codes: kEpiBlocks x 8 bytes of one row, stored at once
+#pragma unroll
       for (int c16 = 0; c16 < kEpiBlocks; ++c16) {
         float y[16];
         tmem_ld16(t_row + 16 * c16, y);
@@ -313,20 +340,20 @@ __global__ void __launch_bounds__(kProducerThreads, kCtasPerSm)
           for (int h = 0; h < 2; ++h) st_v8f(dp + 8 * h, y + 8 * h);
         }
         const BlockScale bs = block_scale_f32(amax, s_t, tab);
-        uint2 c;
         if (inv_overflowed(bs.inv)) {
-          c = overflow_codes_f32(y);
+          cc[c16] = overflow_codes_f32(y);
         } else {
           float v[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i) v[i] = __fmul_rn(y[i], bs.inv);
-          c = pack_codes16(v);
+          cc[c16] = pack_codes16(v);
         }
-        const int64_t blk = blk0 + c16;
-        reinterpret_cast<uint2*>(out.codes)[blk] = c;
         sc |= (uint64_t)bs.sb << (8 * c16);
-        if (HB != 0) store_hint<HB>(out.hints, blk, c);
       }
+      // one row segment per thread: codes kEpiBlocks x 8 bytes (32-byte aligned:
+      // n % 128 == 0), hints kEpiBlocks x (2 / 4 / 8) bytes
+      store_row_segment<kEpiBlocks>(out.codes + blk0 * 8, cc);
+      if (HB != 0) store_hints_segment<HB, kEpiBlocks>(out.hints, blk0, cc);
       if (kEpiBlocks == 8)
         *reinterpret_cast<uint64_t*>(out.scales + blk0) = sc;
       else
