@@ -411,12 +411,16 @@ cudaError_t launch_gemm_hb(const CUtensorMap& ta, const CUtensorMap& tb, const u
                            const uint8_t* b_sf, const float* a_ts, const float* b_ts,
                            const int32_t* group_rows, int groups, int64_t m, int64_t n, int64_t k,
                            uint32_t* ws, const ProducerOut& out, cudaStream_t s) {
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(k_gemm_nvfp4_quantize<HB>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  // The shared-memory opt-in is a property of the function on each device.
+  static bool attr_set[64] = {false};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64 || !attr_set[dev]) {
+    e = cudaFuncSetAttribute(k_gemm_nvfp4_quantize<HB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kSmemBytes);
     if (e != cudaSuccess) return e;
-    attr_set = true;
+    if (dev >= 0 && dev < 64) attr_set[dev] = true;
   }
   const int64_t tiles = (m / kBM) * (n / kBN);
   const int64_t slots = (int64_t)kCtasPerSm * sm_count();
