@@ -166,3 +166,19 @@ def test_moe_gemm_with_one_expert_is_the_plain_gemm():
     d1, a1 = oracle.gemm_nvfp4(ca, sa, ta, cb, sb, tb, m, n, k)
     d2, a2 = oracle.moe_gemm_nvfp4(ca, sa, ta, [cb], [sb], [tb], [0, m], n, k)
     assert np.array_equal(d1, d2) and np.array_equal(a1, a2)
+
+
+@pytest.mark.parametrize("case", range(12))
+def test_gemm_random_shapes_and_kinds(case):
+    rng = np.random.Generator(np.random.PCG64(900 + case))
+    kinds = ["normal", "heavy", "outlier", "tiny", "sparse", "ties", "zeros"]
+    m, n = int(rng.integers(1, 24)), int(rng.integers(1, 24))
+    k = 16 * int(rng.integers(1, 24))                  # ragged: any multiple of 16 up to 368
+    ca, sa, ta = _nvfp4(m, k, 1000 + case, kinds[case % len(kinds)])
+    cb, sb, tb = _nvfp4(n, k, 2000 + case, kinds[(case + 3) % len(kinds)])
+    d, dabs = oracle.gemm_nvfp4(ca, sa, ta, cb, sb, tb, m, n, k)
+    A = _dequant_unit(ca, sa, m, k)
+    B = _dequant_unit(cb, sb, n, k)
+    st = float(ta) * float(tb)
+    assert np.allclose(d, (A @ B.T) * st, rtol=1e-15, atol=0.0)
+    assert np.allclose(dabs, (np.abs(A) @ np.abs(B).T) * abs(st), rtol=1e-15, atol=0.0)
