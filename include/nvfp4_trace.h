@@ -245,10 +245,14 @@ nvfp4_status nvfp4_rht_quantize(const uint16_t* x_bf16, int64_t rows, int64_t co
  *   and outputs are still the caller's device buffers; nothing is allocated.
  *   Limit: batch > NVFP4_SR_NOALLOC_MAX_BATCH returns NVFP4_ERR_SCRATCH_LIMIT
  *   and enqueues nothing.
+ *   Argument checks are those of nvfp4_sr_transpose_requant (same status for
+ *   the same arguments, batch == 0 returns NVFP4_OK), then the limit below.
  *   Set-up: the first call on a device looks up the array's device address
  *   (cudaGetSymbolAddress, with that device current -- call with the stream's
  *   device current) and caches it; make that first call before any stream
- *   capture.
+ *   capture.  The cached address is valid for that device's primary context
+ *   only: after cudaDeviceReset (or any teardown of the primary context) the
+ *   process must not call this entry point again.
  *   Sharing: all calls on a device share the one array; each call clears the
  *   words it uses on `stream` before its kernels read them, and the array keeps
  *   the last call's contents.  Calls whose work overlaps on the GPU (different

@@ -169,3 +169,90 @@ def oracle_guided_parallel(x, hints, hint_bits, A, chunks=16):
     scales = np.concatenate([o[1] for o in outs])
     stats = np.sum([o[3] for o in outs], axis=0).astype(np.uint64)
     return codes, scales, outs[0][2], stats
+
+
+# ----------------------------------------------------------------- RHT tolerance rule
+_E4M3_VALUES = None
+
+
+def _e4m3_midpoints():
+    global _E4M3_VALUES
+    if _E4M3_VALUES is None:
+        e4 = np.array([oracle.e4m3_value(k) for k in range(127)], np.float64)  # 0 .. 448
+        _E4M3_VALUES = (e4, (e4[:-1] + e4[1:]) / 2)
+    return _E4M3_VALUES
+
+
+_E2M1_MIDS = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0])
+
+
+def _nearest_dist(vals, mids):
+    """Distance of each value to the nearest entry of the sorted array mids."""
+    j = np.clip(np.searchsorted(mids, vals), 1, len(mids) - 1)
+    return np.minimum(np.abs(vals - mids[j - 1]), np.abs(vals - mids[j]))
+
+
+def rht_boundary_check(x_rows, yd_rows, oc, osc, ot, g_codes, g_scales, g_ts):
+    """The RHT tolerance rule against the full double-precision oracle, on a
+    row range: the transform may differ from the double one by
+    tol = 1e-6 * ||x_group||_2 per element, so
+      * a block scale may differ only where the oracle's (amax_b / 6) / s_t is
+        within that tolerance (carried into the scale domain) of an E4M3
+        rounding midpoint;
+      * in a block whose scale agrees, a code may differ (as a signed grid
+        position: +0 and -0 are one value) only where the oracle's |v| is
+        within the tolerance (carried into v) of an E2M1 midpoint.
+    A difference between the two tensor scales (they come from the two
+    transforms' maxima) widens both by its relative size.
+    x_rows: BF16 bits [r, cols]; yd_rows: the double transform [r, cols];
+    oc/osc: the oracle's codes/scales of these rows (of y = fl32(yd)), ot its
+    tensor scale; g_*: the GPU's.  -> (scale diffs, code diffs); raises on a
+    difference away from a boundary."""
+    from train_rollout_alignment_b200 import synthetic as syn
+    e4, e4_mid = _e4m3_midpoints()
+    norm = np.linalg.norm(syn.bf16_to_f32(x_rows).astype(np.float64).reshape(-1, 32), axis=1)
+    tol_y = 1e-6 * np.repeat(norm, 2)                       # per 16-block: the bound of its 32-group
+    rel_ts = abs(float(g_ts) - float(ot)) / float(ot) + 1e-6
+    oy = yd_rows.astype(np.float32).astype(np.float64).reshape(-1, 16)
+    amax_b = np.abs(oy).max(axis=1)
+    sbf = amax_b / 6.0 / ot
+    osc = np.asarray(osc).reshape(-1)
+    blk_diff = osc != np.asarray(g_scales).reshape(-1)
+    if blk_diff.any():
+        d = _nearest_dist(sbf[blk_diff], e4_mid)
+        allowed = (tol_y[blk_diff] / 6.0 / ot) * 1.01 + rel_ts * sbf[blk_diff]
+        bad = d > allowed
+        assert not bad.any(), "%d block scales differ away from an E4M3 boundary" % int(bad.sum())
+    pos = lambda c: np.where(c & 8, -(c & 7).astype(np.int8), (c & 7).astype(np.int8))
+    pc_o = pos(oracle.unpack_codes(oc)).reshape(-1, 16)
+    pc_g = pos(oracle.unpack_codes(g_codes)).reshape(-1, 16)
+    diff = (pc_o != pc_g) & ~blk_diff[:, None]
+    n_code = int(diff.sum())
+    if n_code:
+        bi, ki = np.nonzero(diff)
+        sbv = e4[osc[bi]]
+        assert np.all(sbv > 0), "a code differs in a block whose scale is zero"
+        scale = sbv * ot
+        a = np.abs(oy[bi, ki]) / scale
+        d = _nearest_dist(a, _E2M1_MIDS)
+        allowed = tol_y[bi] / scale * 1.01 + rel_ts * a
+        bad = d > allowed
+        assert not bad.any(), "%d codes differ away from an E2M1 boundary" % int(bad.sum())
+    return int(blk_diff.sum()), n_code
+
+
+def oracle_stats_parallel(ca, sa, ta, cb, sb, tb, rows, cols, chunks=16):
+    """Oracle mismatch counters over row chunks (every counter is a sum over rows)."""
+    step = max(1, (rows + chunks - 1) // chunks)
+    ca, sa = np.asarray(ca).reshape(rows, -1), np.asarray(sa).reshape(rows, -1)
+    cb, sb = np.asarray(cb).reshape(rows, -1), np.asarray(sb).reshape(rows, -1)
+    parts = [(r, min(rows, r + step)) for r in range(0, rows, step)]
+    with pool(len(parts)) as ex:
+        outs = list(ex.map(lambda p: oracle.mismatch_stats(ca[p[0]:p[1]], sa[p[0]:p[1]], ta, cb[p[0]:p[1]],
+                                                           sb[p[0]:p[1]], tb, p[1] - p[0], cols), parts))
+    return np.sum(outs, axis=0).astype(np.uint64)
+
+
+def amax_parallel(x, chunks=16):
+    with pool(chunks) as ex:
+        return max(ex.map(oracle.amax_bf16, np.array_split(x, chunks)))

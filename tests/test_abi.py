@@ -180,3 +180,31 @@ def test_validation_of_the_producer_entry_points_without_a_gpu():
     assert mg(f, f, f, f, f, f, None, 4, 256, 256, 512, f, f, f, None, f, None, 0, None, None) == 1  # no offsets
     assert mg(f, f, f, f, f, f, f + 2, 4, 256, 256, 512, f, f, f, None, f, None, 0, None, None) == 2  # offsets align
     assert mg(f, f, f, f, f, f, f, 4, 200, 256, 512, f, f, f, None, f, None, 0, None, None) == 3  # m % 128
+
+
+def test_noalloc_sr_transpose_returns_the_allocating_forms_status_without_a_gpu():
+    """The no-allocation SR transpose checks its arguments exactly as the
+    allocating form does, before it looks up its scratch array: an empty batch
+    is a no-op and bad shapes or pointers give the same status."""
+    lib = ctypes.CDLL(_lib_path())
+    P, I64, U64, U32, I = ctypes.c_void_p, ctypes.c_int64, ctypes.c_uint64, ctypes.c_uint32, ctypes.c_int
+    a = lib.nvfp4_sr_transpose_requant
+    a.restype = I
+    a.argtypes = [P, P, P, I64, I64, I64, U64, U32, P, P, P, P, P]
+    n = lib.nvfp4_sr_transpose_requant_noalloc
+    n.restype = I
+    n.argtypes = [P, P, P, I64, I64, I64, U64, U32, P, P, P, P]
+    fake = 1 << 20
+    cases = [
+        (None, None, None, 0, 16, 16),        # empty batch: nothing to do
+        (fake, fake, fake, 0, 16, 16),
+        (fake, fake, fake, 2, 24, 16),        # rows % 16
+        (fake, fake, fake, -1, 16, 16),       # negative batch
+        (None, fake, fake, 2, 16, 16),        # null input
+        (fake + 4, fake, fake, 2, 16, 16),    # misaligned codes
+    ]
+    for c_, s_, t_, batch, rows, cols in cases:
+        want = a(c_, s_, t_, batch, rows, cols, 2, 0, fake, fake, fake, fake, None)
+        got = n(c_, s_, t_, batch, rows, cols, 2, 0, fake, fake, fake, None)
+        assert got == want, (batch, rows, cols, got, want)
+    assert n(fake, fake, fake, 4097, 16, 16, 2, 0, fake, fake, fake, None) == 6   # over the scratch limit

@@ -11,7 +11,7 @@ import oracle
 from train_rollout_alignment_b200 import synthetic as syn
 
 from _gpu_util import (Buf, assert_codes_equal, dev_bf16, f32_bits, gpu_emit_hint, gpu_guided,
-                       gpu_rht, gpu_rtn, gpu_sr, gpu_stats, lib)
+                       gpu_rht, gpu_rtn, gpu_sr, gpu_stats, lib, rht_boundary_check)
 
 pytestmark = pytest.mark.gpu
 
@@ -196,26 +196,7 @@ def _rht_check(x, seed):
     #    a rounding boundary: an E4M3 midpoint for the block scale, an E2M1
     #    midpoint for the code.
     oc, osc, ot, oy = oracle.rht_quantize(x, seed)
-    tol_y = 1e-6 * np.repeat(norm, 2)  # per 16-block: the bound of its 32-group
-    amax_b = np.abs(oy.reshape(-1, 16)).max(axis=1).astype(np.float64)
-    e4 = np.array([oracle.e4m3_value(k) for k in range(127)])
-    e4_mid = (e4[:-1] + e4[1:]) / 2
-    sbf = amax_b / 6.0 / ot
-    near_sb = np.min(np.abs(sbf[:, None] - e4_mid[None, :]), axis=1) <= (tol_y / 6.0 / ot) * 1.01 + 1e-6 * sbf
-    blk_diff = osc.reshape(-1) != g["scales"].reshape(-1)
-    assert np.all(near_sb[blk_diff])
-    sbv = e4[osc.reshape(-1)].repeat(16)
-    same_blk = np.repeat(~blk_diff, 16)
-    # +0 and -0 are one value: an all-zero group may come out as either sign
-    pos = lambda c: np.where(c & 8, -(c & 7).astype(np.int64), (c & 7).astype(np.int64))
-    diff = np.nonzero((pos(oracle.unpack_codes(oc)) != pos(oracle.unpack_codes(g["codes"]))) & same_blk)[0]
-    if diff.size:
-        assert np.all(sbv[diff] > 0)
-        scale = sbv[diff] * ot
-        a = np.abs(oy.reshape(-1)[diff].astype(np.float64)) / scale
-        mids = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0])
-        dist = np.min(np.abs(a[:, None] - mids[None, :]), axis=1)
-        assert np.all(dist <= np.repeat(tol_y, 16)[diff] / scale * 1.01 + 1e-6 * a)
+    rht_boundary_check(x, yd, oc, osc, ot, g["codes"], g["scales"], g["ts"])
     return g
 
 

@@ -45,6 +45,32 @@ nvfp4_status write_unit_scale(float* tensor_scale, void* stream) {
 
 }  // namespace
 
+namespace nvfp4 {
+
+// Argument checks of the SR transpose entry points other than the scratch
+// words (shared by the allocating and the no-allocation forms, so both return
+// the same status for the same arguments).  batch == 0 passes with any
+// pointers: such a call does nothing.
+nvfp4_status check_sr_transpose_args(const uint8_t* codes, const uint8_t* scales,
+                                     const float* tensor_scale, int64_t batch, int64_t rows,
+                                     int64_t cols, const uint8_t* codes_t, const uint8_t* scales_t,
+                                     const float* tensor_scale_t) {
+  if (batch < 0 || rows < 0 || cols < 0) return NVFP4_ERR_INVALID_ARG;
+  if (rows % 16 != 0 || cols % 16 != 0) return NVFP4_ERR_SHAPE;
+  if (batch > 65535 || rows / 64 >= 65535) return NVFP4_ERR_SHAPE;
+  if (rows != 0 && cols > kMaxElems / rows) return NVFP4_ERR_SHAPE;
+  if (batch != 0 && rows * cols > kMaxElems / batch) return NVFP4_ERR_SHAPE;
+  if (batch == 0) return NVFP4_OK;
+  if (!codes || !scales || !tensor_scale || !codes_t || !scales_t || !tensor_scale_t)
+    return NVFP4_ERR_INVALID_ARG;
+  if (!aligned(codes, 16) || !aligned(scales, 16) || !aligned(codes_t, 16) ||
+      !aligned(scales_t, 16) || !aligned(tensor_scale, 4) || !aligned(tensor_scale_t, 4))
+    return NVFP4_ERR_MISALIGNED;
+  return NVFP4_OK;
+}
+
+}  // namespace nvfp4
+
 extern "C" {
 
 const char* nvfp4_status_string(nvfp4_status status) {
@@ -159,18 +185,11 @@ nvfp4_status nvfp4_sr_transpose_requant(const uint8_t* codes, const uint8_t* sca
                                         int64_t cols, uint64_t seed, uint32_t draw, uint32_t* ws,
                                         uint8_t* codes_t, uint8_t* scales_t,
                                         float* tensor_scale_t, void* stream) {
-  if (batch < 0 || rows < 0 || cols < 0) return NVFP4_ERR_INVALID_ARG;
-  if (rows % 16 != 0 || cols % 16 != 0) return NVFP4_ERR_SHAPE;
-  if (batch > 65535 || rows / 64 >= 65535) return NVFP4_ERR_SHAPE;
-  if (rows != 0 && cols > kMaxElems / rows) return NVFP4_ERR_SHAPE;
-  if (batch != 0 && rows * cols > kMaxElems / batch) return NVFP4_ERR_SHAPE;
-  if (batch == 0) return NVFP4_OK;
-  if (!codes || !scales || !tensor_scale || !ws || !codes_t || !scales_t || !tensor_scale_t)
-    return NVFP4_ERR_INVALID_ARG;
-  if (!aligned(codes, 16) || !aligned(scales, 16) || !aligned(codes_t, 16) ||
-      !aligned(scales_t, 16) || !aligned(ws, 16) || !aligned(tensor_scale, 4) ||
-      !aligned(tensor_scale_t, 4))
-    return NVFP4_ERR_MISALIGNED;
+  nvfp4_status st = nvfp4::check_sr_transpose_args(codes, scales, tensor_scale, batch, rows, cols,
+                                                    codes_t, scales_t, tensor_scale_t);
+  if (st != NVFP4_OK || batch == 0) return st;
+  if (!ws) return NVFP4_ERR_INVALID_ARG;
+  if (!aligned(ws, 16)) return NVFP4_ERR_MISALIGNED;
   return from_cuda(nvfp4::launch_sr_transpose(codes, scales, tensor_scale, batch, rows, cols, seed,
                                               draw, ws, codes_t, scales_t, tensor_scale_t,
                                               static_cast<cudaStream_t>(stream)));

@@ -6,7 +6,16 @@
 #include <cstdint>
 #include <cuda_runtime.h>
 
+#include "../../include/nvfp4_trace.h"
+
 namespace nvfp4 {
+
+// Argument checks shared by nvfp4_sr_transpose_requant and its no-allocation
+// form (everything except the scratch words); NVFP4_OK for batch == 0.
+nvfp4_status check_sr_transpose_args(const uint8_t* codes, const uint8_t* scales,
+                                     const float* tensor_scale, int64_t batch, int64_t rows,
+                                     int64_t cols, const uint8_t* codes_t, const uint8_t* scales_t,
+                                     const float* tensor_scale_t);
 
 // Streaming grid: `ctas_per_sm` resident CTAs on every SM, capped by the work.
 int grid_for(int64_t work_items, int items_per_cta, int ctas_per_sm);

@@ -13,11 +13,16 @@
 //
 // Host code must not use the array's name as a pointer (on the host it is a
 // stand-in, not a device address): its device address is fetched once per
-// device with cudaGetSymbolAddress, with that device current, and cached.
+// device with cudaGetSymbolAddress, with that device current, and cached.  The
+// cached address belongs to the device's primary context as it was at that
+// first call; a process that resets the device (cudaDeviceReset) or otherwise
+// destroys and recreates its primary context must not call this entry point
+// afterwards.
 #include <cstdint>
 #include <mutex>
 
 #include "../../include/nvfp4_trace.h"
+#include "launch.h"
 
 static __device__ __align__(256) uint32_t g_sr_scratch[NVFP4_SR_NOALLOC_MAX_BATCH];
 
@@ -50,13 +55,17 @@ extern "C" nvfp4_status nvfp4_sr_transpose_requant_noalloc(
     const uint8_t* codes, const uint8_t* scales, const float* tensor_scale, int64_t batch,
     int64_t rows, int64_t cols, uint64_t seed, uint32_t draw, uint8_t* codes_t, uint8_t* scales_t,
     float* tensor_scale_t, void* stream) {
-  if (batch < 0) return NVFP4_ERR_INVALID_ARG;
+  // The allocating entry point's own checks first, so both forms return the
+  // same status for the same arguments; an empty batch does nothing and needs
+  // no scratch.
+  nvfp4_status st = nvfp4::check_sr_transpose_args(codes, scales, tensor_scale, batch, rows, cols,
+                                                    codes_t, scales_t, tensor_scale_t);
+  if (st != NVFP4_OK || batch == 0) return st;
   if (batch > NVFP4_SR_NOALLOC_MAX_BATCH) return NVFP4_ERR_SCRATCH_LIMIT;
   uint32_t* ws = nullptr;
-  const nvfp4_status st = scratch_on_current_device(&ws);
-  if (st != NVFP4_OK) return st;
-  // Same validation and kernels as the allocating entry point; it clears the
-  // `batch` scratch words on `stream` before the kernels use them.
+  if ((st = scratch_on_current_device(&ws)) != NVFP4_OK) return st;
+  // Same kernels as the allocating entry point; it clears the `batch`
+  // scratch words on `stream` before the kernels use them.
   return nvfp4_sr_transpose_requant(codes, scales, tensor_scale, batch, rows, cols, seed, draw, ws,
                                     codes_t, scales_t, tensor_scale_t, stream);
 }
