@@ -5,8 +5,9 @@ activations (per-column scales log-uniform in [0.1, 10]), for every layer:
   rollout: tensor amax -> round-to-nearest quantize (+ fused 2-bit hints on
            layers 24..47)
   train:   tensor amax -> guided re-quantize (hints on layers 24..47, plain
-           round-to-nearest before) with its counters
-  both:    mismatch counters between the rollout and the train codes.
+           round-to-nearest before) with its guidance counters, fused with
+           the mismatch counters between the rollout and the train codes
+           (counted from registers: the train codes are not read back).
 Inputs (48 GiB per GPU) are resident in HBM and larger than L2, so no L2 flush
 is needed between steps.  `value` is algorithmic GB/s (bytes each kernel must
 move, summed over the step, divided by the step time), `elements_per_s` the
@@ -51,6 +52,10 @@ BYTES = {
     "quantize_rtn+hint": 2.0 + 0.5 + 1 / 16 + HINT_BITS / 8,
     "guided_requant": 2.0 + 0.5 + 1 / 16,          # no hints: plain RTN
     "guided_requant+hint": 2.0 + HINT_BITS / 8 + 0.5 + 1 / 16,
+    # guided (or RTN) + counters in one pass: BF16 in (+ hints), the rollout's
+    # codes + scales in, the train codes + scales out
+    "guided_requant_stats": 2.0 + 2 * (0.5 + 1 / 16),
+    "guided_requant_stats+hint": 2.0 + HINT_BITS / 8 + 2 * (0.5 + 1 / 16),
     "mismatch_stats": 2 * (0.5 + 1 / 16),
     "emit_hint": 0.5 + HINT_BITS / 8,
 }
@@ -164,24 +169,23 @@ class Stack:
         self.hints = [torch.empty(self.n * HINT_BITS // 8, **u8) if l >= hint_from else None
                       for l in range(layers)]
         self.ts = torch.empty((layers, 2), dtype=torch.float32, device=device)
-        self.ws = torch.zeros((layers, 2, 4), dtype=torch.int32, device=device)
+        self.ws = torch.zeros((layers, 2, 8), dtype=torch.int32, device=device)
         self.stats = torch.zeros((layers, 12), dtype=torch.int64, device=device)
 
     def kernels_of_layer(self, l):
         """(kernel label, algorithmic bytes) in launch order for layer l."""
         q = "quantize_rtn+hint" if l >= self.hint_from else "quantize_rtn"
-        g = "guided_requant+hint" if l >= self.hint_from else "guided_requant"
+        g = "guided_requant_stats+hint" if l >= self.hint_from else "guided_requant_stats"
         return [("amax", BYTES["amax"] * self.n),
                 (q, BYTES[q] * self.n),
                 ("amax", BYTES["amax"] * self.n),
-                (g, BYTES[g] * self.n),
-                ("mismatch_stats", BYTES["mismatch_stats"] * self.n)]
+                (g, BYTES[g] * self.n)]
 
     def step_bytes(self):
         return sum(b for l in range(self.layers) for _, b in self.kernels_of_layer(l))
 
     def run_layer(self, b, l, xr, xt, events=None):
-        """The five kernels of layer l; events: list to append (start, end) pairs to."""
+        """The four kernels of layer l; events: list to append (start, end) pairs to."""
         ws_r, ws_t = self.ws[l, 0], self.ws[l, 1]
         ts_r, ts_t = self.ts[l, 0:1], self.ts[l, 1:2]
         h = self.hints[l]
@@ -192,10 +196,9 @@ class Stack:
             lambda: b.nvfp4_quantize_rtn(xr, ws_r, self.cr[l], self.sr[l], ts_r, h, bits,
                                          flags=b.NVFP4_AMAX_PRECOMPUTED),
             lambda: b.nvfp4_tensor_amax(xt, ws_t),
-            lambda: b.nvfp4_guided_requant(xt, h, HINT_BITS, ws_t, self.ct[l], self.st[l], ts_t, st[8:12],
-                                           flags=b.NVFP4_AMAX_PRECOMPUTED),
-            lambda: b.nvfp4_mismatch_stats(self.cr[l], self.sr[l], ts_r, self.ct[l], self.st[l], ts_t,
-                                           ROWS, COLS, st[0:8]),
+            lambda: b.nvfp4_guided_requant_stats(xt, h, HINT_BITS, ws_t, self.ct[l], self.st[l], ts_t, st[8:12],
+                                                 self.cr[l], self.sr[l], ts_r, st[0:8],
+                                                 flags=b.NVFP4_AMAX_PRECOMPUTED),
         ]
         for fn in calls:
             if events is not None:
@@ -216,7 +219,7 @@ class Stack:
 
     def step_pipelined(self, b, s_roll, s_train):
         """The step on two streams: the rollout chain (amax, quantize + hints)
-        on s_roll, the train chain (amax, guided, counters) on s_train; layer
+        on s_roll, the train chain (amax, guided + counters) on s_train; layer
         l's guided pass waits for layer l's rollout codes and hints.  Kernel
         tails of one chain overlap the other chain's next kernel."""
         main = torch.cuda.current_stream(self.device)
@@ -240,10 +243,9 @@ class Stack:
             with torch.cuda.stream(s_train):
                 b.nvfp4_tensor_amax(self.xt[l], ws_t)
                 s_train.wait_event(rolled)
-                b.nvfp4_guided_requant(self.xt[l], h, HINT_BITS, ws_t, self.ct[l], self.st[l], ts_t,
-                                       st[8:12], flags=b.NVFP4_AMAX_PRECOMPUTED)
-                b.nvfp4_mismatch_stats(self.cr[l], self.sr[l], ts_r, self.ct[l], self.st[l], ts_t,
-                                       ROWS, COLS, st[0:8])
+                b.nvfp4_guided_requant_stats(self.xt[l], h, HINT_BITS, ws_t, self.ct[l], self.st[l], ts_t,
+                                             st[8:12], self.cr[l], self.sr[l], ts_r, st[0:8],
+                                             flags=b.NVFP4_AMAX_PRECOMPUTED)
         for s in (s_roll, s_train):
             done = torch.cuda.Event()
             done.record(s)
@@ -282,8 +284,9 @@ def time_oracle(chunks):
 
 
 def oracle_bytes(chunks):
-    per_elem = (BYTES["amax"] * 2 + BYTES["quantize_rtn+hint"] + BYTES["guided_requant+hint"]
-                + BYTES["mismatch_stats"])
+    """Algorithmic bytes of the oracle's work, counted as for the GPU step of
+    a hinted layer (the same work moves the same algorithmic bytes)."""
+    per_elem = BYTES["amax"] * 2 + BYTES["quantize_rtn+hint"] + BYTES["guided_requant_stats+hint"]
     return sum(c[0].size for c in chunks) * per_elem, sum(c[0].size for c in chunks)
 
 
@@ -420,13 +423,19 @@ def run_ours(args, world, rank, local):
                          % (len(chunks) * 1024, COLS, len(chunks), dt),
                "elements_per_s": round(2 * nel / dt, 1)}
 
-    launches = 5 * args.layers * args.steps
+    launches = 4 * args.layers * args.steps
     out = {
         "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * t_max / args.steps, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
         "data": "synthetic (seeded, generated on the GPU; BF16 inputs, FP32 arithmetic)",
         "config": _config(args.layers),
+        "value_basis": ("algorithmic bytes (what each kernel must read and write, summed over the step) / "
+                        "step time; consecutive kernels can hit in L2 (the quantizer reads the tail of the "
+                        "tensor the amax pass just read), so this is not DRAM traffic: see dram_bytes_per_step "
+                        "and the per-kernel serialized figures"),
+        "algorithmic_bytes_per_step": int(step_bytes),
+        "dram_bytes_per_step": _dram_bytes_per_step(stack),
         "elements_per_s": round(elems, 1),
         "schedule": "rollout chain and train chain on two streams (guided waits for its layer's hints)",
         "serialized": {"ms_per_step": round(1e3 * t_serial / args.steps, 3),
@@ -458,22 +467,41 @@ def _sources_sha(files):
     return h.hexdigest()[:16]
 
 
-def _ncu_traffic(kernel_label):
-    """DRAM bytes per launch of the dominant kernel from the committed ncu
-    summary, if it was taken on the current sources of that kernel (the files
-    its line names; else None)."""
+def _ncu_traffic_all():
+    """DRAM bytes per launch of each kernel of the step from the committed ncu
+    summary, for the kernels whose line was taken on their current sources
+    (the files the line names): {label: bytes}."""
     path = os.path.join(ROOT, "profiles", "ncu_dram_traffic.txt")
+    out = {}
     if not os.path.exists(path):
-        return None
+        return out
     for line in open(path):
         if line.startswith("#") or "=" not in line:
             continue
         kv = dict(tok.split("=", 1) for tok in line.split())
-        if kv.get("label") != kernel_label or "files" not in kv:
+        if "label" not in kv or "files" not in kv:
             continue
         if kv.get("src_sha") == _sources_sha(kv["files"].split(",")):
-            return float(kv["dram_bytes_per_launch"])
-    return None
+            out[kv["label"]] = float(kv["dram_bytes_per_launch"])
+    return out
+
+
+def _ncu_traffic(kernel_label):
+    """DRAM bytes per launch of one kernel (see _ncu_traffic_all), or None."""
+    return _ncu_traffic_all().get(kernel_label)
+
+
+def _dram_bytes_per_step(stack):
+    """DRAM bytes of one step from the per-launch ncu traffic of its kernels,
+    when every kernel of the step has a current line; else None."""
+    per = _ncu_traffic_all()
+    total = 0.0
+    for l in range(stack.layers):
+        for lab, _ in stack.kernels_of_layer(l):
+            if lab not in per:
+                return None
+            total += per[lab]
+    return total
 
 
 def _flush_l2(bufs):
@@ -520,6 +548,32 @@ def time_other_kernels(b, stack, device, peak, sm_mhz, reps=10):
     gbs = BYTES["emit_hint"] * stack.n / t / 1e9
     out["emit_hint"] = {"workload": "%dx%d codes, 2-bit hints" % (ROWS, COLS), "avg_us": round(t * 1e6, 2),
                         "GB/s": round(gbs, 1), "frac": round(gbs / peak, 4), "bytes_per_elem": BYTES["emit_hint"]}
+    # the standalone counters (the step counts inside the guided pass) between
+    # the rollout and train tensors of that layer
+    s8 = torch.zeros(8, dtype=torch.int64, device=device)
+    t = _timed(lambda r: b.nvfp4_mismatch_stats(stack.cr[l], stack.sr[l], stack.ts[l, 0:1], stack.ct[l], stack.st[l],
+                                                stack.ts[l, 1:2], ROWS, COLS, s8), reps, flush)
+    gbs = BYTES["mismatch_stats"] * stack.n / t / 1e9
+    out["mismatch_stats"] = {"workload": "%dx%d rollout vs train NVFP4 (layer %d)" % (ROWS, COLS, l),
+                             "avg_us": round(t * 1e6, 2), "GB/s": round(gbs, 1), "frac": round(gbs / peak, 4),
+                             "bytes_per_elem": BYTES["mismatch_stats"]}
+    # the two quantizers of that layer alone, L2 flushed (in the step they
+    # may find part of their input in L2 behind the amax pass)
+    c_tmp, s_tmp = torch.empty_like(stack.ct[l]), torch.empty_like(stack.st[l])
+    ts_tmp = torch.empty(1, dtype=torch.float32, device=device)
+    s4 = torch.zeros(4, dtype=torch.int64, device=device)
+    for name, fn in (("quantize_rtn+hint", lambda r: b.nvfp4_quantize_rtn(
+                         stack.xr[l], stack.ws[l, 0], c_tmp, s_tmp, ts_tmp, h, HINT_BITS,
+                         flags=b.NVFP4_AMAX_PRECOMPUTED)),
+                     ("guided_requant+hint", lambda r: b.nvfp4_guided_requant(
+                         stack.xt[l], stack.hints[l], HINT_BITS, stack.ws[l, 1], c_tmp, s_tmp, ts_tmp, s4,
+                         flags=b.NVFP4_AMAX_PRECOMPUTED))):
+        t = _timed(fn, reps, flush)
+        gbs = BYTES[name] * stack.n / t / 1e9
+        out[name + " (alone)"] = {"workload": "%dx%d BF16 layer %d, amax precomputed" % (ROWS, COLS, l),
+                                  "avg_us": round(t * 1e6, 2), "GB/s": round(gbs, 1),
+                                  "frac": round(gbs / peak, 4), "bytes_per_elem": BYTES[name]}
+    del c_tmp, s_tmp
     # SR transpose: the expert stack quantized by the library's own RTN path
     batch, er, ec = syn.CFG2_SHAPE
     w = torch.from_numpy(syn.cfg2().view(np.int16)).view(torch.bfloat16).to(device)
@@ -527,7 +581,7 @@ def time_other_kernels(b, stack, device, peak, sm_mhz, reps=10):
     codes = torch.empty(batch * ne // 2, dtype=torch.uint8, device=device)
     scales = torch.empty(batch * ne // 16, dtype=torch.uint8, device=device)
     ts = torch.empty(batch, dtype=torch.float32, device=device)
-    ws = torch.zeros(max(batch, 4), dtype=torch.int32, device=device)
+    ws = torch.zeros(max(batch, 8), dtype=torch.int32, device=device)
     for e in range(batch):
         b.nvfp4_quantize_rtn(w[e], ws, codes[e * ne // 2:(e + 1) * ne // 2],
                              scales[e * ne // 16:(e + 1) * ne // 16], ts[e:e + 1])
@@ -591,7 +645,7 @@ def time_transpose_alternatives(b, stack, w, codes, scales, ts, sr_out, device, 
     tc = torch.empty(n // 2, dtype=torch.uint8, device=device)
     tt = torch.empty(n // 256, dtype=torch.uint8, device=device)
     tts = torch.empty(batch, dtype=torch.float32, device=device)
-    wse = torch.zeros(4, dtype=torch.int32, device=device)
+    wse = torch.zeros(8, dtype=torch.int32, device=device)
     for e in range(batch):
         b.nvfp4_quantize_tile16(w[e], wse, tc[e * ne // 2:(e + 1) * ne // 2], tt[e * ne // 256:(e + 1) * ne // 256],
                                 tts[e:e + 1])

@@ -76,8 +76,14 @@ typedef int nvfp4_status;
 #define NVFP4_ERR_UNSUPPORTED   5   /* hint_bits not in {1, 2, 4} */
 #define NVFP4_ERR_SCRATCH_LIMIT 6   /* batch above NVFP4_SR_NOALLOC_MAX_BATCH (no-allocation entry point) */
 
-/* Scratch words written by the amax pass and read by the quantize pass. */
-#define NVFP4_WS_WORDS          4   /* ws[0] = bits of A (FP32), ws[1] = warning bits */
+/* Scratch words written by the amax pass and read by the quantize pass:
+ *   ws[0] = FP32 bits of A, ws[1] = warning bits, ws[2] = max |D| observed by
+ *   nvfp4_gemm_quantize, ws[3] reserved;
+ *   ws[4], ws[5] = the amax pass's arrival counter and running maximum, which
+ *   must be ZERO before the first call that uses this ws (allocate it zeroed)
+ *   and which every call leaves zero (the pass needs no clearing launch);
+ *   ws[6..7] reserved (left zero). */
+#define NVFP4_WS_WORDS          8
 #define NVFP4_WARN_NONFINITE    1u  /* ws[1]: an input was Inf or NaN */
 #define NVFP4_WARN_TIMEOUT      2u  /* ws[1]: a pipeline wait inside nvfp4_gemm_quantize gave
                                        up (outputs unspecified; the GPU stays usable) */
@@ -106,8 +112,10 @@ typedef int nvfp4_status;
  * nvfp4_tensor_amax -- A = max |x| over n BF16 values.
  *   Defines the per-tensor scale's input ([TML4]: a shared scale needs the
  *   group maximum).  ws[0] receives the FP32 bit pattern of A (exact: the
- *   maximum of BF16 magnitudes is a BF16 value), ws[1] the warning bits.
- *   ws is cleared by this call.  n == 0 gives A = 0.
+ *   maximum of BF16 magnitudes is a BF16 value), ws[1] the warning bits, and
+ *   ws[2], ws[3] are cleared.  One kernel launch: the CTA that finishes last
+ *   publishes the result (ws[4], ws[5] must be zero on entry, see
+ *   NVFP4_WS_WORDS).  n == 0 gives A = 0.
  */
 nvfp4_status nvfp4_tensor_amax(const uint16_t* x_bf16, int64_t n, uint32_t* ws,
                                void* stream);
@@ -179,6 +187,32 @@ nvfp4_status nvfp4_mismatch_stats(const uint8_t* codes_a, const uint8_t* scales_
                                   const float* ts_b,
                                   int64_t rows, int64_t cols, uint64_t* stats8,
                                   void* stream);
+
+/*
+ * nvfp4_guided_requant_stats -- nvfp4_guided_requant and nvfp4_mismatch_stats
+ * against the rollout's tensor in one pass over the train tensor.
+ *   [TRACE]: the train side follows the rollout's cells (prescription
+ *   paragraph), and the train/rollout distance is what the method shrinks
+ *   (opening and compaction paragraphs).  The counters compare the rollout's
+ *   NVFP4 tensor (roll_codes, roll_scales, *roll_tensor_scale: side a) with
+ *   the train codes this call produces (side b), counted while they are still
+ *   in registers instead of being written and read back.
+ *   Outputs, bit for bit: codes, scales, *tensor_scale and stats4 as
+ *   nvfp4_guided_requant with the same arguments; stats8 (required, ADDED to,
+ *   the caller zeroes it; word 7 unchanged) as nvfp4_mismatch_stats(roll_codes,
+ *   roll_scales, roll_tensor_scale, codes, scales, tensor_scale, rows, cols,
+ *   stats8) run afterwards.  roll_codes [rows, cols/2] and roll_scales
+ *   [rows, cols/16] 16-byte aligned, roll_tensor_scale a device float.
+ *   rows == 0 or cols == 0: writes *tensor_scale = 1 and nothing else.
+ */
+nvfp4_status nvfp4_guided_requant_stats(const uint16_t* x_train_bf16, int64_t rows, int64_t cols,
+                                        const uint8_t* hints, int hint_bits,
+                                        uint32_t* ws, int flags,
+                                        uint8_t* codes, uint8_t* scales, float* tensor_scale,
+                                        uint64_t* stats4,
+                                        const uint8_t* roll_codes, const uint8_t* roll_scales,
+                                        const float* roll_tensor_scale, uint64_t* stats8,
+                                        void* stream);
 
 /*
  * nvfp4_sr_transpose_requant -- dequantize, transpose, stochastic-rounding

@@ -65,7 +65,7 @@ def gpu_rtn(x, hint_bits: int = 0, ws=None, flags: int = 0):
     rows, cols = xt.shape
     n = rows * cols
     codes, scales, ts = Buf(n // 2), Buf(n // 16), Buf(4, torch.float32)
-    ws = ws if ws is not None else torch.zeros(4, dtype=torch.int32, device="cuda")
+    ws = ws if ws is not None else torch.zeros(8, dtype=torch.int32, device="cuda")
     hints = Buf((n * hint_bits + 7) // 8) if hint_bits else None
     b.nvfp4_quantize_rtn(xt, ws, codes.t, scales.t, ts.t, hints.t if hints else None, hint_bits, flags)
     torch.cuda.synchronize()
@@ -79,7 +79,7 @@ def gpu_guided(x, hints_np, hint_bits: int, with_stats: bool = True):
     rows, cols = xt.shape
     n = rows * cols
     codes, scales, ts = Buf(n // 2), Buf(n // 16), Buf(4, torch.float32)
-    ws = torch.zeros(4, dtype=torch.int32, device="cuda")
+    ws = torch.zeros(8, dtype=torch.int32, device="cuda")
     hints = torch.from_numpy(np.ascontiguousarray(hints_np)).cuda() if hints_np is not None else None
     stats = torch.zeros(4, dtype=torch.int64, device="cuda") if with_stats else None
     b.nvfp4_guided_requant(xt, hints, hint_bits, ws, codes.t, scales.t, ts.t, stats)
@@ -113,7 +113,7 @@ def gpu_sr(codes, scales, ts, batch, rows, cols, seed, draw):
     dev = lambda a: torch.from_numpy(np.ascontiguousarray(a).reshape(-1)).cuda()
     n = batch * rows * cols
     ct, st, tst = Buf(n // 2), Buf(n // 16), Buf(4 * batch, torch.float32)
-    ws = torch.zeros(max(batch, 4), dtype=torch.int32, device="cuda")
+    ws = torch.zeros(max(batch, 8), dtype=torch.int32, device="cuda")
     b.nvfp4_sr_transpose_requant(dev(codes), dev(scales), dev(np.asarray(ts, np.float32)), batch, rows,
                                  cols, seed, draw, ws, ct.t, st.t, tst.t)
     torch.cuda.synchronize()
@@ -128,7 +128,7 @@ def gpu_rht(x, seed: int, want_y: bool = True):
     n = rows * cols
     codes, scales, ts = Buf(n // 2), Buf(n // 16), Buf(4, torch.float32)
     y = Buf(4 * n, torch.float32) if want_y else None
-    ws = torch.zeros(4, dtype=torch.int32, device="cuda")
+    ws = torch.zeros(8, dtype=torch.int32, device="cuda")
     b.nvfp4_rht_quantize(xt, seed, ws, codes.t, scales.t, ts.t, y.t if y else None)
     torch.cuda.synchronize()
     return dict(codes=codes.np().reshape(rows, cols // 2), scales=scales.np().reshape(rows, cols // 16),
@@ -256,3 +256,26 @@ def oracle_stats_parallel(ca, sa, ta, cb, sb, tb, rows, cols, chunks=16):
 def amax_parallel(x, chunks=16):
     with pool(chunks) as ex:
         return max(ex.map(oracle.amax_bf16, np.array_split(x, chunks)))
+
+
+def gpu_guided_stats(x, hints_np, hint_bits: int, roll, stats8_init=None):
+    """nvfp4_guided_requant_stats on host inputs; roll = (codes, scales, ts) of
+    the rollout side.  -> dict like gpu_guided plus stats8."""
+    b = lib()
+    xt = dev_bf16(x)
+    rows, cols = xt.shape
+    n = rows * cols
+    codes, scales, ts = Buf(n // 2), Buf(n // 16), Buf(4, torch.float32)
+    ws = torch.zeros(8, dtype=torch.int32, device="cuda")
+    hints = torch.from_numpy(np.ascontiguousarray(hints_np)).cuda() if hints_np is not None else None
+    stats4 = torch.zeros(4, dtype=torch.int64, device="cuda")
+    stats8 = (torch.zeros(8, dtype=torch.int64, device="cuda") if stats8_init is None
+              else torch.from_numpy(np.asarray(stats8_init, np.int64)).cuda())
+    dev = lambda a: torch.from_numpy(np.ascontiguousarray(a).reshape(-1)).cuda()
+    rts = torch.tensor([roll[2]], dtype=torch.float32, device="cuda")
+    b.nvfp4_guided_requant_stats(xt, hints, hint_bits, ws, codes.t, scales.t, ts.t, stats4, dev(roll[0]),
+                                 dev(roll[1]), rts, stats8)
+    torch.cuda.synchronize()
+    return dict(codes=codes.np().reshape(rows, cols // 2), scales=scales.np().reshape(rows, cols // 16),
+                ts=float(ts.np()[0]), stats=stats4.cpu().numpy().astype(np.uint64),
+                stats8=stats8.cpu().numpy().astype(np.uint64))

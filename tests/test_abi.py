@@ -208,3 +208,27 @@ def test_noalloc_sr_transpose_returns_the_allocating_forms_status_without_a_gpu(
         got = n(c_, s_, t_, batch, rows, cols, 2, 0, fake, fake, fake, None)
         assert got == want, (batch, rows, cols, got, want)
     assert n(fake, fake, fake, 4097, 16, 16, 2, 0, fake, fake, fake, None) == 6   # over the scratch limit
+
+
+def test_validation_of_the_fused_train_pass_without_a_gpu():
+    lib = ctypes.CDLL(_lib_path())
+    P, I64, I = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
+    f = lib.nvfp4_guided_requant_stats
+    f.restype = I
+    f.argtypes = [P, I64, I64, P, I, P, I, P, P, P, P, P, P, P, P, P]
+    a = 1 << 20  # never dereferenced: every call below fails validation first
+
+    def call(x=a, rows=4, cols=64, hints=None, hb=2, ws=a, flags=0, codes=a, rc=a, rs=a, rts=a, s8=a, s4=None):
+        return f(x, rows, cols, hints, hb, ws, flags, codes, a, a, s4, rc, rs, rts, s8, None)
+
+    assert call(cols=40) == 3                 # cols % 16
+    assert call(rows=-1) == 1                 # negative size
+    assert call(s8=None) == 1                 # the counters are required
+    assert call(rc=None) == 1                 # the rollout tensor is required
+    assert call(rts=None) == 1
+    assert call(flags=2) == 1                 # unknown flag
+    assert call(hints=a, hb=3) == 5           # hint width
+    assert call(x=a + 16) == 2                # BF16 input 32-byte aligned
+    assert call(rc=a + 8) == 2                # rollout codes 16-byte aligned
+    assert call(s8=a + 4) == 2                # counters 8-byte aligned
+    assert call(s4=a + 4) == 2

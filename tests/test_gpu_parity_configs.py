@@ -1,17 +1,19 @@
 """GPU parity on the five synthetic workloads at their full sizes.
 
 * single 1024x2048 tensor: the whole rollout -> hint -> guided -> counters
-  pipeline, every output bit-exact;
+  pipeline, every output bit-exact, the fused train pass included;
 * 24-layer MoE activation stack (8192x2048, Student-t): every layer bit-exact,
   hints on layers 12..23;
 * 128x512x2048 expert stack: SR transpose of draw 0 bit-exact on all experts,
-  draws 0..31 bit-exact on experts 0..1, and the mean of 1024 GPU draws
+  draws 0..1023 bit-exact on experts 0..1, and the mean of 1024 GPU draws
   unbiased (Hoeffding bound per element, z-score overall and per p-bucket);
-* 16384x4096 activation with outliers: RHT + quantize (tolerance rule of the
-  RHT tests);
+* 16384x4096 activation with outliers: RHT + quantize, every element under
+  the RHT tolerance rule (differences only at rounding boundaries);
 * 48-layer 65536x4096 throughput stack, in the launch configuration the bench
-  times: sampled rows of every layer bit-exact against the oracle (which gets
-  the full layer's amax), whole-layer counters checked by invariants.
+  times: layers 0, 23, 24 and 47 bit-exact over every row (codes, scales,
+  hints, both counter sets), sampled rows of every layer bit-exact against the
+  oracle (which gets the full layer's amax), the fused counters equal to the
+  standalone kernel's on every layer.
 """
 import numpy as np
 import pytest
@@ -20,7 +22,7 @@ import torch
 import oracle
 from train_rollout_alignment_b200 import synthetic as syn
 
-from _gpu_util import (assert_codes_equal, dev_bf16, f32_bits, gpu_guided, gpu_rht, gpu_rtn,
+from _gpu_util import (assert_codes_equal, dev_bf16, f32_bits, gpu_guided, gpu_guided_stats, gpu_rht, gpu_rtn,
                        gpu_sr, gpu_stats, lib, oracle_guided_parallel, oracle_rtn_parallel, pool,
                        oracle_stats_parallel, amax_parallel, rht_boundary_check, to_u16)
 
@@ -46,6 +48,13 @@ def _pipeline_check(xt, xr, bits, label):
     s_gpu = gpu_stats(gr["codes"], gr["scales"], gr["ts"], gg["codes"], gg["scales"], gg["ts"], rows, cols)
     s_or = oracle.mismatch_stats(oc, os_, ot, gc, gs, gt, rows, cols)
     assert list(s_gpu[:7]) == list(s_or[:7])
+    # the fused train pass (guided + counters against the rollout tensor)
+    gf = gpu_guided_stats(xt, gr["hints"] if bits else None, bits if bits else 2,
+                          (gr["codes"], gr["scales"], gr["ts"]))
+    assert_codes_equal(gf["codes"], gc, label + " fused guided codes")
+    assert_codes_equal(gf["scales"], gs, label + " fused train scales")
+    assert list(gf["stats"][:3]) == (list(gst[:3]) if bits else [0, 0, 0])
+    assert list(gf["stats8"][:7]) == list(s_or[:7])
     return s_or
 
 
@@ -242,8 +251,8 @@ def test_throughput_stack_sampled_rows_every_layer():
     scales_t = torch.empty_like(scales_r)
     ts_r = torch.empty(1, dtype=torch.float32, device=dev)
     ts_t = torch.empty(1, dtype=torch.float32, device=dev)
-    ws_r = torch.zeros(4, dtype=torch.int32, device=dev)
-    ws_t = torch.zeros(4, dtype=torch.int32, device=dev)
+    ws_r = torch.zeros(8, dtype=torch.int32, device=dev)
+    ws_t = torch.zeros(8, dtype=torch.int32, device=dev)
     hints = torch.empty(n * 2 // 8, dtype=torch.uint8, device=dev)
     for layer in range(L):
         xt_d, xr_d = syn.cfg4_layer_device(layer, dev)
@@ -251,10 +260,15 @@ def test_throughput_stack_sampled_rows_every_layer():
         h = hints if bits else None
         stats4 = torch.zeros(4, dtype=torch.int64, device=dev)
         stats8 = torch.zeros(8, dtype=torch.int64, device=dev)
-        b.nvfp4_quantize_rtn(xr_d, ws_r, codes_r, scales_r, ts_r, h, bits)
-        b.nvfp4_guided_requant(xt_d, h, 2, ws_t, codes_t, scales_t, ts_t, stats4)
-        b.nvfp4_mismatch_stats(codes_r, scales_r, ts_r, codes_t, scales_t, ts_t, rows, cols, stats8)
+        stats8_sep = torch.zeros(8, dtype=torch.int64, device=dev)
+        b.nvfp4_tensor_amax(xr_d, ws_r)
+        b.nvfp4_quantize_rtn(xr_d, ws_r, codes_r, scales_r, ts_r, h, bits, flags=b.NVFP4_AMAX_PRECOMPUTED)
+        b.nvfp4_tensor_amax(xt_d, ws_t)
+        b.nvfp4_guided_requant_stats(xt_d, h, 2, ws_t, codes_t, scales_t, ts_t, stats4, codes_r, scales_r,
+                                     ts_r, stats8, flags=b.NVFP4_AMAX_PRECOMPUTED)
+        b.nvfp4_mismatch_stats(codes_r, scales_r, ts_r, codes_t, scales_t, ts_t, rows, cols, stats8_sep)
         torch.cuda.synchronize()
+        assert torch.equal(stats8, stats8_sep)  # fused counters == the standalone kernel's
         sel = np.unique(np.concatenate([[0, rows - 1], rng.choice(rows, 30, replace=False)]))
         sel_t = torch.from_numpy(sel).to(dev)
         xr, xt = to_u16(xr_d), to_u16(xt_d)
@@ -296,7 +310,8 @@ def test_throughput_stack_full_layer(layer):
     against the oracle over every row: codes, scales, tensor scales, hints,
     the guidance counters and the mismatch counters, all bit-exact, in the
     launch configuration the bench times (amax pass, then the quantizers with
-    the amax precomputed)."""
+    the amax precomputed, the train side fused with its counters); the
+    standalone counter kernel must agree too."""
     b = lib()
     rows, cols = syn.CFG4_SHAPE
     n = rows * cols
@@ -311,9 +326,12 @@ def test_throughput_stack_full_layer(layer):
     b.nvfp4_tensor_amax(xr_d, ws_r)
     b.nvfp4_quantize_rtn(xr_d, ws_r, codes_r, scales_r, ts_r, hints, bits, flags=b.NVFP4_AMAX_PRECOMPUTED)
     b.nvfp4_tensor_amax(xt_d, ws_t)
-    b.nvfp4_guided_requant(xt_d, hints, 2, ws_t, codes_t, scales_t, ts_t, stats4, flags=b.NVFP4_AMAX_PRECOMPUTED)
-    b.nvfp4_mismatch_stats(codes_r, scales_r, ts_r, codes_t, scales_t, ts_t, rows, cols, stats8)
+    b.nvfp4_guided_requant_stats(xt_d, hints, 2, ws_t, codes_t, scales_t, ts_t, stats4, codes_r, scales_r, ts_r,
+                                 stats8, flags=b.NVFP4_AMAX_PRECOMPUTED)
+    stats8_sep = torch.zeros(8, dtype=torch.int64, device=dev)
+    b.nvfp4_mismatch_stats(codes_r, scales_r, ts_r, codes_t, scales_t, ts_t, rows, cols, stats8_sep)
     torch.cuda.synchronize()
+    assert torch.equal(stats8, stats8_sep)
     xr, xt = to_u16(xr_d), to_u16(xt_d)
     del xt_d, xr_d
     A_r, A_t = amax_parallel(xr), amax_parallel(xt)

@@ -28,7 +28,7 @@ def gpu_tile16(x, precomputed=False):
     rows, cols = xt.shape
     n = rows * cols
     codes, tsc, ts = Buf(n // 2), Buf(n // 256), Buf(4, torch.float32)
-    ws = torch.zeros(4, dtype=torch.int32, device="cuda")
+    ws = torch.zeros(8, dtype=torch.int32, device="cuda")
     flags = 0
     if precomputed:
         b.nvfp4_tensor_amax(xt, ws)
@@ -169,7 +169,7 @@ def test_empty_and_invalid_calls_write_nothing():
     b = lib()
     e = torch.empty(0, dtype=torch.uint8, device="cuda")
     ts = Buf(4, torch.float32)
-    ws = torch.zeros(4, dtype=torch.int32, device="cuda")
+    ws = torch.zeros(8, dtype=torch.int32, device="cuda")
     x0 = torch.empty((0, 64), dtype=torch.bfloat16, device="cuda")
     b.nvfp4_quantize_tile16(x0, ws, e, e, ts.t)
     torch.cuda.synchronize()

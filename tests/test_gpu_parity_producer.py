@@ -56,7 +56,7 @@ def gpu_gemm(ca, sa, ta, cb, sb, tb, m, n, k, a_out, hint_bits=2, want_d=True):
     b = lib()
     sfa = _dev_mma_scales(sa, m, k // 16)
     sfb = _dev_mma_scales(sb, n, k // 16)
-    ws = torch.zeros(4, dtype=torch.int32, device="cuda")
+    ws = torch.zeros(8, dtype=torch.int32, device="cuda")
     ws[0] = np.int32(np.uint32(f32_bits(a_out)).view(np.int32))
     codes, scales = Buf(m * n // 2), Buf(m * n // 16)
     smma = Buf(b.mma_scale_bytes(m, n // 16))
@@ -191,7 +191,7 @@ def test_gemm_quantize_without_d_output_matches():
 
 def test_gemm_quantize_empty_rows_only_write_the_tensor_scale():
     b = lib()
-    ws = torch.zeros(4, dtype=torch.int32, device="cuda")
+    ws = torch.zeros(8, dtype=torch.int32, device="cuda")
     ws[0] = np.int32(f32_bits(2688.0 * 2))
     ts = Buf(4, torch.float32)
     b.nvfp4_gemm_quantize(None, None, None, None, None, None, 0, 256, 512, ws, None, None, ts.t)
@@ -227,7 +227,7 @@ def test_bounded_wait_reports_timeout_and_the_gpu_stays_usable():
     a GEMM right after it still matches the oracle."""
     import time
     b = lib()
-    ws = torch.zeros(4, dtype=torch.int32, device="cuda")
+    ws = torch.zeros(8, dtype=torch.int32, device="cuda")
     torch.cuda.synchronize()
     t0 = time.time()
     b.nvfp4_wait_selftest(ws)
@@ -249,7 +249,7 @@ def gpu_moe(ca, sa, ta, experts, rows, n, k, a_out, hint_bits=2):
     w_codes = np.concatenate([np.asarray(w[0]).reshape(n, k // 2) for w in experts])
     w_ts = np.array([w[2] for w in experts], np.float32)
     offs = torch.tensor(rows, dtype=torch.int32, device="cuda")
-    ws = torch.zeros(4, dtype=torch.int32, device="cuda")
+    ws = torch.zeros(8, dtype=torch.int32, device="cuda")
     ws[0] = np.int32(np.uint32(f32_bits(a_out)).view(np.int32))
     codes, scales = Buf(m * n // 2), Buf(m * n // 16)
     smma = Buf(b.mma_scale_bytes(m, n // 16))

@@ -11,7 +11,7 @@ import oracle
 from train_rollout_alignment_b200 import synthetic as syn
 
 from _gpu_util import (Buf, assert_codes_equal, dev_bf16, f32_bits, gpu_emit_hint, gpu_guided,
-                       gpu_rht, gpu_rtn, gpu_sr, gpu_stats, lib, rht_boundary_check)
+                       gpu_guided_stats, gpu_rht, gpu_rtn, gpu_sr, gpu_stats, lib, rht_boundary_check)
 
 pytestmark = pytest.mark.gpu
 
@@ -38,7 +38,7 @@ def test_amax_precomputed_flag_and_standalone_amax():
     b = lib()
     x = syn.random_case((128, 256), 5, "heavy")
     xt = dev_bf16(x)
-    ws = torch.zeros(4, dtype=torch.int32, device="cuda")
+    ws = torch.zeros(8, dtype=torch.int32, device="cuda")
     b.nvfp4_tensor_amax(xt, ws)
     torch.cuda.synchronize()
     assert f32_bits(np.uint32(ws.cpu().numpy()[0]).view(np.float32)) == f32_bits(oracle.amax_bf16(x))
@@ -46,11 +46,41 @@ def test_amax_precomputed_flag_and_standalone_amax():
     c, s, t, _ = oracle.quantize_rtn(x)
     assert_codes_equal(g["codes"], c)
     # a planted amax is used as given: scales follow A = 2 * true amax
-    ws2 = torch.tensor([f32_bits(2 * oracle.amax_bf16(x)), 0, 0, 0], dtype=torch.int64).to(torch.int32).cuda()
+    ws2 = torch.tensor([f32_bits(2 * oracle.amax_bf16(x)), 0, 0, 0, 0, 0, 0, 0], dtype=torch.int64).to(torch.int32).cuda()
     g2 = gpu_rtn(x, 0, ws=ws2, flags=b.NVFP4_AMAX_PRECOMPUTED)
     c2, s2, t2, _ = oracle.quantize_rtn(x, A=2 * oracle.amax_bf16(x))
     assert f32_bits(g2["ts"]) == f32_bits(t2)
     assert_codes_equal(g2["codes"], c2)
+
+
+def test_amax_passes_in_a_row_leave_no_state_behind():
+    """The amax pass publishes A from the CTA that finishes last, without a
+    clearing launch: calls in a row on one scratch buffer must each give their
+    own tensor's amax (a smaller one after a larger one, a non-finite one,
+    then a finite one, an empty one), set the warning bit only when it applies,
+    and leave the arrival counter and the running maximum (words 4 and 5) zero."""
+    b = lib()
+    ws = torch.zeros(8, dtype=torch.int32, device="cuda")
+    ws[2] = 12345  # a result left by another call: cleared by the amax pass
+    big = syn.random_case((1024, 4096), 11, "outlier")          # many CTAs
+    small = (syn.bf16_to_f32(syn.random_case((333, 64), 12, "normal")) * np.float32(1e-3))
+    small = syn.bf16_bits(small)
+    bad = syn.random_case((64, 256), 13, "normal").copy()
+    bad[7, 9] = 0x7FC0  # a NaN pattern
+    for x, warn in ((big, 0), (small, 0), (bad, 1), (small, 0)):
+        b.nvfp4_tensor_amax(dev_bf16(x), ws)
+        torch.cuda.synchronize()
+        w = ws.cpu().numpy().view(np.uint32)
+        if warn:
+            assert w[0] >= 0x7F800000 and w[1] == b.NVFP4_WARN_NONFINITE
+        else:
+            assert f32_bits(np.uint32(w[0]).view(np.float32)) == f32_bits(oracle.amax_bf16(x))
+            assert w[1] == 0
+        assert w[2] == 0 and w[3] == 0
+        assert not w[4:].any()
+    b.nvfp4_tensor_amax(torch.empty(0, dtype=torch.bfloat16, device="cuda"), ws)
+    torch.cuda.synchronize()
+    assert not ws.cpu().numpy().any()
 
 
 @pytest.mark.parametrize("shape", [(1, 16), (37, 528), (129, 2048)])
@@ -109,6 +139,41 @@ def test_emit_hint_matches_oracle(n):
     codes = rng.integers(0, 256, n // 2).astype(np.uint8)
     for bits in (1, 2, 4):
         assert_codes_equal(gpu_emit_hint(codes, n, bits), oracle.emit_hint(codes, n, bits), "hints")
+
+
+@pytest.mark.parametrize("shape", [(1, 16), (37, 528), (129, 2048), (300, 4096)])
+@pytest.mark.parametrize("kind", ["normal", "heavy", "sparse", "ties", "outlier", "tiny"])
+def test_guided_requant_stats_matches_guided_then_stats(shape, kind):
+    """The fused train pass equals the guided re-quantization followed by the
+    counters against the rollout tensor, bit for bit, for every hint width
+    (none = round-to-nearest), with rollout tensors that are a noisy copy (few
+    differing blocks), an unrelated tensor (most blocks differ) and the train
+    side's own round-to-nearest result (equal tensor scales)."""
+    rng = np.random.default_rng(shape[0] + len(kind))
+    rows, cols = shape
+    xt = syn.random_case(shape, 6000 + rows, kind)
+    xr = syn.rollout_copy(xt, rng, 2.0 ** -8)
+    other = syn.random_case(shape, 6100 + rows, "heavy")
+    for bits in (0, 1, 2, 4):
+        hb = bits if bits else 2
+        ro = oracle.quantize_rtn(xr, hint_bits=bits)
+        hints = ro[3] if bits else None
+        gc, gs, gt, gst = oracle.guided_requant(xt, hints, hb)
+        rollouts = [ro[:3], oracle.quantize_rtn(other)[:3]]
+        if bits == 0:
+            rollouts.append(oracle.quantize_rtn(xt)[:3])
+        for roll in rollouts:
+            g = gpu_guided_stats(xt, hints, hb, roll, stats8_init=[5, 0, 0, 0, 0, 0, 0, 77])
+            assert f32_bits(g["ts"]) == f32_bits(gt)
+            assert_codes_equal(g["scales"], gs, "scales")
+            assert_codes_equal(g["codes"], gc, "guided codes")
+            if bits:
+                assert list(g["stats"][:3]) == list(gst[:3])
+            else:
+                assert not g["stats"].any()
+            o = oracle.mismatch_stats(roll[0], roll[1], roll[2], gc, gs, gt, rows, cols)
+            want = [int(o[0]) + 5] + [int(v) for v in o[1:7]] + [77]  # added to; word 7 untouched
+            assert [int(v) for v in g["stats8"]] == want
 
 
 @pytest.mark.parametrize("shape", [(1, 16), (37, 528), (200, 1024)])
@@ -218,7 +283,7 @@ def test_empty_tensors():
     b = lib()
     x = torch.empty((0, 64), dtype=torch.bfloat16, device="cuda")
     ts = torch.zeros(1, dtype=torch.float32, device="cuda")
-    ws = torch.zeros(4, dtype=torch.int32, device="cuda")
+    ws = torch.zeros(8, dtype=torch.int32, device="cuda")
     e = torch.empty(0, dtype=torch.uint8, device="cuda")
     b.nvfp4_quantize_rtn(x, ws, e, e, ts, None, 0)
     torch.cuda.synchronize()
@@ -240,7 +305,7 @@ def test_invalid_arguments_write_nothing():
     codes = Buf(128)
     scales = Buf(16)
     ts = torch.zeros(1, dtype=torch.float32, device="cuda")
-    ws = torch.zeros(4, dtype=torch.int32, device="cuda")
+    ws = torch.zeros(8, dtype=torch.int32, device="cuda")
     raw = torch.zeros(4 * 64 + 16, dtype=torch.int16, device="cuda")
     x_mis = raw[8:8 + 256].view(torch.bfloat16).view(4, 64)  # 16-byte aligned, not 32
     cases = [
@@ -301,7 +366,7 @@ def test_subnormal_tensor_scales_every_path():
     assert_codes_equal(codes.np(), rc.reshape(-1), "row codes")
     # tile quantizer
     tcodes, tsc, tts = Buf(rows * cols // 2), Buf(rows * cols // 256), Buf(4, torch.float32)
-    b.nvfp4_quantize_tile16(xt, torch.zeros(4, dtype=torch.int32, device="cuda"), tcodes.t, tsc.t, tts.t)
+    b.nvfp4_quantize_tile16(xt, torch.zeros(8, dtype=torch.int32, device="cuda"), tcodes.t, tsc.t, tts.t)
     torch.cuda.synchronize()
     tc, tt, tst = oracle.quantize_tile16(x)
     assert_codes_equal(tcodes.np(), tc.reshape(-1), "tile codes")

@@ -98,7 +98,7 @@ def _worker(rank, world, port, q):
     n = rows * COLS
     u8 = dict(dtype=torch.uint8)
     # rollout side on this rank's rows, with 2-bit hints
-    ws = torch.zeros(4, dtype=torch.int32)
+    ws = torch.zeros(8, dtype=torch.int32)
     cr, sr, tr = torch.zeros(n // 2, **u8), torch.zeros(n // 16, **u8), torch.zeros(1)
     h = torch.zeros(n * 2 // 8, **u8)
     sharded.quantize_rtn(_bf16(xr[sl]), ws, cr, sr, tr, h, 2, lib=lib)

@@ -28,7 +28,7 @@ def _stack(batch, rows, cols, seed):
     codes = torch.empty(batch * rows * cols // 2, dtype=torch.uint8, device="cuda")
     scales = torch.empty(batch * rows * cols // 16, dtype=torch.uint8, device="cuda")
     ts = torch.empty(batch, dtype=torch.float32, device="cuda")
-    ws = torch.zeros(4, dtype=torch.int32, device="cuda")
+    ws = torch.zeros(8, dtype=torch.int32, device="cuda")
     n = rows * cols
     for e in range(batch):
         x = (torch.randn(rows, cols, generator=g, device="cuda") * 0.02).to(torch.bfloat16)

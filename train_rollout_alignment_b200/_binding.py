@@ -30,6 +30,8 @@ _SIGS = {
     "nvfp4_emit_hint": (_I, [_P, _I64, _I, _P, _P]),
     "nvfp4_guided_requant": (_I, [_P, _I64, _I64, _P, _I, _P, _I, _P, _P, _P, _P, _P]),
     "nvfp4_mismatch_stats": (_I, [_P, _P, _P, _P, _P, _P, _I64, _I64, _P, _P]),
+    "nvfp4_guided_requant_stats": (
+        _I, [_P, _I64, _I64, _P, _I, _P, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
     "nvfp4_sr_transpose_requant": (
         _I, [_P, _P, _P, _I64, _I64, _I64, ctypes.c_uint64, ctypes.c_uint32, _P, _P, _P, _P, _P]),
     "nvfp4_rht_quantize": (_I, [_P, _I64, _I64, ctypes.c_uint64, _P, _P, _P, _P, _P, _P]),
@@ -56,7 +58,7 @@ for _name, (_res, _args) in _SIGS.items():
     _fn.argtypes = _args
 
 # Constants mirrored from include/nvfp4_trace.h
-NVFP4_WS_WORDS = 4
+NVFP4_WS_WORDS = 8
 NVFP4_STATS8_WORDS = 8
 NVFP4_STATS4_WORDS = 4
 NVFP4_AMAX_PRECOMPUTED = 1
@@ -134,6 +136,15 @@ def nvfp4_guided_requant(x, hints, hint_bits, ws, codes, scales, tensor_scale, s
         _ptr(scales), _ptr(tensor_scale), _ptr(stats4), _stream(stream)))
 
 
+def nvfp4_guided_requant_stats(x, hints, hint_bits, ws, codes, scales, tensor_scale, stats4, roll_codes,
+                               roll_scales, roll_tensor_scale, stats8, flags=0, stream=None):
+    rows, cols = _rows_cols(x)
+    _check("nvfp4_guided_requant_stats", _lib.nvfp4_guided_requant_stats(
+        _ptr(x), rows, cols, _ptr(hints), int(hint_bits), _ptr(ws), int(flags), _ptr(codes),
+        _ptr(scales), _ptr(tensor_scale), _ptr(stats4), _ptr(roll_codes), _ptr(roll_scales),
+        _ptr(roll_tensor_scale), _ptr(stats8), _stream(stream)))
+
+
 def nvfp4_mismatch_stats(codes_a, scales_a, ts_a, codes_b, scales_b, ts_b, rows, cols, stats8,
                          stream=None):
     _check("nvfp4_mismatch_stats", _lib.nvfp4_mismatch_stats(
@@ -174,7 +185,7 @@ def empty_nvfp4(rows: int, cols: int, device, hint_bits: int = 0):
     codes = torch.empty((rows, cols // 2), dtype=torch.uint8, device=device)
     scales = torch.empty((rows, cols // 16), dtype=torch.uint8, device=device)
     ts = torch.empty(1, dtype=torch.float32, device=device)
-    ws = torch.empty(NVFP4_WS_WORDS, dtype=torch.int32, device=device)
+    ws = torch.zeros(NVFP4_WS_WORDS, dtype=torch.int32, device=device)  # words 4..7 must start at zero
     hints = None
     if hint_bits:
         hints = torch.empty(((rows * cols * hint_bits + 7) // 8,), dtype=torch.uint8, device=device)

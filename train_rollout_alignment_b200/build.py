@@ -17,7 +17,7 @@ CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libnvfp4trace.so")
 SOURCES = ["api.cu", "quantize.cu", "stats.cu", "sr_transpose.cu", "rht.cu", "noalloc.cu",
            "next_formats.cu", "producer.cu"]
-HEADERS = ["nvfp4_device.cuh", "launch.h", "umma.cuh"]
+HEADERS = ["nvfp4_device.cuh", "stats_device.cuh", "launch.h", "umma.cuh"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

@@ -93,10 +93,7 @@ nvfp4_status nvfp4_tensor_amax(const uint16_t* x_bf16, int64_t n, uint32_t* ws, 
   if (n < 0) return NVFP4_ERR_INVALID_ARG;
   if (n % 16 != 0 || n >= kMaxElems) return NVFP4_ERR_SHAPE;
   if (!aligned(ws, 16) || !aligned(x_bf16, 32)) return NVFP4_ERR_MISALIGNED;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  cudaError_t e = cudaMemsetAsync(ws, 0, NVFP4_WS_WORDS * sizeof(uint32_t), s);
-  if (e != cudaSuccess) return NVFP4_ERR_CUDA;
-  return from_cuda(nvfp4::launch_amax_bf16(x_bf16, n / 16, ws, s));
+  return from_cuda(nvfp4::launch_amax_bf16(x_bf16, n / 16, ws, static_cast<cudaStream_t>(stream)));
 }
 
 nvfp4_status nvfp4_quantize_rtn(const uint16_t* x_bf16, int64_t rows, int64_t cols, uint32_t* ws,
@@ -160,6 +157,39 @@ nvfp4_status nvfp4_guided_requant(const uint16_t* x_train_bf16, int64_t rows, in
   return from_cuda(nvfp4::launch_guided(x_train_bf16, n / 16, hints, hint_bits, ws, codes, scales,
                                         tensor_scale,
                                         reinterpret_cast<unsigned long long*>(stats4), s));
+}
+
+nvfp4_status nvfp4_guided_requant_stats(const uint16_t* x_train_bf16, int64_t rows, int64_t cols,
+                                        const uint8_t* hints, int hint_bits, uint32_t* ws,
+                                        int flags, uint8_t* codes, uint8_t* scales,
+                                        float* tensor_scale, uint64_t* stats4,
+                                        const uint8_t* roll_codes, const uint8_t* roll_scales,
+                                        const float* roll_tensor_scale, uint64_t* stats8,
+                                        void* stream) {
+  nvfp4_status st = check_shape(rows, cols, 16);
+  if (st != NVFP4_OK) return st;
+  if ((flags & ~NVFP4_AMAX_PRECOMPUTED) != 0) return NVFP4_ERR_INVALID_ARG;
+  if (rows * cols == 0) return write_unit_scale(tensor_scale, stream);
+  if (!x_train_bf16 || !roll_codes || !roll_scales || !roll_tensor_scale || !stats8)
+    return NVFP4_ERR_INVALID_ARG;
+  if ((st = check_quant_outputs(ws, codes, scales, tensor_scale)) != NVFP4_OK) return st;
+  if (hints) {
+    if ((st = check_hint_bits(hint_bits)) != NVFP4_OK) return st;
+    if (!aligned(hints, 16)) return NVFP4_ERR_MISALIGNED;
+  }
+  if (!aligned(x_train_bf16, 32) || !aligned(roll_codes, 16) || !aligned(roll_scales, 16) ||
+      !aligned(roll_tensor_scale, 4) || !aligned(stats8, 8) || (stats4 && !aligned(stats4, 8)))
+    return NVFP4_ERR_MISALIGNED;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int64_t n = rows * cols;
+  if (!(flags & NVFP4_AMAX_PRECOMPUTED)) {
+    st = nvfp4_tensor_amax(x_train_bf16, n, ws, stream);
+    if (st != NVFP4_OK) return st;
+  }
+  return from_cuda(nvfp4::launch_guided_stats(
+      x_train_bf16, n / 16, hints, hint_bits, ws, codes, scales, tensor_scale,
+      reinterpret_cast<unsigned long long*>(stats4), roll_codes, roll_scales, roll_tensor_scale,
+      reinterpret_cast<unsigned long long*>(stats8), s));
 }
 
 nvfp4_status nvfp4_mismatch_stats(const uint8_t* codes_a, const uint8_t* scales_a,
@@ -273,8 +303,6 @@ nvfp4_status nvfp4_quantize_tile16(const uint16_t* x_bf16, int64_t rows, int64_t
   if (!aligned(x_bf16, 32)) return NVFP4_ERR_MISALIGNED;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (!(flags & NVFP4_AMAX_PRECOMPUTED)) {
-    if (cudaMemsetAsync(ws, 0, NVFP4_WS_WORDS * sizeof(uint32_t), s) != cudaSuccess)
-      return NVFP4_ERR_CUDA;
     if ((st = from_cuda(nvfp4::launch_amax_bf16(x_bf16, rows * cols / 16, ws, s))) != NVFP4_OK)
       return st;
   }

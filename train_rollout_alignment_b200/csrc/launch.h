@@ -28,6 +28,14 @@ cudaError_t launch_quantize_rtn(const uint16_t* x, int64_t nblk, const uint32_t*
 cudaError_t launch_guided(const uint16_t* x, int64_t nblk, const uint8_t* hints, int hint_bits,
                           const uint32_t* ws, uint8_t* codes, uint8_t* scales,
                           float* tensor_scale, unsigned long long* stats4, cudaStream_t s);
+// Guided re-quantization (plain round-to-nearest without hints) that also
+// adds the mismatch counters against the rollout tensor (rcodes, rscales,
+// *rts) to stats8.
+cudaError_t launch_guided_stats(const uint16_t* x, int64_t nblk, const uint8_t* hints,
+                                int hint_bits, const uint32_t* ws, uint8_t* codes, uint8_t* scales,
+                                float* tensor_scale, unsigned long long* stats4,
+                                const uint8_t* rcodes, const uint8_t* rscales, const float* rts,
+                                unsigned long long* stats8, cudaStream_t s);
 cudaError_t launch_emit_hint(const uint8_t* codes, int64_t nblk, int hint_bits, uint8_t* hints,
                              cudaStream_t s);
 cudaError_t launch_mismatch_stats(const uint8_t* ca, const uint8_t* sa, const float* ta,

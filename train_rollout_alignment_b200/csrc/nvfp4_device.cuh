@@ -305,6 +305,36 @@ __device__ __forceinline__ uint32_t block_max_u32(uint32_t v, uint32_t* smem32) 
   return v;
 }
 
+// Scratch words of the amax passes (NVFP4_WS_WORDS in all): ws[0] A, ws[1]
+// warnings, ws[2..3] results of other calls, ws[4] arrival counter and ws[5]
+// running maximum of the pass in flight (zero between calls), ws[6..7] unused.
+constexpr int kWsArrivals = 4;
+constexpr int kWsRunningMax = 5;
+
+// Tensor-wide maximum of the CTAs' values (non-negative FP32 bit patterns,
+// NaN patterns above every number), published without clearing ws first:
+// each CTA folds its value into the running maximum ws[5] and then takes a
+// ticket from the arrival counter ws[4]; the CTA that arrives last reads and
+// zeroes the running maximum, writes ws[0] = A, ws[1] = NVFP4_WARN_NONFINITE
+// iff A is an Inf/NaN pattern (the largest patterns, so the maximum shows
+// whether any was seen), ws[2] = ws[3] = 0, and zeroes the counter.  No CTA
+// waits for another.  Needs ws[4] == ws[5] == 0 on entry, which every call
+// leaves behind.  Called once per CTA by one thread.
+__device__ __forceinline__ void grid_max_publish(uint32_t* ws, uint32_t m) {
+  if (m) atomicMax(ws + kWsRunningMax, m);
+  __threadfence();
+  const uint32_t ticket = atomicAdd(ws + kWsArrivals, 1u);
+  if (ticket == gridDim.x - 1) {
+    __threadfence();
+    const uint32_t A = atomicExch(ws + kWsRunningMax, 0u);
+    ws[0] = A;
+    ws[1] = (A >= 0x7F800000u) ? 1u : 0u;
+    ws[2] = 0u;
+    ws[3] = 0u;
+    atomicExch(ws + kWsArrivals, 0u);
+  }
+}
+
 __device__ __forceinline__ unsigned long long warp_sum_u64(unsigned long long v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);

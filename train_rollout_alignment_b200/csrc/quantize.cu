@@ -14,6 +14,7 @@
 // flight.  HBM-bound: no tensor cores.
 #include "launch.h"
 #include "nvfp4_device.cuh"
+#include "stats_device.cuh"
 
 namespace nvfp4 {
 
@@ -24,8 +25,9 @@ constexpr int kAmaxUnroll = 4;  // 128 bytes in flight per thread: the amax pass
 // ----------------------------------------------------------------- amax
 // Max of |x| over BF16 magnitudes: |x| is the 15 low bits, and for non-negative
 // values the bit patterns order like the numbers, so an unsigned max on packed
-// 16-bit halves is exact.  Result: FP32 bits of A in ws[0] (atomicMax), and
-// NVFP4_WARN_NONFINITE in ws[1] when an Inf/NaN pattern was seen.
+// 16-bit halves is exact.  Result: FP32 bits of A in ws[0] and
+// NVFP4_WARN_NONFINITE in ws[1] when an Inf/NaN pattern was seen, published by
+// the last CTA to finish (grid_max_publish: no clearing pass before it).
 template <int U>
 __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     k_amax_bf16(const uint16_t* __restrict__ x, int64_t nblk, uint32_t* __restrict__ ws) {
@@ -49,10 +51,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
   }
   uint32_t m = max(m2 & 0xFFFFu, m2 >> 16) << 16;  // FP32 bits of the max magnitude
   m = block_max_u32(m, red);
-  if (threadIdx.x == 0) {
-    if (m) atomicMax(ws, m);
-    if (m >= 0x7F800000u) atomicOr(ws + 1, 1u);
-  }
+  if (threadIdx.x == 0) grid_max_publish(ws, m);
 }
 
 // Hint bits of one block (16 codes) from its 8 code bytes.
@@ -181,17 +180,11 @@ __device__ __forceinline__ uint32_t hint_field(const uint8_t* __restrict__ hints
   return 0;
 }
 
+// The guided codes of one block given its reciprocal scale inv (no stores).
 template <int HB>
-__device__ __forceinline__ void guided_block_scaled(const Block16& b, uint32_t hw, uint2 h4,
-                                                    BlockScale bs, int64_t blk,
-                                                    uint8_t* __restrict__ codes,
-                                                    uint8_t* __restrict__ scales, GuidedCounts& cnt,
-                                                    uint32_t one) {
-  if (inv_overflowed(bs.inv)) {  // every element saturated or zero: no decision
-    reinterpret_cast<uint2*>(codes)[blk] = overflow_codes_bf16(b);
-    scales[blk] = (uint8_t)bs.sb;
-    return;
-  }
+__device__ __forceinline__ uint2 guided_codes(const Block16& b, uint32_t hw, uint2 h4, float inv,
+                                              GuidedCounts& cnt, uint32_t one) {
+  if (inv_overflowed(inv)) return overflow_codes_bf16(b);  // every element saturated or zero: no decision
   float x[16];
   unpack_block(b, x);
   const uint32_t h1 = HB == 1 ? hint_spread1(hw) : 0u;
@@ -201,7 +194,7 @@ __device__ __forceinline__ void guided_block_scaled(const Block16& b, uint32_t h
     float v[8], p[8];
 #pragma unroll
     for (int t = 0; t < 8; ++t) {
-      v[t] = __fmul_rn(x[8 * half + t], bs.inv);
+      v[t] = __fmul_rn(x[8 * half + t], inv);
       // one ulp toward zero: bits * one - 1 with one == 1 known only at run
       // time, so it issues as a multiply-add on the FP pipe
       p[t] = __uint_as_float(__float_as_uint(v[t]) * one + 0xFFFFFFFFu);
@@ -215,7 +208,27 @@ __device__ __forceinline__ void guided_block_scaled(const Block16& b, uint32_t h
     else hword = half ? (h1 >> 1) : h1;
     out[half] = guided_select<HB>(R, Zs & 0x77777777u, pz, hword, cnt);
   }
-  reinterpret_cast<uint2*>(codes)[blk] = make_uint2(out[0], out[1]);
+  return make_uint2(out[0], out[1]);
+}
+
+// The round-to-nearest codes of one block given inv (no stores).
+__device__ __forceinline__ uint2 rtn_codes(const Block16& b, float inv) {
+  if (inv_overflowed(inv)) return overflow_codes_bf16(b);
+  float x[16];
+  unpack_block(b, x);
+  float v[16];
+#pragma unroll
+  for (int k = 0; k < 16; ++k) v[k] = __fmul_rn(x[k], inv);
+  return pack_codes16(v);
+}
+
+template <int HB>
+__device__ __forceinline__ void guided_block_scaled(const Block16& b, uint32_t hw, uint2 h4,
+                                                    BlockScale bs, int64_t blk,
+                                                    uint8_t* __restrict__ codes,
+                                                    uint8_t* __restrict__ scales, GuidedCounts& cnt,
+                                                    uint32_t one) {
+  reinterpret_cast<uint2*>(codes)[blk] = guided_codes<HB>(b, hw, h4, bs.inv, cnt, one);
   scales[blk] = (uint8_t)bs.sb;
 }
 
@@ -267,6 +280,86 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
   if (stats4 != nullptr) {
     const unsigned long long vals[3] = {cnt.consulted, cnt.changed, cnt.outside};
     block_add_u64<3>(vals, stats4, red);
+  }
+}
+
+// ----------------------------------------------------------------- guided + counters
+// The train side's guided re-quantization (round-to-nearest for HB = 0) that
+// also counts the mismatches against the rollout's NVFP4 tensor while it has
+// its own codes in registers: the counters of nvfp4_mismatch_stats (side a =
+// rollout, side b = train) without writing the train codes and reading them
+// back.  Per block it reads the rollout's 8 code bytes and scale byte beside
+// its own inputs.  The loop runs warp-uniformly (the counters' dirty-block
+// queue needs every lane of the warp); a lane past the end counts a block of
+// zeros against zeros, which adds nothing.
+constexpr int kGsCtasPerSm = 4;
+
+template <int HB, int U>
+__global__ void __launch_bounds__(kThreads, kGsCtasPerSm)
+    k_guided_stats(const uint16_t* __restrict__ x, int64_t nblk, const uint8_t* __restrict__ hints,
+                   const uint32_t* __restrict__ ws, uint8_t* __restrict__ codes,
+                   uint8_t* __restrict__ scales, float* __restrict__ tensor_scale,
+                   unsigned long long* __restrict__ stats4, const uint8_t* __restrict__ rcodes,
+                   const uint8_t* __restrict__ rscales, const float* __restrict__ rts,
+                   unsigned long long* __restrict__ stats8, uint32_t one) {
+  __shared__ ScaleTables tab;
+  __shared__ StatsShared sm;
+  __shared__ unsigned long long red4[3 * 8];
+  const float s_t = tensor_scale_from_amax(__uint_as_float(ws[0]));
+  if (blockIdx.x == 0 && threadIdx.x == 0) *tensor_scale = s_t;
+  scale_tables_init(tab, s_t);
+  const float ts_r = *rts;
+  const bool same_ts = __float_as_uint(ts_r) == __float_as_uint(s_t);
+  const bool far_all = stats_tables_init(sm, ts_r, s_t);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const uint32_t lt_mask = (1u << lane) - 1u;
+  GuidedCounts gcnt{0u, 0u, 0u};
+  MismatchCounts mc{0u, 0u, 0u, 0u, 0u};
+  int qn = 0;  // warp-uniform queue length
+  const int64_t stride = (int64_t)gridDim.x * kThreads;
+  for (int64_t base = (int64_t)blockIdx.x * kThreads + warp * 32; base < nblk; base += U * stride) {
+    Block16 b[U];
+    uint32_t hw[U], rs[U];
+    uint2 h4[U], rc[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int64_t i = base + u * stride + lane;
+      const int64_t blk = nblk - 1 - i;  // backwards, as the other quantizers
+      b[u] = Block16{};
+      hw[u] = 0u;
+      h4[u] = rc[u] = make_uint2(0u, 0u);
+      rs[u] = 0u;
+      if (i < nblk) {
+        b[u] = ld_block(x + blk * 16);
+        if constexpr (HB != 0) hw[u] = hint_field<HB>(hints, blk, h4[u]);
+        rc[u] = __ldg(reinterpret_cast<const uint2*>(rcodes) + blk);
+        rs[u] = __ldg(rscales + blk);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int64_t i = base + u * stride + lane;
+      const bool valid = i < nblk;
+      const int64_t blk = nblk - 1 - i;
+      uint2 c = make_uint2(0u, 0u);
+      uint32_t sb = 0u;
+      if (valid) {
+        const BlockScale bs = block_scale_bf16(block_amax_bits(b[u]), s_t, tab);
+        if constexpr (HB != 0) c = guided_codes<HB>(b[u], hw[u], h4[u], bs.inv, gcnt, one);
+        else c = rtn_codes(b[u], bs.inv);
+        sb = bs.sb;
+        reinterpret_cast<uint2*>(codes)[blk] = c;
+        scales[blk] = (uint8_t)sb;
+      }
+      count_block(sm, rc[u].x, rc[u].y, c.x, c.y, rs[u], sb, valid, same_ts, far_all, ts_r, s_t,
+                  warp, lane, lt_mask, qn, mc);
+    }
+  }
+  stats_finish(sm, warp, lane, qn, mc, stats8);
+  if (blockIdx.x == 0 && threadIdx.x == 0) atomicAdd(stats8, (unsigned long long)nblk * 16ull);
+  if (HB != 0 && stats4 != nullptr) {
+    const unsigned long long vals[3] = {gcnt.consulted, gcnt.changed, gcnt.outside};
+    block_add_u64<3>(vals, stats4, red4);
   }
 }
 
@@ -452,7 +545,7 @@ int grid_for(int64_t work_items, int items_per_cta, int ctas_per_sm) {
 }
 
 cudaError_t launch_amax_bf16(const uint16_t* x, int64_t nblk, uint32_t* ws, cudaStream_t s) {
-  if (nblk == 0) return cudaSuccess;
+  // nblk == 0 still launches one CTA: it publishes A = 0
   k_amax_bf16<kAmaxUnroll><<<grid_for(nblk, kThreads, kCtasPerSm), kThreads, 0, s>>>(x, nblk, ws);
   return cudaGetLastError();
 }
@@ -482,6 +575,22 @@ cudaError_t launch_guided(const uint16_t* x, int64_t nblk, const uint8_t* hints,
     case 1: k_guided<1, kUnroll><<<g, kThreads, 0, s>>>(x, nblk, hints, ws, codes, scales, tensor_scale, stats4, 1u); break;
     case 2: k_guided<2, kUnroll><<<g, kThreads, 0, s>>>(x, nblk, hints, ws, codes, scales, tensor_scale, stats4, 1u); break;
     case 4: k_guided<4, kUnroll><<<g, kThreads, 0, s>>>(x, nblk, hints, ws, codes, scales, tensor_scale, stats4, 1u); break;
+    default: return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_guided_stats(const uint16_t* x, int64_t nblk, const uint8_t* hints,
+                                int hint_bits, const uint32_t* ws, uint8_t* codes, uint8_t* scales,
+                                float* tensor_scale, unsigned long long* stats4,
+                                const uint8_t* rcodes, const uint8_t* rscales, const float* rts,
+                                unsigned long long* stats8, cudaStream_t s) {
+  const int g = grid_for(nblk, kThreads, kGsCtasPerSm);
+  switch (hints ? hint_bits : 0) {
+    case 0: k_guided_stats<0, kUnroll><<<g, kThreads, 0, s>>>(x, nblk, nullptr, ws, codes, scales, tensor_scale, nullptr, rcodes, rscales, rts, stats8, 1u); break;
+    case 1: k_guided_stats<1, kUnroll><<<g, kThreads, 0, s>>>(x, nblk, hints, ws, codes, scales, tensor_scale, stats4, rcodes, rscales, rts, stats8, 1u); break;
+    case 2: k_guided_stats<2, kUnroll><<<g, kThreads, 0, s>>>(x, nblk, hints, ws, codes, scales, tensor_scale, stats4, rcodes, rscales, rts, stats8, 1u); break;
+    case 4: k_guided_stats<4, kUnroll><<<g, kThreads, 0, s>>>(x, nblk, hints, ws, codes, scales, tensor_scale, stats4, rcodes, rscales, rts, stats8, 1u); break;
     default: return cudaErrorInvalidValue;
   }
   return cudaGetLastError();

@@ -121,10 +121,7 @@ __global__ void __launch_bounds__(kThreads, kRhtCtasPerSm)
   const uint32_t zb = __float_as_uint(zmax);
   uint32_t best = zb >= 0x7F800000u ? zb : __float_as_uint(__fmul_rn(zmax, kInvSqrt32));
   best = block_max_u32(best, red);
-  if (threadIdx.x == 0) {
-    if (best) atomicMax(ws, best);
-    if (best >= 0x7F800000u) atomicOr(ws + 1, 1u);
-  }
+  if (threadIdx.x == 0) grid_max_publish(ws, best);
 }
 
 __device__ __forceinline__ void quantize_block_f32(const float* y, float s_t, const ScaleTables& tab,
@@ -177,14 +174,12 @@ __global__ void __launch_bounds__(kThreads, kRhtCtasPerSm)
 cudaError_t launch_rht_quantize(const uint16_t* x, int64_t nblk, uint64_t seed, uint32_t* ws,
                                 uint8_t* codes, uint8_t* scales, float* tensor_scale,
                                 float* y_out, cudaStream_t s) {
-  cudaError_t err = cudaMemsetAsync(ws, 0, 4 * sizeof(uint32_t), s);
-  if (err != cudaSuccess) return err;
   if (nblk == 0) return launch_set_f32(tensor_scale, 1.0f, s);
   const uint32_t lo = (uint32_t)seed, hi = (uint32_t)(seed >> 32);
   const int64_t ngroups = nblk / 2;  // cols % 32 == 0
   const int g = grid_for(ngroups, kThreads, kRhtCtasPerSm);
   k_rht_amax<<<g, kThreads, 0, s>>>(x, ngroups, lo, hi, ws);
-  err = cudaGetLastError();
+  cudaError_t err = cudaGetLastError();
   if (err != cudaSuccess) return err;
   k_rht_quantize<<<g, kThreads, 0, s>>>(x, ngroups, lo, hi, ws, codes, scales, tensor_scale, y_out);
   return cudaGetLastError();
