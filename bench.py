@@ -152,20 +152,25 @@ class ClockSampler:
 class Stack:
     """Device-resident 48-layer workload and its output buffers."""
 
-    def __init__(self, layers: int, hint_from: int, device, rank: int):
+    def __init__(self, layers: int, hint_from: int, device, rank: int, shape=(ROWS, COLS), gen=None):
+        """gen(layer) -> (train, rollout) BF16 device tensors of `shape`; the
+        throughput stack's generator by default."""
         from train_rollout_alignment_b200 import synthetic as syn
         self.layers, self.hint_from, self.device = layers, hint_from, device
-        self.n = ROWS * COLS
+        rows, cols = self.rows, self.cols = shape
+        self.n = rows * cols
+        if gen is None:
+            gen = lambda l: syn.cfg4_layer_device(l, device, rank, shape)
         self.xt, self.xr = [], []
         for l in range(layers):
-            t, r = syn.cfg4_layer_device(l, device, rank)
+            t, r = gen(l)
             self.xt.append(t)
             self.xr.append(r)
         u8 = dict(dtype=torch.uint8, device=device)
-        self.cr = [torch.empty((ROWS, COLS // 2), **u8) for _ in range(layers)]
-        self.sr = [torch.empty((ROWS, COLS // 16), **u8) for _ in range(layers)]
-        self.ct = [torch.empty((ROWS, COLS // 2), **u8) for _ in range(layers)]
-        self.st = [torch.empty((ROWS, COLS // 16), **u8) for _ in range(layers)]
+        self.cr = [torch.empty((rows, cols // 2), **u8) for _ in range(layers)]
+        self.sr = [torch.empty((rows, cols // 16), **u8) for _ in range(layers)]
+        self.ct = [torch.empty((rows, cols // 2), **u8) for _ in range(layers)]
+        self.st = [torch.empty((rows, cols // 16), **u8) for _ in range(layers)]
         self.hints = [torch.empty(self.n * HINT_BITS // 8, **u8) if l >= hint_from else None
                       for l in range(layers)]
         self.ts = torch.empty((layers, 2), dtype=torch.float32, device=device)
@@ -400,8 +405,9 @@ def run_ours(args, world, rank, local):
     sm_mhz = clocks["sm_max_mhz"] if clocks else 1965.0
     other = time_other_kernels(b, stack, device, peak, sm_mhz)
 
-    other["hint_transport"] = time_hint_transport(stack, device)
+    other["hint_transport"] = time_hint_transport(b, stack, device)
     other.update(time_kv_rows(b, device, peak))
+    other["l2_resident_configs"] = time_small_configs(b, device, peak, rank)
     other["rollout_producer"] = time_producer(b, device)
 
     # ---- end to end through the C ABI with host buffers (rank-local)
@@ -416,12 +422,18 @@ def run_ours(args, world, rank, local):
         chunks = oracle_sample(device, rank, rows_per_core=1024, cores=cores)
         nbytes_cpu, nel = oracle_bytes(chunks)
         dt = time_oracle(chunks)
+        one = chunks[:1]
+        nbytes_1, nel_1 = oracle_bytes(one)
+        dt_1 = time_oracle(one)
         cpu = {"value": round(nbytes_cpu / dt / 1e9, 3), "unit": "GB/s", "cores": len(chunks),
                "kind": "oracle",
                "sample": "%d rows x %d cols of layer 24 (train + rollout), split in %d chunks of 1024 "
                          "rows each quantized as its own tensor, one thread per chunk; %.1f s wall"
                          % (len(chunks) * 1024, COLS, len(chunks), dt),
-               "elements_per_s": round(2 * nel / dt, 1)}
+               "elements_per_s": round(2 * nel / dt, 1),
+               "single_thread": {"value": round(nbytes_1 / dt_1 / 1e9, 4), "unit": "GB/s", "cores": 1,
+                                 "elements_per_s": round(2 * nel_1 / dt_1, 1),
+                                 "sample": "one chunk of 1024 rows on one thread; %.1f s wall" % dt_1}}
 
     launches = 4 * args.layers * args.steps
     out = {
@@ -702,6 +714,58 @@ def time_transpose_alternatives(b, stack, w, codes, scales, ts, sr_out, device, 
     return out
 
 
+def time_small_configs(b, device, peak, rank, reps=30):
+    """The whole step on the two smaller activation workloads, whose tensors
+    fit in L2 (126 MB): the single 1024x2048 N(0,1) tensor with 2-bit hints,
+    and the 24-layer 8192x2048 Student-t (nu=4) stack with 16 outlier channels
+    x50 per layer, hints on layers 12-23 (generated on the GPU: the same
+    distribution as the host generator of the parity tests).  Each timed
+    "warm" back to back (median over steps; L2 may hold the inputs) and
+    "flushed" (L2 flushed before every step).  Flagged L2-resident: these
+    numbers can exceed the HBM roofline."""
+    from train_rollout_alignment_b200 import synthetic as syn
+    flush = (torch.zeros(64 << 20, dtype=torch.float32, device=device),
+             torch.ones(64 << 20, dtype=torch.float32, device=device))
+    s_roll, s_train = torch.cuda.Stream(device), torch.cuda.Stream(device)
+    out = {}
+    x0 = syn.cfg0()
+    to_dev = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(device)
+    stacks = {
+        "single_tensor_1024x2048": Stack(1, 0, device, rank, syn.CFG0_SHAPE,
+                                         gen=lambda l: (to_dev(x0[0]), to_dev(x0[1]))),
+        "moe_activation_stack_24x8192x2048": Stack(
+            syn.CFG1_LAYERS, syn.CFG1_HINT_FROM, device, rank, syn.CFG1_SHAPE,
+            gen=lambda l: syn.cfg1_layer_device(l, device, rank)),
+    }
+    for name, st in stacks.items():
+        nbytes, nel = st.step_bytes(), 2 * st.n * st.layers
+        for _ in range(3):
+            st.step_pipelined(b, s_roll, s_train)
+        res = {}
+        for mode in ("warm", "flushed"):
+            times = []
+            for _ in range(reps):
+                if mode == "flushed":
+                    _flush_l2(flush)
+                torch.cuda._sleep(20_000)
+                e0 = torch.cuda.Event(enable_timing=True)
+                e1 = torch.cuda.Event(enable_timing=True)
+                e0.record()
+                st.step_pipelined(b, s_roll, s_train)
+                e1.record()
+                torch.cuda.synchronize()
+                times.append(e0.elapsed_time(e1) / 1e3)
+            t = statistics.median(times)
+            res[mode] = {"us_per_step": round(t * 1e6, 2), "GB/s": round(nbytes / t / 1e9, 1),
+                         "frac": round(nbytes / t / 1e9 / peak, 4), "elements_per_s": round(nel / t, 1)}
+        res.update({"layers": st.layers, "shape": [st.rows, st.cols], "bytes_per_step": int(nbytes),
+                    "l2_resident": True})
+        out[name] = res
+        del st
+    stacks.clear()
+    return out
+
+
 def time_kv_rows(b, device, peak, reps=10):
     """KV-cache layout (one FP32 scale per (token, head) row): a cache of
     65536 tokens x 16 heads x 128 (head_dim), the rollout's RTN + 2-bit hints
@@ -817,34 +881,66 @@ def time_producer(b, device, reps=10, m=8192, n=4096, k=4096):
     return out
 
 
-def time_hint_transport(stack, device, reps=5):
+def time_hint_transport(b, stack, device, reps=5):
     """The guidance that leaves the GPU in one step: the back-half layers'
-    hints copied to pinned host memory on a copy stream (one copy per layer),
-    median of `reps` transfers; with its size against the uncompacted NVFP4 of
-    the same layers (4 + 0.5 bits per element)."""
+    hints to pinned host memory, (1) through the library (nvfp4_hint_pack:
+    one gather kernel into a staging buffer, then one copy) and (2) as one
+    copy per layer on a copy stream; median of `reps` transfers each, with the
+    size against the uncompacted NVFP4 of the same layers (4 + 0.5 bits per
+    element)."""
     hinted = [l for l in range(stack.layers) if stack.hints[l] is not None]
-    nbytes = sum(stack.hints[l].numel() for l in hinted)
-    host = torch.empty(nbytes, dtype=torch.uint8).pin_memory()
+    streams = [stack.hints[l] for l in hinted]
+    nbytes = sum(t.numel() for t in streams)
+    total = b.nvfp4_hint_pack_size([t.numel() for t in streams])
+    staging = torch.empty(total, dtype=torch.uint8, device=device)
+    host = torch.empty(max(total, nbytes), dtype=torch.uint8).pin_memory()
     copy = torch.cuda.Stream(device)
-    times = []
-    for _ in range(reps):
-        torch.cuda.synchronize()
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
-        with torch.cuda.stream(copy):
-            e0.record(copy)
-            off = 0
-            for l in hinted:
-                n = stack.hints[l].numel()
-                host[off:off + n].copy_(stack.hints[l], non_blocking=True)
-                off += n
-            e1.record(copy)
-        torch.cuda.synchronize()
-        times.append(e0.elapsed_time(e1) / 1e3)
-    t = statistics.median(times)
+
+    def timed(fn):
+        times, gather = [], []
+        for _ in range(reps):
+            torch.cuda.synchronize()
+            ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+            with torch.cuda.stream(copy):
+                fn(ev)
+            torch.cuda.synchronize()
+            times.append(ev[0].elapsed_time(ev[2]) / 1e3)
+            gather.append(ev[0].elapsed_time(ev[1]) / 1e3)
+        return statistics.median(times), statistics.median(gather)
+
+    def packed(ev):
+        ev[0].record(copy)
+        b.nvfp4_hint_pack(streams, staging, stream=copy)
+        ev[1].record(copy)
+        host[:total].copy_(staging, non_blocking=True)
+        ev[2].record(copy)
+
+    def per_layer(ev):
+        ev[0].record(copy)
+        ev[1].record(copy)
+        off = 0
+        for t in streams:
+            host[off:off + t.numel()].copy_(t, non_blocking=True)
+            off += t.numel()
+        ev[2].record(copy)
+
+    # the library call as one unit (gather + its own copy), for the record
+    def library(ev):
+        ev[0].record(copy)
+        ev[1].record(copy)
+        b.nvfp4_hint_pack(streams, staging, host, stream=copy)
+        ev[2].record(copy)
+
+    t_lib, _ = timed(library)
+    t_pack, t_gather = timed(packed)
+    t_direct, _ = timed(per_layer)
     uncompacted = stack.n * len(hinted) * 4.5 / 8
     return {"layers": "%d-%d" % (hinted[0], hinted[-1]), "hint_bits": HINT_BITS, "bytes_per_step": nbytes,
-            "seconds": round(t, 5), "d2h_GB/s": round(nbytes / t / 1e9, 2),
+            "library_call": {"entry": "nvfp4_hint_pack (gather kernel + one copy to pinned host memory)",
+                             "seconds": round(t_lib, 5), "GB/s": round(total / t_lib / 1e9, 2)},
+            "gather_kernel": {"seconds": round(t_gather, 6), "GB/s": round(2 * total / t_gather / 1e9, 1),
+                              "note": "device-to-device, read + write"},
+            "per_layer_copies": {"seconds": round(t_direct, 5), "GB/s": round(nbytes / t_direct / 1e9, 2)},
             "uncompacted_nvfp4_bytes": int(uncompacted), "compaction": round(nbytes / uncompacted, 4),
             "context": "the TRACE explainer sizes guidance transport at 300 GB/s GPU->CPU (GB200); "
                        "this is the B200 host link with pinned memory"}

@@ -301,6 +301,39 @@ nvfp4_status nvfp4_sr_transpose_requant_noalloc(const uint8_t* codes, const uint
                                                 float* tensor_scale_t, void* stream);
 
 /* ======================================================================
+ * Hint transport: the guidance leaves the GPU.
+ * ====================================================================== */
+
+/*
+ * nvfp4_hint_pack -- gather the hint streams of several tensors (the layers
+ * that ship guidance) into one contiguous device staging buffer, then copy it
+ * to host memory.
+ *   [TRACE], guidance-volume paragraph: the guidance of every step leaves the
+ *   GPU (to host memory or storage), and its volume and that transfer are the
+ *   cost of naive alignment; compaction paragraph: only the back half of the
+ *   layers ship guidance, as a few low bits per code (the hint streams of
+ *   nvfp4_quantize_rtn / nvfp4_emit_hint; no further compaction here).
+ *   srcs, sizes: HOST arrays of `count` device pointers and byte counts (any
+ *   size >= 0; a non-empty stream 16-byte aligned).  staging: device buffer
+ *   of nvfp4_hint_pack_size(sizes, count) bytes, 16-byte aligned: stream i
+ *   occupies bytes off_i .. off_i + sizes[i] - 1 with off_i = the sum over
+ *   j < i of sizes[j] rounded up to a multiple of 16; the bytes up to the next
+ *   multiple of 16 are written as 0.  One gather kernel per 128 streams.
+ *   host_dst: NULL (staging only), or host memory of the same size that
+ *   receives the staging buffer by one cudaMemcpyAsync on `stream` after the
+ *   gather (page-locked memory keeps the call asynchronous; pageable memory
+ *   makes the copy synchronous with the host).  Total size below 2^40
+ *   (NVFP4_ERR_SHAPE).  count == 0 or all sizes 0: nothing is enqueued.
+ */
+nvfp4_status nvfp4_hint_pack(const uint8_t* const* srcs, const int64_t* sizes, int64_t count,
+                             uint8_t* staging, uint8_t* host_dst, void* stream);
+
+/* Staging size in bytes for nvfp4_hint_pack (sum of sizes rounded up to 16
+ * each), or -1 for a negative count or size, a NULL `sizes` with count > 0,
+ * or a total of 2^40 or more.  Host-only; touches no device. */
+int64_t nvfp4_hint_pack_size(const int64_t* sizes, int64_t count);
+
+/* ======================================================================
  * KV-cache layout: one FP32 scale per row.
  * ====================================================================== */
 

@@ -20,7 +20,7 @@ def _declared():
     for fname in os.listdir(os.path.join(ROOT, "include")):
         if fname.endswith(".h"):
             text = open(os.path.join(ROOT, "include", fname)).read()
-            names += re.findall(r"^\s*(?:nvfp4_status|const char\*)\s+((?:nvfp4|mxfp8)_\w+)\s*\(", text, re.M)
+            names += re.findall(r"^\s*(?:nvfp4_status|const char\*|int64_t)\s+((?:nvfp4|mxfp8)_\w+)\s*\(", text, re.M)
     return sorted(set(names))
 
 
@@ -232,3 +232,32 @@ def test_validation_of_the_fused_train_pass_without_a_gpu():
     assert call(rc=a + 8) == 2                # rollout codes 16-byte aligned
     assert call(s8=a + 4) == 2                # counters 8-byte aligned
     assert call(s4=a + 4) == 2
+
+
+def test_hint_pack_validation_and_size_without_a_gpu():
+    lib = ctypes.CDLL(_lib_path())
+    P, I64, I = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
+    size = lib.nvfp4_hint_pack_size
+    size.restype = I64
+    size.argtypes = [P, I64]
+    pack = lib.nvfp4_hint_pack
+    pack.restype = I
+    pack.argtypes = [P, P, I64, P, P, P]
+    sizes = (ctypes.c_int64 * 4)(16, 1, 0, 33)
+    assert size(sizes, 4) == 16 + 16 + 0 + 48
+    assert size(sizes, 0) == 0
+    assert size(None, 2) == -1
+    assert size((ctypes.c_int64 * 1)(-1), 1) == -1
+    assert size((ctypes.c_int64 * 1)(1 << 40), 1) == -1
+    a = 1 << 20
+    srcs = (ctypes.c_void_p * 4)(a, a + 16, None, a + 32)
+    assert pack(srcs, sizes, 4, None, None, None) == 1            # no staging buffer
+    assert pack(srcs, sizes, 4, a + 8, None, None) == 2           # staging not 16-byte aligned
+    bad = (ctypes.c_void_p * 4)(a, a + 8, None, a + 32)
+    assert pack(bad, sizes, 4, a, None, None) == 2                # a stream not 16-byte aligned
+    nul = (ctypes.c_void_p * 4)(a, None, None, a)
+    assert pack(nul, sizes, 4, a, None, None) == 1                # a non-empty stream without a pointer
+    assert pack(srcs, sizes, -1, a, None, None) == 1
+    assert pack(None, None, 0, None, None, None) == 0             # nothing to do
+    zeros = (ctypes.c_int64 * 2)(0, 0)
+    assert pack((ctypes.c_void_p * 2)(None, None), zeros, 2, None, None, None) == 0

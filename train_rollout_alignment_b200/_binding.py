@@ -47,6 +47,8 @@ _SIGS = {
     "mxfp8_dequantize": (_I, [_P, _P, _I64, _P, _P]),
     "nvfp4_scales_to_mma": (_I, [_P, _I64, _I64, _P, _P]),
     "nvfp4_wait_selftest": (_I, [_P, _P]),
+    "nvfp4_hint_pack": (_I, [_P, _P, _I64, _P, _P, _P]),
+    "nvfp4_hint_pack_size": (_I64, [_P, _I64]),
     "nvfp4_moe_gemm_quantize": (
         _I, [_P, _P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _P, _P, _P, _P, _P, _P, _I, _P, _P]),
     "nvfp4_gemm_quantize": (
@@ -265,6 +267,29 @@ def nvfp4_moe_gemm_quantize(a_codes, a_scales_mma, a_ts, w_codes, w_scales_mma, 
         _ptr(a_codes), _ptr(a_scales_mma), _ptr(a_ts), _ptr(w_codes), _ptr(w_scales_mma), _ptr(w_ts),
         _ptr(expert_rows), int(experts), int(m), int(n), int(k), _ptr(ws), _ptr(codes), _ptr(scales),
         _ptr(scales_mma), _ptr(tensor_scale), _ptr(hints), int(hint_bits), _ptr(d_out), _stream(stream)))
+
+
+def nvfp4_hint_pack_size(sizes) -> int:
+    arr = (ctypes.c_int64 * max(1, len(sizes)))(*[int(v) for v in sizes])
+    total = _lib.nvfp4_hint_pack_size(arr, len(sizes))
+    if total < 0:
+        raise ValueError("invalid hint stream sizes")
+    return int(total)
+
+
+def nvfp4_hint_pack(streams, staging, host_dst=None, stream=None):
+    """Gather the device byte tensors `streams` into `staging` (each stream on
+    a 16-byte boundary, padding zeroed) and copy that to `host_dst` (a CPU
+    uint8 tensor, pinned for an asynchronous copy) when given."""
+    n = len(streams)
+    srcs = (ctypes.c_void_p * max(1, n))(*[_ptr(t) if t.numel() else None for t in streams])
+    sizes = (ctypes.c_int64 * max(1, n))(*[t.numel() * t.element_size() for t in streams])
+    host = None
+    if host_dst is not None:
+        if host_dst.is_cuda or not host_dst.is_contiguous():
+            raise ValueError("host_dst must be a contiguous CPU tensor")
+        host = host_dst.data_ptr()
+    _check("nvfp4_hint_pack", _lib.nvfp4_hint_pack(srcs, sizes, n, _ptr(staging), host, _stream(stream)))
 
 
 def nvfp4_wait_selftest(ws, stream=None):

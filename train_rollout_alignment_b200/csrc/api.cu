@@ -455,6 +455,37 @@ nvfp4_status nvfp4_moe_gemm_quantize(const uint8_t* a_codes, const uint8_t* a_sc
                        scales_mma, tensor_scale, hints, hint_bits, d_out, stream);
 }
 
+int64_t nvfp4_hint_pack_size(const int64_t* sizes, int64_t count) {
+  if (count < 0 || (count > 0 && !sizes)) return -1;
+  int64_t total = 0;
+  for (int64_t i = 0; i < count; ++i) {
+    if (sizes[i] < 0 || sizes[i] >= kMaxElems) return -1;
+    total += (sizes[i] + 15) / 16 * 16;
+    if (total >= kMaxElems) return -1;
+  }
+  return total;
+}
+
+nvfp4_status nvfp4_hint_pack(const uint8_t* const* srcs, const int64_t* sizes, int64_t count,
+                             uint8_t* staging, uint8_t* host_dst, void* stream) {
+  if (count < 0 || (count > 0 && (!srcs || !sizes))) return NVFP4_ERR_INVALID_ARG;
+  for (int64_t i = 0; i < count; ++i) {
+    if (sizes[i] < 0) return NVFP4_ERR_INVALID_ARG;
+    if (sizes[i] > 0 && !srcs[i]) return NVFP4_ERR_INVALID_ARG;
+  }
+  const int64_t total = nvfp4_hint_pack_size(sizes, count);
+  if (total < 0) return NVFP4_ERR_SHAPE;
+  if (total == 0) return NVFP4_OK;
+  if (!staging) return NVFP4_ERR_INVALID_ARG;
+  if (!aligned(staging, 16)) return NVFP4_ERR_MISALIGNED;
+  for (int64_t i = 0; i < count; ++i)
+    if (sizes[i] > 0 && !aligned(srcs[i], 16)) return NVFP4_ERR_MISALIGNED;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  nvfp4_status st = from_cuda(nvfp4::launch_hint_pack(srcs, sizes, count, staging, s));
+  if (st != NVFP4_OK || !host_dst) return st;
+  return from_cuda(cudaMemcpyAsync(host_dst, staging, (size_t)total, cudaMemcpyDeviceToHost, s));
+}
+
 nvfp4_status nvfp4_wait_selftest(uint32_t* ws, void* stream) {
   if (!ws) return NVFP4_ERR_INVALID_ARG;
   if (!aligned(ws, 16)) return NVFP4_ERR_MISALIGNED;

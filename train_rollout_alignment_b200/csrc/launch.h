@@ -78,6 +78,11 @@ cudaError_t launch_gemm_quantize(const uint8_t* a_codes, const uint8_t* a_sf, co
                                  uint8_t* scales_mma, float* tensor_scale, uint8_t* hints,
                                  int hint_bits, float* d_out, cudaStream_t s);
 cudaError_t launch_wait_selftest(uint32_t* ws, cudaStream_t s);
+// Hint transport: gathers `count` device streams (srcs/sizes are host arrays)
+// into `staging`, each stream starting on a 16-byte boundary, padding zeroed.
+constexpr int kPackMaxStreams = 128;  // streams per launch (more take several launches)
+cudaError_t launch_hint_pack(const uint8_t* const* srcs, const int64_t* sizes, int64_t count,
+                             uint8_t* staging, cudaStream_t s);
 cudaError_t launch_set_f32(float* dst, float value, cudaStream_t s);
 
 }  // namespace nvfp4

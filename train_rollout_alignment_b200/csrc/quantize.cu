@@ -18,8 +18,14 @@
 
 namespace nvfp4 {
 
-constexpr int kCtasPerSm = 4;
-constexpr int kUnroll = 2;
+#ifndef NVFP4_STREAM_CTAS
+#define NVFP4_STREAM_CTAS 4
+#endif
+#ifndef NVFP4_STREAM_UNROLL
+#define NVFP4_STREAM_UNROLL 2
+#endif
+constexpr int kCtasPerSm = NVFP4_STREAM_CTAS;
+constexpr int kUnroll = NVFP4_STREAM_UNROLL;
 constexpr int kAmaxUnroll = 4;  // 128 bytes in flight per thread: the amax pass has no other work
 
 // ----------------------------------------------------------------- amax
@@ -292,7 +298,14 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 // its own inputs.  The loop runs warp-uniformly (the counters' dirty-block
 // queue needs every lane of the warp); a lane past the end counts a block of
 // zeros against zeros, which adds nothing.
-constexpr int kGsCtasPerSm = 4;
+#ifndef NVFP4_GS_CTAS
+#define NVFP4_GS_CTAS 4
+#endif
+#ifndef NVFP4_GS_UNROLL
+#define NVFP4_GS_UNROLL 2
+#endif
+constexpr int kGsCtasPerSm = NVFP4_GS_CTAS;
+constexpr int kGsUnroll = NVFP4_GS_UNROLL;
 
 template <int HB, int U>
 __global__ void __launch_bounds__(kThreads, kGsCtasPerSm)
@@ -587,10 +600,10 @@ cudaError_t launch_guided_stats(const uint16_t* x, int64_t nblk, const uint8_t* 
                                 unsigned long long* stats8, cudaStream_t s) {
   const int g = grid_for(nblk, kThreads, kGsCtasPerSm);
   switch (hints ? hint_bits : 0) {
-    case 0: k_guided_stats<0, kUnroll><<<g, kThreads, 0, s>>>(x, nblk, nullptr, ws, codes, scales, tensor_scale, nullptr, rcodes, rscales, rts, stats8, 1u); break;
-    case 1: k_guided_stats<1, kUnroll><<<g, kThreads, 0, s>>>(x, nblk, hints, ws, codes, scales, tensor_scale, stats4, rcodes, rscales, rts, stats8, 1u); break;
-    case 2: k_guided_stats<2, kUnroll><<<g, kThreads, 0, s>>>(x, nblk, hints, ws, codes, scales, tensor_scale, stats4, rcodes, rscales, rts, stats8, 1u); break;
-    case 4: k_guided_stats<4, kUnroll><<<g, kThreads, 0, s>>>(x, nblk, hints, ws, codes, scales, tensor_scale, stats4, rcodes, rscales, rts, stats8, 1u); break;
+    case 0: k_guided_stats<0, kGsUnroll><<<g, kThreads, 0, s>>>(x, nblk, nullptr, ws, codes, scales, tensor_scale, nullptr, rcodes, rscales, rts, stats8, 1u); break;
+    case 1: k_guided_stats<1, kGsUnroll><<<g, kThreads, 0, s>>>(x, nblk, hints, ws, codes, scales, tensor_scale, stats4, rcodes, rscales, rts, stats8, 1u); break;
+    case 2: k_guided_stats<2, kGsUnroll><<<g, kThreads, 0, s>>>(x, nblk, hints, ws, codes, scales, tensor_scale, stats4, rcodes, rscales, rts, stats8, 1u); break;
+    case 4: k_guided_stats<4, kGsUnroll><<<g, kThreads, 0, s>>>(x, nblk, hints, ws, codes, scales, tensor_scale, stats4, rcodes, rscales, rts, stats8, 1u); break;
     default: return cudaErrorInvalidValue;
   }
   return cudaGetLastError();

@@ -18,8 +18,19 @@ def world() -> tuple[int, int, int]:
             int(os.environ.get("LOCAL_RANK", "0")))
 
 
+def nccl_init_log() -> None:
+    """Keep NCCL's communicator set-up log (rank count, transports, NVLS) on,
+    written to stderr so that stdout carries only the result line; a caller's
+    own NCCL_DEBUG settings win."""
+    os.environ.setdefault("NCCL_DEBUG", "INFO")
+    os.environ.setdefault("NCCL_DEBUG_SUBSYS", "INIT")
+    os.environ.setdefault("NCCL_DEBUG_FILE", "/dev/stderr")
+
+
 def init(backend: str, timeout_s: float = 300.0) -> None:
     if not dist.is_initialized():
+        if backend == "nccl":
+            nccl_init_log()
         dist.init_process_group(backend, timeout=datetime.timedelta(seconds=timeout_s))
 
 

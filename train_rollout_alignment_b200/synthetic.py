@@ -158,3 +158,28 @@ def cfg4_layer_device(layer: int, device, rank: int = 0, shape=CFG4_SHAPE):
     rb = eps.to(torch.bfloat16)
     del eps
     return xb, rb
+
+
+def cfg1_layer_device(layer: int, device, rank: int = 0, shape=CFG1_SHAPE):
+    """MoE activation layer generated on the GPU, for timing: Student-t with
+    nu = 4 as z / sqrt(chi2_4 / 4) (z and the four squared normals of chi2_4
+    independent N(0, 1)), 16 random outlier channels x50, rollout copy as
+    everywhere.  Same distribution as cfg1_layer, not the same numbers (the
+    parity tests use cfg1_layer).  Returns (train, rollout) torch.bfloat16."""
+    rows, cols = shape
+    g = torch.Generator(device=device)
+    g.manual_seed((1 << 40) | (rank << 20) | layer)
+    chi2 = torch.zeros(rows, cols, device=device, dtype=torch.float32)
+    for _ in range(4):
+        z = torch.randn(rows, cols, device=device, dtype=torch.float32, generator=g)
+        chi2.addcmul_(z, z)
+    x = torch.randn(rows, cols, device=device, dtype=torch.float32, generator=g)
+    x.div_(chi2.div_(4.0).sqrt_())
+    del chi2
+    ch = torch.randperm(cols, device=device, generator=g)[:16]
+    x[:, ch] *= 50.0
+    xb = x.to(torch.bfloat16)
+    eps = torch.randn(rows, cols, device=device, dtype=torch.float32, generator=g)
+    eps.mul_(ROLLOUT_REL_STD).add_(1.0)
+    eps.mul_(xb.float())
+    return xb, eps.to(torch.bfloat16)
