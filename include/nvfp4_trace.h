@@ -517,10 +517,13 @@ nvfp4_status nvfp4_gemm_quantize(const uint8_t* a_codes, const uint8_t* a_scales
  *   all-to-all that delivers them is not part of this call: A arrives
  *   grouped, expert e owning rows expert_rows[e] .. expert_rows[e + 1] - 1.
  *   expert_rows: device int32 [experts + 1], non-decreasing, expert_rows[0] =
- *   0, expert_rows[experts] = m, every entry a multiple of 128 (pad each
+ *   0, expert_rows[experts] <= m, every entry a multiple of 128 (pad each
  *   expert's tokens to 128 rows); an entry breaking that gives wrong rows,
  *   never an out-of-bounds read (every 128-row tile takes the weight of the
- *   expert owning its first row).
+ *   expert owning its first row).  Rows expert_rows[experts] .. m - 1 are not
+ *   computed and their outputs are left unchanged, so m may be the capacity
+ *   of a grouping the GPU produced (nvfp4_moe_route) without the host
+ *   reading its size back.
  *   w_codes [experts, n, k/2] and w_scales_mma (each expert's scales in the
  *   MMA layout, concatenated, i.e. the MMA layout of [experts * n, k/16]);
  *   w_tensor_scales [experts] floats (device).  D rows follow A's rows, row r
@@ -536,6 +539,54 @@ nvfp4_status nvfp4_moe_gemm_quantize(const uint8_t* a_codes, const uint8_t* a_sc
                                      int64_t n, int64_t k, uint32_t* ws, uint8_t* codes,
                                      uint8_t* scales, uint8_t* scales_mma, float* tensor_scale,
                                      uint8_t* hints, int hint_bits, float* d_out, void* stream);
+
+/*
+ * nvfp4_moe_route -- group the routed tokens by expert, on the GPU.
+ *   [TML4], communication paragraph: tokens are sent to the experts in NVFP4;
+ *   the expert GEMM (nvfp4_moe_gemm_quantize) reads each expert's rows as one
+ *   contiguous group padded to a multiple of 128 rows.  The pages give no
+ *   layout; this is the reading taken: the assignments a = token * top_k +
+ *   slot (topk_ids [tokens, top_k] int32, device) are grouped by expert id,
+ *   in increasing a within an expert (a stable counting sort: every call
+ *   gives the same rows); an id outside 0 .. experts - 1 drops its
+ *   assignment.
+ *   Outputs (device int32): expert_rows [experts + 1] (group offsets, each a
+ *   multiple of 128, expert_rows[0] = 0); row_src [m_cap] (the assignment each
+ *   grouped row holds, -1 for a padding row and for every row from
+ *   expert_rows[experts] on); assign_row [tokens * top_k] (the row of each
+ *   assignment, -1 if dropped).  m_cap >= nvfp4_moe_rows_cap(tokens * top_k,
+ *   experts), the largest grouping possible (NVFP4_ERR_SHAPE otherwise).
+ *   ws: nvfp4_moe_route_ws_words(tokens * top_k, experts) int32 words of
+ *   device scratch, 16-byte aligned (no initial value needed).
+ *   1 <= experts <= 1024, top_k >= 1, tokens * top_k < 2^31 - 2^17.
+ */
+nvfp4_status nvfp4_moe_route(const int32_t* topk_ids, int64_t tokens, int64_t top_k,
+                             int64_t experts, int32_t* ws, int32_t* expert_rows,
+                             int32_t* row_src, int64_t m_cap, int32_t* assign_row, void* stream);
+
+/* Largest number of grouped rows for `assignments` over `experts` experts:
+ * (assignments + 127 * experts) rounded down to a multiple of 128, or -1 for
+ * arguments nvfp4_moe_route rejects.  Host-only. */
+int64_t nvfp4_moe_rows_cap(int64_t assignments, int64_t experts);
+/* Scratch words of nvfp4_moe_route (experts * (ceil(assignments / 2048) + 1),
+ * at least one chunk), or -1.  Host-only. */
+int64_t nvfp4_moe_route_ws_words(int64_t assignments, int64_t experts);
+
+/*
+ * nvfp4_moe_gather -- the routed tokens' NVFP4 rows in the grouped layout of
+ * nvfp4_moe_gemm_quantize's A operand.
+ *   codes [tokens, k/2] and scales [tokens, k/16] (row layout, as the
+ *   quantizers write them) of the tokens; row_src [m_cap] from
+ *   nvfp4_moe_route (any value outside 0 .. tokens * top_k - 1 is a padding
+ *   row); grouped row r holds token row_src[r] / top_k.
+ *   -> a_codes [m_cap, k/2] and a_scales_mma (the tensor-core layout of
+ *   [m_cap, k/16], nvfp4_scales_to_mma's); padding rows are zero codes with
+ *   zero scales (their products are 0).  k % 64 == 0, m_cap % 128 == 0
+ *   (NVFP4_ERR_SHAPE); codes, scales, a_codes, a_scales_mma 16-byte aligned.
+ */
+nvfp4_status nvfp4_moe_gather(const uint8_t* codes, const uint8_t* scales, int64_t tokens,
+                              int64_t k, const int32_t* row_src, int64_t m_cap, int64_t top_k,
+                              uint8_t* a_codes, uint8_t* a_scales_mma, void* stream);
 
 /*
  * nvfp4_wait_selftest -- failure detection of the producer pipeline, without

@@ -425,6 +425,33 @@ def moe_gemm_nvfp4(a_codes, a_scales, a_ts: float, w_codes, w_scales, w_ts, expe
     return d, dabs
 
 
+def moe_route(topk_ids, experts: int):
+    """The dispatch of routed tokens to the experts ("Thinking Machines Lab
+    releases 4-bit training", communication paragraph: tokens are sent to the
+    experts in NVFP4; configuration paragraph: the MoE forward runs in NVFP4).
+    The pages give no layout; the reading taken: the (token, slot)
+    assignments a = token * top_k + slot are grouped by expert, in increasing
+    a within an expert, and every expert's group is padded with empty rows to
+    a multiple of 128 (the tile height of the expert GEMM); an assignment whose
+    expert id is outside 0 .. experts - 1 is dropped.
+
+    -> (expert_rows [experts + 1], row_src [expert_rows[-1]] with the
+    assignment of each grouped row or -1 for a padding row, assign_row [A]
+    with the grouped row of each assignment or -1), all int64."""
+    ids = np.asarray(topk_ids, dtype=np.int64).reshape(-1)
+    rows = [0]
+    row_src = []
+    assign_row = np.full(ids.size, -1, np.int64)
+    for e in range(experts):
+        idx = np.nonzero(ids == e)[0]
+        start = rows[-1]
+        assign_row[idx] = start + np.arange(idx.size)
+        pad = (-idx.size) % 128
+        row_src.extend(idx.tolist() + [-1] * pad)
+        rows.append(start + idx.size + pad)
+    return np.array(rows, np.int64), np.array(row_src, np.int64), assign_row
+
+
 def scales_to_mma(scales, rows: int, sf_cols: int) -> np.ndarray:
     """Row-layout block scales [rows, sf_cols] -> the 128x4-tiled MMA layout."""
     scales = np.ascontiguousarray(scales, dtype=np.uint8).reshape(-1)

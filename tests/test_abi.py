@@ -261,3 +261,33 @@ def test_hint_pack_validation_and_size_without_a_gpu():
     assert pack(None, None, 0, None, None, None) == 0             # nothing to do
     zeros = (ctypes.c_int64 * 2)(0, 0)
     assert pack((ctypes.c_void_p * 2)(None, None), zeros, 2, None, None, None) == 0
+
+
+def test_moe_dispatch_sizes_and_validation_without_a_gpu():
+    lib = ctypes.CDLL(_lib_path())
+    P, I64, I = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
+    cap = lib.nvfp4_moe_rows_cap
+    cap.restype, cap.argtypes = I64, [I64, I64]
+    words = lib.nvfp4_moe_route_ws_words
+    words.restype, words.argtypes = I64, [I64, I64]
+    assert cap(6, 3) == 384 and cap(0, 1) == 0 and cap(256, 1) == 256 and cap(257, 2) == 384
+    assert cap(-1, 3) == -1 and cap(5, 0) == -1 and cap(5, 1025) == -1
+    assert words(6, 3) == 2 * 3 and words(4097, 5) == (3 + 1) * 5
+    route = lib.nvfp4_moe_route
+    route.restype = I
+    route.argtypes = [P, I64, I64, I64, P, P, P, I64, P, P]
+    a = 1 << 20
+    assert route(a, 3, 2, 3, a, a, a, 384, a, None) != 3              # capacity large enough
+    assert route(a, 3, 2, 3, a, a, a, 383, a, None) == 3              # capacity too small
+    assert route(a, 3, 2, 2000, a, a, a, 1 << 20, a, None) == 3       # too many experts
+    assert route(a, 3, 0, 3, a, a, a, 384, a, None) == 1              # top_k 0
+    assert route(a, 3, 2, 3, None, a, a, 384, a, None) == 1           # no scratch
+    assert route(a + 2, 3, 2, 3, a, a, a, 384, a, None) == 2          # ids not 4-byte aligned
+    gather = lib.nvfp4_moe_gather
+    gather.restype = I
+    gather.argtypes = [P, P, I64, I64, P, I64, I64, P, P, P]
+    assert gather(a, a, 3, 96, a, 128, 2, a, a, None) == 3            # k % 64
+    assert gather(a, a, 3, 128, a, 100, 2, a, a, None) == 3           # m_cap % 128
+    assert gather(a, a, 3, 128, a, 128, 2, a + 8, a, None) == 2       # a_codes 16-byte aligned
+    assert gather(a, a, 3, 128, None, 128, 2, a, a, None) == 1
+    assert gather(None, None, 0, 128, None, 0, 2, None, None, None) == 0

@@ -182,3 +182,33 @@ def test_gemm_random_shapes_and_kinds(case):
     st = float(ta) * float(tb)
     assert np.allclose(d, (A @ B.T) * st, rtol=1e-15, atol=0.0)
     assert np.allclose(dabs, (np.abs(A) @ np.abs(B).T) * abs(st), rtol=1e-15, atol=0.0)
+
+
+# ----------------------------------------------------------------- dispatch
+def test_moe_route_worked_example():
+    """3 tokens, top-2, 3 experts, worked by hand: assignments a = 2 t + j
+    with experts [[1, 0], [1, 2], [0, 1]] -> expert 0 gets a = 1, 4; expert 1
+    a = 0, 2, 5; expert 2 a = 3; each group padded to 128 rows."""
+    rows, src, arow = oracle.moe_route([[1, 0], [1, 2], [0, 1]], 3)
+    assert list(rows) == [0, 128, 256, 384]
+    assert list(src[:2]) == [1, 4] and list(src[128:131]) == [0, 2, 5] and src[256] == 3
+    assert np.all(src[2:128] == -1) and np.all(src[131:256] == -1) and np.all(src[257:] == -1)
+    assert list(arow) == [128, 0, 129, 256, 1, 130]
+
+
+def test_moe_route_invariants():
+    rng = np.random.Generator(np.random.PCG64(5))
+    tokens, top_k, E = 500, 3, 7
+    ids = rng.integers(-1, E + 1, (tokens, top_k))     # some ids out of range: dropped
+    rows, src, arow = oracle.moe_route(ids, E)
+    flat = ids.reshape(-1)
+    assert rows[0] == 0 and np.all(np.diff(rows) % 128 == 0) and np.all(np.diff(rows) >= 0)
+    for e in range(E):
+        grp = src[rows[e]:rows[e + 1]]
+        real = grp[grp >= 0]
+        assert np.array_equal(real, np.nonzero(flat == e)[0])      # all of expert e, in order
+        assert np.all(grp[real.size:] == -1) and rows[e + 1] - rows[e] - real.size < 128
+    ok = (flat >= 0) & (flat < E)
+    assert np.all(arow[~ok] == -1)
+    assert np.array_equal(src[arow[ok]], np.nonzero(ok)[0])        # the inverse permutation
+    assert rows[-1] <= ((ok.sum() + 127 * E + 127) // 128) * 128

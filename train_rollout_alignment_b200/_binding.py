@@ -49,6 +49,10 @@ _SIGS = {
     "nvfp4_wait_selftest": (_I, [_P, _P]),
     "nvfp4_hint_pack": (_I, [_P, _P, _I64, _P, _P, _P]),
     "nvfp4_hint_pack_size": (_I64, [_P, _I64]),
+    "nvfp4_moe_rows_cap": (_I64, [_I64, _I64]),
+    "nvfp4_moe_route_ws_words": (_I64, [_I64, _I64]),
+    "nvfp4_moe_route": (_I, [_P, _I64, _I64, _I64, _P, _P, _P, _I64, _P, _P]),
+    "nvfp4_moe_gather": (_I, [_P, _P, _I64, _I64, _P, _I64, _I64, _P, _P, _P]),
     "nvfp4_moe_gemm_quantize": (
         _I, [_P, _P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _P, _P, _P, _P, _P, _P, _I, _P, _P]),
     "nvfp4_gemm_quantize": (
@@ -290,6 +294,34 @@ def nvfp4_hint_pack(streams, staging, host_dst=None, stream=None):
             raise ValueError("host_dst must be a contiguous CPU tensor")
         host = host_dst.data_ptr()
     _check("nvfp4_hint_pack", _lib.nvfp4_hint_pack(srcs, sizes, n, _ptr(staging), host, _stream(stream)))
+
+
+def nvfp4_moe_rows_cap(assignments: int, experts: int) -> int:
+    v = int(_lib.nvfp4_moe_rows_cap(int(assignments), int(experts)))
+    if v < 0:
+        raise ValueError("unsupported routing size")
+    return v
+
+
+def nvfp4_moe_route_ws_words(assignments: int, experts: int) -> int:
+    v = int(_lib.nvfp4_moe_route_ws_words(int(assignments), int(experts)))
+    if v < 0:
+        raise ValueError("unsupported routing size")
+    return v
+
+
+def nvfp4_moe_route(topk_ids, experts, ws, expert_rows, row_src, assign_row, stream=None):
+    """topk_ids: int32 [tokens, top_k] (CUDA)."""
+    tokens, top_k = int(topk_ids.shape[0]), int(topk_ids.shape[1])
+    _check("nvfp4_moe_route", _lib.nvfp4_moe_route(
+        _ptr(topk_ids), tokens, top_k, int(experts), _ptr(ws), _ptr(expert_rows), _ptr(row_src),
+        int(row_src.numel()), _ptr(assign_row), _stream(stream)))
+
+
+def nvfp4_moe_gather(codes, scales, tokens, k, row_src, top_k, a_codes, a_scales_mma, stream=None):
+    _check("nvfp4_moe_gather", _lib.nvfp4_moe_gather(
+        _ptr(codes), _ptr(scales), int(tokens), int(k), _ptr(row_src), int(row_src.numel()), int(top_k),
+        _ptr(a_codes), _ptr(a_scales_mma), _stream(stream)))
 
 
 def nvfp4_wait_selftest(ws, stream=None):

@@ -486,6 +486,55 @@ nvfp4_status nvfp4_hint_pack(const uint8_t* const* srcs, const int64_t* sizes, i
   return from_cuda(cudaMemcpyAsync(host_dst, staging, (size_t)total, cudaMemcpyDeviceToHost, s));
 }
 
+int64_t nvfp4_moe_rows_cap(int64_t assignments, int64_t experts) {
+  if (assignments < 0 || experts < 1 || experts > nvfp4::kRouteMaxExperts ||
+      assignments >= (int64_t(1) << 31) - 128 * 1024)
+    return -1;
+  return (assignments + 127 * experts) / 128 * 128;  // each group adds < 128 padding rows
+}
+
+int64_t nvfp4_moe_route_ws_words(int64_t assignments, int64_t experts) {
+  if (nvfp4_moe_rows_cap(assignments, experts) < 0) return -1;
+  return (nvfp4::route_chunks(assignments) + 1) * experts;
+}
+
+nvfp4_status nvfp4_moe_route(const int32_t* topk_ids, int64_t tokens, int64_t top_k, int64_t experts,
+                             int32_t* ws, int32_t* expert_rows, int32_t* row_src, int64_t m_cap,
+                             int32_t* assign_row, void* stream) {
+  if (tokens < 0 || top_k < 1 || experts < 1) return NVFP4_ERR_INVALID_ARG;
+  if (experts > nvfp4::kRouteMaxExperts || top_k > (int64_t(1) << 20)) return NVFP4_ERR_SHAPE;
+  if (tokens > (int64_t(1) << 31) / top_k) return NVFP4_ERR_SHAPE;
+  const int64_t A = tokens * top_k;
+  const int64_t cap = nvfp4_moe_rows_cap(A, experts);
+  if (cap < 0) return NVFP4_ERR_SHAPE;
+  if (m_cap < cap) return NVFP4_ERR_SHAPE;   // too small to hold every possible grouping
+  if (!ws || !expert_rows || !row_src || (A > 0 && (!topk_ids || !assign_row)))
+    return NVFP4_ERR_INVALID_ARG;
+  if (!aligned(ws, 16) || !aligned(expert_rows, 4) || !aligned(row_src, 4) ||
+      !aligned(topk_ids, 4) || !aligned(assign_row, 4))
+    return NVFP4_ERR_MISALIGNED;
+  return from_cuda(nvfp4::launch_moe_route(topk_ids, A, (int)experts, ws, expert_rows, row_src, m_cap,
+                                           assign_row, static_cast<cudaStream_t>(stream)));
+}
+
+nvfp4_status nvfp4_moe_gather(const uint8_t* codes, const uint8_t* scales, int64_t tokens, int64_t k,
+                              const int32_t* row_src, int64_t m_cap, int64_t top_k, uint8_t* a_codes,
+                              uint8_t* a_scales_mma, void* stream) {
+  if (tokens < 0 || k < 0 || m_cap < 0 || top_k < 1) return NVFP4_ERR_INVALID_ARG;
+  if (k % 64 != 0 || m_cap % 128 != 0) return NVFP4_ERR_SHAPE;
+  if (tokens > (int64_t(1) << 31) / top_k || (k != 0 && m_cap > kMaxElems / k) ||
+      (k != 0 && tokens > kMaxElems / k))
+    return NVFP4_ERR_SHAPE;
+  if (m_cap == 0 || k == 0) return NVFP4_OK;
+  if (!row_src || !a_codes || !a_scales_mma || (tokens > 0 && (!codes || !scales)))
+    return NVFP4_ERR_INVALID_ARG;
+  if (!aligned(codes, 16) || !aligned(scales, 16) || !aligned(row_src, 4) || !aligned(a_codes, 16) ||
+      !aligned(a_scales_mma, 16))
+    return NVFP4_ERR_MISALIGNED;
+  return from_cuda(nvfp4::launch_moe_gather(codes, scales, k, row_src, m_cap, tokens * top_k, top_k,
+                                            a_codes, a_scales_mma, static_cast<cudaStream_t>(stream)));
+}
+
 nvfp4_status nvfp4_wait_selftest(uint32_t* ws, void* stream) {
   if (!ws) return NVFP4_ERR_INVALID_ARG;
   if (!aligned(ws, 16)) return NVFP4_ERR_MISALIGNED;

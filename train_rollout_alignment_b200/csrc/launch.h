@@ -78,6 +78,15 @@ cudaError_t launch_gemm_quantize(const uint8_t* a_codes, const uint8_t* a_sf, co
                                  uint8_t* scales_mma, float* tensor_scale, uint8_t* hints,
                                  int hint_bits, float* d_out, cudaStream_t s);
 cudaError_t launch_wait_selftest(uint32_t* ws, cudaStream_t s);
+// MoE dispatch on one GPU: stable grouping of the top-k assignments by expert
+// (ws: route_ws_words(A, E) words) and the gather of the routed NVFP4 rows.
+constexpr int kRouteMaxExperts = 1024;
+int64_t route_chunks(int64_t assignments);
+cudaError_t launch_moe_route(const int32_t* ids, int64_t A, int E, int32_t* ws, int32_t* expert_rows,
+                             int32_t* row_src, int64_t m_cap, int32_t* assign_row, cudaStream_t s);
+cudaError_t launch_moe_gather(const uint8_t* codes, const uint8_t* scales, int64_t k,
+                              const int32_t* row_src, int64_t m_cap, int64_t A, int64_t top_k,
+                              uint8_t* a_codes, uint8_t* a_scales_mma, cudaStream_t s);
 // Hint transport: gathers `count` device streams (srcs/sizes are host arrays)
 // into `staging`, each stream starting on a 16-byte boundary, padding zeroed.
 constexpr int kPackMaxStreams = 128;  // streams per launch (more take several launches)

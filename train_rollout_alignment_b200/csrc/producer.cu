@@ -226,6 +226,14 @@ __global__ void __launch_bounds__(kProducerThreads, kCtasPerSm)
     tc_fence_before();
   }
   const float s_t = tensor_scale_from_amax(__uint_as_float(ws[0]));
+  // MoE form: the rows past group_rows[groups] (within m) are not computed;
+  // every role reads the same value, so their tile loops agree
+  if (group_rows != nullptr) {
+    const int64_t m_rows = (int64_t)(tiles / n_tiles_n) * kBM;
+    int64_t used = (int64_t)__ldg(group_rows + groups);
+    used = used < 0 ? 0 : (used > m_rows ? m_rows : used);
+    tiles = (int)((used / kBM) * n_tiles_n);
+  }
   scale_tables_init_f32(tab, s_t);  // ends with __syncthreads
   tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + kOffTmemSlot);
