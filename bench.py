@@ -64,19 +64,31 @@ BYTES = {
 SPEC_HBM_GBS = 8000.0  # B200 HBM3e data-sheet bandwidth, reported beside the measured peak
 # Philox-bound kernels: each random word costs 18 32x32->64-bit multiplies per
 # element (10 rounds of 2; the first round's product of the shared draw word is
-# computed once, the last round needs one), and a B200 SM retires such
-# multiplies for 32 lanes per clock (measured with an instruction-throughput
-# probe: mul.wide.u32 30.6, mul.hi.u32 31.8 lanes/clk/SM).
+# computed once, the last round needs one).  The multiply rate per SM is
+# measured in the same run (nvfp4_measure_mul_wide: one 1024-thread CTA per SM,
+# 8 independent multiply chains per thread, SM clock cycles read in the kernel).
 PHILOX_MULS_PER_ELEM = 18
-WIDE_MUL_LANES_PER_CLK = 32
 
 
-def _philox_roofline(elems_per_s, sms, sm_mhz):
-    peak = sms * sm_mhz * 1e6 * WIDE_MUL_LANES_PER_CLK / PHILOX_MULS_PER_ELEM
+def measure_mul_wide(b, device, iters=20000):
+    """32x32->64-bit multiplies per clock per SM, median over the SMs."""
+    sms = torch.cuda.get_device_properties(device).multi_processor_count
+    cycles = torch.zeros(sms, dtype=torch.int64, device=device)
+    sink = torch.zeros(sms, dtype=torch.int32, device=device)
+    b.nvfp4_measure_mul_wide(sms, 100, cycles, sink)           # warm-up
+    b.nvfp4_measure_mul_wide(sms, iters, cycles, sink)
+    torch.cuda.synchronize()
+    c = statistics.median(cycles.cpu().tolist())
+    return 1024 * 8 * iters / c
+
+
+def _philox_roofline(elems_per_s, sms, sm_mhz, lanes_per_clk):
+    peak = sms * sm_mhz * 1e6 * lanes_per_clk / PHILOX_MULS_PER_ELEM
     return {"bound": "alu", "unit": "elements/s", "achieved": round(elems_per_s, 1), "peak": round(peak, 1),
             "frac": round(elems_per_s / peak, 4),
-            "basis": "%d Philox wide multiplies per element at %d lanes/clk/SM, %d SMs, %.0f MHz"
-                     % (PHILOX_MULS_PER_ELEM, WIDE_MUL_LANES_PER_CLK, sms, sm_mhz)}
+            "basis": "%d Philox wide multiplies per element at %.1f lanes/clk/SM (measured in this run by "
+                     "nvfp4_measure_mul_wide), %d SMs, %.0f MHz"
+                     % (PHILOX_MULS_PER_ELEM, lanes_per_clk, sms, sm_mhz)}
 
 
 def _peaks():
@@ -553,6 +565,8 @@ def time_other_kernels(b, stack, device, peak, sm_mhz, reps=10):
     flush = (torch.zeros(64 << 20, dtype=torch.float32, device=device),
              torch.ones(64 << 20, dtype=torch.float32, device=device))
     out = {}
+    mul_rate = measure_mul_wide(b, device)
+    out["mul_wide_lanes_per_clk_per_sm"] = round(mul_rate, 2)
     # hint emit from the codes of a hinted layer
     l = stack.hint_from
     h = torch.empty(stack.n * HINT_BITS // 8, dtype=torch.uint8, device=device)
@@ -607,13 +621,14 @@ def time_other_kernels(b, stack, device, peak, sm_mhz, reps=10):
         "avg_us": round(t * 1e6, 2), "GB/s": round(sr_bytes * n / t / 1e9, 1),
         "frac": round(sr_bytes * n / t / 1e9 / peak, 4), "bytes_per_elem": sr_bytes,
         "elements_per_s": round(n / t, 1),
-        "alu_roofline": _philox_roofline(n / t, torch.cuda.get_device_properties(device).multi_processor_count, sm_mhz)}
+        "alu_roofline": _philox_roofline(n / t, torch.cuda.get_device_properties(device).multi_processor_count, sm_mhz,
+                                         mul_rate)}
     b.nvfp4_sr_transpose_requant(codes, scales, ts, batch, er, ec, syn.CFG2_SR_SEED, 0, ws, ct, st, tst)
     out.update(time_transpose_alternatives(b, stack, w, codes, scales, ts, (ct, st, tst), device, peak, reps,
                                            flush))
     out["mxfp8_sr_transpose_requant"]["alu_roofline"] = _philox_roofline(
         out["mxfp8_sr_transpose_requant"]["elements_per_s"], torch.cuda.get_device_properties(device).multi_processor_count,
-        sm_mhz)
+        sm_mhz, mul_rate)
     del w, codes, scales, ct, st
     # RHT32 + quantize
     x = torch.from_numpy(syn.cfg3().view(np.int16)).view(torch.bfloat16).to(device)

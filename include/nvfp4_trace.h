@@ -598,6 +598,21 @@ nvfp4_status nvfp4_moe_gather(const uint8_t* codes, const uint8_t* scales, int64
  */
 nvfp4_status nvfp4_wait_selftest(uint32_t* ws, void* stream);
 
+/*
+ * nvfp4_measure_mul_wide -- measurement helper (the pages have no
+ * counterpart; not a step of the method): the issue rate of the
+ * 32 x 32 -> 64-bit integer multiply that Philox4x32-10 spends 20 of per
+ * random word, which bounds nvfp4_sr_transpose_requant and
+ * mxfp8_sr_transpose_requant.  `ctas` CTAs of 1024 threads (one per SM when
+ * ctas = the SM count), each thread running 8 independent multiply chains for
+ * `iters` iterations; cycles[i] receives CTA i's SM clock cycles for its loop
+ * (uint64, device).  Multiplies per clock per SM = 1024 * 8 * iters /
+ * cycles[i].  sink: ctas uint32 words the kernel may write (keeps the work
+ * from being optimised away).
+ */
+nvfp4_status nvfp4_measure_mul_wide(int64_t ctas, int64_t iters, uint64_t* cycles, uint32_t* sink,
+                                    void* stream);
+
 /* Human-readable name of a status code (static string, never NULL). */
 const char* nvfp4_status_string(nvfp4_status status);
 

@@ -50,6 +50,7 @@ _SIGS = {
     "nvfp4_hint_pack": (_I, [_P, _P, _I64, _P, _P, _P]),
     "nvfp4_hint_pack_size": (_I64, [_P, _I64]),
     "nvfp4_moe_rows_cap": (_I64, [_I64, _I64]),
+    "nvfp4_measure_mul_wide": (_I, [_I64, _I64, _P, _P, _P]),
     "nvfp4_moe_route_ws_words": (_I64, [_I64, _I64]),
     "nvfp4_moe_route": (_I, [_P, _I64, _I64, _I64, _P, _P, _P, _I64, _P, _P]),
     "nvfp4_moe_gather": (_I, [_P, _P, _I64, _I64, _P, _I64, _I64, _P, _P, _P]),
@@ -322,6 +323,11 @@ def nvfp4_moe_gather(codes, scales, tokens, k, row_src, top_k, a_codes, a_scales
     _check("nvfp4_moe_gather", _lib.nvfp4_moe_gather(
         _ptr(codes), _ptr(scales), int(tokens), int(k), _ptr(row_src), int(row_src.numel()), int(top_k),
         _ptr(a_codes), _ptr(a_scales_mma), _stream(stream)))
+
+
+def nvfp4_measure_mul_wide(ctas, iters, cycles, sink, stream=None):
+    _check("nvfp4_measure_mul_wide", _lib.nvfp4_measure_mul_wide(int(ctas), int(iters), _ptr(cycles), _ptr(sink),
+                                                                 _stream(stream)))
 
 
 def nvfp4_wait_selftest(ws, stream=None):

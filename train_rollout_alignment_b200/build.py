@@ -16,7 +16,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libnvfp4trace.so")
 SOURCES = ["api.cu", "quantize.cu", "stats.cu", "sr_transpose.cu", "rht.cu", "noalloc.cu",
-           "next_formats.cu", "producer.cu", "transport.cu", "moe_dispatch.cu"]
+           "next_formats.cu", "producer.cu", "transport.cu", "moe_dispatch.cu", "measure.cu"]
 HEADERS = ["nvfp4_device.cuh", "stats_device.cuh", "launch.h", "umma.cuh"]
 
 NVCC_FLAGS = [

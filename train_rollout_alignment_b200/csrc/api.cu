@@ -535,6 +535,16 @@ nvfp4_status nvfp4_moe_gather(const uint8_t* codes, const uint8_t* scales, int64
                                             a_codes, a_scales_mma, static_cast<cudaStream_t>(stream)));
 }
 
+nvfp4_status nvfp4_measure_mul_wide(int64_t ctas, int64_t iters, uint64_t* cycles, uint32_t* sink,
+                                    void* stream) {
+  if (ctas < 1 || ctas > 65535 || iters < 1 || iters > (int64_t(1) << 24) || !cycles || !sink)
+    return NVFP4_ERR_INVALID_ARG;
+  if (!aligned(cycles, 8) || !aligned(sink, 4)) return NVFP4_ERR_MISALIGNED;
+  return from_cuda(nvfp4::launch_measure_mul_wide((int)ctas, (int)iters,
+                                                  reinterpret_cast<unsigned long long*>(cycles), sink,
+                                                  static_cast<cudaStream_t>(stream)));
+}
+
 nvfp4_status nvfp4_wait_selftest(uint32_t* ws, void* stream) {
   if (!ws) return NVFP4_ERR_INVALID_ARG;
   if (!aligned(ws, 16)) return NVFP4_ERR_MISALIGNED;

@@ -78,6 +78,8 @@ cudaError_t launch_gemm_quantize(const uint8_t* a_codes, const uint8_t* a_sf, co
                                  uint8_t* scales_mma, float* tensor_scale, uint8_t* hints,
                                  int hint_bits, float* d_out, cudaStream_t s);
 cudaError_t launch_wait_selftest(uint32_t* ws, cudaStream_t s);
+cudaError_t launch_measure_mul_wide(int ctas, int iters, unsigned long long* cycles, uint32_t* sink,
+                                    cudaStream_t s);
 // MoE dispatch on one GPU: stable grouping of the top-k assignments by expert
 // (ws: route_ws_words(A, E) words) and the gather of the routed NVFP4 rows.
 constexpr int kRouteMaxExperts = 1024;

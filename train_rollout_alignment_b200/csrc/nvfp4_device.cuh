@@ -342,21 +342,23 @@ __device__ __forceinline__ unsigned long long warp_sum_u64(unsigned long long v)
 }
 
 // Adds the block-wide sums of `vals[0..N)` to the global counters `dst`.
-template <int N>
+// Warps 0 .. WARPS-1 contribute (a CTA may carry further warps, e.g. a copy
+// producer, which only take part in the barrier); smem holds N x WARPS words.
+template <int N, int WARPS = kThreads / 32>
 __device__ __forceinline__ void block_add_u64(const unsigned long long* vals,
                                               unsigned long long* dst,
-                                              unsigned long long* smem /*[N][8]*/) {
+                                              unsigned long long* smem /*[N][WARPS]*/) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 #pragma unroll
   for (int k = 0; k < N; ++k) {
     unsigned long long s = warp_sum_u64(vals[k]);
-    if (lane == 0) smem[k * 8 + warp] = s;
+    if (lane == 0 && warp < WARPS) smem[k * WARPS + warp] = s;
   }
   __syncthreads();
   if (warp == 0) {
 #pragma unroll
     for (int k = 0; k < N; ++k) {
-      unsigned long long s = (lane < kThreads / 32) ? smem[k * 8 + lane] : 0ull;
+      unsigned long long s = (lane < WARPS) ? smem[k * WARPS + lane] : 0ull;
       s = warp_sum_u64(s);
       if (lane == 0 && s != 0ull) atomicAdd(dst + k, s);
     }

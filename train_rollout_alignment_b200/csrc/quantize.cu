@@ -15,6 +15,7 @@
 #include "launch.h"
 #include "nvfp4_device.cuh"
 #include "stats_device.cuh"
+#include "umma.cuh"
 
 namespace nvfp4 {
 
@@ -376,6 +377,192 @@ __global__ void __launch_bounds__(kThreads, kGsCtasPerSm)
   }
 }
 
+// ----------------------------------------------------------------- staged guided (+ counters)
+// The guided pass with its inputs staged through shared memory by bulk
+// copies: one producer warp streams chunks of kStageBlocks blocks (their BF16
+// values, hint fields and, with counters, the rollout's codes and scale
+// bytes) through a ring of shared-memory stages with cp.async.bulk (one copy
+// per input stream and chunk, completion counted on an mbarrier), and eight
+// compute warps take one block per thread from shared memory.  Global-memory
+// latency is hidden by the ring instead of by registers, so the compute
+// threads never wait on a load and keep the logic pipe busy.  Chunk c holds
+// blocks kStageBlocks * c .. + kStageBlocks - 1 (so every copy starts on a
+// 16-byte boundary, whatever the tensor size); the chunks are visited from
+// the end of the tensor backwards (the amax pass just read its tail), and
+// the blocks after the last whole chunk (nblk % kStageBlocks of them) are
+// done first, by CTA 0, with direct loads.  Every wait is bounded (2 s); a
+// wait that gives up stops the CTA and sets NVFP4_WARN_TIMEOUT in ws[1].
+// HB = 0 (with counters only): round-to-nearest codes.
+constexpr int kStageBlocks = 256;                   // one block per compute thread
+constexpr int kComputeWarps = kThreads / 32;        // 8
+constexpr int kStagedThreads = kThreads + 32;       // + the producer warp
+#ifndef NVFP4_GUIDED_STAGES
+#define NVFP4_GUIDED_STAGES 4
+#endif
+#ifndef NVFP4_GUIDED_CTAS
+#define NVFP4_GUIDED_CTAS 3
+#endif
+constexpr int kGuidedStages = NVFP4_GUIDED_STAGES;
+constexpr int kGuidedCtas = NVFP4_GUIDED_CTAS;
+
+template <int HB, bool STATS>
+struct GuidedStage {
+  static constexpr uint32_t kHintBytes = HB == 0 ? 0u : (HB == 4 ? 8u : (uint32_t)HB * 2u);  // per block
+  static constexpr uint32_t x = 0;
+  static constexpr uint32_t hints = x + kStageBlocks * 32;
+  static constexpr uint32_t rc = hints + kStageBlocks * kHintBytes;
+  static constexpr uint32_t rs = rc + (STATS ? kStageBlocks * 8 : 0);
+  static constexpr uint32_t payload = rs + (STATS ? kStageBlocks : 0);
+  static constexpr uint32_t bytes = (payload + 127) / 128 * 128;
+  static constexpr uint32_t smem = kGuidedStages * bytes + 128;  // + barriers
+};
+
+template <int HB>
+__device__ __forceinline__ uint32_t hint_field_smem(const uint8_t* st, int t, uint2& h4) {
+  if (HB == 1) return *reinterpret_cast<const uint16_t*>(st + 2 * t);
+  if (HB == 2) return *reinterpret_cast<const uint32_t*>(st + 4 * t);
+  if (HB == 4) h4 = *reinterpret_cast<const uint2*>(st + 8 * t);
+  return 0u;
+}
+
+template <int HB, bool STATS>
+__global__ void __launch_bounds__(kStagedThreads, kGuidedCtas)
+    k_guided_staged(const uint16_t* __restrict__ x, int64_t nblk, const uint8_t* __restrict__ hints,
+                    uint32_t* __restrict__ ws, uint8_t* __restrict__ codes,
+                    uint8_t* __restrict__ scales, float* __restrict__ tensor_scale,
+                    unsigned long long* __restrict__ stats4, const uint8_t* __restrict__ rcodes,
+                    const uint8_t* __restrict__ rscales, const float* __restrict__ rts,
+                    unsigned long long* __restrict__ stats8, uint32_t one) {
+  using L = GuidedStage<HB, STATS>;
+  extern __shared__ __align__(128) uint8_t stage_smem[];
+  __shared__ ScaleTables tab;
+  __shared__ StatsShared sm;
+  __shared__ unsigned long long red4[3 * 8];
+  __shared__ int abort_flag;
+  const uint32_t sbase = umma::smem_u32(stage_smem);
+  const uint32_t full = sbase + kGuidedStages * L::bytes, empty = full + 8 * kGuidedStages;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kGuidedStages; ++s) {
+      umma::mbar_init(full + 8 * s, 1);
+      umma::mbar_init(empty + 8 * s, kComputeWarps);
+    }
+    abort_flag = 0;
+    umma::fence_mbar_init();
+  }
+  const float s_t = tensor_scale_from_amax(__uint_as_float(ws[0]));
+  if (blockIdx.x == 0 && threadIdx.x == 0) *tensor_scale = s_t;
+  scale_tables_init(tab, s_t);  // ends in a barrier: the mbarriers are ready too
+  const float ts_r = STATS ? *rts : 0.0f;
+  const bool same_ts = STATS && __float_as_uint(ts_r) == __float_as_uint(s_t);
+  bool far_all = false;
+  if constexpr (STATS) far_all = stats_tables_init(sm, ts_r, s_t);
+  volatile int* abort = &abort_flag;
+  const int64_t nfull = nblk / kStageBlocks;  // whole chunks
+  const int64_t tail0 = nfull * kStageBlocks;  // blocks tail0 .. nblk-1: direct loads, CTA 0
+  GuidedCounts gcnt{0u, 0u, 0u};
+  MismatchCounts mc{0u, 0u, 0u, 0u, 0u};
+  int qn = 0;
+
+  if (warp == kComputeWarps) {
+    // ---------------- producer: one lane issues the bulk copies
+    if (lane == 0) {
+      int it = 0;
+      for (int64_t c = blockIdx.x; c < nfull; c += gridDim.x, ++it) {
+        const int s = it % kGuidedStages;
+        const uint32_t ph = (uint32_t)(it / kGuidedStages) & 1u;
+        if (!umma::mbar_wait(empty + 8 * s, ph ^ 1u, abort)) break;
+        const int64_t b0 = (nfull - 1 - c) * kStageBlocks;
+        const uint32_t bar = full + 8 * s, st = sbase + s * L::bytes;
+        umma::mbar_arrive_expect_tx(bar, L::payload);
+        umma::bulk_load(st + L::x, x + b0 * 16, kStageBlocks * 32, bar);
+        if (HB != 0) umma::bulk_load(st + L::hints, hints + b0 * L::kHintBytes, kStageBlocks * L::kHintBytes, bar);
+        if (STATS) {
+          umma::bulk_load(st + L::rc, rcodes + b0 * 8, kStageBlocks * 8, bar);
+          umma::bulk_load(st + L::rs, rscales + b0, kStageBlocks, bar);
+        }
+      }
+    }
+    __syncwarp();
+  } else {
+    // ---------------- compute: one block per thread per chunk
+    const int t = threadIdx.x;
+    const uint32_t lt_mask = (1u << lane) - 1u;
+    // the blocks after the last whole chunk: CTA 0, direct loads, every lane
+    // of a warp in step (the counters' queue is warp-wide)
+    if (tail0 < nblk && blockIdx.x == 0) {
+      for (int64_t i0 = tail0 + 32 * warp; i0 < nblk; i0 += kThreads) {
+        const int64_t i = i0 + lane;
+        const bool valid = i < nblk;
+        uint2 cw = make_uint2(0u, 0u), rc = make_uint2(0u, 0u);
+        uint32_t sb = 0u, rs = 0u;
+        if (valid) {
+          const Block16 b = ld_block(x + i * 16);
+          uint2 h4 = make_uint2(0u, 0u);
+          uint32_t hw = 0u;
+          if constexpr (HB != 0) hw = hint_field<HB>(hints, i, h4);
+          const BlockScale bs = block_scale_bf16(block_amax_bits(b), s_t, tab);
+          if constexpr (HB != 0) cw = guided_codes<HB>(b, hw, h4, bs.inv, gcnt, one);
+          else cw = rtn_codes(b, bs.inv);
+          sb = bs.sb;
+          reinterpret_cast<uint2*>(codes)[i] = cw;
+          scales[i] = (uint8_t)sb;
+          if (STATS) {
+            rc = __ldg(reinterpret_cast<const uint2*>(rcodes) + i);
+            rs = __ldg(rscales + i);
+          }
+        }
+        if constexpr (STATS)
+          count_block(sm, rc.x, rc.y, cw.x, cw.y, rs, sb, valid, same_ts, far_all, ts_r, s_t, warp,
+                      lane, lt_mask, qn, mc);
+      }
+    }
+    int it = 0;
+    for (int64_t c = blockIdx.x; c < nfull; c += gridDim.x, ++it) {
+      const int s = it % kGuidedStages;
+      const uint32_t ph = (uint32_t)(it / kGuidedStages) & 1u;
+      const bool ok = umma::mbar_wait(full + 8 * s, ph, abort);
+      if (!__all_sync(0xFFFFFFFFu, ok)) break;
+      const uint8_t* st = stage_smem + s * L::bytes;
+      const int64_t blk = (nfull - 1 - c) * kStageBlocks + t;
+      Block16 b;
+      const uint4 lo = *reinterpret_cast<const uint4*>(st + L::x + 32 * t);
+      const uint4 hi = *reinterpret_cast<const uint4*>(st + L::x + 32 * t + 16);
+      b.w[0] = lo.x; b.w[1] = lo.y; b.w[2] = lo.z; b.w[3] = lo.w;
+      b.w[4] = hi.x; b.w[5] = hi.y; b.w[6] = hi.z; b.w[7] = hi.w;
+      uint2 h4 = make_uint2(0u, 0u);
+      const uint32_t hw = hint_field_smem<HB>(st + L::hints, t, h4);
+      uint2 rc = make_uint2(0u, 0u);
+      uint32_t rs = 0u;
+      if (STATS) {
+        rc = *reinterpret_cast<const uint2*>(st + L::rc + 8 * t);
+        rs = st[L::rs + t];
+      }
+      const BlockScale bs = block_scale_bf16(block_amax_bits(b), s_t, tab);
+      uint2 cw;
+      if constexpr (HB != 0) cw = guided_codes<HB>(b, hw, h4, bs.inv, gcnt, one);
+      else cw = rtn_codes(b, bs.inv);
+      reinterpret_cast<uint2*>(codes)[blk] = cw;
+      scales[blk] = (uint8_t)bs.sb;
+      if constexpr (STATS)
+        count_block(sm, rc.x, rc.y, cw.x, cw.y, rs, bs.sb, true, same_ts, far_all, ts_r, s_t, warp,
+                    lane, lt_mask, qn, mc);
+      __syncwarp();
+      if (lane == 0) umma::mbar_arrive(empty + 8 * s);
+    }
+  }
+  if constexpr (STATS) {
+    stats_finish(sm, warp, lane, qn, mc, stats8);
+    if (blockIdx.x == 0 && threadIdx.x == 0) atomicAdd(stats8, (unsigned long long)nblk * 16ull);
+  }
+  if (HB != 0 && stats4 != nullptr) {
+    const unsigned long long vals[3] = {gcnt.consulted, gcnt.changed, gcnt.outside};
+    block_add_u64<3, kComputeWarps>(vals, stats4, red4);
+  }
+  __syncthreads();
+  if (*abort && threadIdx.x == 0) atomicOr(ws + 1, NVFP4_WARN_TIMEOUT);
+}
+
 // ----------------------------------------------------------------- KV-cache rows
 // One FP32 scale per row of [rows, cols] (one token's vector for one head of a
 // KV cache, cols = head_dim), as if every row were its own tensor.  LPR =
@@ -578,11 +765,49 @@ cudaError_t launch_quantize_rtn(const uint16_t* x, int64_t nblk, const uint32_t*
   return cudaGetLastError();
 }
 
+#ifndef NVFP4_GUIDED_STAGED
+#define NVFP4_GUIDED_STAGED 1
+#endif
+
+template <int HB, bool STATS>
+cudaError_t launch_staged(const uint16_t* x, int64_t nblk, const uint8_t* hints, const uint32_t* ws,
+                          uint8_t* codes, uint8_t* scales, float* tensor_scale,
+                          unsigned long long* stats4, const uint8_t* rcodes, const uint8_t* rscales,
+                          const float* rts, unsigned long long* stats8, cudaStream_t s) {
+  using L = GuidedStage<HB, STATS>;
+  // the dynamic shared-memory opt-in is a property of the function on each device
+  static bool attr_set[64] = {false};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64 || !attr_set[dev]) {
+    e = cudaFuncSetAttribute(k_guided_staged<HB, STATS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)L::smem);
+    if (e != cudaSuccess) return e;
+    if (dev >= 0 && dev < 64) attr_set[dev] = true;
+  }
+  const int64_t chunks = nblk / kStageBlocks;
+  const int64_t slots = (int64_t)sm_count() * kGuidedCtas;
+  const int g = (int)(chunks < 1 ? 1 : (chunks < slots ? chunks : slots));
+  k_guided_staged<HB, STATS><<<g, kStagedThreads, L::smem, s>>>(
+      x, nblk, hints, const_cast<uint32_t*>(ws), codes, scales, tensor_scale, stats4, rcodes, rscales,
+      rts, stats8, 1u);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_guided(const uint16_t* x, int64_t nblk, const uint8_t* hints, int hint_bits,
                           const uint32_t* ws, uint8_t* codes, uint8_t* scales,
                           float* tensor_scale, unsigned long long* stats4, cudaStream_t s) {
   if (hints == nullptr)
     return launch_quantize_rtn(x, nblk, ws, codes, scales, tensor_scale, nullptr, 0, s);
+#if NVFP4_GUIDED_STAGED
+  switch (hint_bits) {
+    case 1: return launch_staged<1, false>(x, nblk, hints, ws, codes, scales, tensor_scale, stats4, nullptr, nullptr, nullptr, nullptr, s);
+    case 2: return launch_staged<2, false>(x, nblk, hints, ws, codes, scales, tensor_scale, stats4, nullptr, nullptr, nullptr, nullptr, s);
+    case 4: return launch_staged<4, false>(x, nblk, hints, ws, codes, scales, tensor_scale, stats4, nullptr, nullptr, nullptr, nullptr, s);
+    default: return cudaErrorInvalidValue;
+  }
+#else
   const int g = grid_for(nblk, kThreads, kCtasPerSm);
   switch (hint_bits) {
     case 1: k_guided<1, kUnroll><<<g, kThreads, 0, s>>>(x, nblk, hints, ws, codes, scales, tensor_scale, stats4, 1u); break;
@@ -591,6 +816,7 @@ cudaError_t launch_guided(const uint16_t* x, int64_t nblk, const uint8_t* hints,
     default: return cudaErrorInvalidValue;
   }
   return cudaGetLastError();
+#endif
 }
 
 cudaError_t launch_guided_stats(const uint16_t* x, int64_t nblk, const uint8_t* hints,
@@ -598,6 +824,15 @@ cudaError_t launch_guided_stats(const uint16_t* x, int64_t nblk, const uint8_t* 
                                 float* tensor_scale, unsigned long long* stats4,
                                 const uint8_t* rcodes, const uint8_t* rscales, const float* rts,
                                 unsigned long long* stats8, cudaStream_t s) {
+#if NVFP4_GUIDED_STAGED
+  switch (hints ? hint_bits : 0) {
+    case 0: return launch_staged<0, true>(x, nblk, nullptr, ws, codes, scales, tensor_scale, nullptr, rcodes, rscales, rts, stats8, s);
+    case 1: return launch_staged<1, true>(x, nblk, hints, ws, codes, scales, tensor_scale, stats4, rcodes, rscales, rts, stats8, s);
+    case 2: return launch_staged<2, true>(x, nblk, hints, ws, codes, scales, tensor_scale, stats4, rcodes, rscales, rts, stats8, s);
+    case 4: return launch_staged<4, true>(x, nblk, hints, ws, codes, scales, tensor_scale, stats4, rcodes, rscales, rts, stats8, s);
+    default: return cudaErrorInvalidValue;
+  }
+#else
   const int g = grid_for(nblk, kThreads, kGsCtasPerSm);
   switch (hints ? hint_bits : 0) {
     case 0: k_guided_stats<0, kGsUnroll><<<g, kThreads, 0, s>>>(x, nblk, nullptr, ws, codes, scales, tensor_scale, nullptr, rcodes, rscales, rts, stats8, 1u); break;
@@ -607,6 +842,7 @@ cudaError_t launch_guided_stats(const uint16_t* x, int64_t nblk, const uint8_t* 
     default: return cudaErrorInvalidValue;
   }
   return cudaGetLastError();
+#endif
 }
 
 cudaError_t launch_emit_hint(const uint8_t* codes, int64_t nblk, int hint_bits, uint8_t* hints,

@@ -158,12 +158,12 @@ __device__ __forceinline__ void count_block(StatsShared& sm, uint32_t ax, uint32
 
 // Per-CTA tables of the decoded-value counter for tensor scales tsa (side
 // a) and tsb (side b); returns the CTA-uniform far_all flag (see count_block).
-// Every thread of the CTA calls it (it ends in a barrier); blockDim.x ==
-// kThreads >= 256 covers the 256 significand pairs.
+// Every thread of the CTA calls it (it ends in a barrier); threads 0..255
+// cover the 256 significand pairs, any further threads only vote.
 __device__ __forceinline__ bool stats_tables_init(StatsShared& sm, float tsa, float tsb) {
   const bool same_ts = __float_as_uint(tsa) == __float_as_uint(tsb);
-  const int t = threadIdx.x;
-  if (t < 128) {
+  const int t = threadIdx.x < 256 ? (int)threadIdx.x : 0;
+  if (threadIdx.x < 128) {
     const float sv = e4m3_value(t);
     const float xa = __fmul_rn(sv, tsa), xb = __fmul_rn(sv, tsb);
     // every nonzero decoded value of the block is a normal float
@@ -181,12 +181,12 @@ __device__ __forceinline__ bool stats_tables_init(StatsShared& sm, float tsa, fl
     bool far_ratio = false;
     if (ma != 0u && mb != 0u && tr >= 0x1p-120f && tr <= 0x1p120f)
       far_ratio = !near_grid_ratio(__fmul_rn(__fdiv_rn((float)ma, (float)mb), tr));
-    sm.ratio_far[t] = far_ratio;
+    if (threadIdx.x < 256) sm.ratio_far[t] = far_ratio;
     // the CTA-wide shortcut: every nonzero significand pair far, every
     // nonzero scale byte regular on both sides
     ok = (ma == 0u || mb == 0u || far_ratio);
   }
-  if (t < 128 && t != 0) {
+  if (threadIdx.x < 128 && t != 0) {
     const float sv = e4m3_value(t);
     const float xa = __fmul_rn(sv, tsa), xb = __fmul_rn(sv, tsb);
     ok = ok && xa >= 0x1p-124f && xa <= 0x1p120f && xb >= 0x1p-124f && xb <= 0x1p120f;
@@ -195,13 +195,14 @@ __device__ __forceinline__ bool stats_tables_init(StatsShared& sm, float tsa, fl
 }
 
 // Empties the warp's queue and adds the CTA's six counters to stats8[1..6]
-// (every thread of the CTA calls it).
+// (every thread of the CTA calls it; warps from kWarps on only take part in
+// the barrier).
 __device__ __forceinline__ void stats_finish(StatsShared& sm, int warp, int lane, int qn,
                                              MismatchCounts& c, unsigned long long* stats8) {
   if (qn > 0) flush_queue(sm, warp, lane, qn, qn, c);
   const unsigned long long vals[6] = {c.mism, (unsigned long long)(c.mism - c.far), c.far, c.sumd,
                                       c.scale, c.value};
-  block_add_u64<6>(vals, stats8 + 1, sm.red);
+  block_add_u64<6, kWarps>(vals, stats8 + 1, sm.red);
 }
 
 }  // namespace nvfp4
