@@ -100,7 +100,9 @@ typedef int nvfp4_status;
 #define NVFP4_STAT_SUM_ABS_DELTA 4  /* sum of |pos_a - pos_b| */
 #define NVFP4_STAT_SCALE_MISMATCH 5 /* 16-blocks whose E4M3 scale bytes differ */
 #define NVFP4_STAT_VALUE_MISMATCH 6 /* decoded FP32 values differ (-0 == +0) */
-#define NVFP4_STATS8_WORDS       8  /* word 7 is reserved (left unchanged) */
+#define NVFP4_STATS8_WORDS       8  /* word 7: left unchanged, except that bit 0 is set if a
+                                       bounded wait of the counting pipeline gave up (never
+                                       expected; the counters are then unspecified) */
 
 /* stats4 indices (nvfp4_guided_requant) */
 #define NVFP4_GSTAT_CONSULTED    0  /* off-grid and |v| < 6: the hint decided */

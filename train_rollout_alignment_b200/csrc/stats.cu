@@ -30,6 +30,7 @@
 //    zero/zero rule without table lookups.
 #include "launch.h"
 #include "stats_device.cuh"
+#include "umma.cuh"
 
 namespace nvfp4 {
 
@@ -101,12 +102,143 @@ __global__ void __launch_bounds__(kThreads, kStatsCtasPerSm)
   if (blockIdx.x == 0 && t == 0) atomicAdd(stats8, (unsigned long long)nblk * 16ull);
 }
 
+// The same counters with their inputs staged through shared memory: one
+// producer warp streams chunks of kStatsChunk blocks (both sides' codes and
+// scale bytes, four bulk copies per chunk) through a ring of stages, and
+// each of the eight compute warps' threads takes one pair of adjacent blocks
+// per chunk from shared memory, so no compute thread waits on a global load.
+// The blocks after the last whole chunk are counted by CTA 0 with direct
+// loads.  Every wait is bounded (2 s); a wait that gives up stops the CTA and
+// sets bit 0 of stats8[7].
+constexpr int kStatsChunk = 2 * kThreads;          // 512 blocks: one pair per compute thread
+constexpr int kStatsStagedThreads = kThreads + 32;
+#ifndef NVFP4_STATS_STAGES
+#define NVFP4_STATS_STAGES 4
+#endif
+#ifndef NVFP4_STATS_CTAS
+#define NVFP4_STATS_CTAS 4
+#endif
+constexpr int kStatsStages = NVFP4_STATS_STAGES;
+constexpr int kStatsStagedCtas = NVFP4_STATS_CTAS;
+constexpr uint32_t kSsCa = 0, kSsCb = kStatsChunk * 8, kSsSa = 2 * kStatsChunk * 8,
+                   kSsSb = kSsSa + kStatsChunk, kSsPayload = kSsSb + kStatsChunk;
+constexpr uint32_t kSsBytes = (kSsPayload + 127) / 128 * 128;
+constexpr uint32_t kSsSmem = kStatsStages * kSsBytes + 128;
+
+__global__ void __launch_bounds__(kStatsStagedThreads, kStatsStagedCtas)
+    k_mismatch_stats_staged(const uint8_t* __restrict__ ca, const uint8_t* __restrict__ sa,
+                            const float* __restrict__ ta, const uint8_t* __restrict__ cb,
+                            const uint8_t* __restrict__ sb, const float* __restrict__ tb,
+                            int64_t nblk, unsigned long long* __restrict__ stats8) {
+  extern __shared__ __align__(128) uint8_t stage_smem[];
+  __shared__ StatsShared sm;
+  __shared__ int abort_flag;
+  const uint32_t sbase = umma::smem_u32(stage_smem);
+  const uint32_t full = sbase + kStatsStages * kSsBytes, empty = full + 8 * kStatsStages;
+  const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+  if (t == 0) {
+    for (int s = 0; s < kStatsStages; ++s) {
+      umma::mbar_init(full + 8 * s, 1);
+      umma::mbar_init(empty + 8 * s, kWarps);
+    }
+    abort_flag = 0;
+    umma::fence_mbar_init();
+  }
+  const float tsa = *ta, tsb = *tb;
+  const bool same_ts = __float_as_uint(tsa) == __float_as_uint(tsb);
+  const bool far_all = stats_tables_init(sm, tsa, tsb);  // ends in a barrier
+  volatile int* abort = &abort_flag;
+  const int64_t nfull = nblk / kStatsChunk;
+  MismatchCounts c{0u, 0u, 0u, 0u, 0u};
+  int qn = 0;
+  if (warp == kWarps) {
+    if (lane == 0) {  // producer
+      int it = 0;
+      for (int64_t ch = blockIdx.x; ch < nfull; ch += gridDim.x, ++it) {
+        const int s = it % kStatsStages;
+        const uint32_t ph = (uint32_t)(it / kStatsStages) & 1u;
+        if (!umma::mbar_wait(empty + 8 * s, ph ^ 1u, abort)) break;
+        const int64_t b0 = ch * kStatsChunk;
+        const uint32_t bar = full + 8 * s, st = sbase + s * kSsBytes;
+        umma::mbar_arrive_expect_tx(bar, kSsPayload);
+        umma::bulk_load(st + kSsCa, ca + b0 * 8, kStatsChunk * 8, bar);
+        umma::bulk_load(st + kSsCb, cb + b0 * 8, kStatsChunk * 8, bar);
+        umma::bulk_load(st + kSsSa, sa + b0, kStatsChunk, bar);
+        umma::bulk_load(st + kSsSb, sb + b0, kStatsChunk, bar);
+      }
+    }
+    __syncwarp();
+  } else {
+    const uint32_t lt_mask = (1u << lane) - 1u;
+    int it = 0;
+    for (int64_t ch = blockIdx.x; ch < nfull; ch += gridDim.x, ++it) {
+      const int s = it % kStatsStages;
+      const uint32_t ph = (uint32_t)(it / kStatsStages) & 1u;
+      const bool ok = umma::mbar_wait(full + 8 * s, ph, abort);
+      if (!__all_sync(0xFFFFFFFFu, ok)) break;
+      const uint8_t* st = stage_smem + s * kSsBytes;
+      const uint4 va = *reinterpret_cast<const uint4*>(st + kSsCa + 16 * t);
+      const uint4 vb = *reinterpret_cast<const uint4*>(st + kSsCb + 16 * t);
+      const uint32_t xa = *reinterpret_cast<const uint16_t*>(st + kSsSa + 2 * t);
+      const uint32_t xb = *reinterpret_cast<const uint16_t*>(st + kSsSb + 2 * t);
+      count_block(sm, va.x, va.y, vb.x, vb.y, xa & 0xFFu, xb & 0xFFu, true, same_ts, far_all, tsa,
+                  tsb, warp, lane, lt_mask, qn, c);
+      count_block(sm, va.z, va.w, vb.z, vb.w, xa >> 8, xb >> 8, true, same_ts, far_all, tsa, tsb,
+                  warp, lane, lt_mask, qn, c);
+      __syncwarp();
+      if (lane == 0) umma::mbar_arrive(empty + 8 * s);
+    }
+    // blocks after the last whole chunk: CTA 0, direct loads, warps in step
+    if (blockIdx.x == 0) {
+      for (int64_t i0 = nfull * kStatsChunk + 32 * warp; i0 < nblk; i0 += kThreads) {
+        const int64_t i = i0 + lane;
+        const bool valid = i < nblk;
+        uint2 a = make_uint2(0u, 0u), b = make_uint2(0u, 0u);
+        uint32_t x = 0u, y = 0u;
+        if (valid) {
+          a = __ldg(reinterpret_cast<const uint2*>(ca) + i);
+          b = __ldg(reinterpret_cast<const uint2*>(cb) + i);
+          x = __ldg(sa + i);
+          y = __ldg(sb + i);
+        }
+        count_block(sm, a.x, a.y, b.x, b.y, x, y, valid, same_ts, far_all, tsa, tsb, warp, lane,
+                    lt_mask, qn, c);
+      }
+    }
+  }
+  stats_finish(sm, warp, lane, qn, c, stats8);
+  if (blockIdx.x == 0 && t == 0) atomicAdd(stats8, (unsigned long long)nblk * 16ull);
+  __syncthreads();
+  if (*abort && t == 0) atomicOr(stats8 + 7, 1ull);
+}
+
+#ifndef NVFP4_STATS_STAGED
+#define NVFP4_STATS_STAGED 1
+#endif
+
 cudaError_t launch_mismatch_stats(const uint8_t* ca, const uint8_t* sa, const float* ta,
                                   const uint8_t* cb, const uint8_t* sb, const float* tb,
                                   int64_t nblk, unsigned long long* stats8, cudaStream_t s) {
   if (nblk == 0) return cudaSuccess;
+#if NVFP4_STATS_STAGED
+  static bool attr_set[64] = {false};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64 || !attr_set[dev]) {
+    e = cudaFuncSetAttribute(k_mismatch_stats_staged, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)kSsSmem);
+    if (e != cudaSuccess) return e;
+    if (dev >= 0 && dev < 64) attr_set[dev] = true;
+  }
+  const int64_t chunks = nblk / kStatsChunk;
+  const int64_t slots = (int64_t)sm_count() * kStatsStagedCtas;
+  const int g = (int)(chunks < 1 ? 1 : (chunks < slots ? chunks : slots));
+  k_mismatch_stats_staged<<<g, kStatsStagedThreads, kSsSmem, s>>>(ca, sa, ta, cb, sb, tb, nblk, stats8);
+#else
   k_mismatch_stats<kStatsUnroll><<<grid_for(nblk, kThreads, kStatsCtasPerSm), kThreads, 0, s>>>(
       ca, sa, ta, cb, sb, tb, nblk, stats8);
+#endif
   return cudaGetLastError();
 }
 

@@ -107,16 +107,21 @@ __device__ __forceinline__ int flush_queue(StatsShared& sm, int warp, int lane, 
   return rest;
 }
 
-// Elements of a word whose magnitudes are not both zero (bit 3 per nibble:
-// a nibble value in 0..7 plus 7 sets bit 3 iff it is nonzero).
-__device__ __forceinline__ uint32_t not_both_zero(uint32_t wa, uint32_t wb) {
-  return __popc((((wa | wb) & 0x77777777u) + 0x77777777u) & 0x88888888u);
+// Elements of a block (words x, y of both sides) whose magnitudes are not
+// both zero: bit 3 of each nibble of ((a | b) & 7) + 7 flags the first word's
+// elements, the second word's flags move to bit 2, one popc counts both.
+__device__ __forceinline__ uint32_t not_both_zero2(uint32_t ax, uint32_t ay, uint32_t bx, uint32_t by) {
+  const uint32_t f0 = (((ax | bx) & 0x77777777u) + 0x77777777u) & 0x88888888u;
+  const uint32_t f1 = ((((ay | by) & 0x77777777u) + 0x77777777u) >> 1) & 0x44444444u;
+  return __popc(f0 | f1);
 }
 
-// One block of the stream: queue it if its codes differ; count its scale and
-// (unless positions decide it) its decoded-value mismatches.
+// One block of the stream: count its scale and (unless positions decide it)
+// its decoded-value mismatches, and queue it if its codes differ.
 // far_all: CTA-uniform, the tensor scales differ and every pair of nonzero
-// scale bytes is regular and far from a grid ratio.
+// scale bytes is regular and far from a grid ratio.  The common case -- both
+// scales nonzero under far_all, and no block of the warp step differing --
+// takes no table lookup and no queue work.
 __device__ __forceinline__ void count_block(StatsShared& sm, uint32_t ax, uint32_t ay, uint32_t bx,
                                             uint32_t by, uint32_t sa, uint32_t sb, bool valid,
                                             bool same_ts, bool far_all, float tsa, float tsb,
@@ -125,34 +130,38 @@ __device__ __forceinline__ void count_block(StatsShared& sm, uint32_t ax, uint32
   sa &= 0x7Fu;
   sb &= 0x7Fu;
   const bool fast = far_all && sa != 0u && sb != 0u;
-  uint32_t ka = 0u, kb = 0u;
-  if (!fast) {
-    ka = sm.key_a[sa];
-    kb = sm.key_b[sb];
-  }
-  const bool same = !fast && same_ts && sa == sb && ka < 0x100u;
-  const bool dirty = ((ax ^ bx) | (ay ^ by)) != 0u;
-  const uint32_t m = __ballot_sync(0xFFFFFFFFu, dirty);
-  if (dirty) {
-    const int slot = qn + __popc(m & lt_mask);
-    sm.queue[warp][slot] = make_uint4(ax, ay, bx, by);
-    sm.queue_same[warp][slot] = same;
-  }
-  qn += __popc(m);
-  if (qn >= 32) qn = flush_queue(sm, warp, lane, qn, 32, c);
-  if (valid) {
-    c.scale += (sa != sb) ? 1u : 0u;
-    if (fast) {
-      c.value += not_both_zero(ax, bx) + not_both_zero(ay, by);  // only zero pairs are equal
-    } else if (!same) {
-      const uint32_t k = ka + kb;
-      if (k < 0x100u && sm.ratio_far[k]) {
-        c.value += not_both_zero(ax, bx) + not_both_zero(ay, by);
-      } else {
-        c.value += value_mismatch_slow(make_uint2(ax, ay), make_uint2(bx, by), e4m3_value(sa),
-                                       e4m3_value(sb), tsa, tsb);
+  bool same = false;
+  if (fast) {
+    if (valid) {
+      c.scale += (sa != sb) ? 1u : 0u;
+      c.value += not_both_zero2(ax, ay, bx, by);  // only zero pairs are equal
+    }
+  } else {
+    const uint32_t ka = sm.key_a[sa], kb = sm.key_b[sb];
+    same = same_ts && sa == sb && ka < 0x100u;
+    if (valid) {
+      c.scale += (sa != sb) ? 1u : 0u;
+      if (!same) {
+        const uint32_t k = ka + kb;
+        if (k < 0x100u && sm.ratio_far[k]) {
+          c.value += not_both_zero2(ax, ay, bx, by);
+        } else {
+          c.value += value_mismatch_slow(make_uint2(ax, ay), make_uint2(bx, by), e4m3_value(sa),
+                                         e4m3_value(sb), tsa, tsb);
+        }
       }
     }
+  }
+  const bool dirty = ((ax ^ bx) | (ay ^ by)) != 0u;
+  const uint32_t m = __ballot_sync(0xFFFFFFFFu, dirty);
+  if (m != 0u) {  // warp-uniform
+    if (dirty) {
+      const int slot = qn + __popc(m & lt_mask);
+      sm.queue[warp][slot] = make_uint4(ax, ay, bx, by);
+      sm.queue_same[warp][slot] = same;
+    }
+    qn += __popc(m);
+    if (qn >= 32) qn = flush_queue(sm, warp, lane, qn, 32, c);
   }
 }
 
