@@ -383,7 +383,7 @@ __global__ void __launch_bounds__(kThreads, kGsCtasPerSm)
 // values, hint fields and, with counters, the rollout's codes and scale
 // bytes) through a ring of shared-memory stages with cp.async.bulk (one copy
 // per input stream and chunk, completion counted on an mbarrier), and eight
-// compute warps take one block per thread from shared memory.  Global-memory
+// compute warps take kGuidedBpt blocks per thread from shared memory.  Global-memory
 // latency is hidden by the ring instead of by registers, so the compute
 // threads never wait on a load and keep the logic pipe busy.  Chunk c holds
 // blocks kStageBlocks * c .. + kStageBlocks - 1 (so every copy starts on a
@@ -393,15 +393,19 @@ __global__ void __launch_bounds__(kThreads, kGsCtasPerSm)
 // done first, by CTA 0, with direct loads.  Every wait is bounded (2 s); a
 // wait that gives up stops the CTA and sets NVFP4_WARN_TIMEOUT in ws[1].
 // HB = 0 (with counters only): round-to-nearest codes.
-constexpr int kStageBlocks = 256;                   // one block per compute thread
-constexpr int kComputeWarps = kThreads / 32;        // 8
-constexpr int kStagedThreads = kThreads + 32;       // + the producer warp
+#ifndef NVFP4_GUIDED_BPT
+#define NVFP4_GUIDED_BPT 2
+#endif
 #ifndef NVFP4_GUIDED_STAGES
-#define NVFP4_GUIDED_STAGES 4
+#define NVFP4_GUIDED_STAGES 3
 #endif
 #ifndef NVFP4_GUIDED_CTAS
-#define NVFP4_GUIDED_CTAS 3
+#define NVFP4_GUIDED_CTAS 2
 #endif
+constexpr int kGuidedBpt = NVFP4_GUIDED_BPT;        // blocks per compute thread and chunk
+constexpr int kStageBlocks = kThreads * kGuidedBpt; // blocks per chunk
+constexpr int kComputeWarps = kThreads / 32;        // 8
+constexpr int kStagedThreads = kThreads + 32;       // + the producer warp
 constexpr int kGuidedStages = NVFP4_GUIDED_STAGES;
 constexpr int kGuidedCtas = NVFP4_GUIDED_CTAS;
 
@@ -524,29 +528,41 @@ __global__ void __launch_bounds__(kStagedThreads, kGuidedCtas)
       const bool ok = umma::mbar_wait(full + 8 * s, ph, abort);
       if (!__all_sync(0xFFFFFFFFu, ok)) break;
       const uint8_t* st = stage_smem + s * L::bytes;
-      const int64_t blk = (nfull - 1 - c) * kStageBlocks + t;
-      Block16 b;
-      const uint4 lo = *reinterpret_cast<const uint4*>(st + L::x + 32 * t);
-      const uint4 hi = *reinterpret_cast<const uint4*>(st + L::x + 32 * t + 16);
-      b.w[0] = lo.x; b.w[1] = lo.y; b.w[2] = lo.z; b.w[3] = lo.w;
-      b.w[4] = hi.x; b.w[5] = hi.y; b.w[6] = hi.z; b.w[7] = hi.w;
-      uint2 h4 = make_uint2(0u, 0u);
-      const uint32_t hw = hint_field_smem<HB>(st + L::hints, t, h4);
-      uint2 rc = make_uint2(0u, 0u);
-      uint32_t rs = 0u;
-      if (STATS) {
-        rc = *reinterpret_cast<const uint2*>(st + L::rc + 8 * t);
-        rs = st[L::rs + t];
+      const int64_t blk0 = (nfull - 1 - c) * kStageBlocks;
+      // thread t takes blocks t, t + 256, ... of the chunk: a warp reads 1 KiB
+      // of contiguous values per block slot
+      Block16 b[kGuidedBpt];
+      uint32_t hw[kGuidedBpt], rs[kGuidedBpt];
+      uint2 h4[kGuidedBpt], rc[kGuidedBpt];
+#pragma unroll
+      for (int k = 0; k < kGuidedBpt; ++k) {
+        const int j = k * kThreads + t;
+        const uint4 lo = *reinterpret_cast<const uint4*>(st + L::x + 32 * j);
+        const uint4 hi = *reinterpret_cast<const uint4*>(st + L::x + 32 * j + 16);
+        b[k].w[0] = lo.x; b[k].w[1] = lo.y; b[k].w[2] = lo.z; b[k].w[3] = lo.w;
+        b[k].w[4] = hi.x; b[k].w[5] = hi.y; b[k].w[6] = hi.z; b[k].w[7] = hi.w;
+        h4[k] = make_uint2(0u, 0u);
+        hw[k] = hint_field_smem<HB>(st + L::hints, j, h4[k]);
+        rc[k] = make_uint2(0u, 0u);
+        rs[k] = 0u;
+        if (STATS) {
+          rc[k] = *reinterpret_cast<const uint2*>(st + L::rc + 8 * j);
+          rs[k] = st[L::rs + j];
+        }
       }
-      const BlockScale bs = block_scale_bf16(block_amax_bits(b), s_t, tab);
-      uint2 cw;
-      if constexpr (HB != 0) cw = guided_codes<HB>(b, hw, h4, bs.inv, gcnt, one);
-      else cw = rtn_codes(b, bs.inv);
-      reinterpret_cast<uint2*>(codes)[blk] = cw;
-      scales[blk] = (uint8_t)bs.sb;
-      if constexpr (STATS)
-        count_block(sm, rc.x, rc.y, cw.x, cw.y, rs, bs.sb, true, same_ts, far_all, ts_r, s_t, warp,
-                    lane, lt_mask, qn, mc);
+#pragma unroll
+      for (int k = 0; k < kGuidedBpt; ++k) {
+        const int64_t blk = blk0 + k * kThreads + t;
+        const BlockScale bs = block_scale_bf16(block_amax_bits(b[k]), s_t, tab);
+        uint2 cw;
+        if constexpr (HB != 0) cw = guided_codes<HB>(b[k], hw[k], h4[k], bs.inv, gcnt, one);
+        else cw = rtn_codes(b[k], bs.inv);
+        reinterpret_cast<uint2*>(codes)[blk] = cw;
+        scales[blk] = (uint8_t)bs.sb;
+        if constexpr (STATS)
+          count_block(sm, rc[k].x, rc[k].y, cw.x, cw.y, rs[k], bs.sb, true, same_ts, far_all, ts_r,
+                      s_t, warp, lane, lt_mask, qn, mc);
+      }
       __syncwarp();
       if (lane == 0) umma::mbar_arrive(empty + 8 * s);
     }
@@ -766,7 +782,10 @@ cudaError_t launch_quantize_rtn(const uint16_t* x, int64_t nblk, const uint32_t*
 }
 
 #ifndef NVFP4_GUIDED_STAGED
-#define NVFP4_GUIDED_STAGED 1
+#define NVFP4_GUIDED_STAGED 1   // guided alone: staged (1) or one block per thread from registers (0)
+#endif
+#ifndef NVFP4_GS_STAGED
+#define NVFP4_GS_STAGED 1       // guided + counters: staged (1) or from registers (0)
 #endif
 
 template <int HB, bool STATS>
@@ -824,7 +843,7 @@ cudaError_t launch_guided_stats(const uint16_t* x, int64_t nblk, const uint8_t* 
                                 float* tensor_scale, unsigned long long* stats4,
                                 const uint8_t* rcodes, const uint8_t* rscales, const float* rts,
                                 unsigned long long* stats8, cudaStream_t s) {
-#if NVFP4_GUIDED_STAGED
+#if NVFP4_GS_STAGED
   switch (hints ? hint_bits : 0) {
     case 0: return launch_staged<0, true>(x, nblk, nullptr, ws, codes, scales, tensor_scale, nullptr, rcodes, rscales, rts, stats8, s);
     case 1: return launch_staged<1, true>(x, nblk, hints, ws, codes, scales, tensor_scale, stats4, rcodes, rscales, rts, stats8, s);
