@@ -158,6 +158,11 @@ def test_gemm_quantize_small(hint_bits):
     (384, 512, 1024, ("heavy", "outlier")),        # 3 x 4 tiles, 4 K-blocks: ring wraps
     (128, 256, 4096, ("normal", "tiny")),          # long K, subnormal block scales
     (256, 128, 768, ("sparse", "ties")),           # zeros, -0, grid midpoints
+    # 256 x 256 tiles over CTA pairs (m, n multiples of 256)
+    (512, 768, 2048, ("normal", "heavy")),         # 2 x 3 pair tiles, ring wraps
+    (256, 512, 256, ("outlier", "normal")),        # one K-block per tile
+    (768, 256, 4096, ("tiny", "normal")),          # long K, subnormal block scales
+    (1024, 1024, 512, ("sparse", "ties")),         # 16 pair tiles
 ])
 def test_gemm_quantize_shapes(m, n, k, kinds):
     _run_case(m, n, k, 23 + m + k, kinds)

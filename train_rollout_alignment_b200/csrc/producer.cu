@@ -63,6 +63,9 @@ using namespace umma;
 #ifndef NVFP4_GEMM_EPI_WARPS
 #define NVFP4_GEMM_EPI_WARPS 8
 #endif
+#ifndef NVFP4_GEMM_PAIR
+#define NVFP4_GEMM_PAIR 1   // 256 x 256 tiles over CTA pairs where the shape allows
+#endif
 
 constexpr int kBM = 128, kBN = 128;
 constexpr int kBK = 256;                             // elements per K-block (128 bytes)
@@ -388,6 +391,232 @@ __global__ void __launch_bounds__(kProducerThreads, kCtasPerSm)
   }
 }
 
+// ----------------------------------------------------------------- the CTA-pair form
+// The same GEMM + quantizing epilogue on 256 x 256 output tiles shared by a
+// cluster of two CTAs on two SMs (tcgen05 cta_group::2): each CTA holds
+// 128 rows of A and 128 of the 256 rows of B per K-block, the pair's MMA
+// (issued by the even CTA) computes the 256 x 256 tile, and each CTA's TMEM
+// receives its 128 rows.  Per SM and K-block of 256 this streams 38 KB for
+// 16.8 MFLOP where the 128 x 128 form streams 36 KB for 8.4: half the L2
+// traffic per FLOP, the resource the single-CTA form runs out of.  Each CTA
+// also needs the scales of all 256 rows of B (its TMEM reads the scale of
+// every output column).  TMEM: the 256-column accumulator and the scale
+// factors of every stage (48 columns each); there is no room for a second
+// accumulator, so 16 epilogue warps load their 64 columns each into
+// registers at once and hand the accumulator back before quantizing.  All
+// loads are TMA loads (no multicast) whose completion is counted on the even
+// CTA's barrier; the MMA's completion is signalled to both CTAs.
+constexpr int kPairStages = 4;
+constexpr int kPairBN = 256;                                 // output columns per tile
+constexpr int kPairEpiWarps = 16;
+constexpr int kPairThreads = 32 * (2 + kPairEpiWarps);
+constexpr uint32_t kPairA = 128 * (kBK / 2);                  // 16 KB
+constexpr uint32_t kPairB = 128 * (kBK / 2);                  // 16 KB: this CTA's half of B
+constexpr uint32_t kPairSfa = (kBK / 64) * kScaleTile;        // 2 KB
+constexpr uint32_t kPairSfb = 2 * (kBK / 64) * kScaleTile;    // 4 KB: both 128-row tiles of B
+constexpr uint32_t kPairStageTx = kPairA + kPairB + kPairSfa + kPairSfb;
+constexpr uint32_t kPOffA = 0;
+constexpr uint32_t kPOffB = kPOffA + kPairStages * kPairA;
+constexpr uint32_t kPOffSfa = kPOffB + kPairStages * kPairB;
+constexpr uint32_t kPOffSfb = kPOffSfa + kPairStages * kPairSfa;
+constexpr uint32_t kPOffBar = kPOffSfb + kPairStages * kPairSfb;  // full[S], empty[S], acc_full, acc_empty
+constexpr uint32_t kPOffSlot = kPOffBar + 8 * (2 * kPairStages + 2);
+constexpr uint32_t kPOffAbort = kPOffSlot + 4;
+constexpr uint32_t kPOffTables = (kPOffAbort + 4 + 15) / 16 * 16;
+constexpr uint32_t kPairSmem = kPOffTables + sizeof(ScaleTables) + 1024;
+constexpr uint32_t kPairTmemCols = 512;
+constexpr uint32_t kPairTmemSf = 256;                          // stage s scales at 256 + 48 s
+static_assert(kPairTmemSf + 48 * kPairStages <= kPairTmemCols, "TMEM budget");
+static_assert(kPairSmem <= 227 * 1024, "shared memory");
+static_assert(kPOffB % 1024 == 0 && kPOffSfa % 1024 == 0, "swizzled tiles need 1024-byte bases");
+
+template <int HB>
+__global__ void __launch_bounds__(kPairThreads, 1)
+    k_gemm_nvfp4_quantize_pair(const __grid_constant__ CUtensorMap tm_a,
+                               const __grid_constant__ CUtensorMap tm_b,
+                               const __grid_constant__ CUtensorMap tm_sa,
+                               const __grid_constant__ CUtensorMap tm_sb,
+                               const float* __restrict__ a_ts, const float* __restrict__ b_ts,
+                               int n, int n_tiles_n, int tiles, int kblocks,
+                               uint32_t* __restrict__ ws, ProducerOut out) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const int cluster = blockIdx.x >> 1, clusters = gridDim.x >> 1;
+  const uint32_t base = smem_u32(smem);
+  const uint32_t full = base + kPOffBar, empty = full + 8 * kPairStages;
+  const uint32_t acc_full = empty + 8 * kPairStages, acc_empty = acc_full + 8;
+  volatile int* abort = reinterpret_cast<volatile int*>(smem + kPOffAbort);
+  ScaleTables& tab = *reinterpret_cast<ScaleTables*>(smem + kPOffTables);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kPairStages; ++s) {
+      mbar_init(full + 8 * s, 1);
+      mbar_init(empty + 8 * s, 1);
+    }
+    mbar_init(acc_full, 1);
+    mbar_init(acc_empty, 2 * kPairEpiWarps);
+    *abort = 0;
+    fence_mbar_init();
+    prefetch_tensormap(&tm_a);
+    prefetch_tensormap(&tm_b);
+    prefetch_tensormap(&tm_sa);
+    prefetch_tensormap(&tm_sb);
+  }
+  cluster_sync();  // both CTAs' barriers exist before either signals the other's
+  if (warp == 1) {
+    tmem_alloc_pair(base + kPOffSlot, kPairTmemCols);
+    tc_fence_before();
+  }
+  const float s_t = tensor_scale_from_amax(__uint_as_float(ws[0]));
+  scale_tables_init_f32(tab, s_t);  // ends with __syncthreads
+  tc_fence_after();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + kPOffSlot);
+  const int64_t col_tiles_k = (int64_t)kblocks * (kBK / 64);
+
+  if (warp == 0) {
+    // ---------------- producer (both CTAs): this CTA's halves of A and B, the
+    // scales of its A rows and of all 256 B rows; completion on CTA 0's barrier
+    if (lane == 0) {
+      int it = 0;
+      for (int tile = cluster; tile < tiles && !*abort; tile += clusters) {
+        const int mt = tile / n_tiles_n, nt = tile - mt * n_tiles_n;
+        const int a_row = mt * 256 + (int)rank * 128, b_row = nt * kPairBN + (int)rank * 128;
+        const int sfa_row = (int)(((int64_t)(2 * mt + (int)rank) * col_tiles_k) * 32);
+        const int sfb_row0 = (int)(((int64_t)(2 * nt) * col_tiles_k) * 32);
+        const int sfb_row1 = (int)(((int64_t)(2 * nt + 1) * col_tiles_k) * 32);
+        for (int kb = 0; kb < kblocks; ++kb, ++it) {
+          const int s = it % kPairStages;
+          const uint32_t ph = (uint32_t)(it / kPairStages) & 1u;
+          if (!mbar_wait(empty + 8 * s, ph ^ 1u, abort)) break;
+          if (rank == 0) mbar_arrive_expect_tx(full + 8 * s, 2 * kPairStageTx);
+          const uint32_t bar = mapa_shared(full + 8 * s, 0);
+          tma_load_2d_pair(base + kPOffA + s * kPairA, &tm_a, bar, kb * (kBK / 2), a_row);
+          tma_load_2d_pair(base + kPOffB + s * kPairB, &tm_b, bar, kb * (kBK / 2), b_row);
+          tma_load_2d_pair(base + kPOffSfa + s * kPairSfa, &tm_sa, bar, 0, sfa_row + kb * 128);
+          tma_load_2d_pair(base + kPOffSfb + s * kPairSfb, &tm_sb, bar, 0, sfb_row0 + kb * 128);
+          tma_load_2d_pair(base + kPOffSfb + s * kPairSfb + kPairSfb / 2, &tm_sb, bar, 0,
+                           sfb_row1 + kb * 128);
+        }
+      }
+      // drain: the MMA's completion signal for every stage has reached this
+      // CTA before it can leave the cluster
+      for (int i = 0; i < kPairStages; ++i, ++it) {
+        const int s = it % kPairStages;
+        if (!mbar_wait(empty + 8 * s, ((uint32_t)(it / kPairStages) & 1u) ^ 1u, abort)) break;
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ---------------- MMA issuer: CTA 0 only
+    if (rank == 0 && lane == 0) {
+      constexpr uint32_t idesc = idesc_nvf4(256, kPairBN);
+      int it = 0, tc = 0;
+      for (int tile = cluster; tile < tiles && !*abort; tile += clusters, ++tc) {
+        if (!mbar_wait(acc_empty, ((uint32_t)tc & 1u) ^ 1u, abort)) break;
+        tc_fence_after();
+        for (int kb = 0; kb < kblocks; ++kb, ++it) {
+          const int s = it % kPairStages;
+          const uint32_t ph = (uint32_t)(it / kPairStages) & 1u;
+          if (!mbar_wait(full + 8 * s, ph, abort)) break;
+          tc_fence_after();
+          const uint32_t sf = tmem + kPairTmemSf + 48u * (uint32_t)s;  // SFA +4j, SFB +16+8j
+          const uint32_t sfa_s = base + kPOffSfa + s * kPairSfa;
+          const uint32_t sfb_s = base + kPOffSfb + s * kPairSfb;
+#pragma unroll
+          for (int j = 0; j < kBK / 64; ++j) {
+            cp_32x128b_warpx4_pair(sf + 4 * j, desc_scale_chunk(sfa_s + j * kScaleTile));
+            cp_32x128b_warpx4_pair(sf + 16 + 8 * j, desc_scale_chunk(sfb_s + j * kScaleTile));
+            cp_32x128b_warpx4_pair(sf + 20 + 8 * j,
+                                   desc_scale_chunk(sfb_s + kPairSfb / 2 + j * kScaleTile));
+          }
+          const uint64_t da = desc_kmajor_sw128(base + kPOffA + s * kPairA);
+          const uint64_t db = desc_kmajor_sw128(base + kPOffB + s * kPairB);
+#pragma unroll
+          for (int j = 0; j < kBK / 64; ++j)
+            mma_nvf4_pair(tmem, da + 2 * j, db + 2 * j, idesc, sf + 4 * j, sf + 16 + 8 * j,
+                          (kb | j) != 0);
+          mma_commit_pair(empty + 8 * s, 0x3);
+        }
+        mma_commit_pair(acc_full, 0x3);
+      }
+    }
+    __syncwarp();
+  } else {
+    // ---------------- epilogue (both CTAs): this CTA's 128 rows of the tile
+    const int q = warp & 3;            // TMEM lane quadrant this warp may read
+    const int cg = (warp - 2) >> 2;    // 64-column group
+    const float alpha = __fmul_rn(*a_ts, *b_ts);
+    const int64_t sf_cols_out = n / 16;
+    const int64_t col_tiles_n = n / 64;
+    const uint32_t acc_empty0 = mapa_shared(acc_empty, 0);
+    if (blockIdx.x == 0 && warp == 2 && lane == 0) *out.tensor_scale = s_t;
+    float dmax = 0.0f;
+    int tc = 0;
+    for (int tile = cluster; tile < tiles; tile += clusters, ++tc) {
+      const int mt = tile / n_tiles_n, nt = tile - mt * n_tiles_n;
+      const bool ok = mbar_wait(acc_full, (uint32_t)tc & 1u, abort);
+      __syncwarp();  // tcgen05.ld is warp-collective
+      if (!__all_sync(0xFFFFFFFFu, ok)) break;
+      tc_fence_after();
+      float y[64];
+      tmem_ld64(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(cg * 64), y);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(acc_empty0);  // the accumulator may be overwritten
+      const int64_t row = (int64_t)mt * 256 + rank * 128 + q * 32 + lane;
+      const int64_t col0 = (int64_t)nt * kPairBN + cg * 64;
+      const int64_t blk0 = row * sf_cols_out + col0 / 16;
+      uint32_t sc = 0;
+      uint2 cc[4];
+#pragma unroll
+      for (int c16 = 0; c16 < 4; ++c16) {
+        float* yb = y + 16 * c16;
+        float amax = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          yb[i] = __fmul_rn(yb[i], alpha);
+          amax = fmaxf(amax, fabsf(yb[i]));
+        }
+        dmax = fmaxf(dmax, amax);
+        if (out.d_out != nullptr) {
+          float* dp = out.d_out + row * n + col0 + 16 * c16;
+#pragma unroll
+          for (int h = 0; h < 2; ++h) st_v8f(dp + 8 * h, yb + 8 * h);
+        }
+        const BlockScale bs = block_scale_f32(amax, s_t, tab);
+        if (inv_overflowed(bs.inv)) {
+          cc[c16] = overflow_codes_f32(yb);
+        } else {
+          float v[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) v[i] = __fmul_rn(yb[i], bs.inv);
+          cc[c16] = pack_codes16(v);
+        }
+        sc |= bs.sb << (8 * c16);
+      }
+      store_row_segment<4>(out.codes + blk0 * 8, cc);
+      if (HB != 0) store_hints_segment<HB, 4>(out.hints, blk0, cc);
+      *reinterpret_cast<uint32_t*>(out.scales + blk0) = sc;
+      if (out.scales_mma != nullptr)
+        *reinterpret_cast<uint32_t*>(out.scales_mma + mma_scale_offset(row, col0 / 16, col_tiles_n)) = sc;
+    }
+    const uint32_t wmax = warp_max_u32(__float_as_uint(dmax));
+    if (lane == 0) atomicMax(ws + 2, wmax);
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // every MMA of the pair has completed and been read
+  if (*abort && threadIdx.x == 0) atomicOr(ws + 1, NVFP4_WARN_TIMEOUT);
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem, kPairTmemCols);
+  }
+}
+
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
   if (fn == nullptr) {
@@ -412,6 +641,55 @@ bool codes_tensor_map(CUtensorMap* map, const uint8_t* codes, int64_t rows, int6
   return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(codes), dims, strides,
              box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// The tensor-core scale layout viewed as [bytes / 16, 16]: boxes of 128 x 16
+// bytes, i.e. the 2 KiB of one 128-row tile group for one K-block of 256.
+bool scales_tensor_map(CUtensorMap* map, const uint8_t* sf, int64_t rows, int64_t k) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+  if (enc == nullptr) return false;
+  const int64_t bytes = ((rows + 127) / 128) * (k / 64) * kScaleTile;
+  cuuint64_t dims[2] = {16, (cuuint64_t)(bytes / 16)};
+  cuuint64_t strides[1] = {16};
+  cuuint32_t box[2] = {16, 128};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(sf), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int HB>
+cudaError_t launch_gemm_pair_hb(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tsa,
+                                const CUtensorMap& tsb, const float* a_ts, const float* b_ts,
+                                int64_t m, int64_t n, int64_t k, uint32_t* ws,
+                                const ProducerOut& out, cudaStream_t s) {
+  static bool attr_set[64] = {false};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64 || !attr_set[dev]) {
+    e = cudaFuncSetAttribute(k_gemm_nvfp4_quantize_pair<HB>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, kPairSmem);
+    if (e != cudaSuccess) return e;
+    if (dev >= 0 && dev < 64) attr_set[dev] = true;
+  }
+  const int64_t tiles = (m / 256) * (n / kPairBN);
+  const int64_t pairs = sm_count() / 2;
+  const int clusters = (int)(tiles < pairs ? tiles : pairs);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * clusters, 1, 1);
+  cfg.blockDim = dim3(kPairThreads, 1, 1);
+  cfg.dynamicSmemBytes = kPairSmem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, k_gemm_nvfp4_quantize_pair<HB>, ta, tb, tsa, tsb, a_ts, b_ts, (int)n,
+                            (int)(n / kPairBN), (int)tiles, (int)(k / kBK), ws, out);
 }
 
 template <int HB>
@@ -494,6 +772,20 @@ cudaError_t launch_gemm_quantize(const uint8_t* a_codes, const uint8_t* a_sf, co
     return cudaErrorInvalidValue;
   const ProducerOut out{codes, scales, scales_mma, tensor_scale, hints, d_out};
   const int g = (int)groups;
+#if NVFP4_GEMM_PAIR
+  // the CTA-pair form: plain GEMMs whose tiles of 256 x 256 cover the output
+  if (groups == 1 && m % 256 == 0 && n % kPairBN == 0 && sm_count() >= 2) {
+    CUtensorMap tsa, tsb;
+    if (!scales_tensor_map(&tsa, a_sf, m, k) || !scales_tensor_map(&tsb, b_sf, n, k))
+      return cudaErrorInvalidValue;
+    switch (hints == nullptr ? 0 : hint_bits) {
+      case 1: return launch_gemm_pair_hb<1>(ta, tb, tsa, tsb, a_ts, b_ts, m, n, k, ws, out, s);
+      case 2: return launch_gemm_pair_hb<2>(ta, tb, tsa, tsb, a_ts, b_ts, m, n, k, ws, out, s);
+      case 4: return launch_gemm_pair_hb<4>(ta, tb, tsa, tsb, a_ts, b_ts, m, n, k, ws, out, s);
+      default: return launch_gemm_pair_hb<0>(ta, tb, tsa, tsb, a_ts, b_ts, m, n, k, ws, out, s);
+    }
+  }
+#endif
   switch (hints == nullptr ? 0 : hint_bits) {
     case 1: return launch_gemm_hb<1>(ta, tb, a_sf, b_sf, a_ts, b_ts, group_rows, g, m, n, k, ws, out, s);
     case 2: return launch_gemm_hb<2>(ta, tb, a_sf, b_sf, a_ts, b_ts, group_rows, g, m, n, k, ws, out, s);

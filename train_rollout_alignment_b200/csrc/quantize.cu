@@ -782,7 +782,7 @@ cudaError_t launch_quantize_rtn(const uint16_t* x, int64_t nblk, const uint32_t*
 }
 
 #ifndef NVFP4_GUIDED_STAGED
-#define NVFP4_GUIDED_STAGED 1   // guided alone: staged (1) or one block per thread from registers (0)
+#define NVFP4_GUIDED_STAGED 0   // guided alone: staged (1) or two blocks per thread from registers (0)
 #endif
 #ifndef NVFP4_GS_STAGED
 #define NVFP4_GS_STAGED 1       // guided + counters: staged (1) or from registers (0)
