@@ -76,7 +76,8 @@ constexpr int kEpiWarps = NVFP4_GEMM_EPI_WARPS;
 constexpr int kEpiColGroups = kEpiWarps / 4;         // column slices per lane quadrant
 constexpr int kEpiBlocks = kBN / 16 / kEpiColGroups; // 16-column blocks per epilogue thread
 static_assert(kEpiWarps == 4 || kEpiWarps == 8, "epilogue warps");
-constexpr int kProducerThreads = 32 * (2 + kEpiWarps);
+constexpr int kSfWarp = 2 + kEpiWarps;               // the warp that copies scale factors
+constexpr int kProducerThreads = 32 * (3 + kEpiWarps);
 constexpr uint32_t kTileBytes = kBM * kBK / 2;       // 16 KB for A, same for B (kBN == kBM)
 constexpr uint32_t kScaleTile = 512;                 // 128 rows x 4 scales
 constexpr uint32_t kScaleBytes = (kBK / 64) * kScaleTile;  // 2 KB per operand per stage
@@ -93,9 +94,9 @@ constexpr uint32_t kOffA = 0;
 constexpr uint32_t kOffB = kOffA + kStages * kTileBytes;
 constexpr uint32_t kOffSfa = kOffB + kStages * kTileBytes;
 constexpr uint32_t kOffSfb = kOffSfa + kStages * kScaleBytes;
-// barriers: full[STAGES], empty[STAGES], acc_full[ACC], acc_empty[ACC]
+// barriers: full[STAGES], empty[STAGES], acc_full[ACC], acc_empty[ACC], sf_ready[STAGES]
 constexpr uint32_t kOffBar = kOffSfb + kStages * kScaleBytes;
-constexpr uint32_t kOffTmemSlot = kOffBar + 8 * (2 * kStages + 2 * kAccBufs);
+constexpr uint32_t kOffTmemSlot = kOffBar + 8 * (3 * kStages + 2 * kAccBufs);
 constexpr uint32_t kOffAbort = kOffTmemSlot + 4;
 constexpr uint32_t kOffTables = (kOffAbort + 4 + 15) / 16 * 16;
 constexpr uint32_t kSmemUsed = kOffTables + sizeof(ScaleTables);
@@ -207,6 +208,7 @@ __global__ void __launch_bounds__(kProducerThreads, kCtasPerSm)
   const uint32_t base = smem_u32(smem);
   const uint32_t full = base + kOffBar, empty = full + 8 * kStages;
   const uint32_t acc_full = empty + 8 * kStages, acc_empty = acc_full + 8 * kAccBufs;
+  const uint32_t sf_ready = acc_empty + 8 * kAccBufs;  // [STAGES]: a stage's scales are in TMEM
   volatile int* abort = reinterpret_cast<volatile int*>(smem + kOffAbort);
   ScaleTables& tab = *reinterpret_cast<ScaleTables*>(smem + kOffTables);
 
@@ -214,6 +216,7 @@ __global__ void __launch_bounds__(kProducerThreads, kCtasPerSm)
     for (int s = 0; s < kStages; ++s) {
       mbar_init(full + 8 * s, 1);
       mbar_init(empty + 8 * s, 1);
+      mbar_init(sf_ready + 8 * s, 1);
     }
     for (int b = 0; b < kAccBufs; ++b) {
       mbar_init(acc_full + 8 * b, 1);
@@ -282,16 +285,9 @@ __global__ void __launch_bounds__(kProducerThreads, kCtasPerSm)
         for (int kb = 0; kb < kblocks; ++kb, ++it) {
           const int s = it % kStages;
           const uint32_t ph = (uint32_t)(it / kStages) & 1u;
-          if (!mbar_wait(full + 8 * s, ph, abort)) break;
+          if (!mbar_wait(sf_ready + 8 * s, ph, abort)) break;  // implies the stage has landed
           tc_fence_after();
           const uint32_t sf = tmem + kTmemSfBase + 32u * (uint32_t)s;  // SFA +0, SFB +16
-#pragma unroll
-          for (int j = 0; j < kBK / 64; ++j) {
-            cp_32x128b_warpx4(sf + 4 * j,
-                              desc_scale_chunk(base + kOffSfa + s * kScaleBytes + j * kScaleTile));
-            cp_32x128b_warpx4(sf + 16 + 4 * j,
-                              desc_scale_chunk(base + kOffSfb + s * kScaleBytes + j * kScaleTile));
-          }
           const uint64_t da = desc_kmajor_sw128(base + kOffA + s * kTileBytes);
           const uint64_t db = desc_kmajor_sw128(base + kOffB + s * kTileBytes);
 #pragma unroll
@@ -301,6 +297,32 @@ __global__ void __launch_bounds__(kProducerThreads, kCtasPerSm)
           mma_commit(empty + 8 * s);
         }
         mma_commit(acc_full + 8 * buf);
+      }
+    }
+    __syncwarp();
+  } else if (warp == kSfWarp) {
+    // ---------------- scale-factor copies into TMEM as soon as a stage has
+    // landed, running ahead of the MMA warp (copies issued by the MMA warp
+    // itself stall the tensor pipe between stages).  A stage's TMEM slot is
+    // free then: the stage was reloaded only after the MMAs that last read
+    // the slot had completed.
+    if (lane == 0) {
+      int it = 0;
+      for (int tile = blockIdx.x; tile < tiles && !*abort; tile += gridDim.x) {
+        for (int kb = 0; kb < kblocks; ++kb, ++it) {
+          const int s = it % kStages;
+          if (!mbar_wait(full + 8 * s, (uint32_t)(it / kStages) & 1u, abort)) break;
+          tc_fence_after();
+          const uint32_t sf = tmem + kTmemSfBase + 32u * (uint32_t)s;  // SFA +0, SFB +16
+#pragma unroll
+          for (int j = 0; j < kBK / 64; ++j) {
+            cp_32x128b_warpx4(sf + 4 * j,
+                              desc_scale_chunk(base + kOffSfa + s * kScaleBytes + j * kScaleTile));
+            cp_32x128b_warpx4(sf + 16 + 4 * j,
+                              desc_scale_chunk(base + kOffSfb + s * kScaleBytes + j * kScaleTile));
+          }
+          mma_commit(sf_ready + 8 * s);
+        }
       }
     }
     __syncwarp();
@@ -406,10 +428,14 @@ __global__ void __launch_bounds__(kProducerThreads, kCtasPerSm)
 // registers at once and hand the accumulator back before quantizing.  All
 // loads are TMA loads (no multicast) whose completion is counted on the even
 // CTA's barrier; the MMA's completion is signalled to both CTAs.
-constexpr int kPairStages = 4;
+#ifndef NVFP4_PAIR_STAGES
+#define NVFP4_PAIR_STAGES 4
+#endif
+constexpr int kPairStages = NVFP4_PAIR_STAGES;
 constexpr int kPairBN = 256;                                 // output columns per tile
 constexpr int kPairEpiWarps = 16;
-constexpr int kPairThreads = 32 * (2 + kPairEpiWarps);
+constexpr int kPairSfWarp = 2 + kPairEpiWarps;                // the warp that copies scale factors
+constexpr int kPairThreads = 32 * (3 + kPairEpiWarps);
 constexpr uint32_t kPairA = 128 * (kBK / 2);                  // 16 KB
 constexpr uint32_t kPairB = 128 * (kBK / 2);                  // 16 KB: this CTA's half of B
 constexpr uint32_t kPairSfa = (kBK / 64) * kScaleTile;        // 2 KB
@@ -419,14 +445,14 @@ constexpr uint32_t kPOffA = 0;
 constexpr uint32_t kPOffB = kPOffA + kPairStages * kPairA;
 constexpr uint32_t kPOffSfa = kPOffB + kPairStages * kPairB;
 constexpr uint32_t kPOffSfb = kPOffSfa + kPairStages * kPairSfa;
-constexpr uint32_t kPOffBar = kPOffSfb + kPairStages * kPairSfb;  // full[S], empty[S], acc_full, acc_empty
-constexpr uint32_t kPOffSlot = kPOffBar + 8 * (2 * kPairStages + 2);
+constexpr uint32_t kPOffBar = kPOffSfb + kPairStages * kPairSfb;  // full[S], empty[S], acc_full, acc_empty, sf_ready[S]
+constexpr uint32_t kPOffSlot = kPOffBar + 8 * (3 * kPairStages + 2);
 constexpr uint32_t kPOffAbort = kPOffSlot + 4;
 constexpr uint32_t kPOffTables = (kPOffAbort + 4 + 15) / 16 * 16;
 constexpr uint32_t kPairSmem = kPOffTables + sizeof(ScaleTables) + 1024;
 constexpr uint32_t kPairTmemCols = 512;
 constexpr uint32_t kPairTmemSf = 256;                          // stage s scales at 256 + 48 s
-static_assert(kPairTmemSf + 48 * kPairStages <= kPairTmemCols, "TMEM budget");
+static_assert(kPairTmemSf + 48 * kPairStages <= kPairTmemCols, "TMEM budget");  // at most 5 stages
 static_assert(kPairSmem <= 227 * 1024, "shared memory");
 static_assert(kPOffB % 1024 == 0 && kPOffSfa % 1024 == 0, "swizzled tiles need 1024-byte bases");
 
@@ -448,6 +474,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
   const uint32_t base = smem_u32(smem);
   const uint32_t full = base + kPOffBar, empty = full + 8 * kPairStages;
   const uint32_t acc_full = empty + 8 * kPairStages, acc_empty = acc_full + 8;
+  const uint32_t sf_ready = acc_empty + 8;  // [S]: the stage's scale factors are in TMEM
   volatile int* abort = reinterpret_cast<volatile int*>(smem + kPOffAbort);
   ScaleTables& tab = *reinterpret_cast<ScaleTables*>(smem + kPOffTables);
 
@@ -458,6 +485,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     }
     mbar_init(acc_full, 1);
     mbar_init(acc_empty, 2 * kPairEpiWarps);
+    for (int st = 0; st < kPairStages; ++st) mbar_init(sf_ready + 8 * st, 1);
     *abort = 0;
     fence_mbar_init();
     prefetch_tensormap(&tm_a);
@@ -484,9 +512,10 @@ __global__ void __launch_bounds__(kPairThreads, 1)
       for (int tile = cluster; tile < tiles && !*abort; tile += clusters) {
         const int mt = tile / n_tiles_n, nt = tile - mt * n_tiles_n;
         const int a_row = mt * 256 + (int)rank * 128, b_row = nt * kPairBN + (int)rank * 128;
-        const int sfa_row = (int)(((int64_t)(2 * mt + (int)rank) * col_tiles_k) * 32);
-        const int sfb_row0 = (int)(((int64_t)(2 * nt) * col_tiles_k) * 32);
-        const int sfb_row1 = (int)(((int64_t)(2 * nt + 1) * col_tiles_k) * 32);
+        // scale rows of 256 bytes: tile (rt, kt) starts at row (rt * col_tiles_k + kt) * 2
+        const int sfa_row = (int)(((int64_t)(2 * mt + (int)rank) * col_tiles_k) * 2);
+        const int sfb_row0 = (int)(((int64_t)(2 * nt) * col_tiles_k) * 2);
+        const int sfb_row1 = (int)(((int64_t)(2 * nt + 1) * col_tiles_k) * 2);
         for (int kb = 0; kb < kblocks; ++kb, ++it) {
           const int s = it % kPairStages;
           const uint32_t ph = (uint32_t)(it / kPairStages) & 1u;
@@ -495,10 +524,10 @@ __global__ void __launch_bounds__(kPairThreads, 1)
           const uint32_t bar = mapa_shared(full + 8 * s, 0);
           tma_load_2d_pair(base + kPOffA + s * kPairA, &tm_a, bar, kb * (kBK / 2), a_row);
           tma_load_2d_pair(base + kPOffB + s * kPairB, &tm_b, bar, kb * (kBK / 2), b_row);
-          tma_load_2d_pair(base + kPOffSfa + s * kPairSfa, &tm_sa, bar, 0, sfa_row + kb * 128);
-          tma_load_2d_pair(base + kPOffSfb + s * kPairSfb, &tm_sb, bar, 0, sfb_row0 + kb * 128);
+          tma_load_2d_pair(base + kPOffSfa + s * kPairSfa, &tm_sa, bar, 0, sfa_row + kb * 8);
+          tma_load_2d_pair(base + kPOffSfb + s * kPairSfb, &tm_sb, bar, 0, sfb_row0 + kb * 8);
           tma_load_2d_pair(base + kPOffSfb + s * kPairSfb + kPairSfb / 2, &tm_sb, bar, 0,
-                           sfb_row1 + kb * 128);
+                           sfb_row1 + kb * 8);
         }
       }
       // drain: the MMA's completion signal for every stage has reached this
@@ -510,7 +539,9 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     }
     __syncwarp();
   } else if (warp == 1) {
-    // ---------------- MMA issuer: CTA 0 only
+    // ---------------- MMA issuer: CTA 0 only.  It waits for a stage's scale
+    // factors to be in TMEM (copied by the scale-factor warp, which runs ahead)
+    // and issues the stage's four MMAs.
     if (rank == 0 && lane == 0) {
       constexpr uint32_t idesc = idesc_nvf4(256, kPairBN);
       int it = 0, tc = 0;
@@ -520,18 +551,9 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         for (int kb = 0; kb < kblocks; ++kb, ++it) {
           const int s = it % kPairStages;
           const uint32_t ph = (uint32_t)(it / kPairStages) & 1u;
-          if (!mbar_wait(full + 8 * s, ph, abort)) break;
+          if (!mbar_wait(sf_ready + 8 * s, ph, abort)) break;  // implies the stage's data is in
           tc_fence_after();
           const uint32_t sf = tmem + kPairTmemSf + 48u * (uint32_t)s;  // SFA +4j, SFB +16+8j
-          const uint32_t sfa_s = base + kPOffSfa + s * kPairSfa;
-          const uint32_t sfb_s = base + kPOffSfb + s * kPairSfb;
-#pragma unroll
-          for (int j = 0; j < kBK / 64; ++j) {
-            cp_32x128b_warpx4_pair(sf + 4 * j, desc_scale_chunk(sfa_s + j * kScaleTile));
-            cp_32x128b_warpx4_pair(sf + 16 + 8 * j, desc_scale_chunk(sfb_s + j * kScaleTile));
-            cp_32x128b_warpx4_pair(sf + 20 + 8 * j,
-                                   desc_scale_chunk(sfb_s + kPairSfb / 2 + j * kScaleTile));
-          }
           const uint64_t da = desc_kmajor_sw128(base + kPOffA + s * kPairA);
           const uint64_t db = desc_kmajor_sw128(base + kPOffB + s * kPairB);
 #pragma unroll
@@ -541,6 +563,32 @@ __global__ void __launch_bounds__(kPairThreads, 1)
           mma_commit_pair(empty + 8 * s, 0x3);
         }
         mma_commit_pair(acc_full, 0x3);
+      }
+    }
+    __syncwarp();
+  } else if (warp == kPairSfWarp) {
+    // ---------------- scale-factor copies: CTA 0 only, as soon as a stage has
+    // landed.  Its TMEM slot is free then: the stage was reloaded only after
+    // the MMAs that read the slot last had completed.
+    if (rank == 0 && lane == 0) {
+      int it = 0;
+      for (int tile = cluster; tile < tiles && !*abort; tile += clusters) {
+        for (int kb = 0; kb < kblocks; ++kb, ++it) {
+          const int s = it % kPairStages;
+          if (!mbar_wait(full + 8 * s, (uint32_t)(it / kPairStages) & 1u, abort)) break;
+          tc_fence_after();
+          const uint32_t sf = tmem + kPairTmemSf + 48u * (uint32_t)s;
+          const uint32_t sfa_s = base + kPOffSfa + s * kPairSfa;
+          const uint32_t sfb_s = base + kPOffSfb + s * kPairSfb;
+#pragma unroll
+          for (int j = 0; j < kBK / 64; ++j) {
+            cp_32x128b_warpx4_pair(sf + 4 * j, desc_scale_chunk(sfa_s + j * kScaleTile));
+            cp_32x128b_warpx4_pair(sf + 16 + 8 * j, desc_scale_chunk(sfb_s + j * kScaleTile));
+            cp_32x128b_warpx4_pair(sf + 20 + 8 * j,
+                                   desc_scale_chunk(sfb_s + kPairSfb / 2 + j * kScaleTile));
+          }
+          mma_commit_pair(sf_ready + 8 * s, 0x1);
+        }
       }
     }
     __syncwarp();
@@ -643,15 +691,18 @@ bool codes_tensor_map(CUtensorMap* map, const uint8_t* codes, int64_t rows, int6
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// The tensor-core scale layout viewed as [bytes / 16, 16]: boxes of 128 x 16
-// bytes, i.e. the 2 KiB of one 128-row tile group for one K-block of 256.
+// The tensor-core scale layout viewed as [bytes / 256, 256]: boxes of 8 rows
+// of 256 bytes, i.e. the 2 KiB of one 128-row tile group for one K-block of
+// 256 (every span starts on a 512-byte tile boundary), fetched as eight
+// 256-byte requests.
+constexpr int kSfRow = 256;
 bool scales_tensor_map(CUtensorMap* map, const uint8_t* sf, int64_t rows, int64_t k) {
   PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
   if (enc == nullptr) return false;
   const int64_t bytes = ((rows + 127) / 128) * (k / 64) * kScaleTile;
-  cuuint64_t dims[2] = {16, (cuuint64_t)(bytes / 16)};
-  cuuint64_t strides[1] = {16};
-  cuuint32_t box[2] = {16, 128};
+  cuuint64_t dims[2] = {kSfRow, (cuuint64_t)(bytes / kSfRow)};
+  cuuint64_t strides[1] = {kSfRow};
+  cuuint32_t box[2] = {kSfRow, (cuuint32_t)((kBK / 64) * kScaleTile / kSfRow)};
   cuuint32_t estr[2] = {1, 1};
   return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(sf), dims, strides, box, estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
