@@ -556,11 +556,34 @@ def _timed(fn, reps, flush):
     return statistics.median(times) / 1e3
 
 
+def _timed_b2b(fn, count=10, reps=3):
+    """Device time per call of `count` calls launched back to back between one
+    pair of events (median over `reps` such runs), no L2 flush: for kernels
+    whose inputs are more than twice the L2, so a call cannot find its input
+    left in L2 by the one before.  Each call also pays for writing back the
+    previous call's output, as it would in a stream of work; and the event
+    timer's granularity (about a microsecond) is spread over `count` calls."""
+    times = []
+    for r in range(reps):
+        torch.cuda._sleep(100_000)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for i in range(count):
+            fn(i)
+        e1.record()
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1) / count)
+    return statistics.median(times) / 1e3
+
+
 def time_other_kernels(b, stack, device, peak, sm_mhz, reps=10):
     """Standalone hint emit (throughput stack, layer 24), SR transpose
     re-quantize (128 x 512 x 2048 expert stack) and RHT32 + quantize
     (16384 x 4096 activation with outliers): seconds per call and algorithmic
-    GB/s (median of `reps` calls), L2 flushed before every call."""
+    GB/s (median of `reps` calls), L2 flushed before every call; kernels whose
+    inputs are more than twice the L2 (the counters, the two quantizers alone,
+    tile quantize) are timed back to back, the flushed figure beside it."""
     from train_rollout_alignment_b200 import synthetic as syn
     flush = (torch.zeros(64 << 20, dtype=torch.float32, device=device),
              torch.ones(64 << 20, dtype=torch.float32, device=device))
@@ -576,15 +599,21 @@ def time_other_kernels(b, stack, device, peak, sm_mhz, reps=10):
                         "GB/s": round(gbs, 1), "frac": round(gbs / peak, 4), "bytes_per_elem": BYTES["emit_hint"]}
     # the standalone counters (the step counts inside the guided pass) between
     # the rollout and train tensors of that layer
+    # (inputs of 302 MB: timed back to back, the L2-flushed figure beside it)
     s8 = torch.zeros(8, dtype=torch.int64, device=device)
-    t = _timed(lambda r: b.nvfp4_mismatch_stats(stack.cr[l], stack.sr[l], stack.ts[l, 0:1], stack.ct[l], stack.st[l],
-                                                stack.ts[l, 1:2], ROWS, COLS, s8), reps, flush)
+    stats_call = lambda r: b.nvfp4_mismatch_stats(stack.cr[l], stack.sr[l], stack.ts[l, 0:1], stack.ct[l],
+                                                  stack.st[l], stack.ts[l, 1:2], ROWS, COLS, s8)
+    t = _timed_b2b(stats_call)
+    t_f = _timed(stats_call, reps, flush)
     gbs = BYTES["mismatch_stats"] * stack.n / t / 1e9
     out["mismatch_stats"] = {"workload": "%dx%d rollout vs train NVFP4 (layer %d)" % (ROWS, COLS, l),
+                             "timing": "10 calls back to back, inputs > 2x L2",
                              "avg_us": round(t * 1e6, 2), "GB/s": round(gbs, 1), "frac": round(gbs / peak, 4),
+                             "flushed_us": round(t_f * 1e6, 2),
+                             "flushed_frac": round(BYTES["mismatch_stats"] * stack.n / t_f / 1e9 / peak, 4),
                              "bytes_per_elem": BYTES["mismatch_stats"]}
-    # the two quantizers of that layer alone, L2 flushed (in the step they
-    # may find part of their input in L2 behind the amax pass)
+    # the two quantizers of that layer alone (in the step they may find part
+    # of their input in L2 behind the amax pass): back to back and L2-flushed
     c_tmp, s_tmp = torch.empty_like(stack.ct[l]), torch.empty_like(stack.st[l])
     ts_tmp = torch.empty(1, dtype=torch.float32, device=device)
     s4 = torch.zeros(4, dtype=torch.int64, device=device)
@@ -594,11 +623,15 @@ def time_other_kernels(b, stack, device, peak, sm_mhz, reps=10):
                      ("guided_requant+hint", lambda r: b.nvfp4_guided_requant(
                          stack.xt[l], stack.hints[l], HINT_BITS, stack.ws[l, 1], c_tmp, s_tmp, ts_tmp, s4,
                          flags=b.NVFP4_AMAX_PRECOMPUTED))):
-        t = _timed(fn, reps, flush)
+        t = _timed_b2b(fn)
+        t_f = _timed(fn, reps, flush)
         gbs = BYTES[name] * stack.n / t / 1e9
         out[name + " (alone)"] = {"workload": "%dx%d BF16 layer %d, amax precomputed" % (ROWS, COLS, l),
+                                  "timing": "10 calls back to back, inputs > 2x L2",
                                   "avg_us": round(t * 1e6, 2), "GB/s": round(gbs, 1),
-                                  "frac": round(gbs / peak, 4), "bytes_per_elem": BYTES[name]}
+                                  "frac": round(gbs / peak, 4), "flushed_us": round(t_f * 1e6, 2),
+                                  "flushed_frac": round(BYTES[name] * stack.n / t_f / 1e9 / peak, 4),
+                                  "bytes_per_elem": BYTES[name]}
     del c_tmp, s_tmp
     # SR transpose: the expert stack quantized by the library's own RTN path
     batch, er, ec = syn.CFG2_SHAPE
@@ -661,12 +694,15 @@ def time_transpose_alternatives(b, stack, w, codes, scales, ts, sr_out, device, 
     ts16 = torch.empty(1, dtype=torch.float32, device=device)
     wsl = stack.ws[l, 1]
     b.nvfp4_tensor_amax(stack.xt[l], wsl)
-    t = _timed(lambda r: b.nvfp4_quantize_tile16(stack.xt[l], wsl, ct16, tt16, ts16, flags=b.NVFP4_AMAX_PRECOMPUTED),
-               reps, flush)
+    tile_call = lambda r: b.nvfp4_quantize_tile16(stack.xt[l], wsl, ct16, tt16, ts16, flags=b.NVFP4_AMAX_PRECOMPUTED)
+    t = _timed_b2b(tile_call)
+    t_f = _timed(tile_call, reps, flush)
     qb = 2 + 0.5 + 1 / 256
     out["quantize_tile16"] = {"workload": "%dx%d BF16 layer, amax precomputed" % (ROWS, COLS),
+                              "timing": "10 calls back to back, inputs > 2x L2",
                               "avg_us": round(t * 1e6, 2), "GB/s": round(qb * stack.n / t / 1e9, 1),
-                              "frac": round(qb * stack.n / t / 1e9 / peak, 4), "bytes_per_elem": qb}
+                              "frac": round(qb * stack.n / t / 1e9 / peak, 4), "flushed_us": round(t_f * 1e6, 2),
+                              "bytes_per_elem": qb}
     del ct16, tt16
     # tile codes of the expert stack, then the lossless transpose
     tc = torch.empty(n // 2, dtype=torch.uint8, device=device)
@@ -847,13 +883,16 @@ def time_producer(b, device, reps=10, m=8192, n=4096, k=4096):
     gen = torch.Generator(device=device).manual_seed(8)
     u8 = dict(dtype=torch.uint8, device=device)
 
-    def nvfp4_operand(rows, std):
-        x = (torch.randn((rows, k), device=device, generator=gen) * std).to(torch.bfloat16)
-        codes, scales, ts, ws, _ = b.empty_nvfp4(rows, k, device)
+    def nvfp4_operand_k(rows, kk, std):
+        x = (torch.randn((rows, kk), device=device, generator=gen) * std).to(torch.bfloat16)
+        codes, scales, ts, ws, _ = b.empty_nvfp4(rows, kk, device)
         b.nvfp4_quantize_rtn(x, ws, codes, scales, ts)
-        smma = torch.empty(b.mma_scale_bytes(rows, k // 16), **u8)
-        b.nvfp4_scales_to_mma(scales, rows, k // 16, smma)
+        smma = torch.empty(b.mma_scale_bytes(rows, kk // 16), **u8)
+        b.nvfp4_scales_to_mma(scales, rows, kk // 16, smma)
         return codes, smma, ts
+
+    def nvfp4_operand(rows, std):
+        return nvfp4_operand_k(rows, k, std)
 
     a_codes, a_sf, a_ts = nvfp4_operand(m, 1.0)
     w_codes, w_sf, w_ts = nvfp4_operand(n, 0.02)
@@ -886,7 +925,31 @@ def time_producer(b, device, reps=10, m=8192, n=4096, k=4096):
            "epilogue_out_bytes": int(out_bytes),
            "with_fp32_D_written_us": round(t_d * 1e6, 2),
            "warning_bits": warn}
-    del a_codes, a_sf, codes, scales, smma, d, hints
+    del a_codes, a_sf, w_codes, w_sf, codes, scales, smma, d, hints
+
+    # the same product with a 4x longer reduction (k = 16384): the epilogue's
+    # share shrinks and the main loop's rate shows
+    k_long = 4 * k
+    a_codes, a_sf, a_ts = nvfp4_operand_k(m, k_long, 1.0)
+    w_codes, w_sf, w_ts = nvfp4_operand_k(n, k_long, 0.02)
+    codes, scales, ts, ws, hints = b.empty_nvfp4(m, n, device, hint_bits=HINT_BITS)
+    smma = torch.empty(b.mma_scale_bytes(m, n // 16), **u8)
+    ws.zero_()
+
+    def call_long(r):
+        b.nvfp4_gemm_quantize(a_codes, a_sf, a_ts, w_codes, w_sf, w_ts, m, n, k_long, ws, codes, scales,
+                              ts, scales_mma=smma, hints=hints, hint_bits=HINT_BITS)
+
+    call_long(0)
+    torch.cuda.synchronize()
+    ws[0] = ws[2]
+    t_l = _timed(call_long, reps, flush)
+    tf_l = 2.0 * m * n * k_long / t_l / 1e12
+    out["long_k"] = {"workload": "NVFP4 [%d x %d] x NVFP4 weight [%d x %d]^T -> NVFP4 + %d-bit hints"
+                                 % (m, k_long, n, k_long, HINT_BITS),
+                     "avg_us": round(t_l * 1e6, 2), "TFLOP/s": round(tf_l, 1), "frac": round(tf_l / peak, 4),
+                     "warning_bits": int(ws[1].item())}
+    del a_codes, a_sf, w_codes, w_sf, codes, scales, smma, hints
 
     # MoE form: 8 experts x 2048 routed rows (8192 tokens, top-2), hidden k ->
     # expert width n_e, one launch for all experts, each expert its own scale

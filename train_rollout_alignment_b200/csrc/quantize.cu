@@ -107,18 +107,28 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
                    uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
                    float* __restrict__ tensor_scale, uint8_t* __restrict__ hints) {
   __shared__ ScaleTables tab;
+  const int64_t stride = (int64_t)gridDim.x * kThreads;
+  int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x;
+  // the first step's loads are issued before the tables are built
+  Block16 b[U];
+  bool step = i + (U - 1) * stride < nblk;
+  if (step) {
+#pragma unroll
+    for (int u = 0; u < U; ++u) b[u] = ld_block(x + (nblk - 1 - (i + u * stride)) * 16);
+  }
   const float s_t = tensor_scale_from_amax(__uint_as_float(ws[0]));
   if (blockIdx.x == 0 && threadIdx.x == 0) *tensor_scale = s_t;
   scale_tables_init(tab, s_t);
-  const int64_t stride = (int64_t)gridDim.x * kThreads;
-  int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x;
-  for (; i + (U - 1) * stride < nblk; i += U * stride) {
-    Block16 b[U];
-#pragma unroll
-    for (int u = 0; u < U; ++u) b[u] = ld_block(x + (nblk - 1 - (i + u * stride)) * 16);
+  while (step) {
 #pragma unroll
     for (int u = 0; u < U; ++u)
       rtn_block<HB>(b[u], s_t, tab, nblk - 1 - (i + u * stride), codes, scales, hints);
+    i += U * stride;
+    step = i + (U - 1) * stride < nblk;
+    if (step) {
+#pragma unroll
+      for (int u = 0; u < U; ++u) b[u] = ld_block(x + (nblk - 1 - (i + u * stride)) * 16);
+    }
   }
   for (; i < nblk; i += stride)
     rtn_block<HB>(ld_block(x + (nblk - 1 - i) * 16), s_t, tab, nblk - 1 - i, codes, scales, hints);
@@ -257,26 +267,34 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
              unsigned long long* __restrict__ stats4, uint32_t one) {
   __shared__ unsigned long long red[3 * 8];
   __shared__ ScaleTables tab;
-  const float s_t = tensor_scale_from_amax(__uint_as_float(ws[0]));
-  if (blockIdx.x == 0 && threadIdx.x == 0) *tensor_scale = s_t;
-  scale_tables_init(tab, s_t);
   GuidedCounts cnt{0u, 0u, 0u};
   const int64_t stride = (int64_t)gridDim.x * kThreads;
   int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x;
-  for (; i + (U - 1) * stride < nblk; i += U * stride) {
-    Block16 b[U];
-    uint32_t hw[U];
-    uint2 h4[U];
+  Block16 b[U];
+  uint32_t hw[U];
+  uint2 h4[U];
+  auto load_step = [&]() {
 #pragma unroll
     for (int u = 0; u < U; ++u) {
       const int64_t blk = nblk - 1 - (i + u * stride);
       b[u] = ld_block(x + blk * 16);
       hw[u] = hint_field<HB>(hints, blk, h4[u]);
     }
+  };
+  // the first step's loads are issued before the tables are built
+  bool step = i + (U - 1) * stride < nblk;
+  if (step) load_step();
+  const float s_t = tensor_scale_from_amax(__uint_as_float(ws[0]));
+  if (blockIdx.x == 0 && threadIdx.x == 0) *tensor_scale = s_t;
+  scale_tables_init(tab, s_t);
+  while (step) {
 #pragma unroll
     for (int u = 0; u < U; ++u)
       guided_block<HB>(b[u], hw[u], h4[u], s_t, tab, nblk - 1 - (i + u * stride), codes, scales, cnt,
                        one);
+    i += U * stride;
+    step = i + (U - 1) * stride < nblk;
+    if (step) load_step();
   }
   for (; i < nblk; i += stride) {
     const int64_t blk = nblk - 1 - i;
@@ -446,13 +464,32 @@ __global__ void __launch_bounds__(kStagedThreads, kGuidedCtas)
   const uint32_t sbase = umma::smem_u32(stage_smem);
   const uint32_t full = sbase + kGuidedStages * L::bytes, empty = full + 8 * kGuidedStages;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  if (threadIdx.x == 0) {
+  const int64_t nfull = nblk / kStageBlocks;  // whole chunks
+  const int64_t tail0 = nfull * kStageBlocks;  // blocks tail0 .. nblk-1: direct loads, CTA 0
+  const bool producer = warp == kComputeWarps && lane == 0;
+  auto load_chunk = [&](int64_t c, int s) {  // chunks are visited from the end backwards
+    const int64_t b0 = (nfull - 1 - c) * kStageBlocks;
+    const uint32_t bar = full + 8 * s, st = sbase + s * L::bytes;
+    umma::mbar_arrive_expect_tx(bar, L::payload);
+    umma::bulk_load(st + L::x, x + b0 * 16, kStageBlocks * 32, bar);
+    if (HB != 0) umma::bulk_load(st + L::hints, hints + b0 * L::kHintBytes, kStageBlocks * L::kHintBytes, bar);
+    if (STATS) {
+      umma::bulk_load(st + L::rc, rcodes + b0 * 8, kStageBlocks * 8, bar);
+      umma::bulk_load(st + L::rs, rscales + b0, kStageBlocks, bar);
+    }
+  };
+  // The producer sets up the ring and fills every stage before the CTA
+  // builds its tables, so the first loads overlap that set-up.
+  int64_t c0 = blockIdx.x;
+  int it0 = 0;
+  if (producer) {
     for (int s = 0; s < kGuidedStages; ++s) {
       umma::mbar_init(full + 8 * s, 1);
       umma::mbar_init(empty + 8 * s, kComputeWarps);
     }
     abort_flag = 0;
     umma::fence_mbar_init();
+    for (; it0 < kGuidedStages && c0 < nfull; ++it0, c0 += gridDim.x) load_chunk(c0, it0);
   }
   const float s_t = tensor_scale_from_amax(__uint_as_float(ws[0]));
   if (blockIdx.x == 0 && threadIdx.x == 0) *tensor_scale = s_t;
@@ -462,29 +499,19 @@ __global__ void __launch_bounds__(kStagedThreads, kGuidedCtas)
   bool far_all = false;
   if constexpr (STATS) far_all = stats_tables_init(sm, ts_r, s_t);
   volatile int* abort = &abort_flag;
-  const int64_t nfull = nblk / kStageBlocks;  // whole chunks
-  const int64_t tail0 = nfull * kStageBlocks;  // blocks tail0 .. nblk-1: direct loads, CTA 0
   GuidedCounts gcnt{0u, 0u, 0u};
   MismatchCounts mc{0u, 0u, 0u, 0u, 0u};
   int qn = 0;
 
   if (warp == kComputeWarps) {
     // ---------------- producer: one lane issues the bulk copies
-    if (lane == 0) {
-      int it = 0;
-      for (int64_t c = blockIdx.x; c < nfull; c += gridDim.x, ++it) {
+    if (producer) {
+      int it = it0;
+      for (int64_t c = c0; c < nfull; c += gridDim.x, ++it) {
         const int s = it % kGuidedStages;
         const uint32_t ph = (uint32_t)(it / kGuidedStages) & 1u;
         if (!umma::mbar_wait(empty + 8 * s, ph ^ 1u, abort)) break;
-        const int64_t b0 = (nfull - 1 - c) * kStageBlocks;
-        const uint32_t bar = full + 8 * s, st = sbase + s * L::bytes;
-        umma::mbar_arrive_expect_tx(bar, L::payload);
-        umma::bulk_load(st + L::x, x + b0 * 16, kStageBlocks * 32, bar);
-        if (HB != 0) umma::bulk_load(st + L::hints, hints + b0 * L::kHintBytes, kStageBlocks * L::kHintBytes, bar);
-        if (STATS) {
-          umma::bulk_load(st + L::rc, rcodes + b0 * 8, kStageBlocks * 8, bar);
-          umma::bulk_load(st + L::rs, rscales + b0, kStageBlocks, bar);
-        }
+        load_chunk(c, s);
       }
     }
     __syncwarp();

@@ -136,35 +136,44 @@ __global__ void __launch_bounds__(kStatsStagedThreads, kStatsStagedCtas)
   const uint32_t sbase = umma::smem_u32(stage_smem);
   const uint32_t full = sbase + kStatsStages * kSsBytes, empty = full + 8 * kStatsStages;
   const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
-  if (t == 0) {
+  const int64_t nfull = nblk / kStatsChunk;
+  const bool producer = warp == kWarps && lane == 0;
+  auto load_chunk = [&](int64_t ch, int s) {
+    const int64_t b0 = ch * kStatsChunk;
+    const uint32_t bar = full + 8 * s, st = sbase + s * kSsBytes;
+    umma::mbar_arrive_expect_tx(bar, kSsPayload);
+    umma::bulk_load(st + kSsCa, ca + b0 * 8, kStatsChunk * 8, bar);
+    umma::bulk_load(st + kSsCb, cb + b0 * 8, kStatsChunk * 8, bar);
+    umma::bulk_load(st + kSsSa, sa + b0, kStatsChunk, bar);
+    umma::bulk_load(st + kSsSb, sb + b0, kStatsChunk, bar);
+  };
+  // The producer sets up the ring and fills every stage before the CTA
+  // builds its tables, so the first loads overlap that set-up.
+  int64_t ch0 = blockIdx.x;
+  int it0 = 0;
+  if (producer) {
     for (int s = 0; s < kStatsStages; ++s) {
       umma::mbar_init(full + 8 * s, 1);
       umma::mbar_init(empty + 8 * s, kWarps);
     }
     abort_flag = 0;
     umma::fence_mbar_init();
+    for (; it0 < kStatsStages && ch0 < nfull; ++it0, ch0 += gridDim.x) load_chunk(ch0, it0);
   }
   const float tsa = *ta, tsb = *tb;
   const bool same_ts = __float_as_uint(tsa) == __float_as_uint(tsb);
   const bool far_all = stats_tables_init(sm, tsa, tsb);  // ends in a barrier
   volatile int* abort = &abort_flag;
-  const int64_t nfull = nblk / kStatsChunk;
   MismatchCounts c{0u, 0u, 0u, 0u, 0u};
   int qn = 0;
   if (warp == kWarps) {
-    if (lane == 0) {  // producer
-      int it = 0;
-      for (int64_t ch = blockIdx.x; ch < nfull; ch += gridDim.x, ++it) {
+    if (producer) {
+      int it = it0;
+      for (int64_t ch = ch0; ch < nfull; ch += gridDim.x, ++it) {
         const int s = it % kStatsStages;
         const uint32_t ph = (uint32_t)(it / kStatsStages) & 1u;
         if (!umma::mbar_wait(empty + 8 * s, ph ^ 1u, abort)) break;
-        const int64_t b0 = ch * kStatsChunk;
-        const uint32_t bar = full + 8 * s, st = sbase + s * kSsBytes;
-        umma::mbar_arrive_expect_tx(bar, kSsPayload);
-        umma::bulk_load(st + kSsCa, ca + b0 * 8, kStatsChunk * 8, bar);
-        umma::bulk_load(st + kSsCb, cb + b0 * 8, kStatsChunk * 8, bar);
-        umma::bulk_load(st + kSsSa, sa + b0, kStatsChunk, bar);
-        umma::bulk_load(st + kSsSb, sb + b0, kStatsChunk, bar);
+        load_chunk(ch, s);
       }
     }
     __syncwarp();
