@@ -618,6 +618,16 @@ nvfp4_status nvfp4_measure_mul_wide(int64_t ctas, int64_t iters, uint64_t* cycle
 /* Human-readable name of a status code (static string, never NULL). */
 const char* nvfp4_status_string(nvfp4_status status);
 
+/*
+ * nvfp4_last_cuda_error -- the cudaError_t value (as int) behind the most
+ * recent NVFP4_ERR_CUDA returned on the calling host thread; 0 if no call on
+ * this thread has returned NVFP4_ERR_CUDA.  Not reset by later successful
+ * calls.  nvfp4_last_cuda_error_string: the CUDA runtime's text for it
+ * ("no error" for 0; static string, never NULL).
+ */
+int nvfp4_last_cuda_error(void);
+const char* nvfp4_last_cuda_error_string(void);
+
 #ifdef __cplusplus
 }
 #endif

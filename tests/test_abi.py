@@ -20,7 +20,7 @@ def _declared():
     for fname in os.listdir(os.path.join(ROOT, "include")):
         if fname.endswith(".h"):
             text = open(os.path.join(ROOT, "include", fname)).read()
-            names += re.findall(r"^\s*(?:nvfp4_status|const char\*|int64_t)\s+((?:nvfp4|mxfp8)_\w+)\s*\(", text, re.M)
+            names += re.findall(r"^\s*(?:nvfp4_status|const char\*|int64_t|int)\s+((?:nvfp4|mxfp8)_\w+)\s*\(", text, re.M)
     return sorted(set(names))
 
 
@@ -41,12 +41,55 @@ def test_library_exports_every_declared_symbol():
     assert not missing, missing
 
 
+def test_library_exports_only_the_c_abi():
+    """Everything but the C ABI is local to the library, so two copies loaded
+    in one process (or another library) cannot share its internals, e.g. the
+    launchers' per-device shared-memory opt-in flags."""
+    import shutil
+    import subprocess
+    if shutil.which("nm") is None:
+        pytest.skip("nm not available")
+    out = subprocess.run(["nm", "-D", "--defined-only", _lib_path()], capture_output=True, text=True,
+                         check=True).stdout
+    names = [line.split()[-1] for line in out.splitlines() if line.strip()]
+    extra = [n for n in names if not (n.startswith("nvfp4_") or n.startswith("mxfp8_"))]
+    assert not extra, extra[:10]
+    assert set(_declared()) <= set(names)
+
+
 def test_status_strings():
     lib = ctypes.CDLL(_lib_path())
     lib.nvfp4_status_string.restype = ctypes.c_char_p
     for s in range(6):
         assert lib.nvfp4_status_string(s)
     assert b"unknown" in lib.nvfp4_status_string(99)
+
+
+def test_last_cuda_error_names_the_failure_without_a_gpu():
+    """A call that passes validation but cannot launch (no driver or no GPU
+    here) returns NVFP4_ERR_CUDA, and nvfp4_last_cuda_error keeps the CUDA
+    error behind it; the binding puts its text into the exception."""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("needs a machine without a usable GPU (the call would launch)")
+    lib = ctypes.CDLL(_lib_path())
+    lib.nvfp4_last_cuda_error.restype = ctypes.c_int
+    lib.nvfp4_last_cuda_error_string.restype = ctypes.c_char_p
+    f = lib.nvfp4_tensor_amax
+    f.restype = ctypes.c_int
+    f.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p]
+    fake = 1 << 20  # the launch fails before any kernel could touch it
+    assert f(fake, 16, fake, None) == 4
+    err = lib.nvfp4_last_cuda_error()
+    assert err != 0
+    assert lib.nvfp4_last_cuda_error_string() not in (b"", b"no error")
+    # not reset by a later call that fails validation
+    assert f(fake, 15, fake, None) == 3
+    assert lib.nvfp4_last_cuda_error() == err
+    from train_rollout_alignment_b200 import _binding as b
+    with pytest.raises(b.Nvfp4Error) as ei:
+        b._check("nvfp4_tensor_amax", 4)
+    assert ei.value.cuda_error == err and "CUDA error %d" % err in str(ei.value)
 
 
 def test_validation_rejects_bad_arguments_without_a_gpu():

@@ -25,6 +25,8 @@ _I64 = ctypes.c_int64
 _I = ctypes.c_int
 _SIGS = {
     "nvfp4_status_string": (ctypes.c_char_p, [_I]),
+    "nvfp4_last_cuda_error": (_I, []),
+    "nvfp4_last_cuda_error_string": (ctypes.c_char_p, []),
     "nvfp4_tensor_amax": (_I, [_P, _I64, _P, _P]),
     "nvfp4_quantize_rtn": (_I, [_P, _I64, _I64, _P, _I, _P, _P, _P, _P, _I, _P]),
     "nvfp4_emit_hint": (_I, [_P, _I64, _I, _P, _P]),
@@ -77,10 +79,17 @@ NVFP4_SCALES_BLOCK16 = 0
 NVFP4_SCALES_TILE16 = 1
 
 
+NVFP4_ERR_CUDA = 4
+
+
 class Nvfp4Error(RuntimeError):
     def __init__(self, fn: str, status: int):
         self.status = status
-        super().__init__("%s: %s (status %d)" % (fn, nvfp4_status_string(status), status))
+        msg = "%s: %s (status %d)" % (fn, nvfp4_status_string(status), status)
+        if status == NVFP4_ERR_CUDA:
+            self.cuda_error = nvfp4_last_cuda_error()
+            msg += ": CUDA error %d, %s" % (self.cuda_error, nvfp4_last_cuda_error_string())
+        super().__init__(msg)
 
 
 def library_path() -> str:
@@ -89,6 +98,14 @@ def library_path() -> str:
 
 def nvfp4_status_string(status: int) -> str:
     return _lib.nvfp4_status_string(int(status)).decode()
+
+
+def nvfp4_last_cuda_error() -> int:
+    return int(_lib.nvfp4_last_cuda_error())
+
+
+def nvfp4_last_cuda_error_string() -> str:
+    return _lib.nvfp4_last_cuda_error_string().decode()
 
 
 def _ptr(t) -> int | None:

@@ -23,6 +23,7 @@ NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
     "-O3", "-lineinfo", "-std=c++17", "-fmad=false",
     "-Xcompiler", "-fPIC", "-shared", "-cudart", "static",
+    "-Xlinker", "--version-script=" + os.path.join(CSRC, "exports.map"),
 ]
 
 
@@ -32,7 +33,7 @@ def _nvcc() -> str:
 
 
 def _inputs():
-    files = [os.path.join(CSRC, f) for f in SOURCES + HEADERS]
+    files = [os.path.join(CSRC, f) for f in SOURCES + HEADERS + ["exports.map"]]
     files.append(os.path.join(ROOT, "include", "nvfp4_trace.h"))
     return files
 

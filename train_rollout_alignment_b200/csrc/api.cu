@@ -8,12 +8,23 @@
 #include "launch.h"
 
 namespace {
+// The CUDA error behind the calling thread's most recent NVFP4_ERR_CUDA.
+thread_local int g_last_cuda_error = 0;
+}  // namespace
+
+nvfp4_status nvfp4::status_from_cuda(cudaError_t e) {
+  if (e == cudaSuccess) return NVFP4_OK;
+  g_last_cuda_error = static_cast<int>(e);
+  return NVFP4_ERR_CUDA;
+}
+
+namespace {
 
 constexpr int64_t kMaxElems = int64_t(1) << 40;
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
-nvfp4_status from_cuda(cudaError_t e) { return e == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA; }
+nvfp4_status from_cuda(cudaError_t e) { return nvfp4::status_from_cuda(e); }
 
 // Shape checks shared by the [rows, cols] entry points.
 nvfp4_status check_shape(int64_t rows, int64_t cols, int64_t col_multiple) {
@@ -86,6 +97,12 @@ const char* nvfp4_status_string(nvfp4_status status) {
              "(NVFP4_SR_NOALLOC_MAX_BATCH matrices)";
     default: return "unknown status";
   }
+}
+
+int nvfp4_last_cuda_error(void) { return g_last_cuda_error; }
+
+const char* nvfp4_last_cuda_error_string(void) {
+  return g_last_cuda_error == 0 ? "no error" : cudaGetErrorString(static_cast<cudaError_t>(g_last_cuda_error));
 }
 
 nvfp4_status nvfp4_tensor_amax(const uint16_t* x_bf16, int64_t n, uint32_t* ws, void* stream) {

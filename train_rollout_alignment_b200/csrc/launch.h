@@ -96,4 +96,8 @@ cudaError_t launch_hint_pack(const uint8_t* const* srcs, const int64_t* sizes, i
                              uint8_t* staging, cudaStream_t s);
 cudaError_t launch_set_f32(float* dst, float value, cudaStream_t s);
 
+// Records e (when not cudaSuccess) as the calling thread's last CUDA error
+// (nvfp4_last_cuda_error) and returns the matching status.
+nvfp4_status status_from_cuda(cudaError_t e);
+
 }  // namespace nvfp4

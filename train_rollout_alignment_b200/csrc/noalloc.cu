@@ -35,13 +35,16 @@ uint32_t* g_scratch_addr[kMaxDevices] = {};
 // Device address of g_sr_scratch on the current device (set up on first use).
 nvfp4_status scratch_on_current_device(uint32_t** out) {
   int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return NVFP4_ERR_CUDA;
+  const cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return nvfp4::status_from_cuda(e);
+  if (dev < 0 || dev >= kMaxDevices) return nvfp4::status_from_cuda(cudaErrorInvalidDevice);
   std::lock_guard<std::mutex> lock(g_scratch_mu);
   if (g_scratch_addr[dev] == nullptr) {
     void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_sr_scratch) != cudaSuccess || p == nullptr) {
+    const cudaError_t ea = cudaGetSymbolAddress(&p, g_sr_scratch);
+    if (ea != cudaSuccess || p == nullptr) {
       cudaGetLastError();
-      return NVFP4_ERR_CUDA;
+      return nvfp4::status_from_cuda(ea != cudaSuccess ? ea : cudaErrorInvalidSymbol);
     }
     g_scratch_addr[dev] = static_cast<uint32_t*>(p);
   }

@@ -25,8 +25,12 @@ namespace nvfp4 {
 #ifndef NVFP4_STREAM_UNROLL
 #define NVFP4_STREAM_UNROLL 2
 #endif
+#ifndef NVFP4_GUIDED_UNROLL
+#define NVFP4_GUIDED_UNROLL 3   // guided alone: three blocks in flight per thread (measured best)
+#endif
 constexpr int kCtasPerSm = NVFP4_STREAM_CTAS;
 constexpr int kUnroll = NVFP4_STREAM_UNROLL;
+constexpr int kGuidedUnroll = NVFP4_GUIDED_UNROLL;
 constexpr int kAmaxUnroll = 4;  // 128 bytes in flight per thread: the amax pass has no other work
 
 // ----------------------------------------------------------------- amax
@@ -415,10 +419,10 @@ __global__ void __launch_bounds__(kThreads, kGsCtasPerSm)
 #define NVFP4_GUIDED_BPT 2
 #endif
 #ifndef NVFP4_GUIDED_STAGES
-#define NVFP4_GUIDED_STAGES 3
+#define NVFP4_GUIDED_STAGES 2
 #endif
 #ifndef NVFP4_GUIDED_CTAS
-#define NVFP4_GUIDED_CTAS 2
+#define NVFP4_GUIDED_CTAS 3
 #endif
 constexpr int kGuidedBpt = NVFP4_GUIDED_BPT;        // blocks per compute thread and chunk
 constexpr int kStageBlocks = kThreads * kGuidedBpt; // blocks per chunk
@@ -856,9 +860,9 @@ cudaError_t launch_guided(const uint16_t* x, int64_t nblk, const uint8_t* hints,
 #else
   const int g = grid_for(nblk, kThreads, kCtasPerSm);
   switch (hint_bits) {
-    case 1: k_guided<1, kUnroll><<<g, kThreads, 0, s>>>(x, nblk, hints, ws, codes, scales, tensor_scale, stats4, 1u); break;
-    case 2: k_guided<2, kUnroll><<<g, kThreads, 0, s>>>(x, nblk, hints, ws, codes, scales, tensor_scale, stats4, 1u); break;
-    case 4: k_guided<4, kUnroll><<<g, kThreads, 0, s>>>(x, nblk, hints, ws, codes, scales, tensor_scale, stats4, 1u); break;
+    case 1: k_guided<1, kGuidedUnroll><<<g, kThreads, 0, s>>>(x, nblk, hints, ws, codes, scales, tensor_scale, stats4, 1u); break;
+    case 2: k_guided<2, kGuidedUnroll><<<g, kThreads, 0, s>>>(x, nblk, hints, ws, codes, scales, tensor_scale, stats4, 1u); break;
+    case 4: k_guided<4, kGuidedUnroll><<<g, kThreads, 0, s>>>(x, nblk, hints, ws, codes, scales, tensor_scale, stats4, 1u); break;
     default: return cudaErrorInvalidValue;
   }
   return cudaGetLastError();
