@@ -156,7 +156,10 @@ __global__ void __launch_bounds__(kThreads, kRhtCtasPerSm)
   scale_tables_init_f32(tab, s_t);
   const f32x2 c2 = pack2(kInvSqrt32, kInvSqrt32);
   const int64_t stride = (int64_t)gridDim.x * kThreads;
-  for (int64_t g = (int64_t)blockIdx.x * kThreads + threadIdx.x; g < ngroups; g += stride) {
+  // Groups are visited from the END of the tensor backwards: the amax pass
+  // just before streamed forwards, so the tail it read last is still in L2.
+  for (int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x; i < ngroups; i += stride) {
+    const int64_t g = ngroups - 1 - i;
     f32x2 P[16];
     hadamard32(x + g * 32, masks, P);
     float z[32];
