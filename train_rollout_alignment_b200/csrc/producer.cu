@@ -429,7 +429,7 @@ __global__ void __launch_bounds__(kProducerThreads, kCtasPerSm)
 // loads are TMA loads (no multicast) whose completion is counted on the even
 // CTA's barrier; the MMA's completion is signalled to both CTAs.
 #ifndef NVFP4_PAIR_STAGES
-#define NVFP4_PAIR_STAGES 4
+#define NVFP4_PAIR_STAGES 5
 #endif
 constexpr int kPairStages = NVFP4_PAIR_STAGES;
 constexpr int kPairBN = 256;                                 // output columns per tile
