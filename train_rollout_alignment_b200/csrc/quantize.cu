@@ -328,7 +328,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 #define NVFP4_GS_UNROLL 2
 #endif
 constexpr int kGsCtasPerSm = NVFP4_GS_CTAS;
-constexpr int kGsUnroll = NVFP4_GS_UNROLL;
+[[maybe_unused]] constexpr int kGsUnroll = NVFP4_GS_UNROLL;  // register form only
 
 template <int HB, int U>
 __global__ void __launch_bounds__(kThreads, kGsCtasPerSm)

@@ -35,7 +35,7 @@
 namespace nvfp4 {
 
 constexpr int kStatsCtasPerSm = 4;
-constexpr int kStatsUnroll = 2;  // two pairs (four blocks) in flight per lane
+[[maybe_unused]] constexpr int kStatsUnroll = 2;  // register form: two pairs (four blocks) in flight per lane
 
 template <int U>
 __global__ void __launch_bounds__(kThreads, kStatsCtasPerSm)
