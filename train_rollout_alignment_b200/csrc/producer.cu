@@ -431,11 +431,22 @@ __global__ void __launch_bounds__(kProducerThreads, kCtasPerSm)
 #ifndef NVFP4_PAIR_STAGES
 #define NVFP4_PAIR_STAGES 5
 #endif
+// Scale factors into TMEM: 0 = one thread of a dedicated warp issues
+// tcgen05.cp copies (the default); 1 = four warps (one per lane quadrant)
+// load them from shared memory and write them with tcgen05.st.  Both give the
+// same results; the stores measured slower (123 against 85 us at 8192 x 4096
+// x 4096, 422 against 270 us at K = 16384), and with four more warps the
+// block's register budget leaves 80 per thread (the epilogue then reads the
+// accumulator in two 32-column loads).
+#ifndef NVFP4_PAIR_SF_ST
+#define NVFP4_PAIR_SF_ST 0
+#endif
 constexpr int kPairStages = NVFP4_PAIR_STAGES;
 constexpr int kPairBN = 256;                                 // output columns per tile
 constexpr int kPairEpiWarps = 16;
-constexpr int kPairSfWarp = 2 + kPairEpiWarps;                // the warp that copies scale factors
-constexpr int kPairThreads = 32 * (3 + kPairEpiWarps);
+constexpr int kPairSfWarp = 2 + kPairEpiWarps;                // the first scale-factor warp
+constexpr int kPairSfWarps = NVFP4_PAIR_SF_ST ? 4 : 1;
+constexpr int kPairThreads = 32 * (2 + kPairEpiWarps + kPairSfWarps);
 constexpr uint32_t kPairA = 128 * (kBK / 2);                  // 16 KB
 constexpr uint32_t kPairB = 128 * (kBK / 2);                  // 16 KB: this CTA's half of B
 constexpr uint32_t kPairSfa = (kBK / 64) * kScaleTile;        // 2 KB
@@ -445,8 +456,9 @@ constexpr uint32_t kPOffA = 0;
 constexpr uint32_t kPOffB = kPOffA + kPairStages * kPairA;
 constexpr uint32_t kPOffSfa = kPOffB + kPairStages * kPairB;
 constexpr uint32_t kPOffSfb = kPOffSfa + kPairStages * kPairSfa;
-constexpr uint32_t kPOffBar = kPOffSfb + kPairStages * kPairSfb;  // full[S], empty[S], acc_full, acc_empty, sf_ready[S]
-constexpr uint32_t kPOffSlot = kPOffBar + 8 * (3 * kPairStages + 2);
+// barriers: full[S], empty[S], acc_full, acc_empty, sf_ready[S], sf_landed[S]
+constexpr uint32_t kPOffBar = kPOffSfb + kPairStages * kPairSfb;
+constexpr uint32_t kPOffSlot = kPOffBar + 8 * (4 * kPairStages + 2);
 constexpr uint32_t kPOffAbort = kPOffSlot + 4;
 constexpr uint32_t kPOffTables = (kPOffAbort + 4 + 15) / 16 * 16;
 constexpr uint32_t kPairSmem = kPOffTables + sizeof(ScaleTables) + 1024;
@@ -475,6 +487,8 @@ __global__ void __launch_bounds__(kPairThreads, 1)
   const uint32_t full = base + kPOffBar, empty = full + 8 * kPairStages;
   const uint32_t acc_full = empty + 8 * kPairStages, acc_empty = acc_full + 8;
   const uint32_t sf_ready = acc_empty + 8;  // [S]: the stage's scale factors are in TMEM
+  // [S], per CTA: this CTA's scale tiles of the stage have landed (SF_ST form)
+  const uint32_t sf_landed = sf_ready + 8 * kPairStages;
   volatile int* abort = reinterpret_cast<volatile int*>(smem + kPOffAbort);
   ScaleTables& tab = *reinterpret_cast<ScaleTables*>(smem + kPOffTables);
 
@@ -485,7 +499,10 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     }
     mbar_init(acc_full, 1);
     mbar_init(acc_empty, 2 * kPairEpiWarps);
-    for (int st = 0; st < kPairStages; ++st) mbar_init(sf_ready + 8 * st, 1);
+    for (int st = 0; st < kPairStages; ++st) {
+      mbar_init(sf_ready + 8 * st, NVFP4_PAIR_SF_ST ? 2 * kPairSfWarps : 1);
+      mbar_init(sf_landed + 8 * st, 1);
+    }
     *abort = 0;
     fence_mbar_init();
     prefetch_tensormap(&tm_a);
@@ -520,14 +537,27 @@ __global__ void __launch_bounds__(kPairThreads, 1)
           const int s = it % kPairStages;
           const uint32_t ph = (uint32_t)(it / kPairStages) & 1u;
           if (!mbar_wait(empty + 8 * s, ph ^ 1u, abort)) break;
-          if (rank == 0) mbar_arrive_expect_tx(full + 8 * s, 2 * kPairStageTx);
           const uint32_t bar = mapa_shared(full + 8 * s, 0);
+#if NVFP4_PAIR_SF_ST
+          // A and B of both CTAs on CTA 0's barrier; this CTA's scale tiles on
+          // its own barrier, for its scale-factor warps
+          if (rank == 0) mbar_arrive_expect_tx(full + 8 * s, 2 * (kPairA + kPairB));
+          tma_load_2d_pair(base + kPOffA + s * kPairA, &tm_a, bar, kb * (kBK / 2), a_row);
+          tma_load_2d_pair(base + kPOffB + s * kPairB, &tm_b, bar, kb * (kBK / 2), b_row);
+          const uint32_t lb = sf_landed + 8 * s;
+          mbar_arrive_expect_tx(lb, kPairSfa + kPairSfb);
+          tma_load_2d(base + kPOffSfa + s * kPairSfa, &tm_sa, lb, 0, sfa_row + kb * 8);
+          tma_load_2d(base + kPOffSfb + s * kPairSfb, &tm_sb, lb, 0, sfb_row0 + kb * 8);
+          tma_load_2d(base + kPOffSfb + s * kPairSfb + kPairSfb / 2, &tm_sb, lb, 0, sfb_row1 + kb * 8);
+#else
+          if (rank == 0) mbar_arrive_expect_tx(full + 8 * s, 2 * kPairStageTx);
           tma_load_2d_pair(base + kPOffA + s * kPairA, &tm_a, bar, kb * (kBK / 2), a_row);
           tma_load_2d_pair(base + kPOffB + s * kPairB, &tm_b, bar, kb * (kBK / 2), b_row);
           tma_load_2d_pair(base + kPOffSfa + s * kPairSfa, &tm_sa, bar, 0, sfa_row + kb * 8);
           tma_load_2d_pair(base + kPOffSfb + s * kPairSfb, &tm_sb, bar, 0, sfb_row0 + kb * 8);
           tma_load_2d_pair(base + kPOffSfb + s * kPairSfb + kPairSfb / 2, &tm_sb, bar, 0,
                            sfb_row1 + kb * 8);
+#endif
         }
       }
       // drain: the MMA's completion signal for every stage has reached this
@@ -551,7 +581,12 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         for (int kb = 0; kb < kblocks; ++kb, ++it) {
           const int s = it % kPairStages;
           const uint32_t ph = (uint32_t)(it / kPairStages) & 1u;
+#if NVFP4_PAIR_SF_ST
+          if (!mbar_wait(full + 8 * s, ph, abort)) break;
+          if (!mbar_wait_cluster(sf_ready + 8 * s, ph, abort)) break;  // both CTAs' scale factors
+#else
           if (!mbar_wait(sf_ready + 8 * s, ph, abort)) break;  // implies the stage's data is in
+#endif
           tc_fence_after();
           const uint32_t sf = tmem + kPairTmemSf + 48u * (uint32_t)s;  // SFA +4j, SFB +16+8j
           const uint64_t da = desc_kmajor_sw128(base + kPOffA + s * kPairA);
@@ -566,7 +601,51 @@ __global__ void __launch_bounds__(kPairThreads, 1)
       }
     }
     __syncwarp();
-  } else if (warp == kPairSfWarp) {
+  } else if (warp >= kPairSfWarp) {
+#if NVFP4_PAIR_SF_ST
+    // ---------------- scale factors (both CTAs): the warp of lane quadrant q
+    // writes the stage's scale factors into its 32 TMEM lanes as soon as this
+    // CTA's scale tiles have landed: lane l takes the 16-byte row l of each
+    // 512-byte scale tile (the scales of rows l, l + 32, l + 64, l + 96) into
+    // 4 columns, the layout the MMA reads (every quadrant holds the same).
+    // The slot is free then: the tiles were reloaded only after the MMAs that
+    // read the slot last had completed.  Each warp then arrives on CTA 0's
+    // sf_ready.
+    const int q = warp & 3;
+    const uint32_t ready0 = mapa_shared(sf_ready, 0);
+    int it = 0;
+    bool go = true;
+    for (int tile = cluster; go && tile < tiles && !*abort; tile += clusters) {
+      for (int kb = 0; kb < kblocks; ++kb, ++it) {
+        const int s = it % kPairStages;
+        const bool ok = mbar_wait(sf_landed + 8 * s, (uint32_t)(it / kPairStages) & 1u, abort);
+        if (!__all_sync(0xFFFFFFFFu, ok)) {
+          go = false;
+          break;
+        }
+        const uint8_t* sa = smem + kPOffSfa + s * kPairSfa + 16 * lane;
+        const uint8_t* sb = smem + kPOffSfb + s * kPairSfb + 16 * lane;
+        uint32_t va[16], vb[32];
+#pragma unroll
+        for (int j = 0; j < kBK / 64; ++j) {
+          const uint4 a = *reinterpret_cast<const uint4*>(sa + j * kScaleTile);
+          const uint4 b0 = *reinterpret_cast<const uint4*>(sb + j * kScaleTile);
+          const uint4 b1 = *reinterpret_cast<const uint4*>(sb + kPairSfb / 2 + j * kScaleTile);
+          va[4 * j] = a.x; va[4 * j + 1] = a.y; va[4 * j + 2] = a.z; va[4 * j + 3] = a.w;
+          vb[8 * j] = b0.x; vb[8 * j + 1] = b0.y; vb[8 * j + 2] = b0.z; vb[8 * j + 3] = b0.w;
+          vb[8 * j + 4] = b1.x; vb[8 * j + 5] = b1.y; vb[8 * j + 6] = b1.z; vb[8 * j + 7] = b1.w;
+        }
+        const uint32_t taddr = tmem + ((uint32_t)(32 * q) << 16) + kPairTmemSf + 48u * (uint32_t)s;
+        tmem_st16(taddr, va);        // SFA: columns 4j .. 4j + 3
+        tmem_st32(taddr + 16, vb);   // SFB: columns 16 + 8j (rows 0-127), 20 + 8j (rows 128-255)
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(ready0 + 8 * s);
+      }
+    }
+    __syncwarp();
+#else
     // ---------------- scale-factor copies: CTA 0 only, as soon as a stage has
     // landed.  Its TMEM slot is free then: the stage was reloaded only after
     // the MMAs that read the slot last had completed.
@@ -592,6 +671,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
       }
     }
     __syncwarp();
+#endif
   } else {
     // ---------------- epilogue (both CTAs): this CTA's 128 rows of the tile
     const int q = warp & 3;            // TMEM lane quadrant this warp may read
@@ -610,7 +690,14 @@ __global__ void __launch_bounds__(kPairThreads, 1)
       if (!__all_sync(0xFFFFFFFFu, ok)) break;
       tc_fence_after();
       float y[64];
+#if NVFP4_PAIR_SF_ST
+      // two loads of 32 columns: with four scale-factor warps the block's
+      // register budget leaves too few for one 64-column load
+      tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(cg * 64), y);
+      tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(cg * 64 + 32), y + 32);
+#else
       tmem_ld64(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(cg * 64), y);
+#endif
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(acc_empty0);  // the accumulator may be overwritten
