@@ -105,14 +105,18 @@ __global__ void __launch_bounds__(kThreads)
     const int64_t r = r0 + row, c = c0 + 32 * q;
     uint4 v = make_uint4(0u, 0u, 0u, 0u);
     if (r < rows && c < cols) {
-      const uint2* p = reinterpret_cast<const uint2*>(src + r * (cols / 2) + c / 2);
-      const uint2 lo = __ldg(p);
-      v.x = lo.x;
-      v.y = lo.y;
-      if (c + 32 <= cols) {  // else cols % 32 == 16: the row ends after 16 elements
-        const uint2 hi = __ldg(p + 1);
-        v.z = hi.x;
-        v.w = hi.y;
+      if ((cols & 31) == 0) {  // 16-byte row segments: one load (codes are 16-byte aligned)
+        v = __ldg(reinterpret_cast<const uint4*>(src + r * (cols / 2) + c / 2));
+      } else {
+        const uint2* p = reinterpret_cast<const uint2*>(src + r * (cols / 2) + c / 2);
+        const uint2 lo = __ldg(p);
+        v.x = lo.x;
+        v.y = lo.y;
+        if (c + 32 <= cols) {  // else the row ends after 16 elements
+          const uint2 hi = __ldg(p + 1);
+          v.z = hi.x;
+          v.w = hi.y;
+        }
       }
     }
     sq[row][4 * q] = v.x;
@@ -132,12 +136,22 @@ __global__ void __launch_bounds__(kThreads)
   uint32_t m[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) m[i] = sq[8 * br + i][bc];
+  // 4x4 and 2x2 nibble blocks move as whole half-words and bytes (one byte
+  // permute per output word); single nibbles by masked swaps
 #pragma unroll
-  for (int i = 0; i < 4; ++i) nib_swap(m[i], m[i + 4], 16, 0x0000FFFFu);
+  for (int i = 0; i < 4; ++i) {
+    const uint32_t a = m[i], b = m[i + 4];
+    m[i] = __byte_perm(a, b, 0x5410);      // low halves of a, b
+    m[i + 4] = __byte_perm(a, b, 0x7632);  // high halves
+  }
 #pragma unroll
   for (int i = 0; i < 8; i += 4) {
-    nib_swap(m[i], m[i + 2], 8, 0x00FF00FFu);
-    nib_swap(m[i + 1], m[i + 3], 8, 0x00FF00FFu);
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const uint32_t a = m[i + k], b = m[i + k + 2];
+      m[i + k] = __byte_perm(a, b, 0x6240);      // bytes a0 b0 a2 b2
+      m[i + k + 2] = __byte_perm(a, b, 0x7351);  // bytes a1 b1 a3 b3
+    }
   }
 #pragma unroll
   for (int i = 0; i < 8; i += 2) nib_swap(m[i], m[i + 1], 4, 0x0F0F0F0Fu);
