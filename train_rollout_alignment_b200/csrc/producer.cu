@@ -427,7 +427,8 @@ __global__ void __launch_bounds__(kProducerThreads, kCtasPerSm)
 // accumulator, so 16 epilogue warps load their 64 columns each into
 // registers at once and hand the accumulator back before quantizing.  All
 // loads are TMA loads (no multicast) whose completion is counted on the even
-// CTA's barrier; the MMA's completion is signalled to both CTAs.
+// CTA's barrier (in the tcgen05.st form below, the scale tiles on each CTA's
+// own); the MMA's completion is signalled to both CTAs.
 #ifndef NVFP4_PAIR_STAGES
 #define NVFP4_PAIR_STAGES 5
 #endif
