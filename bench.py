@@ -584,8 +584,9 @@ def time_other_kernels(b, stack, device, peak, sm_mhz, reps=10):
     re-quantize (128 x 512 x 2048 expert stack) and RHT32 + quantize
     (16384 x 4096 activation with outliers): seconds per call and algorithmic
     GB/s (median of `reps` calls), L2 flushed before every call; kernels whose
-    inputs are more than twice the L2 (the counters, the two quantizers alone,
-    tile quantize) are timed back to back, the flushed figure beside it."""
+    inputs are more than twice the L2 (the amax pass, the counters, the two
+    quantizers alone, tile quantize) are timed back to back, the flushed
+    figure beside it."""
     from train_rollout_alignment_b200 import synthetic as syn
     flush = (torch.zeros(64 << 20, dtype=torch.float32, device=device),
              torch.ones(64 << 20, dtype=torch.float32, device=device))
@@ -599,6 +600,19 @@ def time_other_kernels(b, stack, device, peak, sm_mhz, reps=10):
     gbs = BYTES["emit_hint"] * stack.n / t / 1e9
     out["emit_hint"] = {"workload": "%dx%d codes, 2-bit hints" % (ROWS, COLS), "avg_us": round(t * 1e6, 2),
                         "GB/s": round(gbs, 1), "frac": round(gbs / peak, 4), "bytes_per_elem": BYTES["emit_hint"]}
+    # the amax pass alone on that layer's rollout input (in the step each launch
+    # follows a writer and pays for its output write-back): back to back and flushed
+    ws_tmp = torch.zeros(8, dtype=torch.int32, device=device)
+    amax_call = lambda r: b.nvfp4_tensor_amax(stack.xr[l], ws_tmp)
+    t = _timed_b2b(amax_call)
+    t_f = _timed(amax_call, reps, flush)
+    gbs = BYTES["amax"] * stack.n / t / 1e9
+    out["amax (alone)"] = {"workload": "%dx%d BF16 layer %d" % (ROWS, COLS, l),
+                           "timing": "10 calls back to back, inputs > 2x L2",
+                           "avg_us": round(t * 1e6, 2), "GB/s": round(gbs, 1), "frac": round(gbs / peak, 4),
+                           "flushed_us": round(t_f * 1e6, 2),
+                           "flushed_frac": round(BYTES["amax"] * stack.n / t_f / 1e9 / peak, 4),
+                           "bytes_per_elem": BYTES["amax"]}
     # the standalone counters (the step counts inside the guided pass) between
     # the rollout and train tensors of that layer
     # (inputs of 302 MB: timed back to back, the L2-flushed figure beside it)
